@@ -1,0 +1,457 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE routing hot path on B200.
+
+Workload (one step): moe_route on the DeepSeek-V3-style grouped sigmoid batch --
+T=16384 tokens, E=256 experts, top-8, 8 groups keep 4 (group score = sum of the
+top-2 biased scores), bf16 logits ~N(0,2), fp32 correction bias ~U(-0.1,0.1),
+renormalised weights x 2.5 stored bf16, tile 128 -- i.e. selection, weights and
+the full permutation bookkeeping in one launch.
+
+Metric: routed tokens/s (and us per call); the roofline object reports the
+route kernel's algorithmic bytes / event-timed duration against the measured
+HBM copy bandwidth.  L2: every timed step reads and writes one of ROTATE input
+and output sets whose total exceeds the 126 MB L2.
+
+Multi-GPU: one process per GPU (torchrun); each rank routes its own batch of
+the same shape (data-parallel, no collective on the path; weak scaling).  The
+timed region is bracketed by a barrier and a device synchronize; the max over
+ranks is reported.
+
+--impl reference times the CPU oracle (test infrastructure) on the same
+workload: this pages' methods have no runnable reference implementation.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "routed tokens/s (moe_route, grouped sigmoid top-8 of 256 + permutation bookkeeping)"
+UNIT = "tokens/s"
+ROTATE = 24
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=("cuda", "reference"), default="cuda")
+    ap.add_argument("--no-extra", action="store_true", help="skip the secondary workloads")
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+def route_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("route.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "top_expert_selection_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic_per_launch():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this exact source."""
+    path = os.path.join(ROOT, "profiles", "route_kernel_dsv3_grouped_sigmoid.txt")
+    try:
+        kv = {}
+        with open(path) as f:
+            for line in f:
+                if ":" in line:
+                    k, _, v = line.partition(":")
+                    kv[k.strip()] = v.strip()
+        if kv.get("source_sha256_16") != route_source_hash():
+            return None
+        return int(kv["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"moe_bench_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}",
+                 "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "20"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    mx.append(float(parts[1]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[4:8]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def algorithmic_bytes(T, E, k, P, ntiles, logits_bytes=2, bias_bytes=4, w_bytes=2):
+    """Bytes the route step must move once: inputs read, outputs written, no intermediates."""
+    return (T * E * logits_bytes + E * bias_bytes            # logits, bias
+            + T * k * 4 + T * k * w_bytes                     # ids, weights
+            + E * 4 + (E + 1) * 4 + 2 * 4                     # counts, offsets, totals
+            + T * k * 4 + P * 4                               # expanded->permuted, permuted->token
+            + 2 * ntiles * 4)                                 # tile expert, tile row limit
+
+
+def cpu_baseline(budget_s: float = 12.0):
+    """The CPU oracle (single thread, as it stands) on the same workload, repeated up to ~budget_s."""
+    import oracle
+    from top_expert_selection_b200 import workloads as W
+    spec = W.DSV3_GROUPED_SIGMOID
+    inp = W.route_inputs(spec)
+    lg, b = oracle.as_numpy(inp["logits"]), oracle.as_numpy(inp["bias"])
+    n = 0
+    t0 = time.perf_counter()
+    while True:
+        sel = oracle.route_select(lg, k=spec.k, score_fn=spec.score_fn, n_group=spec.n_group,
+                                  topk_group=spec.topk_group, renormalize=1, scaling_factor=spec.scaling_factor, bias=b)
+        oracle.f32_to_bf16(sel["weights"][:1])
+        oracle.route_bookkeeping(sel["ids"], spec.E, spec.tile_tokens_dim)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or n >= 50:
+            break
+    return {"value": spec.T * n / el, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"the full {spec.T}-token batch routed {n}x (selection, weights, bookkeeping) "
+                      f"by the single-threaded C oracle, {el:.1f} s"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    from top_expert_selection_b200 import workloads as W
+    spec = W.DSV3_GROUPED_SIGMOID
+    for _ in range(max(0, min(args.warmup, 1))):
+        cpu_baseline(budget_s=0.0)
+    cb = cpu_baseline()
+    line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * spec.T / cb["value"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": workload_config(), "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config():
+    return {"workload": "dsv3_grouped_sigmoid_route: T=16384 E=256 top_k=8 n_group=8 topk_group=4 "
+                        "(top-2 group score) bf16 logits N(0,2) fp32 bias U(-0.1,0.1) renorm scale=2.5 tile=128 "
+                        "bf16 weights",
+            "global_batch": 16384, "parallelism": "data-parallel replicas (one batch per GPU)",
+            "l2": f"inputs/outputs rotated over {ROTATE} sets (> 126 MB L2); launches replayed from a CUDA graph"}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    from top_expert_selection_b200 import binding as B
+    from top_expert_selection_b200 import workloads as W
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        pg = dist
+
+    spec = W.DSV3_GROUPED_SIGMOID.with_(seed=W.DSV3_GROUPED_SIGMOID.seed + rank)
+    inp = W.route_inputs(spec)
+    p = B.route_params(spec.T, spec.E, spec.k, score_fn=spec.score_fn, n_group=spec.n_group,
+                       topk_group=spec.topk_group, group_score_topn=spec.group_score_topn, renormalize=1,
+                       scaling_factor=spec.scaling_factor, tile_tokens_dim=spec.tile_tokens_dim,
+                       logits_dtype=spec.logits_dtype, bias_dtype=spec.bias_dtype, weights_dtype=spec.weights_dtype)
+    routers = [B.Router(p, dev) for _ in range(ROTATE)]
+    logits = [inp["logits"].to(dev) for _ in range(ROTATE)]
+    bias = inp["bias"].to(dev)
+    stream = torch.cuda.Stream(dev)
+    with torch.cuda.stream(stream):
+        for i in range(ROTATE):
+            routers[i](logits[i], bias)
+    torch.cuda.synchronize()
+
+    chunk = ROTATE
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(chunk):
+            routers[i](logits[i], bias)
+    torch.cuda.synchronize()
+
+    def run_steps(n):
+        full, rest = divmod(n, chunk)
+        for _ in range(full):
+            graph.replay()
+        for i in range(rest):
+            routers[i](logits[i], bias)
+
+    # warm-up
+    with torch.cuda.stream(stream):
+        run_steps(args.warmup)
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.05)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        run_steps(args.steps)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if pg:
+        pg.barrier()
+    ms_total = e0.elapsed_time(e1)
+    if pg:
+        t = torch.tensor([ms_total], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    value = world * spec.T / (ms_step / 1000.0)
+
+    # correctness of what was timed: every rotated output set reports OK and the same bookkeeping
+    ok = all(B.status(r.ws) == B.MOE_OK for r in routers)
+    tot = routers[0].out["totals"].tolist()
+    P, ntiles = int(tot[0]), int(tot[1])
+    alg = algorithmic_bytes(spec.T, spec.E, spec.k, P, ntiles)
+    hbm, tflops, peak_kind = load_peaks()
+    achieved = alg / (ms_step / 1000.0) / 1e9
+
+    # end to end through host buffers: pinned inputs -> device, route, outputs -> pinned host, every step
+    e2e = None
+    if rank == 0 or True:
+        h_logits = inp["logits"].pin_memory()
+        h_bias = inp["bias"].pin_memory()
+        r0 = routers[0]
+        out_names = ("ids", "weights", "counts", "offsets", "e2p", "p2t", "tile_expert", "tile_mn_limit", "totals")
+        h_out = {n: torch.empty_like(r0.out[n], device="cpu").pin_memory() for n in out_names}
+        d_logits = logits[0]
+        d_bias = torch.empty_like(bias)
+        n_e2e = max(20, min(2000, args.steps // 10))
+        h2d = h_logits.numel() * h_logits.element_size() + h_bias.numel() * h_bias.element_size()
+        d2h = sum(h_out[n].numel() * h_out[n].element_size() for n in out_names)
+
+        def e2e_step():
+            d_logits.copy_(h_logits, non_blocking=True)
+            d_bias.copy_(h_bias, non_blocking=True)
+            o = r0(d_logits, d_bias)
+            for n in out_names:
+                h_out[n].copy_(o[n], non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            for _ in range(5):
+                e2e_step()
+        torch.cuda.synchronize()
+        if pg:
+            pg.barrier()
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            f0.record(stream)
+            for _ in range(n_e2e):
+                e2e_step()
+            f1.record(stream)
+        torch.cuda.synchronize()
+        ms_e2e = f0.elapsed_time(f1) / n_e2e
+        if pg:
+            t = torch.tensor([ms_e2e], device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        e2e = {"value": world * spec.T / (ms_e2e / 1000.0), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": ms_e2e, "steps": n_e2e}
+
+    extra = None
+    if rank == 0 and not args.no_extra:
+        try:
+            extra = secondary_rows(dev, hbm)
+        except Exception as exc:  # reported, never hides the headline
+            extra = {"error": repr(exc)}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "us_per_call": ms_step * 1000.0,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; shapes and distributions of the grouped-sigmoid routing workload)",
+            "config": workload_config(),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                         "frac": achieved / hbm, "traffic": ncu_traffic_per_launch(),
+                         "algorithmic_bytes_per_launch": alg, "peak_kind": f"{peak_kind} HBM copy bandwidth",
+                         "kernel": "route_kernel (selection + bookkeeping, one launch)",
+                         "frac_of_8TBps": achieved / 8000.0},
+            "e2e": e2e, "gpu_launches": args.steps, "status_ok": ok,
+            "clocks": clocks,
+            "cpu_baseline": cpu_baseline() if world == 1 else None,
+            "other_rows": extra,
+        }
+        print(json.dumps(line), flush=True)
+    for r in routers:
+        del r
+    if pg:
+        pg.destroy_process_group()
+
+
+def _time_graph(fn, n_iter, stream):
+    import torch
+    with torch.cuda.stream(stream):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    torch.cuda.synchronize()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n_iter):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) * 1000.0 / n_iter  # us
+
+
+def secondary_rows(dev, hbm):
+    """The other workloads of the path, timed the same way (for context; not the headline)."""
+    import torch
+    from top_expert_selection_b200 import binding as B
+    from top_expert_selection_b200 import workloads as W
+    stream = torch.cuda.Stream(dev)
+    rows = {}
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    # Mixtral-style route + dispatch + combine (T=65536, E=8, k=2, H=4096)
+    spec = W.MIXTRAL_ROUTE
+    mi = W.mixtral_inputs()
+    p = B.route_params(spec.T, spec.E, spec.k, score_fn=W.SOFTMAX, softmax_before_topk=0, renormalize=0,
+                       tile_tokens_dim=128, logits_dtype=W.BF16, weights_dtype=W.F32)
+    r = B.Router(p, dev)
+    lg = mi["logits"].to(dev)
+    o = r(lg)
+    torch.cuda.synchronize()
+    P = int(o["totals"][0])
+    H = W.MIXTRAL_HIDDEN
+    hid = mi["hidden"].to(dev)
+    disp = torch.empty((r.max_padded, H), dtype=torch.bfloat16, device=dev)
+    eo = torch.randn((r.max_padded, H), device=dev).to(torch.bfloat16)
+    comb = torch.empty((spec.T, H), dtype=torch.bfloat16, device=dev)
+    us_route = _time_graph(lambda: r(lg), 200, stream)
+    us_disp = _time_graph(lambda: B.dispatch_into(hid, o["e2p"], o["p2t"], o["totals"], 2, disp), 20, stream)
+    us_comb = _time_graph(lambda: B.combine_into(eo, o["e2p"], o["weights"], 2, comb), 20, stream)
+    disp_bytes = spec.T * H * 2 + P * H * 2 + spec.T * 2 * 4 + P * 4
+    comb_bytes = spec.T * 2 * H * 2 + spec.T * 2 * 8 + spec.T * H * 2
+    rows["mixtral_route_us"] = us_route
+    rows["mixtral_dispatch"] = {"us": us_disp, "GBps": disp_bytes / us_disp / 1e3, "frac": disp_bytes / us_disp / 1e3 / hbm}
+    rows["mixtral_combine"] = {"us": us_comb, "GBps": comb_bytes / us_comb / 1e3, "frac": comb_bytes / us_comb / 1e3 / hbm}
+    del disp, eo, comb, hid
+    # aux loss (T=32768, E=128, k=8)
+    a = W.QWEN3_AUX
+    alg = W.aux_inputs(a)["logits"].to(dev)
+    ws = B.aux_workspace(a.T, a.E, dev)
+    sc = B.aux_scores(alg, a.k, ws=ws)
+    loss = torch.empty(1, device=dev)
+    glog = torch.empty_like(alg)
+    gl = torch.ones(1, device=dev)
+
+    def aux_scores_fn():
+        flush.zero_()
+        B.aux_scores_into(alg, a.k, sc["probs"], sc["routing_map"], sc["tokens_per_expert"], ws)
+
+    def loss_fn():
+        flush.zero_()
+        B.aux_loss_fwd_into(sc["probs"], sc["tokens_per_expert"], a.T, a.k, a.coeff, loss, ws)
+
+    def bwd_fn():
+        flush.zero_()
+        B.aux_loss_bwd_into(gl, sc["probs"], sc["tokens_per_expert"], a.T, a.k, a.coeff, None, glog)
+
+    us_flush = _time_graph(lambda: flush.zero_(), 20, stream)
+    rows["aux_scores_us"] = _time_graph(aux_scores_fn, 20, stream) - us_flush
+    rows["aux_loss_fwd_us"] = _time_graph(loss_fn, 20, stream) - us_flush
+    rows["aux_loss_bwd_us"] = _time_graph(bwd_fn, 20, stream) - us_flush
+    # decode fused (T=128, H=7168, E=256, k=8)
+    d = W.DECODE_FUSED
+    di = W.decode_inputs(d)
+    x, gam, Wm, bb = (di[n].to(dev) for n in ("hidden", "gamma", "W", "bias"))
+    res = B.rmsnorm_router_topk(x, gam, Wm, bb, k=d.k)
+
+    def dec_fn():
+        flush.zero_()
+        B.rmsnorm_router_topk_into(x, gam, Wm, bb, d.k, d.eps, d.act, res["out_norm"], res["ids"], res["affinities"],
+                                   None, res["ws"])
+
+    rows["decode_us"] = _time_graph(dec_fn, 20, stream) - us_flush
+    rows["note"] = ("us per call, device time from CUDA graph replays; dispatch/combine inputs exceed L2; "
+                    "aux and decode calls follow an L2 flush whose time is subtracted")
+    return rows
+
+
+if __name__ == "__main__":
+    main()

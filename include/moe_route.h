@@ -1,0 +1,278 @@
+/*
+ * moe_route.h -- C ABI of the B200 (sm_100a) MoE routing library.
+ *
+ * The library computes, on one GPU, the Mixture-of-Experts routing hot path
+ * described by these pages (cited by title and section):
+ *   [TE]  Implementation:NVIDIA TransformerEngine Fused Router
+ *   [TRT] flashinfer.fused_moe.trtllm_gen_routing
+ *   [NKI] RMSNorm Router Top-K A2AV Kernel API Reference
+ *   [LMD] Implementation:InternLM Lmdeploy Gemm MoeUtils
+ *   [MAX] max.nn.moe.SigmoidTopKRouter
+ *
+ * Conventions for every entry point:
+ *   - Buffers are caller-owned.  Pointers named as device pointers must point
+ *     to device memory of the current CUDA device; the library never
+ *     allocates, frees or synchronises (except moe_status, which reads one
+ *     word back).  Tensors are row-major with the last dimension contiguous.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every call is asynchronous and stream-ordered.
+ *   - Arguments are validated before any launch; a failed check returns a
+ *     negative MOE_ERR_* code and launches nothing.  MOE_ERR_CUDA reports a
+ *     launch failure (cudaGetLastError after the launch).
+ *   - Kernels that wait on other thread blocks (a grid barrier, a
+ *     last-block reduction) wait at most a bounded time; on expiry they record
+ *     MOE_ERR_DEVICE_TIMEOUT in the status word at the start of their
+ *     workspace and return, leaving outputs undefined.  Read it with
+ *     moe_status().  After a timeout the workspace must be zero-filled again
+ *     before its next use.
+ *   - A workspace must be zero-filled once before its first use
+ *     (moe_workspace_init or any memset); the library leaves it consistent
+ *     for the next call.  One workspace serves one stream at a time: calls
+ *     that may overlap on the GPU need separate workspaces.
+ *   - Inputs must be finite (no NaN or Inf logits or hidden states).
+ */
+#ifndef MOE_ROUTE_H
+#define MOE_ROUTE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---- */
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG (-1)    /* an argument breaks a documented constraint */
+#define MOE_ERR_UNSUPPORTED (-2)    /* valid per the pages but outside this build's limits */
+#define MOE_ERR_WORKSPACE (-3)      /* workspace missing or smaller than required */
+#define MOE_ERR_CUDA (-4)           /* a CUDA runtime call or launch failed */
+#define MOE_ERR_DEVICE_TIMEOUT (-5) /* a bounded device-side wait expired (status word) */
+#define MOE_ERR_DEVICE_BOUNDS (-6)  /* a kernel's own bounds check skipped an out-of-range index
+                                       (status word; indicates a library bug; outputs undefined) */
+
+/* ---- element types and score functions ---- */
+#define MOE_F32 0
+#define MOE_BF16 1
+#define MOE_SOFTMAX 0
+#define MOE_SIGMOID 1
+
+/* Limits of this build. */
+#define MOE_MAX_EXPERTS 1024
+#define MOE_MAX_TOPK 32
+
+/*
+ * Parameters of one routing call.  Field meanings follow [TE: Signature,
+ * I/O Contract], [TRT: Parameters] and [MAX: steps 1-4].
+ */
+typedef struct moe_route_params {
+  int32_t num_tokens;          /* T >= 0 */
+  int32_t num_experts;         /* E, 1..MOE_MAX_EXPERTS */
+  int32_t top_k;               /* k, 1..min(E, MOE_MAX_TOPK) [TE: topk; TRT: top_k] */
+  int32_t score_fn;            /* MOE_SOFTMAX | MOE_SIGMOID [TE: score_function] */
+  int32_t softmax_before_topk; /* 1: score, then top-k on score (+bias) [TE: use_pre_softmax];
+                                  0: top-k on logit (+bias), then the score function over the
+                                  k selected (softmax over the k, or sigmoid each) */
+  int32_t n_group;             /* grouped routing; n_group <= 1 or topk_group == 0 disables
+                                  [TRT: n_group, topk_group; TE: num_groups, group_topk] */
+  int32_t topk_group;          /* groups kept per token */
+  int32_t group_score_topn;    /* a group's score = sum of its top-n keys; 1 or 2 */
+  int32_t renormalize;         /* selected weights divided by their sum [TRT: norm_topk_prob;
+                                  MAX: norm_topk_prob] */
+  float scaling_factor;        /* weights times this [TRT: routed_scaling_factor; TE:
+                                  scaling_factor] */
+  int32_t tile_tokens_dim;     /* power of two, 1..4096 [TRT: tile_tokens_dim] */
+  int32_t logits_dtype;        /* MOE_F32 | MOE_BF16 [TRT: routing_logits] */
+  int32_t bias_dtype;          /* MOE_F32 | MOE_BF16 [TRT: routing_bias] */
+  int32_t weights_dtype;       /* MOE_F32 | MOE_BF16 [TRT: Notes, topk_weights dtype] */
+} moe_route_params;
+
+/* Human-readable name of a status code (static string). */
+const char* moe_error_string(int code);
+
+/* Zero-fill `bytes` of workspace on `stream` (what a workspace needs once). */
+int moe_workspace_init(void* ws, size_t bytes, void* stream);
+
+/*
+ * Read and optionally clear the status word at the start of a workspace.
+ * Synchronises `stream`.  *status receives MOE_OK or MOE_ERR_DEVICE_TIMEOUT.
+ */
+int moe_status(void* ws, void* stream, int32_t* status, int clear);
+
+/*
+ * Upper bounds for the permutation outputs of moe_route:
+ *   max_padded = T*k + min(E, T*k) * (tile - 1)   (rows of permuted_to_token)
+ *   max_tiles  = max_padded / tile                (entries of the tile tables)
+ * [TRT: tile_tokens_dim -- each expert's rows are padded to the tile].
+ */
+int moe_route_capacity(const moe_route_params* p, int64_t* max_padded, int64_t* max_tiles);
+
+/* Workspace bytes moe_route needs on the current device for these parameters. */
+int moe_route_workspace_bytes(const moe_route_params* p, size_t* bytes);
+
+/*
+ * moe_route -- expert selection, routing weights and permutation bookkeeping
+ * [TE: Description, fused_topk_with_score_function; TRT: standalone routing
+ * (expert selection + permutation), Returns, Notes; MAX: steps 2-4; LMD:
+ * invokeMoeGate_V2].
+ *
+ * Per token t:
+ *   score   s_e = softmax(logits_t)_e, sigmoid(logit_te), or the logit itself
+ *                 when softmax_before_topk == 0; computed in fp32
+ *   key     s_e + bias_e (bias only selects; NULL = no bias)
+ *   groups  (optional) experts in n_group contiguous groups; group score =
+ *           sum of its group_score_topn largest keys; the topk_group best
+ *           groups (ties -> lower group) stay selectable
+ *   top-k   the k largest keys, ties -> lower expert index; slot order =
+ *           descending key
+ *   weight  w_j = v_j / sum(v) * scale (renormalize) or v_j * scale, where v_j
+ *           is the selected expert's unbiased score (softmax_before_topk == 0:
+ *           the score function applied to the k selected logits)
+ * Bookkeeping over all T*k selections (token-major order):
+ *   expert_counts[e]          rows routed to e
+ *   padded_offsets[e]         exclusive prefix of ceil(count/tile)*tile; [E] = P
+ *   expanded_to_permuted[i]   row of selection i = t*k + j in the expert-
+ *                             contiguous padded layout; rows of one expert
+ *                             follow token order
+ *   permuted_to_token[p]      source token of row p, -1 on padding rows (p < P)
+ *   tile_expert[c]            expert of tile c (rows c*tile .. c*tile+tile-1)
+ *   tile_mn_limit[c]          exclusive end of tile c's valid rows
+ *   totals[0] = P (total_num_padded_tokens), totals[1] = P / tile
+ *                             (num_non_exiting_ctas); device-resident, so a
+ *                             consumer sized for the capacity can exit early
+ * Entries of permuted_to_token at or past P, and of the tile tables at or past
+ * P/tile, are not written.
+ *
+ * Device pointers (caller-owned):
+ *   logits [T,E] (logits_dtype), bias [E] (bias_dtype) or NULL,
+ *   topk_ids [T,k] int32, topk_weights [T,k] (weights_dtype),
+ *   expert_counts [E], padded_offsets [E+1], expanded_to_permuted [T*k],
+ *   permuted_to_token [max_padded], tile_expert [max_tiles],
+ *   tile_mn_limit [max_tiles], totals [2] -- all int32,
+ *   ws [ws_bytes] from moe_route_workspace_bytes (zero-filled before first use).
+ * Errors: MOE_ERR_INVALID_ARG (sizes, k > E, tile not a power of two, groups
+ * not dividing E, k > topk_group * E / n_group, NULL outputs),
+ * MOE_ERR_UNSUPPORTED (E or k past the build limits, a group layout the
+ * kernels do not map), MOE_ERR_WORKSPACE, MOE_ERR_CUDA; device timeout via
+ * moe_status.
+ */
+int moe_route(const moe_route_params* p, const void* logits, const void* bias, int32_t* topk_ids,
+              void* topk_weights, int32_t* expert_counts, int32_t* padded_offsets,
+              int32_t* expanded_to_permuted, int32_t* permuted_to_token, int32_t* tile_expert,
+              int32_t* tile_mn_limit, int32_t* totals, void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes of the aux-loss entry points (scores, loss forward). */
+int moe_aux_workspace_bytes(int32_t num_tokens, int32_t num_experts, size_t* bytes);
+
+/*
+ * moe_aux_scores -- scores and routing map for the load-balancing loss
+ * [TE: Description, fused_compute_score_for_moe_aux_loss; Signature].
+ *   probs [T,E] fp32      = softmax(logits_t) (MOE_SIGMOID: sigmoid / row sum)
+ *   routing_map [T,E] u8  = 1 at the token's k largest probs (ties -> lower e)
+ *   tokens_per_expert [E] = column sums of routing_map (int32)
+ * logits [T,E] fp32.  All pointers device, caller-owned; ws as above.
+ */
+int moe_aux_scores(int32_t T, int32_t E, int32_t k, int32_t score_fn, const float* logits,
+                   float* probs, uint8_t* routing_map, int32_t* tokens_per_expert, void* ws,
+                   size_t ws_bytes, void* stream);
+
+/*
+ * moe_aux_loss_fwd -- load-balancing loss [TE: Description, fused_moe_aux_loss;
+ * Signature (probs, tokens_per_expert, total_num_tokens, num_experts, topk,
+ * coeff)]:
+ *   loss = coeff * E / (T_total * k) * sum_e ( sum_t probs[t,e] ) * tpe[e]
+ * probs [T_rows,E] fp32, tokens_per_expert [E] int32, loss: one fp32 on the
+ * device.  Deterministic (fixed reduction order).
+ */
+int moe_aux_loss_fwd(int32_t T_rows, int32_t T_total, int32_t E, int32_t k, float coeff,
+                     const float* probs, const int32_t* tokens_per_expert, float* loss, void* ws,
+                     size_t ws_bytes, void* stream);
+
+/*
+ * moe_aux_loss_bwd -- gradient of the loss [TE: Description, forward and
+ * backward].  With C = coeff * E / (T_total * k) and g = *grad_loss (device):
+ *   grad_probs[t,e]  = g * C * tpe[e]                       (optional, may be NULL)
+ *   grad_logits[t,e] = p[t,e] * (grad_probs[t,e] - sum_j p[t,j] grad_probs[t,j])
+ *                      (softmax backward; optional, may be NULL)
+ * tokens_per_expert is treated as a constant.  No workspace.
+ */
+int moe_aux_loss_bwd(int32_t T_rows, int32_t T_total, int32_t E, int32_t k, float coeff,
+                     const float* grad_loss, const float* probs, const int32_t* tokens_per_expert,
+                     float* grad_probs, float* grad_logits, void* stream);
+
+/*
+ * moe_dispatch -- gather token rows into the expert-contiguous padded buffer
+ * [LMD: invokeMoeDispatch].
+ *   out[expanded_to_permuted[t*k+j], :] = hidden[t, :]
+ *   out[p, :] = 0 for padding rows p < P (permuted_to_token[p] == -1)
+ * Rows at or past P (= totals[0], read on the device) are not written.
+ * hidden [T,H], out [max_padded,H] (dtype MOE_BF16 or MOE_F32),
+ * expanded_to_permuted [T*k], permuted_to_token [max_padded], totals [2]: the
+ * outputs of moe_route.  H * element size must be a multiple of 16 bytes and
+ * hidden/out 16-byte aligned.
+ */
+int moe_dispatch(int32_t T, int32_t H, int32_t k, int32_t dtype, const void* hidden,
+                 const int32_t* expanded_to_permuted, const int32_t* permuted_to_token,
+                 const int32_t* totals, int64_t max_padded, void* out, void* stream);
+
+/*
+ * moe_combine -- weighted sum of each token's k expert rows back in token
+ * order [LMD: invokeMoeCombine, routing scales]:
+ *   out[t, :] = round( sum_j w[t,j] * expert_out[expanded_to_permuted[t*k+j], :] )
+ * accumulated in fp32 in slot order, stored in `dtype` (bf16: round to
+ * nearest even).  Slots whose expanded_to_permuted is negative are skipped.
+ * expert_out [max_padded,H], out [T,H] (dtype MOE_BF16 or MOE_F32), weights
+ * [T,k] (weights_dtype).  Padding rows of expert_out are never read.
+ * H * element size must be a multiple of 16 bytes and rows 16-byte aligned.
+ */
+int moe_combine(int32_t T, int32_t H, int32_t k, int32_t dtype, const void* expert_out,
+                const int32_t* expanded_to_permuted, const void* weights, int32_t weights_dtype,
+                void* out, void* stream);
+
+/* Workspace bytes of moe_rmsnorm_router_topk. */
+int moe_rmsnorm_router_topk_workspace_bytes(int32_t T, int32_t H, int32_t E, size_t* bytes);
+
+/*
+ * moe_rmsnorm_router_topk -- fused RMSNorm + router projection + top-k for
+ * small decode batches [NKI: Background; Parameters; Returns; Notes].
+ *   out_norm[t,h] = bf16( x[t,h] / sqrt(mean_h x[t,h]^2 + eps) * gamma[h] )
+ *   logit[t,e]    = sum_h out_norm[t,h] * W[h,e] + bias[e]   (fp32 accumulate,
+ *                   tensor cores)
+ *   ids[t,:]      = top-k on the raw logits, ties -> lower expert (ACT2:
+ *                   activation after top-k)
+ *   affinities    = bf16(sigmoid(logit)) at the selected experts (MOE_SOFTMAX:
+ *                   softmax over the k selected logits), 0 elsewhere
+ * hidden [T,H], gamma [H], W [H,E], bias [E] or NULL, out_norm [T,H],
+ * affinities [T,E] -- bf16; ids [T,k] int32; debug_logits [T,E] fp32 or NULL
+ * (receives the logits when given).  T <= 128 and H % 128 == 0 [NKI: Notes];
+ * this build also needs E % 16 == 0 and E <= 256.
+ */
+int moe_rmsnorm_router_topk(int32_t T, int32_t H, int32_t E, int32_t k, float eps, int32_t act,
+                            const void* hidden, const void* gamma, const void* W, const void* bias,
+                            void* out_norm, int32_t* ids, void* affinities, float* debug_logits,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Test hook for the bounded grid barrier used by moe_route: launches
+ * `blocks` co-resident blocks that wait for `blocks + extra_arrivals`
+ * arrivals, giving up after timeout_ns.  With extra_arrivals > 0 the wait
+ * cannot complete, so the status word must read MOE_ERR_DEVICE_TIMEOUT
+ * afterwards; the kernel returns normally either way.  ws needs 64 bytes.
+ */
+int moe_debug_barrier_wait(int32_t blocks, int32_t extra_arrivals, int64_t timeout_ns, void* ws,
+                           size_t ws_bytes, void* stream);
+
+/*
+ * Test hook for the sigmoid fast path of moe_route: for each x[i] writes
+ * proxy(x) - sigmoid(x), where proxy(x) = 0.5 * tanh.approx(x / 2) + 0.5 is
+ * the approximate key that chooses candidates and sigmoid(x) = 1 / (1 +
+ * exp(-x)) in fp32 is the exact one.  moe_route assumes |difference| <= 2^-12
+ * and keeps a 2^-10 margin.  x and out are device arrays of n floats.
+ */
+int moe_debug_sigmoid_proxy_error(const float* x, int64_t n, float* out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_ROUTE_H */

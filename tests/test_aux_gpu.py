@@ -1,0 +1,122 @@
+"""GPU parity of the aux-loss path (scores, loss forward, loss backward) against the CPU oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import near_tie_ok, to_np
+from top_expert_selection_b200 import binding as B
+from top_expert_selection_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+RTOL = 1e-5
+
+
+def check_scores(logits, k, score_fn=W.SOFTMAX):
+    T, E = logits.shape
+    g = B.aux_scores(logits.cuda(), k, score_fn)
+    torch.cuda.synchronize()
+    o = oracle.aux_scores(logits, k, score_fn)
+    probs = to_np(g["probs"])
+    ref = o["probs"]
+    assert np.all(np.abs(probs - ref) <= RTOL * np.abs(ref) + 1e-30), "probs off by more than 1e-5 relative"
+    gm = to_np(g["routing_map"])
+    om = o["routing_map"]
+    flips = 0
+    for t in np.nonzero((gm != om).any(1))[0]:
+        gsel = np.nonzero(gm[t])[0]
+        osel = sorted(np.nonzero(om[t])[0].tolist(), key=lambda e: (-ref[t, e], e))
+        gsel = sorted(gsel.tolist(), key=lambda e: (-ref[t, e], e))
+        assert near_tie_ok(ref[t], gsel, osel, k, False, 0, 0, None), f"token {t} routing map not a near tie"
+        flips += 1
+    assert flips <= max(1, T // 1000)
+    assert np.all(gm.sum(1) == k)
+    tpe = to_np(g["tokens_per_expert"])
+    assert np.array_equal(tpe, gm.sum(0).astype(np.int32)), "tokens_per_expert != column sums of routing_map"
+    if flips == 0:
+        assert np.array_equal(tpe, o["tokens_per_expert"])
+    return g, o, flips
+
+
+def test_aux_workload_full_size():
+    spec = W.QWEN3_AUX
+    lg = W.aux_inputs(spec)["logits"]
+    g, o, flips = check_scores(lg, spec.k)
+    print("aux scores flips:", flips)
+    # loss forward on the GPU's own probs / counts vs the oracle on the same inputs, and from scratch
+    loss = B.aux_loss_fwd(g["probs"], g["tokens_per_expert"], spec.T, spec.k, spec.coeff)
+    torch.cuda.synchronize()
+    ref_same = oracle.aux_loss_fwd(to_np(g["probs"]), to_np(g["tokens_per_expert"]), spec.T, spec.k, spec.coeff)
+    ref_scratch = oracle.aux_loss_fwd(o["probs"], o["tokens_per_expert"], spec.T, spec.k, spec.coeff)
+    got = float(loss.item())
+    assert abs(got - ref_same) <= RTOL * abs(ref_same)
+    assert abs(got - ref_scratch) <= RTOL * abs(ref_scratch)
+    # determinism of the reduction
+    loss2 = B.aux_loss_fwd(g["probs"], g["tokens_per_expert"], spec.T, spec.k, spec.coeff)
+    assert float(loss2.item()) == got
+    # backward with upstream grad 1.0
+    gl = torch.tensor([spec.grad_loss], dtype=torch.float32, device="cuda")
+    gr = B.aux_loss_bwd(gl, g["probs"], g["tokens_per_expert"], spec.T, spec.k, spec.coeff)
+    torch.cuda.synchronize()
+    check_backward(to_np(g["probs"]), to_np(g["tokens_per_expert"]), spec.T, spec.k, spec.coeff, spec.grad_loss,
+                   to_np(gr["grad_probs"]), to_np(gr["grad_logits"]))
+
+
+def check_backward(p, tpe, T_total, k, coeff, grad, got_gp, got_gl):
+    ref = oracle.aux_loss_bwd(p, tpe, T_total, k, coeff, grad)
+    assert np.all(np.abs(got_gp - ref["grad_probs"]) <= RTOL * np.abs(ref["grad_probs"]) + 1e-30)
+    # relative to the terms before cancellation: |p * g_e| + |p * sum_j p_j g_j|
+    E = p.shape[1]
+    C = coeff * E / (T_total * k)
+    ge = grad * C * tpe.astype(np.float64)
+    dot = (p.astype(np.float64) * ge).sum(1, keepdims=True)
+    scale = np.abs(p * ge) + np.abs(p * dot)
+    err = np.abs(got_gl.astype(np.float64) - ref["grad_logits"])
+    assert np.all(err <= RTOL * scale + 1e-30), f"grad_logits err/scale max {np.max(err / (scale + 1e-30))}"
+
+
+@pytest.mark.parametrize("T,E,k", [(1, 8, 2), (33, 64, 6), (1000, 128, 8), (257, 96, 4), (300, 256, 8),
+                                   (129, 1024, 16), (77, 33, 3)])
+def test_aux_shapes(T, E, k):
+    g = torch.Generator().manual_seed(T + E)
+    lg = torch.randn(T, E, generator=g) * 1.5
+    gg, o, _ = check_scores(lg, k)
+    probs, tpe = gg["probs"], gg["tokens_per_expert"]
+    for T_total in (T, 3 * T):
+        loss = B.aux_loss_fwd(probs, tpe, T_total, k, 0.37)
+        ref = oracle.aux_loss_fwd(to_np(probs), to_np(tpe), T_total, k, 0.37)
+        assert abs(float(loss.item()) - ref) <= RTOL * abs(ref)
+        gl = torch.tensor([0.75], dtype=torch.float32, device="cuda")
+        gr = B.aux_loss_bwd(gl, probs, tpe, T_total, k, 0.37)
+        check_backward(to_np(probs), to_np(tpe), T_total, k, 0.37, 0.75, to_np(gr["grad_probs"]),
+                       to_np(gr["grad_logits"]))
+
+
+def test_aux_uniform_closed_form_on_gpu():
+    T, E, k, coeff = 4096, 128, 8, 1e-2
+    g = B.aux_scores(torch.zeros(T, E, device="cuda"), k)
+    loss = B.aux_loss_fwd(g["probs"], g["tokens_per_expert"], T, k, coeff)
+    assert abs(float(loss.item()) - coeff * T) <= 1e-6 * coeff * T
+    assert to_np(g["tokens_per_expert"]).tolist() == [T] * k + [0] * (E - k)
+    gr = B.aux_loss_bwd(torch.ones(1, device="cuda"), g["probs"], g["tokens_per_expert"], T, k, coeff)
+    rs = gr["grad_logits"].double().sum(1).abs().max().item()
+    assert rs < 1e-9
+
+
+def test_aux_sigmoid_scores():
+    g = torch.Generator().manual_seed(1)
+    lg = torch.randn(500, 64, generator=g)
+    check_scores(lg, 4, W.SIGMOID)
+
+
+def test_aux_repeated_calls_reuse_workspace():
+    g = torch.Generator().manual_seed(2)
+    lg = (torch.randn(2000, 128, generator=g)).cuda()
+    ws = B.aux_workspace(2000, 128, "cuda")
+    a = B.aux_scores(lg, 8, ws=ws)
+    b = B.aux_scores(lg, 8, ws=ws)
+    assert torch.equal(a["tokens_per_expert"], b["tokens_per_expert"])
+    l1 = B.aux_loss_fwd(a["probs"], a["tokens_per_expert"], 2000, 8, 0.01, ws=ws)
+    l2 = B.aux_loss_fwd(a["probs"], a["tokens_per_expert"], 2000, 8, 0.01, ws=ws)
+    assert torch.equal(l1, l2)
+    assert B.status(ws) == B.MOE_OK

@@ -1,0 +1,234 @@
+"""GPU parity of moe_route against the CPU oracle (through the C ABI)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import compare_route, to_np
+from top_expert_selection_b200 import binding as B
+from top_expert_selection_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+GUARD = 64
+SENT = -123456789
+
+
+def _guarded(n, dtype, dev):
+    """A buffer of n elements with GUARD sentinel elements on each side; returns (full, view)."""
+    full = torch.empty(n + 2 * GUARD, dtype=dtype, device=dev)
+    if dtype == torch.int32:
+        full.fill_(SENT)
+    elif dtype == torch.bfloat16:
+        full.view(torch.int16).fill_(0x7FC1)
+    else:
+        full.view(torch.int32).fill_(0x7FC00001)
+    return full, full[GUARD:GUARD + n]
+
+
+def _guards_intact(full, n):
+    f = full.detach().cpu()
+    if f.dtype == torch.bfloat16:
+        f = f.view(torch.int16)
+        sent = 0x7FC1
+    elif f.dtype == torch.float32:
+        f = f.view(torch.int32)
+        sent = 0x7FC00001
+    else:
+        sent = SENT
+    return bool((f[:GUARD] == sent).all() and (f[GUARD + n:] == sent).all())
+
+
+def run_route(spec: W.RouteSpec, logits=None, bias=None):
+    inp = W.route_inputs(spec)
+    if logits is None:
+        logits, bias = inp["logits"], inp["bias"]
+    dev = torch.device("cuda")
+    p = B.route_params(spec.T, spec.E, spec.k, score_fn=spec.score_fn, softmax_before_topk=spec.softmax_before_topk,
+                       n_group=spec.n_group, topk_group=spec.topk_group, group_score_topn=spec.group_score_topn,
+                       renormalize=spec.renormalize, scaling_factor=spec.scaling_factor,
+                       tile_tokens_dim=spec.tile_tokens_dim, logits_dtype=spec.logits_dtype,
+                       bias_dtype=spec.bias_dtype, weights_dtype=spec.weights_dtype)
+    max_padded, max_tiles = B.route_capacity(p)
+    T, E, k = spec.T, spec.E, spec.k
+    wdt = torch.bfloat16 if spec.weights_dtype == W.BF16 else torch.float32
+    sizes = {"ids": (T * k, torch.int32), "weights": (T * k, wdt), "counts": (E, torch.int32),
+             "offsets": (E + 1, torch.int32), "e2p": (T * k, torch.int32), "p2t": (max_padded, torch.int32),
+             "tile_expert": (max_tiles, torch.int32), "tile_mn_limit": (max_tiles, torch.int32),
+             "totals": (2, torch.int32)}
+    fulls, views = {}, {}
+    for name, (n, dt) in sizes.items():
+        fulls[name], views[name] = _guarded(n, dt, dev)
+    ws = B.make_workspace(B.route_workspace_bytes(p), dev)
+    lg_d = logits.to(dev)
+    b_d = bias.to(dev) if bias is not None else None
+    B.route_into(p, lg_d, b_d, views, ws)
+    torch.cuda.synchronize()
+    assert B.status(ws) == B.MOE_OK
+    for name, (n, _) in sizes.items():
+        assert _guards_intact(fulls[name], n), f"guard zone of {name} overwritten"
+    P = int(views["totals"][0])
+    # rows of permuted_to_token at or past P are not written
+    assert bool((views["p2t"][P:].cpu() == SENT).all())
+    gpu = {n: v for n, v in views.items()}
+    gpu["ids"] = views["ids"].view(T, k)
+    gpu["weights"] = views["weights"].view(T, k)
+    orc = oracle.route_select(logits, k=k, score_fn=spec.score_fn, softmax_before_topk=spec.softmax_before_topk,
+                              n_group=spec.n_group, topk_group=spec.topk_group,
+                              group_score_topn=spec.group_score_topn, renormalize=spec.renormalize,
+                              scaling_factor=spec.scaling_factor, bias=bias)
+    sp = {"k": k, "E": E, "tile": spec.tile_tokens_dim, "n_group": spec.n_group, "topk_group": spec.topk_group}
+    rep = compare_route(sp, gpu, orc)
+    return rep, gpu, (p, lg_d, b_d, ws, views)
+
+
+def test_tiny_softmax_workload():
+    rep, _, _ = run_route(W.TINY_SOFTMAX)
+    assert rep["flips"] == 0
+
+
+def test_dsv3_grouped_sigmoid_full_size():
+    rep, gpu, _ = run_route(W.DSV3_GROUPED_SIGMOID)
+    print("dsv3 grouped sigmoid:", rep)
+
+
+def test_mixtral_route_full_size():
+    rep, _, _ = run_route(W.MIXTRAL_ROUTE)
+    print("mixtral route:", rep)
+
+
+EDGE = []
+for T in (1, 31, 33, 4097):
+    EDGE.append(W.RouteSpec(T=T, E=8, k=2, tile_tokens_dim=4, seed=T))
+    EDGE.append(W.RouteSpec(T=T, E=256, k=8, score_fn=W.SIGMOID, n_group=8, topk_group=4, renormalize=1,
+                            scaling_factor=2.5, tile_tokens_dim=128, logits_dtype=W.BF16, weights_dtype=W.BF16,
+                            has_bias=True, logit_std=2.0, seed=T + 1))
+for E, k in ((4, 1), (16, 6), (64, 8), (72, 6), (128, 8), (384, 8), (1024, 32), (33, 2), (100, 3)):
+    EDGE.append(W.RouteSpec(T=257, E=E, k=k, tile_tokens_dim=8, seed=E))
+    EDGE.append(W.RouteSpec(T=257, E=E, k=k, score_fn=W.SIGMOID, has_bias=True, renormalize=0,
+                            scaling_factor=1.5, tile_tokens_dim=1, seed=E + 7))
+    EDGE.append(W.RouteSpec(T=129, E=E, k=k, softmax_before_topk=0, renormalize=0, logits_dtype=W.BF16,
+                            tile_tokens_dim=4, seed=E + 9))
+for E, ng, tg, k in ((64, 8, 4, 8), (128, 4, 2, 6), (256, 16, 4, 8), (16, 4, 2, 3), (384, 8, 3, 8),
+                     (64, 32, 8, 4), (256, 8, 8, 8)):
+    EDGE.append(W.RouteSpec(T=300, E=E, k=k, score_fn=W.SIGMOID, n_group=ng, topk_group=tg, has_bias=True,
+                            logits_dtype=W.BF16, logit_std=2.0, tile_tokens_dim=8, seed=E + ng))
+    EDGE.append(W.RouteSpec(T=300, E=E, k=k, score_fn=W.SOFTMAX, n_group=ng, topk_group=tg, group_score_topn=1,
+                            tile_tokens_dim=16, seed=E + ng + 1))
+
+
+@pytest.mark.parametrize("spec", EDGE, ids=lambda s: f"T{s.T}-E{s.E}-k{s.k}-sf{s.score_fn}-pre{s.softmax_before_topk}"
+                         f"-g{s.n_group}.{s.topk_group}-tile{s.tile_tokens_dim}-dt{s.logits_dtype}")
+def test_route_edge_sweep(spec):
+    run_route(spec)
+
+
+def test_all_equal_logits_tie_break():
+    spec = W.RouteSpec(T=64, E=256, k=8, score_fn=W.SIGMOID, n_group=8, topk_group=4, tile_tokens_dim=8,
+                       logits_dtype=W.BF16, weights_dtype=W.BF16)
+    lg = torch.full((64, 256), 0.5).to(torch.bfloat16)
+    rep, gpu, _ = run_route(spec, lg, None)
+    assert rep["flips"] == 0
+    assert to_np(gpu["ids"]).tolist() == [list(range(8))] * 64
+    spec = W.RouteSpec(T=40, E=8, k=3, tile_tokens_dim=4)
+    rep, gpu, _ = run_route(spec, torch.zeros(40, 8), None)
+    assert to_np(gpu["ids"]).tolist() == [[0, 1, 2]] * 40
+
+
+def test_bf16_logits_with_many_exact_ties():
+    g = torch.Generator().manual_seed(9)
+    lg = torch.randint(-3, 4, (500, 128), generator=g).float().to(torch.bfloat16)
+    spec = W.RouteSpec(T=500, E=128, k=8, score_fn=W.SOFTMAX, tile_tokens_dim=8, logits_dtype=W.BF16)
+    rep, _, _ = run_route(spec, lg, None)
+    assert rep["flips"] == 0
+
+
+def test_hot_expert_skew_and_empty_experts():
+    spec = W.RouteSpec(T=4000, E=64, k=4, score_fn=W.SIGMOID, has_bias=True, tile_tokens_dim=128, seed=5)
+    inp = W.route_inputs(spec)
+    bias = inp["bias"].clone()
+    bias[17] = 5.0     # every token picks expert 17
+    bias[40:] = -5.0   # experts 40.. are never picked
+    rep, gpu, _ = run_route(spec, inp["logits"], bias)
+    counts = to_np(gpu["counts"])
+    assert counts[17] == 4000 and counts[40:].sum() == 0
+
+
+def test_grouped_all_kept_equals_ungrouped_on_gpu():
+    base = W.DSV3_GROUPED_SIGMOID.with_(T=2048)
+    _, a, _ = run_route(base.with_(topk_group=8))
+    _, b, _ = run_route(base.with_(n_group=0, topk_group=0))
+    assert torch.equal(a["ids"].cpu(), b["ids"].cpu()) and torch.equal(a["weights"].cpu(), b["weights"].cpu())
+
+
+def test_repeated_calls_are_deterministic():
+    spec = W.DSV3_GROUPED_SIGMOID
+    _, gpu, (p, lg, b, ws, views) = run_route(spec)
+    first = {n: v.clone() for n, v in views.items()}
+    other = W.route_inputs(spec.with_(seed=77))
+    B.route_into(p, other["logits"].cuda(), other["bias"].cuda(), views, ws)
+    for _ in range(3):
+        B.route_into(p, lg, b, views, ws)
+    torch.cuda.synchronize()
+    for n in first:
+        assert torch.equal(first[n], views[n]), n
+
+
+def test_zero_tokens():
+    p = B.route_params(0, 16, 2, tile_tokens_dim=4)
+    dev = torch.device("cuda")
+    views = {"ids": None, "weights": None, "e2p": None, "p2t": None, "tile_expert": None, "tile_mn_limit": None,
+             "counts": torch.full((16,), 5, dtype=torch.int32, device=dev),
+             "offsets": torch.full((17,), 5, dtype=torch.int32, device=dev),
+             "totals": torch.full((2,), 5, dtype=torch.int32, device=dev)}
+    ws = B.make_workspace(B.route_workspace_bytes(p), dev)
+    B.route_into(p, torch.empty(0, 16, device=dev), None, views, ws)
+    torch.cuda.synchronize()
+    assert views["counts"].sum().item() == 0 and views["offsets"].sum().item() == 0
+    assert views["totals"].tolist() == [0, 0]
+
+
+def test_bounded_barrier_times_out_cleanly():
+    """A grid barrier asked for one arrival more than it has blocks gives up after its limit and
+    records a timeout in the status word; the context stays usable."""
+    dev = torch.device("cuda")
+    ws = B.make_workspace(64, dev)
+    B.debug_barrier_wait(4, 1, 20_000_000, ws)
+    torch.cuda.synchronize()
+    assert B.status(ws, clear=True) == B.MOE_ERR_DEVICE_TIMEOUT
+    ws.zero_()
+    B.debug_barrier_wait(4, 0, 20_000_000, ws)
+    torch.cuda.synchronize()
+    assert B.status(ws) == B.MOE_OK
+    run_route(W.TINY_SOFTMAX)
+
+
+def test_sigmoid_proxy_error_bound_exhaustive_bf16():
+    """The fast path's proxy key is within 2^-12 of the exact fp32 sigmoid for every finite bf16
+    input (it assumes that bound and keeps a 2^-10 margin); also checked on random fp32 inputs."""
+    bits = torch.arange(0, 1 << 16, dtype=torch.int32).to(torch.int16)
+    x = bits.view(torch.bfloat16).float()
+    x = x[torch.isfinite(x)]
+    g = torch.Generator().manual_seed(0)
+    x = torch.cat([x, torch.randn(1 << 20, generator=g) * 8, torch.rand(1 << 20, generator=g) * 60 - 30])
+    err = B.debug_sigmoid_proxy_error(x.cuda()).abs().max().item()
+    print("max |proxy - sigmoid| =", err)
+    assert err <= 2.0 ** -12
+
+
+def test_fast_path_group_ties_and_fallbacks():
+    """Sigmoid fast path: exactly tied groups (slow path, lower group wins), k = 16 with 4 kept groups
+    (candidate bound unavailable -> slow path), k = 1, and fp32 logits."""
+    base = W.DSV3_GROUPED_SIGMOID.with_(T=1024, seed=21)
+    inp = W.route_inputs(base)
+    lg = inp["logits"].clone()
+    lg[:, 3 * 32:4 * 32] = lg[:, 5 * 32:6 * 32]  # groups 3 and 5 identical logits
+    bias = inp["bias"].clone()
+    bias[3 * 32:4 * 32] = bias[5 * 32:6 * 32]
+    run_route(base, lg, bias)
+    run_route(base.with_(k=16, seed=22))
+    run_route(base.with_(k=1, seed=23))
+    run_route(base.with_(logits_dtype=W.F32, E=128, n_group=8, topk_group=3, k=6, seed=24))
+    run_route(base.with_(n_group=0, topk_group=0, k=8, seed=25))
+    # saturated sigmoids: many keys equal 1 + bias exactly
+    run_route(base.with_(logit_std=40.0, seed=26))

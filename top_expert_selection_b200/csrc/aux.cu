@@ -1,0 +1,338 @@
+// Aux-loss path: scores + routing map, load-balancing loss, and its backward.
+//
+// Sources: Implementation:NVIDIA TransformerEngine Fused Router -- Description
+// (fused_compute_score_for_moe_aux_loss: scores and routing map;
+// fused_moe_aux_loss: loss from probs and tokens_per_expert; forward and
+// backward), Signature (probs, tokens_per_expert, total_num_tokens,
+// num_experts, topk, coeff).
+//
+// loss = coeff * E / (T_total * k) * sum_e (sum_t probs[t,e]) * tpe[e]
+//      = C * sum_t sum_e probs[t,e] * tpe[e]
+// computed in one pass over probs (no column-sum intermediate).
+//
+// Determinism: tokens_per_expert is an integer sum (order-free).  The loss is
+// reduced from per-thread fp32 partials to per-block double partials over a
+// fixed grid, and the last block to finish adds the block partials in index
+// order, so the result does not depend on scheduling.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kAuxThreads = 256;
+constexpr int kAuxWarps = kAuxThreads / 32;
+constexpr int kLossBlocks = 296;  // fixed: 2 per SM on a 148-SM part; the reduction order depends on it
+
+// workspace layout after the 64-byte header
+struct AuxWs {
+  int32_t* tpe_acc;    // [E] running integer counts
+  double* partials;    // [kLossBlocks]
+};
+
+__host__ __device__ inline size_t aux_ws_bytes(int E) {
+  return sizeof(WsHeader) + (((size_t)E * 4 + 255) & ~(size_t)255) + (size_t)kLossBlocks * sizeof(double);
+}
+
+__device__ inline AuxWs aux_ws(void* ws, int E) {
+  AuxWs w;
+  uint8_t* base = reinterpret_cast<uint8_t*>(ws) + sizeof(WsHeader);
+  w.tpe_acc = reinterpret_cast<int32_t*>(base);
+  w.partials = reinterpret_cast<double*>(base + (((size_t)E * 4 + 255) & ~(size_t)255));
+  return w;
+}
+
+__device__ __forceinline__ float sigmoid_f32(float x) { return 1.0f / (1.0f + expf(-x)); }
+
+// --------------------------------------------------------------------------
+// scores: warp per token, lane l owns experts [l*VPL, l*VPL + VPL)
+// --------------------------------------------------------------------------
+template <int VPL>
+__global__ void __launch_bounds__(kAuxThreads) aux_scores_kernel(int T, int E, int k, int score_fn,
+                                                                 const float* __restrict__ logits,
+                                                                 float* __restrict__ probs,
+                                                                 uint8_t* __restrict__ rmap,
+                                                                 int32_t* __restrict__ tpe, void* ws) {
+  extern __shared__ int hist[];  // [E]
+  const unsigned FULL = 0xffffffffu;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
+  AuxWs w = aux_ws(ws, E);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+
+  for (long long t = (long long)blockIdx.x * kAuxWarps + warp; t < T; t += (long long)gridDim.x * kAuxWarps) {
+    const float* row = logits + t * E;
+    float x[VPL], p[VPL];
+    uint32_t valid = 0;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int e = lane * VPL + i;
+      const bool v = e < E;
+      x[i] = v ? __ldcs(row + e) : 0.0f;
+      valid |= (v ? 1u : 0u) << i;
+    }
+    float sum = 0.0f;
+    if (score_fn == MOE_SOFTMAX) {
+      float m = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i)
+        if (valid & (1u << i)) m = fmaxf(m, x[i]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, off));
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        p[i] = (valid & (1u << i)) ? expf(x[i] - m) : 0.0f;
+        sum += p[i];
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        p[i] = (valid & (1u << i)) ? sigmoid_f32(x[i]) : 0.0f;
+        sum += p[i];
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(FULL, sum, off);
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) p[i] = p[i] / sum;
+
+    // top-k mask over probs: k rounds of warp argmax, ties -> lower expert
+    uint32_t avail = valid, chosen = 0;
+    for (int j = 0; j < k; ++j) {
+      unsigned long long best = 0ull;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i)
+        if (avail & (1u << i)) {
+          const unsigned long long pk = pack_key(p[i], lane * VPL + i);
+          best = pk > best ? pk : best;
+        }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const unsigned long long o = shfl_xor_u64(FULL, best, off);
+        best = o > best ? o : best;
+      }
+      const int win = packed_expert(best);
+      if (win / VPL == lane) {
+        const uint32_t bit = 1u << (win - lane * VPL);
+        avail &= ~bit;
+        chosen |= bit;
+      }
+    }
+    float* prow = probs + t * E;
+    uint8_t* mrow = rmap + t * E;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int e = lane * VPL + i;
+      if (valid & (1u << i)) {
+        __stcs(prow + e, p[i]);
+        const bool c = (chosen >> i) & 1u;
+        mrow[e] = c ? 1 : 0;
+        if (c) atomicAdd(&hist[e], 1);
+      }
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    if (hist[e]) atomicAdd(&w.tpe_acc[e], hist[e]);
+  // the last block to finish publishes the counts and clears the accumulator
+  __shared__ int last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = (atomicAdd(&hdr->ticket, 1u) == gridDim.x - 1);
+  __syncthreads();
+  if (last) {
+    __threadfence();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      tpe[e] = __ldcg(&w.tpe_acc[e]);
+      w.tpe_acc[e] = 0;
+    }
+    if (threadIdx.x == 0) hdr->ticket = 0;
+  }
+}
+
+// --------------------------------------------------------------------------
+// loss forward: one pass over probs; fixed grid; deterministic reduction
+// --------------------------------------------------------------------------
+__global__ void __launch_bounds__(kAuxThreads) aux_loss_fwd_kernel(long long n, int E, double C,
+                                                                   const float* __restrict__ probs,
+                                                                   const int32_t* __restrict__ tpe, float* loss,
+                                                                   void* ws) {
+  extern __shared__ float tpe_s[];  // [E]
+  __shared__ double red[kAuxWarps];
+  __shared__ int last;
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
+  AuxWs w = aux_ws(ws, E);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) tpe_s[e] = (float)tpe[e];
+  __syncthreads();
+  // each block owns a contiguous range of elements; threads stride through it
+  const long long per = (((n + gridDim.x - 1) / gridDim.x) + 3) & ~3LL;  // multiple of 4: float4 ranges
+  const long long b0 = (long long)blockIdx.x * per, b1 = min(n, b0 + per);
+  float acc = 0.0f;
+  if ((E & 3) == 0 && (b0 & 3) == 0) {
+    const long long q1 = b1 >> 2;
+    for (long long q = (b0 >> 2) + threadIdx.x; q < q1; q += blockDim.x) {
+      const float4 v = __ldcs(reinterpret_cast<const float4*>(probs) + q);
+      const int e = (int)((q << 2) % E);
+      acc = fmaf(v.x, tpe_s[e], acc);
+      acc = fmaf(v.y, tpe_s[e + 1], acc);
+      acc = fmaf(v.z, tpe_s[e + 2], acc);
+      acc = fmaf(v.w, tpe_s[e + 3], acc);
+    }
+    for (long long i = (q1 << 2) + threadIdx.x; i < b1; i += blockDim.x) acc = fmaf(probs[i], tpe_s[i % E], acc);
+  } else {
+    for (long long i = b0 + threadIdx.x; i < b1; i += blockDim.x) acc = fmaf(probs[i], tpe_s[i % E], acc);
+  }
+  double d = (double)acc;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = d;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double s = 0.0;
+    for (int i = 0; i < kAuxWarps; ++i) s += red[i];
+    w.partials[blockIdx.x] = s;
+    __threadfence();
+    last = (atomicAdd(&hdr->ticket, 1u) == gridDim.x - 1);
+  }
+  __syncthreads();
+  if (last && threadIdx.x == 0) {
+    __threadfence();
+    double s = 0.0;
+    for (unsigned b = 0; b < gridDim.x; ++b) s += __ldcg(&w.partials[b]);
+    *loss = (float)(C * s);
+    hdr->ticket = 0;
+  }
+}
+
+// --------------------------------------------------------------------------
+// loss backward: warp per row
+// --------------------------------------------------------------------------
+template <int VPL>
+__global__ void __launch_bounds__(kAuxThreads) aux_loss_bwd_kernel(int T, int E, float C,
+                                                                   const float* __restrict__ grad_loss,
+                                                                   const float* __restrict__ probs,
+                                                                   const int32_t* __restrict__ tpe,
+                                                                   float* __restrict__ grad_probs,
+                                                                   float* __restrict__ grad_logits) {
+  extern __shared__ float gp_s[];  // [E] = g * C * tpe[e]
+  const float g = *grad_loss;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) gp_s[e] = g * C * (float)tpe[e];
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (long long t = (long long)blockIdx.x * kAuxWarps + warp; t < T; t += (long long)gridDim.x * kAuxWarps) {
+    const float* prow = probs + t * E;
+    float p[VPL], gp[VPL];
+    float dot = 0.0f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int e = lane * VPL + i;
+      p[i] = e < E ? __ldcs(prow + e) : 0.0f;
+      gp[i] = e < E ? gp_s[e] : 0.0f;
+      dot = fmaf(p[i], gp[i], dot);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int e = lane * VPL + i;
+      if (e < E) {
+        if (grad_probs) __stcs(grad_probs + t * E + e, gp[i]);
+        if (grad_logits) __stcs(grad_logits + t * E + e, p[i] * (gp[i] - dot));
+      }
+    }
+  }
+}
+
+int sm_count() {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+int pick_vpl(int E) {
+  for (int v : {1, 2, 3, 4, 6, 8, 12, 16, 24, 32})
+    if (v * 32 >= E) return v;
+  return -1;
+}
+
+#define MOE_VPL_SWITCH(vpl, KERNEL_CALL) \
+  switch (vpl) {                         \
+    case 1: { constexpr int V = 1; KERNEL_CALL; } break;  \
+    case 2: { constexpr int V = 2; KERNEL_CALL; } break;  \
+    case 3: { constexpr int V = 3; KERNEL_CALL; } break;  \
+    case 4: { constexpr int V = 4; KERNEL_CALL; } break;  \
+    case 6: { constexpr int V = 6; KERNEL_CALL; } break;  \
+    case 8: { constexpr int V = 8; KERNEL_CALL; } break;  \
+    case 12: { constexpr int V = 12; KERNEL_CALL; } break; \
+    case 16: { constexpr int V = 16; KERNEL_CALL; } break; \
+    case 24: { constexpr int V = 24; KERNEL_CALL; } break; \
+    case 32: { constexpr int V = 32; KERNEL_CALL; } break; \
+    default: return MOE_ERR_UNSUPPORTED;  \
+  }
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" int moe_aux_workspace_bytes(int32_t num_tokens, int32_t num_experts, size_t* bytes) {
+  if (num_tokens < 0 || num_experts <= 0 || !bytes) return MOE_ERR_INVALID_ARG;
+  if (num_experts > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+  *bytes = aux_ws_bytes(num_experts);
+  return MOE_OK;
+}
+
+extern "C" int moe_aux_scores(int32_t T, int32_t E, int32_t k, int32_t score_fn, const float* logits, float* probs,
+                              uint8_t* routing_map, int32_t* tokens_per_expert, void* ws, size_t ws_bytes,
+                              void* stream) {
+  if (T < 0 || E <= 0 || k <= 0 || k > E) return MOE_ERR_INVALID_ARG;
+  if (score_fn != MOE_SOFTMAX && score_fn != MOE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+  if (!tokens_per_expert || (T > 0 && (!logits || !probs || !routing_map))) return MOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < aux_ws_bytes(E)) return MOE_ERR_WORKSPACE;
+  const int vpl = pick_vpl(E);
+  const int grid = std::max(1, std::min((T + kAuxWarps - 1) / kAuxWarps, sm_count() * 8));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t smem = (size_t)E * sizeof(int);
+  MOE_VPL_SWITCH(vpl, (aux_scores_kernel<V><<<grid, kAuxThreads, smem, st>>>(T, E, k, score_fn, logits, probs,
+                                                                            routing_map, tokens_per_expert, ws)));
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+extern "C" int moe_aux_loss_fwd(int32_t T_rows, int32_t T_total, int32_t E, int32_t k, float coeff,
+                                const float* probs, const int32_t* tokens_per_expert, float* loss, void* ws,
+                                size_t ws_bytes, void* stream) {
+  if (T_rows < 0 || T_total <= 0 || E <= 0 || k <= 0) return MOE_ERR_INVALID_ARG;
+  if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+  if (!loss || !tokens_per_expert || (T_rows > 0 && !probs)) return MOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < aux_ws_bytes(E)) return MOE_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(probs) & 15) return MOE_ERR_INVALID_ARG;
+  const double C = (double)coeff * (double)E / ((double)T_total * (double)k);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  aux_loss_fwd_kernel<<<kLossBlocks, kAuxThreads, (size_t)E * sizeof(float), st>>>((long long)T_rows * E, E, C, probs,
+                                                                                 tokens_per_expert, loss, ws);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+extern "C" int moe_aux_loss_bwd(int32_t T_rows, int32_t T_total, int32_t E, int32_t k, float coeff,
+                                const float* grad_loss, const float* probs, const int32_t* tokens_per_expert,
+                                float* grad_probs, float* grad_logits, void* stream) {
+  if (T_rows < 0 || T_total <= 0 || E <= 0 || k <= 0) return MOE_ERR_INVALID_ARG;
+  if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+  if (!grad_loss || !tokens_per_expert || (T_rows > 0 && !probs)) return MOE_ERR_INVALID_ARG;
+  if (T_rows == 0 || (!grad_probs && !grad_logits)) return MOE_OK;
+  const float C = (float)((double)coeff * (double)E / ((double)T_total * (double)k));
+  const int vpl = pick_vpl(E);
+  const int grid = std::max(1, std::min((T_rows + kAuxWarps - 1) / kAuxWarps, sm_count() * 8));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t smem = (size_t)E * sizeof(float);
+  MOE_VPL_SWITCH(vpl, (aux_loss_bwd_kernel<V><<<grid, kAuxThreads, smem, st>>>(T_rows, E, C, grad_loss, probs,
+                                                                               tokens_per_expert, grad_probs,
+                                                                               grad_logits)));
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
