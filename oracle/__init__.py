@@ -57,6 +57,8 @@ def _lib():
         L.oracle_dispatch.argtypes = [i32, i32, i32, P, P, P, i32, P]
         L.oracle_combine.argtypes = [i32, i32, i32, P, P, P, i32, P]
         L.oracle_rmsnorm_router_topk.argtypes = [i32, i32, i32, i32, f32, i32, P, P, P, P, P, P, P, P]
+        L.oracle_router_logits.argtypes = [i32, i32, i32, P, P, P, P]
+        L.oracle_router_logits.restype = i32
         L.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
         L.oracle_bf16_to_f32.restype = f32
         L.oracle_f32_to_bf16.argtypes = [f32]
@@ -250,3 +252,15 @@ def rmsnorm_router_topk(hidden, gamma, W, bias, *, k: int, eps: float = 1e-6, ac
                                            _ptr(xn), _ptr(ids), _ptr(aff), _ptr(lg))
     _check(rc, "rmsnorm_router_topk")
     return {"out_norm": xn, "ids": ids, "affinities": aff, "logits": lg}
+
+
+def router_logits(xn, W, bias=None) -> np.ndarray:
+    x = as_numpy(xn)
+    w = as_numpy(W)
+    b = as_numpy(bias) if bias is not None else None
+    T, H = x.shape
+    E = w.shape[1]
+    out = np.zeros((T, E), np.float32)
+    rc = _lib().oracle_router_logits(T, H, E, _ptr(x), _ptr(w), _ptr(b), _ptr(out))
+    _check(rc, "router_logits")
+    return out

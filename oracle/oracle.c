@@ -427,25 +427,30 @@ int oracle_dispatch(int T, int H, int k, const uint16_t* hidden, const int32_t* 
 }
 
 /*
- * Combine [LMD: invokeMoeCombine, routing scales]: out[t,:] = bf16( sum_j
- * w[t,j] * expert_out[e2p[t*k+j], :] ), the weighted sum of the token's k
- * expert rows in the weights' stored dtype, summed in double and rounded once
- * to bf16.  Slots with e2p < 0 contribute nothing.
+ * Combine [LMD: invokeMoeCombine, routing scales]: out[t,:] = bf16( the
+ * fp32-accumulated weighted sum of the token's k expert rows ).  READING: the
+ * accumulation is fp32 in slot order, acc = acc + w_j * x (a rounded product,
+ * then a rounded add; no fused multiply-add), starting from 0, with the weights
+ * read in their stored dtype; the sum is rounded once to bf16 (nearest even).
+ * Slots with e2p < 0 contribute nothing.
  */
 int oracle_combine(int T, int H, int k, const uint16_t* expert_out, const int32_t* e2p,
                    const void* weights, int weights_dtype, uint16_t* out) {
   if (T < 0 || H <= 0 || k <= 0) return -1;
-  double* acc = (double*)malloc(sizeof(double) * (size_t)H);
+  float* acc = (float*)malloc(sizeof(float) * (size_t)H);
   for (int t = 0; t < T; ++t) {
-    for (int h = 0; h < H; ++h) acc[h] = 0.0;
+    for (int h = 0; h < H; ++h) acc[h] = 0.0f;
     for (int j = 0; j < k; ++j) {
       int32_t p = e2p[(size_t)t * k + j];
       if (p < 0) continue;
-      double w = (double)load_elem(weights, weights_dtype, (size_t)t * k + j);
+      float w = load_elem(weights, weights_dtype, (size_t)t * k + j);
       const uint16_t* row = expert_out + (size_t)p * H;
-      for (int h = 0; h < H; ++h) acc[h] += w * (double)bf16_to_f32(row[h]);
+      for (int h = 0; h < H; ++h) {
+        float prod = w * bf16_to_f32(row[h]);
+        acc[h] = acc[h] + prod;
+      }
     }
-    for (int h = 0; h < H; ++h) out[(size_t)t * H + h] = f64_to_bf16(acc[h]);
+    for (int h = 0; h < H; ++h) out[(size_t)t * H + h] = f32_to_bf16(acc[h]);
   }
   free(acc);
   return 0;
@@ -511,5 +516,25 @@ int oracle_rmsnorm_router_topk(int T, int H, int E, int k, float eps, int act,
     }
   }
   free(lg); free(xnf); free(sel); free(v);
+  return 0;
+}
+
+/*
+ * Router projection alone [NKI: Parameters, router_weights [H,E], router_bias]:
+ * logit[t,e] = fp32( sum_h xn[t,h] * W[h,e] + b[e] ), double accumulation, one
+ * rounding; xn given as bf16 (lets a test isolate the projection from the
+ * normalisation).
+ */
+int oracle_router_logits(int T, int H, int E, const uint16_t* xn, const uint16_t* W, const uint16_t* bias,
+                         float* logits) {
+  if (T < 0 || H <= 0 || E <= 0) return -1;
+  for (int t = 0; t < T; ++t)
+    for (int e = 0; e < E; ++e) {
+      double acc = 0.0;
+      for (int h = 0; h < H; ++h)
+        acc += (double)bf16_to_f32(xn[(size_t)t * H + h]) * (double)bf16_to_f32(W[(size_t)h * E + e]);
+      if (bias) acc += (double)bf16_to_f32(bias[e]);
+      logits[(size_t)t * E + e] = (float)acc;
+    }
   return 0;
 }

@@ -385,6 +385,13 @@ def test_combine_closed_forms():
     assert oracle.combine(eo, e2p, w, 2)[0, 2] == _bf([1.0])[0]
     w = np.array([[1.0, 3 * 2 ** -8]], np.float32)
     assert oracle.combine(eo, e2p, w, 2)[0, 2] == _bf([1.0 + 2 ** -6])[0]
+    # fp32 accumulation (rounded product, rounded add): w0 = 1 + 2^-23, x = 1 + 2^-7 gives the
+    # product 1 + 2^-7 + 2^-23 (the 2^-30 term is rounded away); adding -(1 + 2^-7) leaves 2^-23.
+    # An exact (double) sum would give 2^-23 + 2^-30, a different bf16 value.
+    x = _bf([1.0 + 2 ** -7])
+    eo2 = np.stack([x, x])
+    w = np.array([[np.float32(1.0 + 2 ** -23), -1.0]], np.float32)
+    assert oracle.combine(eo2, e2p, w, 2)[0, 0] == _bf([2.0 ** -23])[0]
     # k=1 with weight 1 is a copy; bf16 weights are read as bf16
     assert np.array_equal(oracle.combine(eo, np.array([1], np.int32), np.array([[1.0]], np.float32), 1), eo[1:2])
     wb = _bf([0.5, 0.5]).reshape(1, 2)
@@ -445,6 +452,13 @@ def test_decode_one_hot_projection_and_affinity():
                 assert abs(aff[e] - ref) <= 2 ** -8 * ref
             else:
                 assert aff[e] == 0.0
+
+
+def test_router_logits_alone_matches_fused_oracle():
+    spec = W.DecodeSpec(T=4, H=256, E=32, k=4)
+    inp = W.decode_inputs(spec)
+    out = oracle.rmsnorm_router_topk(inp["hidden"], inp["gamma"], inp["W"], inp["bias"], k=4)
+    assert np.array_equal(oracle.router_logits(out["out_norm"], inp["W"], inp["bias"]), out["logits"])
 
 
 def test_decode_projection_matches_library_matmul():

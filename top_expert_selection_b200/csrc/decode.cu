@@ -13,10 +13,11 @@
 //   phase 1  W slice -> shared memory by 2-D TMA (128-byte swizzle, the
 //            canonical MN-major operand layout of tcgen05.mma); 256 TMEM
 //            columns allocated; per-token partial sum of squares of the slice
-//            -> workspace.  Bounded grid barrier.
+//            (double) -> workspace.  Bounded grid barrier.
 //   phase 2  every block adds the partial sums in block order (deterministic)
-//            and forms r_t = 1/sqrt(mean + eps); normalises its slice
-//            (x*gamma is exact in fp32, then *r_t, RNE to bf16), writes
+//            and forms r_t = 1/sqrt(mean + eps) in double; normalises its
+//            slice (x*gamma exact in fp32, times r_t in double, one rounding to
+//            bf16), writes
 //            out_norm and the same bf16 values to shared memory in the
 //            K-major 128-byte-swizzled layout; one thread issues the
 //            M=128 x N=E x K=16 tcgen05.mma steps into TMEM; the partial logits
@@ -129,6 +130,18 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
 
 __device__ __forceinline__ float sigmoid_f32(float x) { return 1.0f / (1.0f + expf(-x)); }
 
+// double -> bf16 bits, one rounding to nearest-even: truncate to fp32 and set
+// the last bit if anything was cut (round to odd), then round to nearest-even
+// at bf16 precision; with >= 2 extra bits this equals direct rounding (Boldo &
+// Melquiond, "Emulation of FMA and correctly rounded sums: proved algorithms
+// using rounding to odd", IEEE Trans. Computers 2008).
+__device__ __forceinline__ uint16_t f64_to_bf16_bits(double y) {
+  float f = __double2float_rz(y);
+  if ((double)f != y) f = __uint_as_float(__float_as_uint(f) | 1u);
+  const __nv_bfloat16 h = __float2bfloat16_rn(f);
+  return *reinterpret_cast<const uint16_t*>(&h);
+}
+
 __global__ void __launch_bounds__(kDecThreads, 1)
     decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap wmap) {
   extern __shared__ uint8_t smem_raw[];
@@ -143,7 +156,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   uint64_t* mma_bar = tma_bar + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tail + 16);
   int* flag = reinterpret_cast<int*>(tail + 32);    // [0] barrier scratch, [1] failure
-  float* r_s = reinterpret_cast<float*>(tail + 64); // [kM]
+  double* r_s = reinterpret_cast<double*>(tail + 64); // [kM]
 
   const int c = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -168,10 +181,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   // ---------------- phase 1: partial sums of squares ----------------
-  // two threads per token, 64 columns each per slice
+  // two threads per token, 64 columns each per slice; squares of bf16 values
+  // are exact, and are summed in double
   {
     const int t = tid >> 1, half = tid & 1;
-    float acc = 0.0f;
+    double acc = 0.0;
     if (t < a.T) {
       for (int sl = sl0; sl < sl1; ++sl) {
         const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)t * a.H + sl * kKC + half * 64);
@@ -182,13 +196,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xffff0000u);
-            acc = fmaf(lo, lo, acc);
-            acc = fmaf(hi, hi, acc);
+            acc += (double)(lo * lo);
+            acc += (double)(hi * hi);
           }
         }
       }
     }
-    double d = (double)acc;
+    double d = acc;
     d += __shfl_xor_sync(0xffffffffu, d, 1);
     if (half == 0 && t < kM) a.sumsq[(size_t)c * kM + t] = d;
   }
@@ -199,7 +213,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     if (tid < a.T) {
       double s = 0.0;
       for (int cp = 0; cp < a.G; ++cp) s += __ldcg(&a.sumsq[(size_t)cp * kM + tid]);
-      r_s[tid] = (float)(1.0 / sqrt(s / (double)a.H + (double)a.eps));
+      r_s[tid] = 1.0 / sqrt(s / (double)a.H + (double)a.eps);
     }
     __syncthreads();
     const uint32_t idesc = idesc_bf16_f32(a.N);
@@ -218,15 +232,17 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         const size_t off = (size_t)t * a.H + sl * kKC + q * 8;
         const uint4 xv = __ldg(reinterpret_cast<const uint4*>(a.x + off));
         const uint4 gv = __ldg(reinterpret_cast<const uint4*>(a.gamma + sl * kKC + q * 8));
-        const float r = r_s[t];
+        const double r = r_s[t];
         const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
         uint32_t ow[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const float x0 = __uint_as_float(xw[j] << 16), x1 = __uint_as_float(xw[j] & 0xffff0000u);
           const float g0 = __uint_as_float(gw[j] << 16), g1 = __uint_as_float(gw[j] & 0xffff0000u);
-          const __nv_bfloat162 h = __floats2bfloat162_rn((x0 * g0) * r, (x1 * g1) * r);
-          ow[j] = *reinterpret_cast<const uint32_t*>(&h);
+          // x*gamma is exact in fp32; the product with r is formed in double and
+          // rounded once to bf16
+          ow[j] = (uint32_t)f64_to_bf16_bits((double)(x0 * g0) * r) |
+                  ((uint32_t)f64_to_bf16_bits((double)(x1 * g1) * r) << 16);
         }
         const uint4 o = make_uint4(ow[0], ow[1], ow[2], ow[3]);
         *reinterpret_cast<uint4*>(a.out_norm + off) = o;
@@ -412,7 +428,7 @@ size_t dec_ws_bytes(int H, int E) {
 
 int dec_smem(int E) {
   const int NB = (E + 63) / 64;
-  const int need = 1024 + 32 * 1024 + NB * 16 * 1024 + 64 + kM * 4;
+  const int need = 1024 + 32 * 1024 + NB * 16 * 1024 + 64 + kM * 8;
   return std::max(need, kSmemMin);
 }
 

@@ -8,7 +8,8 @@
 // Both are HBM-bound.  Work is token-major so each hidden row is read once:
 // a warp owns a token row, moves it in 16-byte vectors with UNROLL vectors per
 // lane in flight, and writes it to each of its k permuted rows (dispatch) or
-// accumulates its k expert rows in fp32 in slot order (combine).
+// accumulates its k expert rows in fp32 in slot order (combine: acc = acc + w*x
+// with a rounded product and a rounded add, then one RNE rounding to bf16).
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -162,8 +163,9 @@ __global__ void __launch_bounds__(kDcThreads) combine_kernel(CombineArgs a) {
               x[2] = __uint_as_float(buf[u].z);
               x[3] = __uint_as_float(buf[u].w);
             }
+            // fp32 accumulation in slot order: a rounded product, then a rounded add
 #pragma unroll
-            for (int i = 0; i < ELEMS; ++i) acc[u][i] = fmaf(w[j], x[i], acc[u][i]);
+            for (int i = 0; i < ELEMS; ++i) acc[u][i] = __fadd_rn(acc[u][i], __fmul_rn(w[j], x[i]));
           }
         }
       }
