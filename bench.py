@@ -46,6 +46,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=("cuda", "reference"), default="cuda")
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary workloads")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg (profiling runs)")
     return ap.parse_args()
 
 
@@ -347,7 +348,7 @@ def main():
                          "frac_of_8TBps": achieved / 8000.0},
             "e2e": e2e, "gpu_launches": args.steps, "status_ok": ok,
             "clocks": clocks,
-            "cpu_baseline": cpu_baseline() if world == 1 else None,
+            "cpu_baseline": cpu_baseline() if (world == 1 and not args.no_cpu) else None,
             "other_rows": extra,
         }
         print(json.dumps(line), flush=True)

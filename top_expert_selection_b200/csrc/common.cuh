@@ -18,11 +18,10 @@ constexpr long long kDefaultTimeoutNs = 1000LL * 1000 * 1000;  // 1 s; a healthy
 
 // Header at the start of every workspace that has device-side waits.
 struct WsHeader {
-  int32_t status;      // MOE_OK or MOE_ERR_DEVICE_TIMEOUT
-  uint32_t bar_count;  // grid barrier: arrivals in the current generation
-  uint32_t bar_gen;    // grid barrier: generation, bumped by the last arrival
-  uint32_t ticket;     // last-block-done counter (reductions)
-  uint32_t pad[12];    // keeps the header 64 bytes
+  int32_t status;              // MOE_OK or a MOE_ERR_DEVICE_* code
+  uint32_t ticket;             // last-block-done counter (reductions)
+  unsigned long long barrier;  // grid barrier: generation (high 32 bits) | arrivals (low 32 bits)
+  uint32_t pad[12];            // keeps the header 64 bytes
 };
 static_assert(sizeof(WsHeader) == 64, "workspace header is 64 bytes");
 
@@ -46,9 +45,22 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
   return v;
 }
 
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// The barrier generation a block must pass: read before the block arrives
+// (the generation only moves once every block has arrived).
+__device__ __forceinline__ uint32_t barrier_generation(WsHeader* h) {
+  return (uint32_t)(ld_acquire_u64(&h->barrier) >> 32);
+}
+
 // Grid-wide barrier for a co-resident (cooperatively launched) grid of
-// `nblocks` blocks.  `gen_at_entry` must be read (ld_acquire) by the block
-// before it arrives: the generation only moves once every block has arrived.
+// `nblocks` blocks.  One 64-bit word holds generation | arrivals: a block adds
+// 1; the last arrival adds 2^32 - nblocks, which bumps the generation and
+// clears the count in the same atomic.  Waiters poll the generation.
 // Returns false (and records a timeout) if the wait exceeded timeout_ns.
 // Must be called by all threads of the block.
 __device__ __forceinline__ bool grid_barrier(WsHeader* h, uint32_t nblocks, uint32_t gen_at_entry,
@@ -57,20 +69,19 @@ __device__ __forceinline__ bool grid_barrier(WsHeader* h, uint32_t nblocks, uint
   if (threadIdx.x == 0) {
     int ok = 1;
     __threadfence();
-    uint32_t arrived = atomicAdd(&h->bar_count, 1u);
-    if (arrived == nblocks - 1) {
-      atomicExch(&h->bar_count, 0u);
-      __threadfence();
-      atomicAdd(&h->bar_gen, 1u);
+    const unsigned long long old = atomicAdd(&h->barrier, 1ull);
+    if ((uint32_t)old == nblocks - 1) {
+      atomicAdd(&h->barrier, (1ull << 32) - (unsigned long long)nblocks);
     } else {
-      unsigned long long t0 = globaltimer_ns();
-      while (ld_acquire_u32(&h->bar_gen) == gen_at_entry) {
-        if ((long long)(globaltimer_ns() - t0) > timeout_ns) {
+      unsigned long long t0 = 0;
+      int spins = 0;
+      while ((uint32_t)(ld_acquire_u64(&h->barrier) >> 32) == gen_at_entry) {
+        if (++spins == 64) t0 = globaltimer_ns();
+        if (spins > 64 && (long long)(globaltimer_ns() - t0) > timeout_ns) {
           record_timeout(h);
           ok = 0;
           break;
         }
-        __nanosleep(64);
       }
     }
     __threadfence();

@@ -160,7 +160,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
   const int c = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint32_t gen = ld_acquire_u32(&a.hdr->bar_gen);
+  const uint32_t gen = barrier_generation(a.hdr);
   const uint32_t ncols = a.N <= 32 ? 32u : (a.N <= 64 ? 64u : (a.N <= 128 ? 128u : 256u));
   const int sl0 = (int)((long long)a.nslices * c / a.G), sl1 = (int)((long long)a.nslices * (c + 1) / a.G);
 

@@ -73,8 +73,7 @@ struct RouteArgs {
   int32_t* tile_mn;
   int32_t* totals;
   WsHeader* hdr;
-  int32_t* gcount;   // [2][E]
-  uint32_t* table;   // [G][E]
+  uint32_t* table;   // [G][row_stride bytes]: per-block expert counts
   int T, E, k;
   int score_fn, pre, grouped, n_group, topk_group, topn;
   int renorm;
@@ -91,17 +90,18 @@ struct RouteArgs {
   int cnt_bytes;   // width of a block's histogram entry in the table: 1, 2 or 4
   int row_stride;  // bytes per table row (16-byte multiple)
   int fast;        // 1: sigmoid fast path
+  int ids_in_smem; // 1: the block's selections also kept in shared memory (u16)
   long long timeout_ns;
 };
 
 struct RouteSmem {
   // offsets (bytes) inside dynamic shared memory
-  int stage, cand, bias, hist_cta, hist_w, offs, cnt, bar, flag, scan, total;
+  int stage, cand, bias, hist_cta, hist_w, offs, cnt, bar, flag, scan, ids, total;
 };
 
 __host__ __device__ inline int cand_bytes_per_warp() { return 4 * kCandStride * 12; }
 
-__host__ __device__ inline RouteSmem route_smem_layout(int E, int stage_bytes) {
+__host__ __device__ inline RouteSmem route_smem_layout(int E, int stage_bytes, int ids_bytes) {
   RouteSmem L;
   int o = 0;
   L.stage = o;
@@ -124,6 +124,8 @@ __host__ __device__ inline RouteSmem route_smem_layout(int E, int stage_bytes) {
   o += 16;
   L.scan = o;
   o += 32 * 4;
+  L.ids = o;
+  o += (ids_bytes + 15) & ~15;
   L.total = o;
   return L;
 }
@@ -182,9 +184,15 @@ __device__ __forceinline__ float sigmoid_f32(float x) { return 1.0f / (1.0f + ex
 // -------------------------------------------------------------------------
 // warp per token (E > 32): lane l owns experts [l*VPL, l*VPL + VPL)
 // -------------------------------------------------------------------------
+// keep a copy of a selection in the block's shared-memory id list (phase 2
+// reads it instead of global memory)
+__device__ __forceinline__ void keep_id(uint16_t* ids_s, int local_item, int e) {
+  if (ids_s) ids_s[local_item] = (uint16_t)e;
+}
+
 template <int VPL>
 __device__ void select_token_warp(const RouteArgs& a, const uint8_t* row, int t, const float* bias_s,
-                                  int* hist_cta, int lane) {
+                                  int* hist_cta, int lane, uint16_t* ids_s, int t_base) {
   const int E = a.E;
   const unsigned FULL = 0xffffffffu;
   float lg[VPL], s[VPL], key[VPL];
@@ -363,6 +371,7 @@ __device__ void select_token_warp(const RouteArgs& a, const uint8_t* row, int t,
   if (has_slot) {
     const size_t o = (size_t)t * a.k + lane;
     a.ids[o] = my_id;
+    keep_id(ids_s, (t - t_base) * a.k + lane, my_id);
     store_from_f32(a.weights, a.weights_dtype, o, v);
     if ((unsigned)my_id < (unsigned)E) atomicAdd(&hist_cta[my_id], 1); else record_bounds(a.hdr);
   }
@@ -373,7 +382,7 @@ __device__ void select_token_warp(const RouteArgs& a, const uint8_t* row, int t,
 // -------------------------------------------------------------------------
 template <int EMAX>
 __device__ void select_token_thread(const RouteArgs& a, const uint8_t* row, int t, const float* bias_s,
-                                    int* hist_cta) {
+                                    int* hist_cta, uint16_t* ids_s, int t_base) {
   const int E = a.E;
   float lg[EMAX], s[EMAX], key[EMAX];
 #pragma unroll
@@ -490,6 +499,7 @@ __device__ void select_token_thread(const RouteArgs& a, const uint8_t* row, int 
       const float w = a.renorm ? (val[j] / norm) * a.scale : val[j] * a.scale;
       const size_t o = (size_t)t * a.k + j;
       a.ids[o] = sel[j];
+      keep_id(ids_s, (t - t_base) * a.k + j, sel[j]);
       store_from_f32(a.weights, a.weights_dtype, o, w);
       if ((unsigned)sel[j] < (unsigned)E) atomicAdd(&hist_cta[sel[j]], 1); else record_bounds(a.hdr);
     }
@@ -523,7 +533,7 @@ __device__ __forceinline__ int expert_slot(int g, int rot, int e) {
 template <int V, int ESZ>
 __device__ void select_quad_fast(const RouteArgs& a, const uint8_t* stage, int lt_base, int n, int t_round0,
                                  const float (&cb)[V], const float* bias_s, float* cand, int* hist_cta,
-                                 int lane) {
+                                 int lane, uint16_t* ids_s, int t_base) {
   constexpr int EPC = 16 / ESZ, NC = V / EPC;
   constexpr uint32_t VMASK = (V >= 32) ? 0xffffffffu : ((1u << V) - 1u);
   const unsigned FULL = 0xffffffffu;
@@ -685,6 +695,7 @@ __device__ void select_quad_fast(const RouteArgs& a, const uint8_t* stage, int l
         const size_t o = (size_t)t * a.k + my_rank[r];
         const float wv = a.renorm ? (my_s[r] / sel_sum) * a.scale : my_s[r] * a.scale;
         a.ids[o] = my_e[r];
+        keep_id(ids_s, (int)(t - t_base) * a.k + my_rank[r], my_e[r]);
         store_from_f32(a.weights, a.weights_dtype, o, wv);
         atomicAdd(&hist_cta[my_e[r]], 1);
       }
@@ -737,6 +748,7 @@ __device__ void select_quad_fast(const RouteArgs& a, const uint8_t* stage, int l
       if (g == 0) {
         const float sg = sigmoid_f32(stage_val(a, row, win));
         a.ids[(size_t)t * a.k + jr] = win;
+        keep_id(ids_s, (int)(t - t_base) * a.k + jr, win);
         ssum = ssum + sg;
         if ((unsigned)win < (unsigned)a.E) atomicAdd(&hist_cta[win], 1); else record_bounds(a.hdr);
       }
@@ -800,7 +812,14 @@ template <int VPL, int FAST_ESZ>
 __global__ void __launch_bounds__(kThreads, 1) route_kernel(RouteArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int E = a.E;
-  const RouteSmem L = route_smem_layout(E, a.stage_bytes);
+  const int c = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  // contiguous token range of this block
+  const int base_n = a.T / a.G, rem = a.T % a.G;
+  const int t_begin = c * base_n + min(c, rem);
+  const int t_end = t_begin + base_n + (c < rem ? 1 : 0);
+  const int n_items = (t_end - t_begin) * a.k;
+  const RouteSmem L = route_smem_layout(E, a.stage_bytes, a.ids_in_smem ? n_items * 2 : 0);
   uint8_t* stage = smem + L.stage;
   float* bias_s = reinterpret_cast<float*>(smem + L.bias);
   int* hist_cta = reinterpret_cast<int*>(smem + L.hist_cta);
@@ -810,19 +829,18 @@ __global__ void __launch_bounds__(kThreads, 1) route_kernel(RouteArgs a) {
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L.bar);
   int* flag = reinterpret_cast<int*>(smem + L.flag);
   int* scan_scratch = reinterpret_cast<int*>(smem + L.scan);
+  uint16_t* ids_s = a.ids_in_smem ? reinterpret_cast<uint16_t*>(smem + L.ids) : nullptr;
 
-  const int c = blockIdx.x;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint32_t gen = ld_acquire_u32(&a.hdr->bar_gen);
-  const int par = (int)(gen & 1u);
+  const uint32_t gen = barrier_generation(a.hdr);
 
-  // contiguous token range of this block
-  const int base_n = a.T / a.G, rem = a.T % a.G;
-  const int t_begin = c * base_n + min(c, rem);
-  const int t_end = t_begin + base_n + (c < rem ? 1 : 0);
-
-  if (threadIdx.x < kMaxSub) mbar_init(&bar[threadIdx.x], 1);
-  if (threadIdx.x == 0) flag[1] = 0;  // set when a staging wait gave up
+  // the first round's logits start streaming before anything else
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kMaxSub; ++s) mbar_init(&bar[s], 1);
+    flag[1] = 0;  // set when a staging wait gave up
+  }
+  __syncthreads();
+  const int n0 = min(a.chunk_tokens, t_end - t_begin);
+  int nsub = (n0 > 0) ? stage_issue(a, stage, bar, t_begin, n0) : 0;
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     bias_s[e] = a.has_bias ? load_as_f32(a.bias, a.bias_dtype, e) : 0.0f;
     hist_cta[e] = 0;
@@ -844,7 +862,7 @@ __global__ void __launch_bounds__(kThreads, 1) route_kernel(RouteArgs a) {
   uint32_t round = 0;
   for (int t0 = t_begin; t0 < t_end; t0 += a.chunk_tokens, ++round) {
     const int n = min(a.chunk_tokens, t_end - t0);
-    const int nsub = stage_issue(a, stage, bar, t0, n);
+    if (round > 0) nsub = stage_issue(a, stage, bar, t0, n);
     const uint32_t parity = round & 1u;
     if constexpr (FAST_ESZ > 0) {
       const int nquads = (n + 3) >> 2;
@@ -854,7 +872,7 @@ __global__ void __launch_bounds__(kThreads, 1) route_kernel(RouteArgs a) {
           for (int sb = s0; sb <= s1; ++sb)
             if (!stage_wait(a, bar, sb, parity)) flag[1] = 1;
         }
-        select_quad_fast<FV, FAST_ESZ>(a, stage, qd * 4, n, t0, cb, bias_s, cand, hist_cta, lane);
+        select_quad_fast<FV, FAST_ESZ>(a, stage, qd * 4, n, t0, cb, bias_s, cand, hist_cta, lane, ids_s, t_begin);
       }
     } else {
       for (int sb = 0; sb < nsub; ++sb)
@@ -863,15 +881,16 @@ __global__ void __launch_bounds__(kThreads, 1) route_kernel(RouteArgs a) {
         for (int lt = threadIdx.x; lt < n; lt += blockDim.x) {
           const uint8_t* row = stage + (size_t)lt * a.row_bytes;
           if (E <= 8)
-            select_token_thread<8>(a, row, t0 + lt, bias_s, hist_cta);
+            select_token_thread<8>(a, row, t0 + lt, bias_s, hist_cta, ids_s, t_begin);
           else if (E <= 16)
-            select_token_thread<16>(a, row, t0 + lt, bias_s, hist_cta);
+            select_token_thread<16>(a, row, t0 + lt, bias_s, hist_cta, ids_s, t_begin);
           else
-            select_token_thread<32>(a, row, t0 + lt, bias_s, hist_cta);
+            select_token_thread<32>(a, row, t0 + lt, bias_s, hist_cta, ids_s, t_begin);
         }
       } else {
         for (int lt = warp; lt < n; lt += kWarps)
-          select_token_warp<VPL>(a, stage + (size_t)lt * a.row_bytes, t0 + lt, bias_s, hist_cta, lane);
+          select_token_warp<VPL>(a, stage + (size_t)lt * a.row_bytes, t0 + lt, bias_s, hist_cta, lane, ids_s,
+                                 t_begin);
       }
     }
     __syncthreads();
@@ -885,73 +904,105 @@ __global__ void __launch_bounds__(kThreads, 1) route_kernel(RouteArgs a) {
     if (a.cnt_bytes == 1) trow[e] = (uint8_t)h;
     else if (a.cnt_bytes == 2) reinterpret_cast<uint16_t*>(trow)[e] = (uint16_t)h;
     else reinterpret_cast<uint32_t*>(trow)[e] = (uint32_t)h;
-    if (h) atomicAdd(&a.gcount[par * E + e], h);
   }
   if (!grid_barrier(a.hdr, (uint32_t)a.G, gen, a.timeout_ns, flag)) return;
   if (!staged_ok) return;  // a staging wait gave up (recorded); outputs undefined
 
-  // ---------------- phase 2: offsets, slots, tiles ----------------
-  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = __ldcg(&a.gcount[par * E + e]);
-  // rows of earlier blocks: 16-byte vectors, rows spread over thread groups
-  const int vpr = a.row_stride >> 4;
-  const int epv = 16 / a.cnt_bytes;
-  const int rpr = max(1, min((int)blockDim.x / vpr, c));  // row groups actually used
+  // ---------------- phase 2: totals and block base from the table ----------------
+  // Every block reads every row (16-byte vectors, all loads in flight): the sum
+  // of all rows gives the expert counts, the sum of rows before this block its
+  // base.  Integer sums in a fixed order: deterministic, no atomics.
+  const int vpr = a.row_stride >> 4;          // vectors per row
+  const int epv = 16 / a.cnt_bytes;           // entries per vector
+  const int rpr = max(1, min((int)blockDim.x / vpr, a.G));  // row groups
   const int tr = threadIdx.x / vpr, tq = threadIdx.x % vpr;
-  int acc[16];
+  int tot[16], pre[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) acc[i] = 0;
+  for (int i = 0; i < 16; ++i) tot[i] = pre[i] = 0;
   if (tr < rpr) {
-    for (int cp = tr; cp < c; cp += rpr) {
-      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(a.table) +
-                                                            (size_t)cp * a.row_stride) + tq);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-      if (a.cnt_bytes == 1) {
+    constexpr int kBatch = 8;
+    for (int cp0 = tr; cp0 < a.G; cp0 += rpr * kBatch) {
+      uint4 v[kBatch];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) acc[i] += (w[i >> 2] >> (8 * (i & 3))) & 0xffu;
-      } else if (a.cnt_bytes == 2) {
+      for (int b = 0; b < kBatch; ++b) {
+        const int cp = cp0 + b * rpr;
+        v[b] = cp < a.G ? __ldcg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(a.table) +
+                                                                (size_t)cp * a.row_stride) + tq)
+                        : make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] += (w[i >> 1] >> (16 * (i & 1))) & 0xffffu;
-      } else {
+      for (int b = 0; b < kBatch; ++b) {
+        const int cp = cp0 + b * rpr;
+        const bool before = cp < c;
+        const uint32_t w[4] = {v[b].x, v[b].y, v[b].z, v[b].w};
+        if (a.cnt_bytes == 1) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[i] += (int)w[i];
+          for (int i = 0; i < 16; ++i) {
+            const int x = (w[i >> 2] >> (8 * (i & 3))) & 0xff;
+            tot[i] += x;
+            pre[i] += before ? x : 0;
+          }
+        } else if (a.cnt_bytes == 2) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int x = (w[i >> 1] >> (16 * (i & 1))) & 0xffff;
+            tot[i] += x;
+            pre[i] += before ? x : 0;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            tot[i] += (int)w[i];
+            pre[i] += before ? (int)w[i] : 0;
+          }
+        }
+      }
+    }
+  }
+  // reduce the row groups through shared memory (the stage is free now)
+  int* part_t = reinterpret_cast<int*>(stage);  // [rpr][E]
+  int* part_p = part_t + rpr * E;               // [rpr][E]
+  if (tr < rpr) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int e = tq * epv + i;
+      if (i < epv && e < E) {
+        part_t[tr * E + e] = tot[i];
+        part_p[tr * E + e] = pre[i];
       }
     }
   }
   __syncthreads();
-  int* part = reinterpret_cast<int*>(stage);  // the stage is free now: [rpr][E]
-  if (tr < rpr) {  // (zeros when c == 0)
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int e = tq * epv + i;
-      if (i < epv && e < E) part[tr * E + e] = acc[i];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int st = 0, sp = 0;
+    for (int r = 0; r < rpr; ++r) {
+      st += part_t[r * E + e];
+      sp += part_p[r * E + e];
     }
+    cnt[e] = st;
+    hist_cta[e] = sp;  // earlier blocks' rows (offsets added below)
   }
   __syncthreads();
   scan_padded_offsets(cnt, offs, E, a.tile, scan_scratch);
   const int P = offs[E];
   const int ntiles = P / a.tile;
 
-  // block base per expert = padded offset + rows of earlier blocks
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int base = offs[e];
-    for (int r = 0; r < rpr; ++r) base += part[r * E + e];
-    hist_cta[e] = base;  // reuse as the block's running base
-  }
+  // ---------------- phase 2: slots in token order ----------------
+  // per-warp counts over a contiguous split of the block's selections, their
+  // exclusive prefix over warps, then a walk that ranks equal experts inside
+  // each 32-item chunk (match + popcount)
   for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) hist_w[i] = 0;
   __syncthreads();
-
-  // per-warp counts over a contiguous split of the block's selections
-  const long long i_begin = (long long)t_begin * a.k, i_end = (long long)t_end * a.k;
-  const long long ni = i_end - i_begin;
-  const long long w_begin = i_begin + ni * warp / kWarps;
-  const long long w_end = i_begin + ni * (warp + 1) / kWarps;
-  for (long long i = w_begin + lane; i < w_end; i += 32) {
-    const int e = a.ids[i];
+  const long long i_begin = (long long)t_begin * a.k;
+  const int w_begin = (int)((long long)n_items * warp / kWarps);
+  const int w_end = (int)((long long)n_items * (warp + 1) / kWarps);
+  for (int i = w_begin + lane; i < w_end; i += 32) {
+    const int e = ids_s ? (int)ids_s[i] : a.ids[i_begin + i];
     if ((unsigned)e < (unsigned)E) atomicAdd(&hist_w[warp * E + e], 1); else record_bounds(a.hdr);
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int run = hist_cta[e];
+    int run = offs[e] + hist_cta[e];
     for (int w = 0; w < kWarps; ++w) {
       const int h = hist_w[w * E + e];
       hist_w[w * E + e] = run;
@@ -959,14 +1010,12 @@ __global__ void __launch_bounds__(kThreads, 1) route_kernel(RouteArgs a) {
     }
   }
   __syncthreads();
-
-  // token-order walk: rank among equal experts inside each 32-item chunk
-  for (long long i0 = w_begin; i0 < w_end; i0 += 32) {
-    const long long i = i0 + lane;
+  for (int i0 = w_begin; i0 < w_end; i0 += 32) {
+    const int i = i0 + lane;
     const bool act = i < w_end;
     const unsigned amask = __ballot_sync(0xffffffffu, act);
     if (act) {
-      int e = a.ids[i];
+      int e = ids_s ? (int)ids_s[i] : a.ids[i_begin + i];
       if ((unsigned)e >= (unsigned)E) {
         record_bounds(a.hdr);
         e = 0;
@@ -977,37 +1026,37 @@ __global__ void __launch_bounds__(kThreads, 1) route_kernel(RouteArgs a) {
       const int slot = hist_w[warp * E + e] + rank;
       __syncwarp(amask);
       if (lane == leader) hist_w[warp * E + e] += __popc(m);
-      a.e2p[i] = slot;
-      if ((unsigned)slot < (unsigned)a.max_padded) a.p2t[slot] = (int)(i / a.k); else record_bounds(a.hdr);
+      a.e2p[i_begin + i] = slot;
+      if ((unsigned)slot < (unsigned)a.max_padded) a.p2t[slot] = (int)((i_begin + i) / a.k); else record_bounds(a.hdr);
     }
     __syncwarp();
   }
 
-  // tile tables and padding rows: tiles split evenly over blocks
+  // ---------------- tile tables and padding rows (a warp per tile) ----------------
   if (ntiles > a.max_tiles || P > a.max_padded) {
     if (threadIdx.x == 0) record_bounds(a.hdr);
     return;
   }
   const int tc0 = (int)((long long)ntiles * c / a.G), tc1 = (int)((long long)ntiles * (c + 1) / a.G);
-  for (int tc = tc0 + threadIdx.x; tc < tc1; tc += blockDim.x) {
+  for (int tc = tc0 + warp; tc < tc1; tc += kWarps) {
     const int row = tc * a.tile;
     int lo = 0, hi = E - 1;  // largest e with offs[e] <= row
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
       if (offs[mid] <= row) lo = mid; else hi = mid - 1;
     }
-    const int e = lo;
-    const int lim = min(row + a.tile, offs[e] + cnt[e]);
-    a.tile_expert[tc] = e;
-    a.tile_mn[tc] = lim;
-    for (int r = lim; r < row + a.tile; ++r) a.p2t[r] = -1;
+    const int lim = min(row + a.tile, offs[lo] + cnt[lo]);
+    if (lane == 0) {
+      a.tile_expert[tc] = lo;
+      a.tile_mn[tc] = lim;
+    }
+    for (int r = lim + lane; r < row + a.tile; r += 32) a.p2t[r] = -1;
   }
 
   if (c == 0) {
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
       a.counts[e] = cnt[e];
       a.offsets[e] = offs[e];
-      a.gcount[(par ^ 1) * E + e] = 0;  // the next call's counters
     }
     if (threadIdx.x == 0) {
       a.offsets[E] = P;
@@ -1096,9 +1145,9 @@ int grid_for(const moe_route_params* p, const DevInfo& d) {
   return g;
 }
 
-// workspace: header | counters [2][E] | table [G][row] (256-byte aligned, rows
-// sized for the widest 4-byte entries; read with 16-byte vector loads)
-size_t table_offset(int E) { return (sizeof(WsHeader) + (size_t)2 * E * sizeof(int32_t) + 255) & ~(size_t)255; }
+// workspace: header | table [G][row] (256-byte aligned, rows sized for the
+// widest 4-byte entries; read with 16-byte vector loads)
+size_t table_offset(int) { return 256; }
 
 size_t ws_bytes_for(int E, int G) {
   const size_t row = ((size_t)E * 4 + 15) & ~(size_t)15;
@@ -1198,7 +1247,6 @@ extern "C" int moe_route(const moe_route_params* p, const void* logits, const vo
   a.tile_mn = tile_mn_limit;
   a.totals = totals;
   a.hdr = reinterpret_cast<WsHeader*>(ws);
-  a.gcount = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(ws) + sizeof(WsHeader));
   a.table = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(ws) + table_offset(p->num_experts));
   if ((reinterpret_cast<uintptr_t>(ws) & 15) != 0) return MOE_ERR_WORKSPACE;
   a.T = T;
@@ -1231,11 +1279,12 @@ extern "C" int moe_route(const moe_route_params* p, const void* logits, const vo
   a.row_stride = (p->num_experts * a.cnt_bytes + 15) & ~15;
   a.fast = fast_path_ok(p) ? 1 : 0;
   a.timeout_ns = kDefaultTimeoutNs;
-  // the stage region also holds phase 2's per-row-group partial sums
+  // the stage region also holds phase 2's per-row-group partial sums (two sets)
   const int vpr = a.row_stride / 16;
-  const int part_bytes = (kThreads / vpr) * a.E * 4;
+  const int part_bytes = 2 * std::max(1, std::min(kThreads / vpr, a.G)) * a.E * 4;
   a.stage_bytes = (std::max(a.chunk_tokens * a.row_bytes, part_bytes) + 15) & ~15;
-  const RouteSmem L = route_smem_layout(a.E, a.stage_bytes);
+  a.ids_in_smem = ((long long)per_block * a.k * 2 <= 32 * 1024) ? 1 : 0;
+  const RouteSmem L = route_smem_layout(a.E, a.stage_bytes, a.ids_in_smem ? per_block * a.k * 2 : 0);
   const int smem = L.total;
   if (smem > d.smem_optin || smem > kStageBytesMax + 128 * 1024) return MOE_ERR_UNSUPPORTED;
 
@@ -1274,7 +1323,7 @@ namespace moe {
 namespace {
 __global__ void barrier_probe_kernel(WsHeader* hdr, uint32_t expected, long long timeout_ns) {
   __shared__ int flag;
-  const uint32_t gen = ld_acquire_u32(&hdr->bar_gen);
+  const uint32_t gen = barrier_generation(hdr);
   grid_barrier(hdr, expected, gen, timeout_ns, &flag);
 }
 }  // namespace
