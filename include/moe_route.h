@@ -161,6 +161,30 @@ int moe_route(const moe_route_params* p, const void* logits, const void* bias, i
               int32_t* expanded_to_permuted, int32_t* permuted_to_token, int32_t* tile_expert,
               int32_t* tile_mn_limit, int32_t* totals, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * moe_route_no_alloc -- moe_route for callers that cannot allocate device
+ * memory: serving runtimes whose memory manager owns the whole GPU and forbids
+ * allocations outside its pool, plugin or custom-op interfaces that provide
+ * inputs and outputs but no workspace, plain C callers without a device
+ * allocator, and latency-critical paths that cannot pay for cudaMalloc.  (The
+ * pages have no counterpart; this is an interface convenience.)
+ *
+ * Same arguments, results and errors as moe_route, without ws/ws_bytes: the
+ * workspace is a library-owned __device__ array of 512 KB that every GPU loading
+ * the library holds until the process exits.  Calls needing more (the workspace
+ * grows with E and the SM count; moe_route_workspace_bytes reports it) return
+ * MOE_ERR_WORKSPACE.  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress); later calls reuse it.  Each call clears the
+ * array's 64-byte header on `stream` before launching.  All calls share the one
+ * array: calls that may overlap on the GPU (different streams, or several host
+ * threads) race and must be serialised by the caller.  The call allocates no
+ * device memory.  Device-side status (timeouts, bounds) is not reported.
+ */
+int moe_route_no_alloc(const moe_route_params* p, const void* logits, const void* bias, int32_t* topk_ids,
+                       void* topk_weights, int32_t* expert_counts, int32_t* padded_offsets,
+                       int32_t* expanded_to_permuted, int32_t* permuted_to_token, int32_t* tile_expert,
+                       int32_t* tile_mn_limit, int32_t* totals, void* stream);
+
 /* Workspace bytes of the aux-loss entry points (scores, loss forward). */
 int moe_aux_workspace_bytes(int32_t num_tokens, int32_t num_experts, size_t* bytes);
 

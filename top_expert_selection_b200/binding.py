@@ -38,7 +38,7 @@ EXPORTED = (
     "moe_route_workspace_bytes", "moe_route", "moe_aux_workspace_bytes", "moe_aux_scores",
     "moe_aux_loss_fwd", "moe_aux_loss_bwd", "moe_dispatch", "moe_combine",
     "moe_rmsnorm_router_topk_workspace_bytes", "moe_rmsnorm_router_topk", "moe_debug_barrier_wait",
-    "moe_debug_sigmoid_proxy_error",
+    "moe_debug_sigmoid_proxy_error", "moe_route_no_alloc",
 )
 
 
@@ -82,6 +82,7 @@ def lib() -> ctypes.CDLL:
             "moe_route_capacity": ([RP, ctypes.POINTER(i64), ctypes.POINTER(i64)], ctypes.c_int),
             "moe_route_workspace_bytes": ([RP, ctypes.POINTER(sz)], ctypes.c_int),
             "moe_route": ([RP, P, P, P, P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
+            "moe_route_no_alloc": ([RP, P, P, P, P, P, P, P, P, P, P, P, P], ctypes.c_int),
             "moe_aux_workspace_bytes": ([i32, i32, ctypes.POINTER(sz)], ctypes.c_int),
             "moe_aux_scores": ([i32, i32, i32, i32, P, P, P, P, P, sz, P], ctypes.c_int),
             "moe_aux_loss_fwd": ([i32, i32, i32, i32, f32, P, P, P, P, sz, P], ctypes.c_int),
@@ -341,3 +342,12 @@ def rmsnorm_router_topk(hidden, gamma, W, bias=None, *, k: int, eps: float = 1e-
     ws = decode_workspace(T, H, E, dev) if ws is None else ws
     rmsnorm_router_topk_into(hidden, gamma, W, bias, k, eps, act, out_norm, ids, aff, lg, ws)
     return {"out_norm": out_norm, "ids": ids, "affinities": aff, "logits": lg, "ws": ws}
+
+
+def route_no_alloc_into(p: RouteParams, logits: torch.Tensor, bias: Optional[torch.Tensor],
+                        out: Dict[str, torch.Tensor], stream=None) -> None:
+    """moe_route_no_alloc: like route_into, with the library's own static workspace (no allocation)."""
+    names = ("ids", "weights", "counts", "offsets", "e2p", "p2t", "tile_expert", "tile_mn_limit", "totals")
+    rc = lib().moe_route_no_alloc(ctypes.byref(p), _p(logits), _p(bias), *[_p(out[n]) for n in names],
+                                  _stream(stream))
+    _check(rc, "moe_route_no_alloc")

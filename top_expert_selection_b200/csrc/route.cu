@@ -1372,3 +1372,56 @@ extern "C" int moe_debug_sigmoid_proxy_error(const float* x, int64_t n, float* o
   proxy_error_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, (long long)n, out);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
+
+// ---------------------------------------------------------------------------
+// moe_route_no_alloc: moe_route with a library-owned, statically allocated
+// workspace.
+//
+// Some callers cannot allocate device memory when they route: code running
+// under a memory manager that owns all device memory (a serving runtime that
+// reserves the GPU's memory up front and forbids allocations outside its own
+// pool), plugin or custom-op interfaces that hand the operator its inputs and
+// outputs but no workspace, plain C callers with no device allocator, and
+// latency-critical paths that cannot afford cudaMalloc's synchronisation.
+// For them the workspace lives in a file-scope __device__ array that every GPU
+// loading this library holds until the process exits.
+// ---------------------------------------------------------------------------
+namespace moe {
+namespace {
+
+constexpr size_t kStaticScratchBytes = 512 * 1024;  // the route workspace for E up to a few hundred experts
+__device__ __align__(256) uint8_t g_route_scratch[kStaticScratchBytes];
+
+struct ScratchSlot {
+  std::once_flag once;
+  void* ptr = nullptr;
+  cudaError_t err = cudaSuccess;
+};
+ScratchSlot g_scratch_slot[64];
+
+}  // namespace
+}  // namespace moe
+
+extern "C" int moe_route_no_alloc(const moe_route_params* p, const void* logits, const void* bias,
+                                  int32_t* topk_ids, void* topk_weights, int32_t* expert_counts,
+                                  int32_t* padded_offsets, int32_t* expanded_to_permuted,
+                                  int32_t* permuted_to_token, int32_t* tile_expert, int32_t* tile_mn_limit,
+                                  int32_t* totals, void* stream) {
+  const int v = validate(p);
+  if (v != MOE_OK) return v;
+  const DevInfo d = device_info();
+  if (d.sms <= 0) return MOE_ERR_CUDA;
+  if (ws_bytes_for(p->num_experts, d.sms) > kStaticScratchBytes) return MOE_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+  ScratchSlot& slot = g_scratch_slot[dev];
+  // set-up, once per device, with that device current: the array's device address
+  std::call_once(slot.once, [&slot] { slot.err = cudaGetSymbolAddress(&slot.ptr, g_route_scratch); });
+  if (slot.err != cudaSuccess || slot.ptr == nullptr) return MOE_ERR_CUDA;
+  // the array keeps the previous call's contents: its header (status word and
+  // barrier state) must start at zero
+  if (cudaMemsetAsync(slot.ptr, 0, sizeof(WsHeader), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return moe_route(p, logits, bias, topk_ids, topk_weights, expert_counts, padded_offsets, expanded_to_permuted,
+                   permuted_to_token, tile_expert, tile_mn_limit, totals, slot.ptr, kStaticScratchBytes, stream);
+}
