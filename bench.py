@@ -358,99 +358,100 @@ def main():
         pg.destroy_process_group()
 
 
-def _time_graph(fn, n_iter, stream):
+def _time_calls(calls, n_rep, stream):
+    """Device time per call of a list of calls (each on its own input/output set), captured once in a
+    CUDA graph and replayed n_rep times; us per call."""
     import torch
     with torch.cuda.stream(stream):
-        fn()
+        for f in calls:
+            f()
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
-        fn()
+        for f in calls:
+            f()
     torch.cuda.synchronize()
-    for _ in range(3):
+    for _ in range(2):
         g.replay()
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record()
-    for _ in range(n_iter):
+    for _ in range(n_rep):
         g.replay()
     e1.record()
     torch.cuda.synchronize()
-    return e0.elapsed_time(e1) * 1000.0 / n_iter  # us
+    return e0.elapsed_time(e1) * 1000.0 / (n_rep * len(calls))
 
 
 def secondary_rows(dev, hbm):
-    """The other workloads of the path, timed the same way (for context; not the headline)."""
+    """The other workloads of the path, timed like the headline (inputs/outputs rotated over more than
+    the L2 capacity, CUDA-graph replay); for context, not the headline."""
     import torch
     from top_expert_selection_b200 import binding as B
     from top_expert_selection_b200 import workloads as W
     stream = torch.cuda.Stream(dev)
     rows = {}
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    # Mixtral-style route + dispatch + combine (T=65536, E=8, k=2, H=4096)
+    # Mixtral-style route + dispatch + combine (T=65536, E=8, k=2, H=4096); the hidden / expert rows
+    # (>= 0.5 GB) exceed L2 by themselves
     spec = W.MIXTRAL_ROUTE
     mi = W.mixtral_inputs()
     p = B.route_params(spec.T, spec.E, spec.k, score_fn=W.SOFTMAX, softmax_before_topk=0, renormalize=0,
                        tile_tokens_dim=128, logits_dtype=W.BF16, weights_dtype=W.F32)
-    r = B.Router(p, dev)
-    lg = mi["logits"].to(dev)
-    o = r(lg)
+    rts = [B.Router(p, dev) for _ in range(24)]
+    lgs = [mi["logits"].to(dev) for _ in range(24)]
+    o = rts[0](lgs[0])
     torch.cuda.synchronize()
     P = int(o["totals"][0])
     H = W.MIXTRAL_HIDDEN
     hid = mi["hidden"].to(dev)
-    disp = torch.empty((r.max_padded, H), dtype=torch.bfloat16, device=dev)
-    eo = torch.randn((r.max_padded, H), device=dev).to(torch.bfloat16)
+    disp = torch.empty((rts[0].max_padded, H), dtype=torch.bfloat16, device=dev)
+    eo = torch.randn((rts[0].max_padded, H), device=dev).to(torch.bfloat16)
     comb = torch.empty((spec.T, H), dtype=torch.bfloat16, device=dev)
-    us_route = _time_graph(lambda: r(lg), 200, stream)
-    us_disp = _time_graph(lambda: B.dispatch_into(hid, o["e2p"], o["p2t"], o["totals"], 2, disp), 20, stream)
-    us_comb = _time_graph(lambda: B.combine_into(eo, o["e2p"], o["weights"], 2, comb), 20, stream)
+    rows["mixtral_route_us"] = _time_calls([(lambda i=i: rts[i](lgs[i])) for i in range(24)], 20, stream)
+    us_disp = _time_calls([lambda: B.dispatch_into(hid, o["e2p"], o["p2t"], o["totals"], 2, disp)], 20, stream)
+    us_comb = _time_calls([lambda: B.combine_into(eo, o["e2p"], o["weights"], 2, comb)], 20, stream)
     disp_bytes = spec.T * H * 2 + P * H * 2 + spec.T * 2 * 4 + P * 4
     comb_bytes = spec.T * 2 * H * 2 + spec.T * 2 * 8 + spec.T * H * 2
-    rows["mixtral_route_us"] = us_route
-    rows["mixtral_dispatch"] = {"us": us_disp, "GBps": disp_bytes / us_disp / 1e3, "frac": disp_bytes / us_disp / 1e3 / hbm}
-    rows["mixtral_combine"] = {"us": us_comb, "GBps": comb_bytes / us_comb / 1e3, "frac": comb_bytes / us_comb / 1e3 / hbm}
-    del disp, eo, comb, hid
-    # aux loss (T=32768, E=128, k=8)
+    rows["mixtral_dispatch"] = {"us": us_disp, "GBps": disp_bytes / us_disp / 1e3,
+                                "frac": disp_bytes / us_disp / 1e3 / hbm}
+    rows["mixtral_combine"] = {"us": us_comb, "GBps": comb_bytes / us_comb / 1e3,
+                               "frac": comb_bytes / us_comb / 1e3 / hbm}
+    del disp, eo, comb, hid, rts, lgs
+    # aux loss (T=32768, E=128, k=8): 10 rotated sets of 16 MB logits / probs / gradients
     a = W.QWEN3_AUX
+    R = 10
     alg = W.aux_inputs(a)["logits"].to(dev)
-    ws = B.aux_workspace(a.T, a.E, dev)
-    sc = B.aux_scores(alg, a.k, ws=ws)
-    loss = torch.empty(1, device=dev)
-    glog = torch.empty_like(alg)
+    sets = []
+    for _ in range(R):
+        lg = alg.clone()
+        ws = B.aux_workspace(a.T, a.E, dev)
+        sc = B.aux_scores(lg, a.k, ws=ws)
+        sets.append((lg, ws, sc, torch.empty(1, device=dev), torch.empty_like(lg)))
     gl = torch.ones(1, device=dev)
-
-    def aux_scores_fn():
-        flush.zero_()
-        B.aux_scores_into(alg, a.k, sc["probs"], sc["routing_map"], sc["tokens_per_expert"], ws)
-
-    def loss_fn():
-        flush.zero_()
-        B.aux_loss_fwd_into(sc["probs"], sc["tokens_per_expert"], a.T, a.k, a.coeff, loss, ws)
-
-    def bwd_fn():
-        flush.zero_()
-        B.aux_loss_bwd_into(gl, sc["probs"], sc["tokens_per_expert"], a.T, a.k, a.coeff, None, glog)
-
-    us_flush = _time_graph(lambda: flush.zero_(), 20, stream)
-    rows["aux_scores_us"] = _time_graph(aux_scores_fn, 20, stream) - us_flush
-    rows["aux_loss_fwd_us"] = _time_graph(loss_fn, 20, stream) - us_flush
-    rows["aux_loss_bwd_us"] = _time_graph(bwd_fn, 20, stream) - us_flush
-    # decode fused (T=128, H=7168, E=256, k=8)
+    rows["aux_scores_us"] = _time_calls(
+        [(lambda z=z: B.aux_scores_into(z[0], a.k, z[2]["probs"], z[2]["routing_map"], z[2]["tokens_per_expert"],
+                                        z[1])) for z in sets], 20, stream)
+    rows["aux_loss_fwd_us"] = _time_calls(
+        [(lambda z=z: B.aux_loss_fwd_into(z[2]["probs"], z[2]["tokens_per_expert"], a.T, a.k, a.coeff, z[3], z[1]))
+         for z in sets], 20, stream)
+    rows["aux_loss_bwd_us"] = _time_calls(
+        [(lambda z=z: B.aux_loss_bwd_into(gl, z[2]["probs"], z[2]["tokens_per_expert"], a.T, a.k, a.coeff, None,
+                                          z[4])) for z in sets], 20, stream)
+    del sets
+    # decode fused (T=128, H=7168, E=256, k=8): 24 rotated sets of hidden states and router weights
     d = W.DECODE_FUSED
     di = W.decode_inputs(d)
-    x, gam, Wm, bb = (di[n].to(dev) for n in ("hidden", "gamma", "W", "bias"))
-    res = B.rmsnorm_router_topk(x, gam, Wm, bb, k=d.k)
-
-    def dec_fn():
-        flush.zero_()
-        B.rmsnorm_router_topk_into(x, gam, Wm, bb, d.k, d.eps, d.act, res["out_norm"], res["ids"], res["affinities"],
-                                   None, res["ws"])
-
-    rows["decode_us"] = _time_graph(dec_fn, 20, stream) - us_flush
-    rows["note"] = ("us per call, device time from CUDA graph replays; dispatch/combine inputs exceed L2; "
-                    "aux and decode calls follow an L2 flush whose time is subtracted")
+    dsets = []
+    for _ in range(24):
+        x, gam, Wm, bb = (di[n].to(dev) for n in ("hidden", "gamma", "W", "bias"))
+        dsets.append((x, gam, Wm, bb, B.rmsnorm_router_topk(x, gam, Wm, bb, k=d.k)))
+    rows["decode_us"] = _time_calls(
+        [(lambda z=z: B.rmsnorm_router_topk_into(z[0], z[1], z[2], z[3], d.k, d.eps, d.act, z[4]["out_norm"],
+                                                 z[4]["ids"], z[4]["affinities"], None, z[4]["ws"]))
+         for z in dsets], 20, stream)
+    rows["note"] = ("us per call, device time of CUDA-graph replays over input/output sets rotated past the "
+                    "126 MB L2 (dispatch/combine inputs exceed it alone)")
     return rows
 
 

@@ -50,8 +50,10 @@ __device__ __forceinline__ float sigmoid_f32(float x) { return 1.0f / (1.0f + ex
 // --------------------------------------------------------------------------
 // scores: warp per token, lane l owns experts [l*VPL, l*VPL + VPL)
 // --------------------------------------------------------------------------
+constexpr int kScoreThreads = 512;
+
 template <int VPL>
-__global__ void __launch_bounds__(kAuxThreads) aux_scores_kernel(int T, int E, int k, int score_fn,
+__global__ void __launch_bounds__(kScoreThreads) aux_scores_kernel(int T, int E, int k, int score_fn,
                                                                  const float* __restrict__ logits,
                                                                  float* __restrict__ probs,
                                                                  uint8_t* __restrict__ rmap,
@@ -64,16 +66,35 @@ __global__ void __launch_bounds__(kAuxThreads) aux_scores_kernel(int T, int E, i
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
 
-  for (long long t = (long long)blockIdx.x * kAuxWarps + warp; t < T; t += (long long)gridDim.x * kAuxWarps) {
+  const int nw = blockDim.x >> 5;
+  for (long long t = (long long)blockIdx.x * nw + warp; t < T; t += (long long)gridDim.x * nw) {
     const float* row = logits + t * E;
     float x[VPL], p[VPL];
     uint32_t valid = 0;
+    if constexpr (VPL % 4 == 0) {
+      // a lane's VPL experts are contiguous: 16-byte loads when the row allows it
+      const bool vec = ((E & 3) == 0) && (lane * VPL + VPL <= E);
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      const int e = lane * VPL + i;
-      const bool v = e < E;
-      x[i] = v ? __ldcs(row + e) : 0.0f;
-      valid |= (v ? 1u : 0u) << i;
+      for (int i = 0; i < VPL; i += 4) {
+        const int e = lane * VPL + i;
+        if (vec) {
+          const float4 q = __ldcs(reinterpret_cast<const float4*>(row + e));
+          x[i] = q.x; x[i + 1] = q.y; x[i + 2] = q.z; x[i + 3] = q.w;
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) x[i + j] = (e + j < E) ? __ldcs(row + e + j) : 0.0f;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) valid |= ((lane * VPL + i < E) ? 1u : 0u) << i;
+    } else {
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const int e = lane * VPL + i;
+        const bool v = e < E;
+        x[i] = v ? __ldcs(row + e) : 0.0f;
+        valid |= (v ? 1u : 0u) << i;
+      }
     }
     float sum = 0.0f;
     if (score_fn == MOE_SOFTMAX) {
@@ -124,6 +145,23 @@ __global__ void __launch_bounds__(kAuxThreads) aux_scores_kernel(int T, int E, i
     }
     float* prow = probs + t * E;
     uint8_t* mrow = rmap + t * E;
+    if constexpr (VPL % 4 == 0) {
+      const bool vec = ((E & 3) == 0) && (lane * VPL + VPL <= E);
+      if (vec) {
+#pragma unroll
+        for (int i = 0; i < VPL; i += 4) {
+          const int e = lane * VPL + i;
+          __stcs(reinterpret_cast<float4*>(prow + e), make_float4(p[i], p[i + 1], p[i + 2], p[i + 3]));
+          const uint32_t m4 = ((chosen >> i) & 1u) | (((chosen >> (i + 1)) & 1u) << 8) |
+                              (((chosen >> (i + 2)) & 1u) << 16) | (((chosen >> (i + 3)) & 1u) << 24);
+          *reinterpret_cast<uint32_t*>(mrow + e) = m4;
+        }
+#pragma unroll
+        for (int i = 0; i < VPL; ++i)
+          if ((chosen >> i) & 1u) atomicAdd(&hist[lane * VPL + i], 1);
+        continue;
+      }
+    }
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       const int e = lane * VPL + i;
@@ -174,13 +212,25 @@ __global__ void __launch_bounds__(kAuxThreads) aux_loss_fwd_kernel(long long n, 
   float acc = 0.0f;
   if ((E & 3) == 0 && (b0 & 3) == 0) {
     const long long q1 = b1 >> 2;
-    for (long long q = (b0 >> 2) + threadIdx.x; q < q1; q += blockDim.x) {
-      const float4 v = __ldcs(reinterpret_cast<const float4*>(probs) + q);
-      const int e = (int)((q << 2) % E);
-      acc = fmaf(v.x, tpe_s[e], acc);
-      acc = fmaf(v.y, tpe_s[e + 1], acc);
-      acc = fmaf(v.z, tpe_s[e + 2], acc);
-      acc = fmaf(v.w, tpe_s[e + 3], acc);
+    constexpr int kB = 8;  // independent 16-byte loads in flight per thread
+    for (long long q0 = (b0 >> 2) + threadIdx.x; q0 < q1; q0 += (long long)blockDim.x * kB) {
+      float4 v[kB];
+#pragma unroll
+      for (int b = 0; b < kB; ++b) {
+        const long long q = q0 + (long long)b * blockDim.x;
+        v[b] = q < q1 ? __ldcs(reinterpret_cast<const float4*>(probs) + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int b = 0; b < kB; ++b) {
+        const long long q = q0 + (long long)b * blockDim.x;
+        const int e = (int)((q << 2) % E);
+        if (q < q1) {
+          acc = fmaf(v[b].x, tpe_s[e], acc);
+          acc = fmaf(v[b].y, tpe_s[e + 1], acc);
+          acc = fmaf(v[b].z, tpe_s[e + 2], acc);
+          acc = fmaf(v[b].w, tpe_s[e + 3], acc);
+        }
+      }
     }
     for (long long i = (q1 << 2) + threadIdx.x; i < b1; i += blockDim.x) acc = fmaf(probs[i], tpe_s[i % E], acc);
   } else {
@@ -199,12 +249,18 @@ __global__ void __launch_bounds__(kAuxThreads) aux_loss_fwd_kernel(long long n, 
     last = (atomicAdd(&hdr->ticket, 1u) == gridDim.x - 1);
   }
   __syncthreads();
-  if (last && threadIdx.x == 0) {
+  if (last && threadIdx.x < 32) {
+    // warp 0 adds the block partials: lane l takes blocks l, l+32, ... (all
+    // loads in flight), then a fixed shuffle tree -- the same order every call
     __threadfence();
     double s = 0.0;
-    for (unsigned b = 0; b < gridDim.x; ++b) s += __ldcg(&w.partials[b]);
-    *loss = (float)(C * s);
-    hdr->ticket = 0;
+    for (unsigned b = threadIdx.x; b < gridDim.x; b += 32) s += __ldcg(&w.partials[b]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (threadIdx.x == 0) {
+      *loss = (float)(C * s);
+      hdr->ticket = 0;
+    }
   }
 }
 
@@ -227,19 +283,36 @@ __global__ void __launch_bounds__(kAuxThreads) aux_loss_bwd_kernel(int T, int E,
     const float* prow = probs + t * E;
     float p[VPL], gp[VPL];
     float dot = 0.0f;
+    const bool vec = (VPL % 4 == 0) && ((E & 3) == 0) && (lane * VPL + VPL <= E);
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       const int e = lane * VPL + i;
-      p[i] = e < E ? __ldcs(prow + e) : 0.0f;
+      if (vec && (i & 3) == 0) {
+        const float4 q = __ldcs(reinterpret_cast<const float4*>(prow + e));
+        p[i] = q.x;
+        if (i + 1 < VPL) p[i + 1] = q.y;
+        if (i + 2 < VPL) p[i + 2] = q.z;
+        if (i + 3 < VPL) p[i + 3] = q.w;
+      } else if (!vec) {
+        p[i] = e < E ? __ldcs(prow + e) : 0.0f;
+      }
       gp[i] = e < E ? gp_s[e] : 0.0f;
-      dot = fmaf(p[i], gp[i], dot);
     }
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) dot = fmaf(p[i], gp[i], dot);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       const int e = lane * VPL + i;
-      if (e < E) {
+      if (vec && (i & 3) == 0 && i + 3 < VPL) {
+        if (grad_probs)
+          __stcs(reinterpret_cast<float4*>(grad_probs + t * E + e), make_float4(gp[i], gp[i + 1], gp[i + 2], gp[i + 3]));
+        if (grad_logits)
+          __stcs(reinterpret_cast<float4*>(grad_logits + t * E + e),
+                 make_float4(p[i] * (gp[i] - dot), p[i + 1] * (gp[i + 1] - dot), p[i + 2] * (gp[i + 2] - dot),
+                             p[i + 3] * (gp[i + 3] - dot)));
+      } else if (!vec && e < E) {
         if (grad_probs) __stcs(grad_probs + t * E + e, gp[i]);
         if (grad_logits) __stcs(grad_logits + t * E + e, p[i] * (gp[i] - dot));
       }
@@ -296,10 +369,10 @@ extern "C" int moe_aux_scores(int32_t T, int32_t E, int32_t k, int32_t score_fn,
   if (!tokens_per_expert || (T > 0 && (!logits || !probs || !routing_map))) return MOE_ERR_INVALID_ARG;
   if (!ws || ws_bytes < aux_ws_bytes(E)) return MOE_ERR_WORKSPACE;
   const int vpl = pick_vpl(E);
-  const int grid = std::max(1, std::min((T + kAuxWarps - 1) / kAuxWarps, sm_count() * 8));
+  const int grid = std::max(1, std::min((T + 15) / 16, sm_count() * 2));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const size_t smem = (size_t)E * sizeof(int);
-  MOE_VPL_SWITCH(vpl, (aux_scores_kernel<V><<<grid, kAuxThreads, smem, st>>>(T, E, k, score_fn, logits, probs,
+  MOE_VPL_SWITCH(vpl, (aux_scores_kernel<V><<<grid, kScoreThreads, smem, st>>>(T, E, k, score_fn, logits, probs,
                                                                             routing_map, tokens_per_expert, ws)));
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

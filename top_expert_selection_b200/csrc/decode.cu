@@ -210,10 +210,20 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
   // ---------------- phase 2: normalise, project ----------------
   if (ok) {
-    if (tid < a.T) {
-      double s = 0.0;
-      for (int cp = 0; cp < a.G; ++cp) s += __ldcg(&a.sumsq[(size_t)cp * kM + tid]);
-      r_s[tid] = 1.0 / sqrt(s / (double)a.H + (double)a.eps);
+    // warp w reduces tokens w, w+8, ...: lane l adds the partials of blocks
+    // l, l+32, ... (all loads in flight), then a fixed shuffle tree; every
+    // block computes the same r_t
+    for (int t = warp; t < a.T; t += kDecWarps) {
+      double sv[5];
+#pragma unroll
+      for (int i = 0; i < 5; ++i) {
+        const int cp = lane + 32 * i;
+        sv[i] = cp < a.G ? __ldcg(&a.sumsq[(size_t)cp * kM + t]) : 0.0;
+      }
+      double s = (sv[0] + sv[1]) + (sv[2] + sv[3]) + sv[4];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+      if (lane == 0) r_s[t] = 1.0 / sqrt(s / (double)a.H + (double)a.eps);
     }
     __syncthreads();
     const uint32_t idesc = idesc_bf16_f32(a.N);
@@ -226,12 +236,25 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           for (int nb = 0; nb < NB; ++nb)
             tma_load_2d(sB + (kb * NB + nb) * 8192, &wmap, nb * 64, sl * kKC + kb * 64, tma_bar);
       }
-      // normalised slice: (token, 16-byte group) pairs; 16 groups per token row
-      for (int i = tid; i < a.T * 16; i += kDecThreads) {
+      // normalised slice: (token, 16-byte group) pairs, 16 groups per token row;
+      // a thread's loads are all issued before any is used
+      constexpr int kPer = (kM * 16) / kDecThreads;  // pairs per thread (8)
+      uint4 xb[kPer];
+      const uint4 gv = __ldg(reinterpret_cast<const uint4*>(a.gamma + sl * kKC + (tid & 15) * 8));
+#pragma unroll
+      for (int b = 0; b < kPer; ++b) {
+        const int i = tid + b * kDecThreads;
         const int t = i >> 4, q = i & 15;
+        xb[b] = t < a.T ? __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)t * a.H + sl * kKC + q * 8))
+                        : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int b = 0; b < kPer; ++b) {
+        const int i = tid + b * kDecThreads;
+        const int t = i >> 4, q = i & 15;
+        if (t >= a.T) continue;
         const size_t off = (size_t)t * a.H + sl * kKC + q * 8;
-        const uint4 xv = __ldg(reinterpret_cast<const uint4*>(a.x + off));
-        const uint4 gv = __ldg(reinterpret_cast<const uint4*>(a.gamma + sl * kKC + q * 8));
+        const uint4 xv = xb[b];
         const double r = r_s[t];
         const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
         uint32_t ow[4];
@@ -311,8 +334,46 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   if (!grid_barrier(a.hdr, (uint32_t)a.G, gen + 1, a.timeout_ns, flag)) return;
 
   // ---------------- phase 3: reduce partial logits, top-k, affinities ----------------
+  // For each token of this block, warp w adds the partial logits of blocks
+  // w, w+8, ... (lane = 8 experts; all loads of a warp in flight), the 8 warp
+  // sums meet in shared memory and warp 0 adds them in warp order.
+  float* red = reinterpret_cast<float*>(sA);  // [kDecWarps][NP], the operand tiles are free now
   const int t0 = (int)((long long)a.T * c / a.G), t1 = (int)((long long)a.T * (c + 1) / a.G);
-  for (int t = t0 + warp; t < t1; t += kDecWarps) {
+  for (int t = t0; t < t1; ++t) {
+    {
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+      if (lane * 8 < a.NP) {
+        constexpr int kB = 8;
+        for (int cp0 = warp; cp0 < a.G; cp0 += kDecWarps * kB) {
+          float4 u[kB], w[kB];
+#pragma unroll
+          for (int b = 0; b < kB; ++b) {
+            const int cp = cp0 + b * kDecWarps;
+            if (cp < a.G) {
+              const float* src = a.plogits + ((size_t)cp * kM + t) * a.NP + lane * 8;
+              u[b] = __ldcg(reinterpret_cast<const float4*>(src));
+              w[b] = __ldcg(reinterpret_cast<const float4*>(src + 4));
+            } else {
+              u[b] = w[b] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+          }
+#pragma unroll
+          for (int b = 0; b < kB; ++b) {
+            acc[0] += u[b].x; acc[1] += u[b].y; acc[2] += u[b].z; acc[3] += u[b].w;
+            acc[4] += w[b].x; acc[5] += w[b].y; acc[6] += w[b].z; acc[7] += w[b].w;
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) red[warp * a.NP + lane * 8 + i] = acc[i];
+      }
+    }
+    __syncthreads();
+    if (warp != 0) {
+      __syncthreads();
+      continue;
+    }
     float lg[8];
     float bsum[8];
 #pragma unroll
@@ -321,14 +382,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       const int e = lane * 8 + i;
       bsum[i] = (a.bias && e < a.E) ? bf16_bits_to_f32(a.bias[e]) : 0.0f;
     }
-    for (int cp = 0; cp < a.G; ++cp) {
-      const float* src = a.plogits + ((size_t)cp * kM + t) * a.NP + lane * 8;
-      if (lane * 8 < a.NP) {
-        const float4 u = __ldcg(reinterpret_cast<const float4*>(src));
-        const float4 w = __ldcg(reinterpret_cast<const float4*>(src + 4));
-        lg[0] += u.x; lg[1] += u.y; lg[2] += u.z; lg[3] += u.w;
-        lg[4] += w.x; lg[5] += w.y; lg[6] += w.z; lg[7] += w.w;
-      }
+    if (lane * 8 < a.NP) {
+      for (int w = 0; w < kDecWarps; ++w)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) lg[i] += red[w * a.NP + lane * 8 + i];
     }
     uint32_t valid = 0;
 #pragma unroll
@@ -387,6 +444,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         a.aff[(size_t)t * a.E + e] = *reinterpret_cast<const uint16_t*>(&hb);
       }
     }
+    __syncthreads();
   }
 }
 

@@ -48,8 +48,11 @@ namespace moe {
 
 namespace {
 
-constexpr int kThreads = 512;
-constexpr int kWarps = kThreads / 32;
+// threads per block: the sigmoid fast path keeps few registers and runs 24
+// warps per SM; the generic paths keep larger per-thread arrays and run 16
+constexpr int kThreadsFast = 768;
+constexpr int kThreadsGeneric = 512;
+constexpr int kWarpsMax = kThreadsFast / 32;
 constexpr int kStageBytesMax = 96 * 1024;
 constexpr int kMaxSub = 8;         // bulk copies (and mbarriers) per staged round
 constexpr int kCandMax = 32;       // fast path: candidate slots per token
@@ -96,24 +99,26 @@ struct RouteArgs {
 
 struct RouteSmem {
   // offsets (bytes) inside dynamic shared memory
-  int stage, cand, bias, hist_cta, hist_w, offs, cnt, bar, flag, scan, ids, total;
+  int stage, cand, bias, hist_cta, hist_w, offs, cnt, bar, flag, scan, ids, lut, total;
 };
 
+// per warp: 4 tokens x kCandStride packed u64 keys, then 4 x kCandStride fp32 scores
 __host__ __device__ inline int cand_bytes_per_warp() { return 4 * kCandStride * 12; }
 
-__host__ __device__ inline RouteSmem route_smem_layout(int E, int stage_bytes, int ids_bytes) {
+__host__ __device__ inline RouteSmem route_smem_layout(int E, int stage_bytes, int ids_bytes, int nwarps,
+                                                       int lut_bytes) {
   RouteSmem L;
   int o = 0;
   L.stage = o;
   o += (stage_bytes + 127) & ~127;
   L.cand = o;
-  o += kWarps * cand_bytes_per_warp();
+  o += nwarps * cand_bytes_per_warp() + 8 * (32 + 4) * 4;  // + the fast path's per-lane bias table
   L.bias = o;
   o += ((E * 4) + 15) & ~15;
   L.hist_cta = o;
   o += ((E * 4) + 15) & ~15;
   L.hist_w = o;
-  o += ((kWarps * E * 4) + 15) & ~15;
+  o += ((nwarps * E * 4) + 15) & ~15;
   L.offs = o;
   o += (((E + 1) * 4) + 15) & ~15;
   L.cnt = o;
@@ -126,6 +131,8 @@ __host__ __device__ inline RouteSmem route_smem_layout(int E, int stage_bytes, i
   o += 32 * 4;
   L.ids = o;
   o += (ids_bytes + 15) & ~15;
+  L.lut = o;
+  o += (lut_bytes + 15) & ~15;
   L.total = o;
   return L;
 }
@@ -180,6 +187,33 @@ __device__ __forceinline__ float stage_val(const RouteArgs& a, const uint8_t* ro
 }
 
 __device__ __forceinline__ float sigmoid_f32(float x) { return 1.0f / (1.0f + expf(-x)); }
+
+// Exact sigmoid of a bf16 input by table: the kernel fills the table with the
+// very expression above for every bf16 value with biased exponent in
+// [kLutExpLo, kLutExpHi], both signs (8448 entries, 33 KB), so a lookup returns
+// exactly what sigmoid_f32 returns.  Inputs outside the range (|x| < 2^-25 or
+// |x| >= 2^8, and non-finite) are evaluated directly.
+constexpr int kLutExpLo = 102, kLutExpHi = 134;
+constexpr int kLutPerSign = (kLutExpHi - kLutExpLo + 1) * 128;
+constexpr int kLutEntries = 2 * kLutPerSign;
+
+__device__ __forceinline__ int lut_index(uint32_t b16) {
+  const int ex = (int)((b16 >> 7) & 0xffu);
+  if (ex < kLutExpLo || ex > kLutExpHi) return -1;
+  return (int)(b16 >> 15) * kLutPerSign + (ex - kLutExpLo) * 128 + (int)(b16 & 0x7fu);
+}
+
+__device__ __forceinline__ uint32_t lut_bits(int idx) {
+  const int sgn = idx / kLutPerSign, r = idx % kLutPerSign;
+  return ((uint32_t)sgn << 15) | ((uint32_t)(r / 128 + kLutExpLo) << 7) | (uint32_t)(r % 128);
+}
+
+// exact score of expert e of a staged bf16 row: table when available
+__device__ __forceinline__ float sigmoid_bf16_row(const float* lut, const uint8_t* row, int e) {
+  const uint32_t b16 = reinterpret_cast<const uint16_t*>(row)[e];
+  const int idx = lut ? lut_index(b16) : -1;
+  return idx >= 0 ? lut[idx] : sigmoid_f32(bf16_bits_to_f32((uint16_t)b16));
+}
 
 // -------------------------------------------------------------------------
 // warp per token (E > 32): lane l owns experts [l*VPL, l*VPL + VPL)
@@ -530,10 +564,79 @@ __device__ __forceinline__ int expert_slot(int g, int rot, int e) {
   return (((r / EPC) - rot + NC) & (NC - 1)) * EPC + (r % EPC);
 }
 
+// Per-lane constants 0.5 + bias of the lane's experts, in register-slot order,
+// one padded row of V + 4 floats per lane position g: the 16-byte loads of the
+// 8 lanes of a token fall in distinct bank groups.
+template <int V>
+__host__ __device__ constexpr int cb_stride() { return V + 4; }
+
+// Out-of-line exact selection of one token (rare): exact keys for all experts
+// of the lane, exact group scores, k rounds of segment argmax.
+template <int V, int ESZ>
+__device__ __noinline__ void select_token_exact8(const RouteArgs& a, const uint8_t* row, long long t, int g, int rot,
+                                                 int seg, unsigned smask, const float* bias_s, int* hist_cta,
+                                                 uint16_t* ids_s, int t_base) {
+  constexpr uint32_t VMASK = (V >= 32) ? 0xffffffffu : ((1u << V) - 1u);
+  float p[V];
+#pragma unroll
+  for (int j = 0; j < V; ++j) {
+    const int e = slot_expert<V, ESZ>(g, rot, j);
+    p[j] = sigmoid_f32(stage_val(a, row, e)) + bias_s[e];
+  }
+  uint32_t allowed = VMASK;
+  if (a.grouped) {
+    float e1 = -INFINITY, e2 = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      const float hi = fmaxf(e1, p[j]);
+      e2 = fmaxf(e2, fminf(e1, p[j]));
+      e1 = hi;
+    }
+    const float gsc = (a.topn == 1) ? e1 : (e1 + e2);
+    int rank = 0;
+    for (int h = 0; h < 8; ++h) {
+      const float o = __shfl_sync(smask, gsc, seg | h);
+      rank += (o > gsc || (o == gsc && h < g)) ? 1 : 0;
+    }
+    if (rank >= a.topk_group) allowed = 0;
+  }
+  float ssum = 0.0f;
+  for (int jr = 0; jr < a.k; ++jr) {
+    unsigned long long best = 0ull;
+#pragma unroll
+    for (int j = 0; j < V; ++j)
+      if ((allowed >> j) & 1u) {
+        const unsigned long long pk = pack_key(p[j], slot_expert<V, ESZ>(g, rot, j));
+        best = pk > best ? pk : best;
+      }
+#pragma unroll
+    for (int off = 1; off < 8; off <<= 1) {
+      const unsigned long long o = shfl_xor_u64(smask, best, off);
+      best = o > best ? o : best;
+    }
+    const int win = packed_expert(best);
+    if (win / V == g) allowed &= ~(1u << expert_slot<V, ESZ>(g, rot, win));
+    if (g == 0) {
+      const float sg = sigmoid_f32(stage_val(a, row, win));
+      a.ids[(size_t)t * a.k + jr] = win;
+      keep_id(ids_s, (int)(t - t_base) * a.k + jr, win);
+      ssum = ssum + sg;
+      if ((unsigned)win < (unsigned)a.E) atomicAdd(&hist_cta[win], 1); else record_bounds(a.hdr);
+    }
+  }
+  if (g == 0) {
+    for (int jr = 0; jr < a.k; ++jr) {
+      const size_t o = (size_t)t * a.k + jr;
+      const float sg = sigmoid_f32(stage_val(a, row, a.ids[o]));
+      store_from_f32(a.weights, a.weights_dtype, o, a.renorm ? (sg / ssum) * a.scale : sg * a.scale);
+    }
+  }
+}
+
 template <int V, int ESZ>
 __device__ void select_quad_fast(const RouteArgs& a, const uint8_t* stage, int lt_base, int n, int t_round0,
-                                 const float (&cb)[V], const float* bias_s, float* cand, int* hist_cta,
-                                 int lane, uint16_t* ids_s, int t_base) {
+                                 const float* cb_s, const float* bias_s, float* cand, int* hist_cta,
+                                 int lane, uint16_t* ids_s, int t_base, const float* lut) {
   constexpr int EPC = 16 / ESZ, NC = V / EPC;
   constexpr uint32_t VMASK = (V >= 32) ? 0xffffffffu : ((1u << V) - 1u);
   const unsigned FULL = 0xffffffffu;
@@ -546,12 +649,19 @@ __device__ void select_quad_fast(const RouteArgs& a, const uint8_t* stage, int l
 
   // ---- proxy keys (|p - key| <= kProxyDelta) and their top-2 ----
   float p[V];
-  float m1 = -INFINITY, m2 = -INFINITY;
+  float m1 = -INFINITY, m2 = -INFINITY, n1 = -INFINITY, n2 = -INFINITY;
+  const float* cbl = cb_s + g * cb_stride<V>();
 #pragma unroll
   for (int c = 0; c < NC; ++c) {
     const int cc = (c + rot) & (NC - 1);
     const uint4 v = *reinterpret_cast<const uint4*>(row + (size_t)g * V * ESZ + cc * 16);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float cbv[EPC];
+#pragma unroll
+    for (int i = 0; i < EPC; i += 4) {
+      const float4 b4 = *reinterpret_cast<const float4*>(cbl + c * EPC + i);
+      cbv[i] = b4.x; cbv[i + 1] = b4.y; cbv[i + 2] = b4.z; cbv[i + 3] = b4.w;
+    }
 #pragma unroll
     for (int i = 0; i < EPC; ++i) {
       float x;
@@ -560,12 +670,24 @@ __device__ void select_quad_fast(const RouteArgs& a, const uint8_t* stage, int l
       else
         x = __uint_as_float(w[i]);
       const int j = c * EPC + i;
-      const float pj = fmaf(0.5f, tanh_approx(0.5f * x), cb[j]);
+      const float pj = fmaf(0.5f, tanh_approx(0.5f * x), cbv[i]);
       p[j] = pj;
-      const float hi = fmaxf(m1, pj);
-      m2 = fmaxf(m2, fminf(m1, pj));
-      m1 = hi;
+      // two independent top-2 trackers (even / odd slots) shorten the dependency chain
+      if ((i & 1) == 0) {
+        const float hi = fmaxf(m1, pj);
+        m2 = fmaxf(m2, fminf(m1, pj));
+        m1 = hi;
+      } else {
+        const float hi = fmaxf(n1, pj);
+        n2 = fmaxf(n2, fminf(n1, pj));
+        n1 = hi;
+      }
     }
+  }
+  {
+    const float hi = fmaxf(m1, n1);
+    m2 = fmaxf(fminf(m1, n1), fmaxf(m2, n2));
+    m1 = hi;
   }
 
   // ---- exact top-2 keys of the lane: evaluated where the proxy is within
@@ -574,14 +696,15 @@ __device__ void select_quad_fast(const RouteArgs& a, const uint8_t* stage, int l
   int j1 = -1, j2 = -1;
   if (tv) {
     const float th = m2 - 2.0f * kProxyDelta;
-    uint32_t m = 0;
+    uint32_t mq[4] = {0u, 0u, 0u, 0u};  // independent partial masks
 #pragma unroll
-    for (int j = 0; j < V; ++j) m |= (p[j] >= th ? 1u : 0u) << j;
+    for (int j = 0; j < V; ++j) mq[j & 3] |= (p[j] >= th ? 1u : 0u) << j;
+    uint32_t m = (mq[0] | mq[1]) | (mq[2] | mq[3]);
     while (m) {
       const int j = __ffs(m) - 1;
       m &= m - 1;
       const int e = slot_expert<V, ESZ>(g, rot, j);
-      const float sg = sigmoid_f32(stage_val(a, row, e));
+      const float sg = (ESZ == 2) ? sigmoid_bf16_row(lut, row, e) : sigmoid_f32(stage_val(a, row, e));
       const float K = sg + bias_s[e];
       if (K > K1) {
         K2 = K1; S2 = S1; j2 = j1;
@@ -618,8 +741,10 @@ __device__ void select_quad_fast(const RouteArgs& a, const uint8_t* stage, int l
   const float tau = (2 * nkept >= a.k) ? (k2min - kProxyDelta) : -INFINITY;
   uint32_t mask = 0;
   if (kept && tv) {
+    uint32_t mq[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int j = 0; j < V; ++j) mask |= (p[j] >= tau ? 1u : 0u) << j;
+    for (int j = 0; j < V; ++j) mq[j & 3] |= (p[j] >= tau ? 1u : 0u) << j;
+    mask = (mq[0] | mq[1]) | (mq[2] | mq[3]);
     if (j1 >= 0) mask |= 1u << j1;
     if (j2 >= 0) mask |= 1u << j2;
   }
@@ -633,10 +758,10 @@ __device__ void select_quad_fast(const RouteArgs& a, const uint8_t* stage, int l
   const int total = __shfl_sync(FULL, incl, seg | 7);
   const bool slow = tv && (total > kCandMax);
 
-  // ---- fast: exact keys of the candidates, ranked by counting ----
-  float* ckey = cand + q * kCandStride;
-  float* cs = cand + 4 * kCandStride + q * kCandStride;
-  int* ce = reinterpret_cast<int*>(cand + 8 * kCandStride) + q * kCandStride;
+  // ---- fast: exact keys of the candidates, ranked by counting on packed
+  //      (ordered key, ~expert) words: larger key first, then lower expert ----
+  unsigned long long* ck = reinterpret_cast<unsigned long long*>(cand) + q * kCandStride;
+  float* cs = cand + 8 * kCandStride + q * kCandStride;
   if (tv && !slow) {
     int pos = incl - cnt;
     uint32_t m = mask;
@@ -650,12 +775,11 @@ __device__ void select_quad_fast(const RouteArgs& a, const uint8_t* stage, int l
       } else if (j == j2) {
         sg = S2; K = K2;
       } else {
-        sg = sigmoid_f32(stage_val(a, row, e));
+        sg = (ESZ == 2) ? sigmoid_bf16_row(lut, row, e) : sigmoid_f32(stage_val(a, row, e));
         K = sg + bias_s[e];
       }
-      ckey[pos] = K;
+      ck[pos] = pack_key(K, e);
       cs[pos] = sg;
-      ce[pos] = e;
       ++pos;
     }
   }
@@ -671,16 +795,11 @@ __device__ void select_quad_fast(const RouteArgs& a, const uint8_t* stage, int l
     my_s[r] = 0.0f;
     const int i = g + 8 * r;
     if (tv && !slow && i < total) {
-      const float Ki = ckey[i];
-      const int ei = ce[i];
+      const unsigned long long ki = ck[i];
       int rank = 0;
-      for (int jj = 0; jj < total; ++jj) {
-        const float Kj = ckey[jj];
-        const int ej = ce[jj];
-        rank += (Kj > Ki || (Kj == Ki && ej < ei)) ? 1 : 0;
-      }
+      for (int jj = 0; jj < total; ++jj) rank += (ck[jj] > ki) ? 1 : 0;
       my_rank[r] = rank;
-      my_e[r] = ei;
+      my_e[r] = packed_expert(ki);
       my_s[r] = cs[i];
       if (rank < a.k) sel_sum += my_s[r];
     }
@@ -703,64 +822,9 @@ __device__ void select_quad_fast(const RouteArgs& a, const uint8_t* stage, int l
   }
   __syncwarp();
 
-  // ---- slow: exact keys for every expert of the token ----
+  // ---- slow: exact keys for every expert of the token (rare) ----
   const unsigned smask = __ballot_sync(FULL, slow);
-  if (slow) {
-#pragma unroll
-    for (int j = 0; j < V; ++j) {
-      const int e = slot_expert<V, ESZ>(g, rot, j);
-      p[j] = sigmoid_f32(stage_val(a, row, e)) + bias_s[e];
-    }
-    uint32_t allowed = VMASK;
-    if (a.grouped) {
-      float e1 = -INFINITY, e2 = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < V; ++j) {
-        const float hi = fmaxf(e1, p[j]);
-        e2 = fmaxf(e2, fminf(e1, p[j]));
-        e1 = hi;
-      }
-      const float gsc = (a.topn == 1) ? e1 : (e1 + e2);
-      int rank = 0;
-#pragma unroll
-      for (int h = 0; h < 8; ++h) {
-        const float o = __shfl_sync(smask, gsc, seg | h);
-        rank += (o > gsc || (o == gsc && h < g)) ? 1 : 0;
-      }
-      if (rank >= a.topk_group) allowed = 0;
-    }
-    float ssum = 0.0f;
-    for (int jr = 0; jr < a.k; ++jr) {
-      unsigned long long best = 0ull;
-#pragma unroll
-      for (int j = 0; j < V; ++j)
-        if ((allowed >> j) & 1u) {
-          const unsigned long long pk = pack_key(p[j], slot_expert<V, ESZ>(g, rot, j));
-          best = pk > best ? pk : best;
-        }
-#pragma unroll
-      for (int off = 1; off < 8; off <<= 1) {
-        const unsigned long long o = shfl_xor_u64(smask, best, off);
-        best = o > best ? o : best;
-      }
-      const int win = packed_expert(best);
-      if (win / V == g) allowed &= ~(1u << expert_slot<V, ESZ>(g, rot, win));
-      if (g == 0) {
-        const float sg = sigmoid_f32(stage_val(a, row, win));
-        a.ids[(size_t)t * a.k + jr] = win;
-        keep_id(ids_s, (int)(t - t_base) * a.k + jr, win);
-        ssum = ssum + sg;
-        if ((unsigned)win < (unsigned)a.E) atomicAdd(&hist_cta[win], 1); else record_bounds(a.hdr);
-      }
-    }
-    if (g == 0) {
-      for (int jr = 0; jr < a.k; ++jr) {
-        const size_t o = (size_t)t * a.k + jr;
-        const float sg = sigmoid_f32(stage_val(a, row, a.ids[o]));
-        store_from_f32(a.weights, a.weights_dtype, o, a.renorm ? (sg / ssum) * a.scale : sg * a.scale);
-      }
-    }
-  }
+  if (slow) select_token_exact8<V, ESZ>(a, row, t, g, rot, seg, smask, bias_s, hist_cta, ids_s, t_base);
   __syncwarp();
 }
 
@@ -809,7 +873,8 @@ __device__ void scan_padded_offsets(const int* cnt, int* offs, int E, int tile, 
 // VPL: experts per lane (0 = a thread per token).  FAST_ESZ: 0 = generic exact
 // path; 2 or 4 = sigmoid fast path with V = VPL and that logits element size.
 template <int VPL, int FAST_ESZ>
-__global__ void __launch_bounds__(kThreads, 1) route_kernel(RouteArgs a) {
+__global__ void __launch_bounds__((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneric, 1) route_kernel(RouteArgs a) {
+  constexpr int kWarps = ((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneric) / 32;
   extern __shared__ __align__(128) uint8_t smem[];
   const int E = a.E;
   const int c = blockIdx.x;
@@ -819,7 +884,8 @@ __global__ void __launch_bounds__(kThreads, 1) route_kernel(RouteArgs a) {
   const int t_begin = c * base_n + min(c, rem);
   const int t_end = t_begin + base_n + (c < rem ? 1 : 0);
   const int n_items = (t_end - t_begin) * a.k;
-  const RouteSmem L = route_smem_layout(E, a.stage_bytes, a.ids_in_smem ? n_items * 2 : 0);
+  const RouteSmem L = route_smem_layout(E, a.stage_bytes, a.ids_in_smem ? n_items * 2 : 0, kWarps,
+                                       FAST_ESZ == 2 ? kLutEntries * 4 : 0);
   uint8_t* stage = smem + L.stage;
   float* bias_s = reinterpret_cast<float*>(smem + L.bias);
   int* hist_cta = reinterpret_cast<int*>(smem + L.hist_cta);
@@ -833,13 +899,13 @@ __global__ void __launch_bounds__(kThreads, 1) route_kernel(RouteArgs a) {
 
   const uint32_t gen = barrier_generation(a.hdr);
 
-  // the first round's logits start streaming before anything else
+  // the first round's logits start streaming before anything else: thread 0
+  // initialises the mbarriers and issues the bulk copies itself
+  const int n0 = min(a.chunk_tokens, t_end - t_begin);
   if (threadIdx.x == 0) {
     for (int s = 0; s < kMaxSub; ++s) mbar_init(&bar[s], 1);
     flag[1] = 0;  // set when a staging wait gave up
   }
-  __syncthreads();
-  const int n0 = min(a.chunk_tokens, t_end - t_begin);
   int nsub = (n0 > 0) ? stage_issue(a, stage, bar, t_begin, n0) : 0;
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     bias_s[e] = a.has_bias ? load_as_f32(a.bias, a.bias_dtype, e) : 0.0f;
@@ -847,16 +913,26 @@ __global__ void __launch_bounds__(kThreads, 1) route_kernel(RouteArgs a) {
   }
   __syncthreads();
 
-  // fast path: per-lane constants 0.5 + bias of the lane's experts
+  // fast path: per-lane constants 0.5 + bias, in register-slot order
   constexpr int FV = (FAST_ESZ > 0) ? VPL : 1;
-  float cb[FV];
+  float* cb_s = reinterpret_cast<float*>(smem + L.cand + kWarps * cand_bytes_per_warp());
   if constexpr (FAST_ESZ > 0) {
-    const int g = lane & 7;
-    const int rot = (g * (VPL / (16 / FAST_ESZ))) >> 3;
-#pragma unroll
-    for (int j = 0; j < FV; ++j) cb[j] = 0.5f + bias_s[slot_expert<FV, FAST_ESZ>(g, rot, j)];
+    for (int idx = threadIdx.x; idx < 8 * FV; idx += blockDim.x) {
+      const int g = idx / FV, j = idx % FV;
+      const int rot = (g * (FV / (16 / FAST_ESZ))) >> 3;
+      cb_s[g * cb_stride<FV>() + j] = 0.5f + bias_s[slot_expert<FV, FAST_ESZ>(g, rot, j)];
+    }
+    __syncthreads();
   }
   float* cand = reinterpret_cast<float*>(smem + L.cand + warp * cand_bytes_per_warp());
+  // bf16 fast path: exact-sigmoid table, filled while the logits stream in
+  float* lut = nullptr;
+  if constexpr (FAST_ESZ == 2) {
+    lut = reinterpret_cast<float*>(smem + L.lut);
+    for (int i = threadIdx.x; i < kLutEntries; i += blockDim.x)
+      lut[i] = sigmoid_f32(bf16_bits_to_f32((uint16_t)lut_bits(i)));
+    __syncthreads();
+  }
 
   // ---------------- phase 1: select ----------------
   uint32_t round = 0;
@@ -872,7 +948,8 @@ __global__ void __launch_bounds__(kThreads, 1) route_kernel(RouteArgs a) {
           for (int sb = s0; sb <= s1; ++sb)
             if (!stage_wait(a, bar, sb, parity)) flag[1] = 1;
         }
-        select_quad_fast<FV, FAST_ESZ>(a, stage, qd * 4, n, t0, cb, bias_s, cand, hist_cta, lane, ids_s, t_begin);
+        select_quad_fast<FV, FAST_ESZ>(a, stage, qd * 4, n, t0, cb_s, bias_s, cand, hist_cta, lane, ids_s, t_begin,
+                                       lut);
       }
     } else {
       for (int sb = 0; sb < nsub; ++sb)
@@ -909,93 +986,114 @@ __global__ void __launch_bounds__(kThreads, 1) route_kernel(RouteArgs a) {
   if (!staged_ok) return;  // a staging wait gave up (recorded); outputs undefined
 
   // ---------------- phase 2: totals and block base from the table ----------------
-  // Every block reads every row (16-byte vectors, all loads in flight): the sum
-  // of all rows gives the expert counts, the sum of rows before this block its
-  // base.  Integer sums in a fixed order: deterministic, no atomics.
-  const int vpr = a.row_stride >> 4;          // vectors per row
-  const int epv = 16 / a.cnt_bytes;           // entries per vector
-  const int rpr = max(1, min((int)blockDim.x / vpr, a.G));  // row groups
-  const int tr = threadIdx.x / vpr, tq = threadIdx.x % vpr;
-  int tot[16], pre[16];
+  // Every block reads every row of the table: the sum of all rows gives the
+  // expert counts, the sum of the rows of earlier blocks this block's base.
+  // Thread (row group rg, word w) reads 32-bit word w of rows rg, rg + R, ...
+  // (a warp reads consecutive words: coalesced), all loads in flight, and
+  // keeps per-entry sums; the partial sums go to shared memory word-major so
+  // the stores and the reduction reads hit distinct banks.  Integer sums in a
+  // fixed order: deterministic, no atomics.
+  const long long i_begin = (long long)t_begin * a.k;
+  const int w_begin = (int)((long long)n_items * warp / kWarps);
+  const int w_end = (int)((long long)n_items * (warp + 1) / kWarps);
+  int P = 0;
+  {
+    const int WPR = a.row_stride >> 2;                     // 32-bit words per row
+    const int EPW = 4 / a.cnt_bytes;                       // entries per word
+    const int R = max(1, min((int)blockDim.x / WPR, a.G));  // row groups
+    const int rg = threadIdx.x / WPR, w = threadIdx.x % WPR;
+    int tot[4] = {0, 0, 0, 0}, pre[4] = {0, 0, 0, 0};
+    if (rg < R) {
+      constexpr int kBatch = 20;
+      for (int cp0 = rg; cp0 < a.G; cp0 += R * kBatch) {
+        uint32_t v[kBatch];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) tot[i] = pre[i] = 0;
-  if (tr < rpr) {
-    constexpr int kBatch = 8;
-    for (int cp0 = tr; cp0 < a.G; cp0 += rpr * kBatch) {
-      uint4 v[kBatch];
-#pragma unroll
-      for (int b = 0; b < kBatch; ++b) {
-        const int cp = cp0 + b * rpr;
-        v[b] = cp < a.G ? __ldcg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(a.table) +
-                                                                (size_t)cp * a.row_stride) + tq)
-                        : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int b = 0; b < kBatch; ++b) {
-        const int cp = cp0 + b * rpr;
-        const bool before = cp < c;
-        const uint32_t w[4] = {v[b].x, v[b].y, v[b].z, v[b].w};
+        for (int b = 0; b < kBatch; ++b) {
+          const int cp = cp0 + b * R;
+          v[b] = cp < a.G ? __ldcg(reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint8_t*>(a.table) +
+                                                                     (size_t)cp * a.row_stride) + w)
+                          : 0u;
+        }
         if (a.cnt_bytes == 1) {
+          // byte entries: two 16-bit lanes per 32-bit add (entries 0,2 and
+          // 1,3); totals stay below 65536 because a block holds <= 255 tokens
+          uint32_t t02 = 0, t13 = 0, p02 = 0, p13 = 0;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int x = (w[i >> 2] >> (8 * (i & 3))) & 0xff;
-            tot[i] += x;
-            pre[i] += before ? x : 0;
+          for (int b = 0; b < kBatch; ++b) {
+            const uint32_t e02 = v[b] & 0x00ff00ffu, e13 = (v[b] >> 8) & 0x00ff00ffu;
+            t02 += e02;
+            t13 += e13;
+            if (cp0 + b * R < c) {
+              p02 += e02;
+              p13 += e13;
+            }
           }
-        } else if (a.cnt_bytes == 2) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int x = (w[i >> 1] >> (16 * (i & 1))) & 0xffff;
-            tot[i] += x;
-            pre[i] += before ? x : 0;
-          }
+          tot[0] += (int)(t02 & 0xffffu); tot[2] += (int)(t02 >> 16);
+          tot[1] += (int)(t13 & 0xffffu); tot[3] += (int)(t13 >> 16);
+          pre[0] += (int)(p02 & 0xffffu); pre[2] += (int)(p02 >> 16);
+          pre[1] += (int)(p13 & 0xffffu); pre[3] += (int)(p13 >> 16);
         } else {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            tot[i] += (int)w[i];
-            pre[i] += before ? (int)w[i] : 0;
+          for (int b = 0; b < kBatch; ++b) {
+            const bool before = cp0 + b * R < c;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              if (i < EPW) {
+                const int x = a.cnt_bytes == 2 ? (int)((v[b] >> (16 * i)) & 0xffffu) : (int)v[b];
+                tot[i] += x;
+                pre[i] += before ? x : 0;
+              }
+            }
           }
         }
       }
     }
-  }
-  // reduce the row groups through shared memory (the stage is free now)
-  int* part_t = reinterpret_cast<int*>(stage);  // [rpr][E]
-  int* part_p = part_t + rpr * E;               // [rpr][E]
-  if (tr < rpr) {
+    int* part_t = reinterpret_cast<int*>(stage);   // [R][EPW][WPR]
+    int* part_p = part_t + R * EPW * WPR;          // [R][EPW][WPR]
+    if (rg < R) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int e = tq * epv + i;
-      if (i < epv && e < E) {
-        part_t[tr * E + e] = tot[i];
-        part_p[tr * E + e] = pre[i];
+      for (int i = 0; i < 4; ++i)
+        if (i < EPW) {
+          part_t[(rg * EPW + i) * WPR + w] = tot[i];
+          part_p[(rg * EPW + i) * WPR + w] = pre[i];
+        }
+    }
+    __syncthreads();
+    for (int x = threadIdx.x; x < EPW * WPR; x += blockDim.x) {
+      const int i = x / WPR, ww = x % WPR;
+      const int e = ww * EPW + i;
+      if (e < E) {
+        int st = 0, sp = 0;
+        for (int r = 0; r < R; ++r) {
+          st += part_t[(r * EPW + i) * WPR + ww];
+          sp += part_p[(r * EPW + i) * WPR + ww];
+        }
+        cnt[e] = st;
+        hist_cta[e] = sp;
+      }
+    }
+    for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) hist_w[i] = 0;
+    __syncthreads();
+    scan_padded_offsets(cnt, offs, E, a.tile, scan_scratch);
+    P = offs[E];
+    if (c == 0) {
+      for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        a.counts[e] = cnt[e];
+        a.offsets[e] = offs[e];
+      }
+      if (threadIdx.x == 0) {
+        a.offsets[E] = P;
+        a.totals[0] = P;
+        a.totals[1] = P / a.tile;
       }
     }
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int st = 0, sp = 0;
-    for (int r = 0; r < rpr; ++r) {
-      st += part_t[r * E + e];
-      sp += part_p[r * E + e];
-    }
-    cnt[e] = st;
-    hist_cta[e] = sp;  // earlier blocks' rows (offsets added below)
-  }
-  __syncthreads();
-  scan_padded_offsets(cnt, offs, E, a.tile, scan_scratch);
-  const int P = offs[E];
   const int ntiles = P / a.tile;
 
   // ---------------- phase 2: slots in token order ----------------
   // per-warp counts over a contiguous split of the block's selections, their
   // exclusive prefix over warps, then a walk that ranks equal experts inside
   // each 32-item chunk (match + popcount)
-  for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) hist_w[i] = 0;
-  __syncthreads();
-  const long long i_begin = (long long)t_begin * a.k;
-  const int w_begin = (int)((long long)n_items * warp / kWarps);
-  const int w_end = (int)((long long)n_items * (warp + 1) / kWarps);
   for (int i = w_begin + lane; i < w_end; i += 32) {
     const int e = ids_s ? (int)ids_s[i] : a.ids[i_begin + i];
     if ((unsigned)e < (unsigned)E) atomicAdd(&hist_w[warp * E + e], 1); else record_bounds(a.hdr);
@@ -1053,17 +1151,6 @@ __global__ void __launch_bounds__(kThreads, 1) route_kernel(RouteArgs a) {
     for (int r = lim + lane; r < row + a.tile; r += 32) a.p2t[r] = -1;
   }
 
-  if (c == 0) {
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-      a.counts[e] = cnt[e];
-      a.offsets[e] = offs[e];
-    }
-    if (threadIdx.x == 0) {
-      a.offsets[E] = P;
-      a.totals[0] = P;
-      a.totals[1] = ntiles;
-    }
-  }
 }
 
 // ---------------------------------------------------------------------------
@@ -1146,7 +1233,7 @@ int grid_for(const moe_route_params* p, const DevInfo& d) {
 }
 
 // workspace: header | table [G][row] (256-byte aligned, rows sized for the
-// widest 4-byte entries; read with 16-byte vector loads)
+// widest 4-byte entries; read as 32-bit words)
 size_t table_offset(int) { return 256; }
 
 size_t ws_bytes_for(int E, int G) {
@@ -1179,7 +1266,7 @@ cudaError_t launch_route(const RouteArgs& a, int smem, cudaStream_t st) {
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.G);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneric);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -1279,12 +1366,15 @@ extern "C" int moe_route(const moe_route_params* p, const void* logits, const vo
   a.row_stride = (p->num_experts * a.cnt_bytes + 15) & ~15;
   a.fast = fast_path_ok(p) ? 1 : 0;
   a.timeout_ns = kDefaultTimeoutNs;
+  const int nthreads = a.fast ? kThreadsFast : kThreadsGeneric;
   // the stage region also holds phase 2's per-row-group partial sums (two sets)
-  const int vpr = a.row_stride / 16;
-  const int part_bytes = 2 * std::max(1, std::min(kThreads / vpr, a.G)) * a.E * 4;
+  const int wpr = a.row_stride / 4;
+  const int part_bytes = 2 * std::max(1, std::min(nthreads / wpr, a.G)) * (4 / a.cnt_bytes) * wpr * 4;
   a.stage_bytes = (std::max(a.chunk_tokens * a.row_bytes, part_bytes) + 15) & ~15;
   a.ids_in_smem = ((long long)per_block * a.k * 2 <= 32 * 1024) ? 1 : 0;
-  const RouteSmem L = route_smem_layout(a.E, a.stage_bytes, a.ids_in_smem ? per_block * a.k * 2 : 0);
+  const bool lut = a.fast && p->logits_dtype == MOE_BF16;
+  const RouteSmem L = route_smem_layout(a.E, a.stage_bytes, a.ids_in_smem ? per_block * a.k * 2 : 0, nthreads / 32,
+                                        lut ? kLutEntries * 4 : 0);
   const int smem = L.total;
   if (smem > d.smem_optin || smem > kStageBytesMax + 128 * 1024) return MOE_ERR_UNSUPPORTED;
 
