@@ -253,7 +253,11 @@ int moe_combine(int32_t T, int32_t H, int32_t k, int32_t dtype, const void* expe
                 const int32_t* expanded_to_permuted, const void* weights, int32_t weights_dtype,
                 void* out, void* stream);
 
-/* Workspace bytes of moe_rmsnorm_router_topk. */
+/*
+ * Workspace bytes of moe_rmsnorm_router_topk (header, fp32 logits [T,E] and
+ * per-token-run tickets).  The workspace must be zero before its first use
+ * (moe_workspace_init); each call leaves its tickets at zero again.
+ */
 int moe_rmsnorm_router_topk_workspace_bytes(int32_t T, int32_t H, int32_t E, size_t* bytes);
 
 /*
@@ -269,7 +273,14 @@ int moe_rmsnorm_router_topk_workspace_bytes(int32_t T, int32_t H, int32_t E, siz
  * hidden [T,H], gamma [H], W [H,E], bias [E] or NULL, out_norm [T,H],
  * affinities [T,E] -- bf16; ids [T,k] int32; debug_logits [T,E] fp32 or NULL
  * (receives the logits when given).  T <= 128 and H % 128 == 0 [NKI: Notes];
- * this build also needs E % 16 == 0 and E <= 256.
+ * this build also needs E % 16 == 0, E <= 256 and H <= 32768, and every
+ * pointer 16-byte aligned.  The launch is a grid of thread-block clusters
+ * (16 CTAs each where the GPU can place them, else 8) that never wait on one
+ * another; device-side waits are bounded and a wait that gives up leaves
+ * MOE_ERR_DEVICE_TIMEOUT in the workspace status word (outputs undefined).
+ * Returns MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED / MOE_ERR_WORKSPACE for
+ * bad arguments, MOE_ERR_CUDA when the launch fails.  Calls sharing one
+ * workspace must not overlap in time.
  */
 int moe_rmsnorm_router_topk(int32_t T, int32_t H, int32_t E, int32_t k, float eps, int32_t act,
                             const void* hidden, const void* gamma, const void* W, const void* bias,

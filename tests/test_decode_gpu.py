@@ -66,8 +66,11 @@ def test_decode_workload_full_size():
 
 @pytest.mark.parametrize("T,H,E,k,act,bias", [
     (1, 128, 16, 1, W.SIGMOID, False), (7, 256, 64, 4, W.SIGMOID, True), (128, 7168, 256, 8, W.SOFTMAX, True),
-    (33, 1024, 96, 6, W.SIGMOID, False), (128, 19200, 128, 8, W.SIGMOID, True), (64, 640, 48, 3, W.SOFTMAX, False)])
+    (33, 1024, 96, 6, W.SIGMOID, False), (128, 19200, 128, 8, W.SIGMOID, True), (64, 640, 48, 3, W.SOFTMAX, False),
+    (100, 2048, 160, 6, W.SIGMOID, True), (65, 512, 256, 8, W.SIGMOID, True), (128, 32768, 64, 4, W.SIGMOID, True)])
 def test_decode_shapes(T, H, E, k, act, bias):
+    # cluster sizes 2..16 (H/64 chunks), one or two 64-token groups, partial expert groups, and slices
+    # longer than the staging ring (H=19200, 32768)
     run_decode(W.DecodeSpec(T=T, H=H, E=E, k=k, act=act, has_bias=bias, seed=T + H + E))
 
 

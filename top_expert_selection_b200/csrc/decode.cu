@@ -8,23 +8,40 @@
 // Returns, Notes (T <= 128; H % 128 == 0; ACT2: top-K on raw logits, then the
 // activation on the selected experts only).
 //
-// One cooperative launch over G blocks; block c owns K-slice(s) of 128 hidden
-// columns and the matching 128 rows of W.
-//   phase 1  W slice -> shared memory by 2-D TMA (128-byte swizzle, the
-//            canonical MN-major operand layout of tcgen05.mma); 256 TMEM
-//            columns allocated; per-token partial sum of squares of the slice
-//            (double) -> workspace.  Bounded grid barrier.
-//   phase 2  every block adds the partial sums in block order (deterministic)
-//            and forms r_t = 1/sqrt(mean + eps) in double; normalises its
-//            slice (x*gamma exact in fp32, times r_t in double, one rounding to
-//            bf16), writes
-//            out_norm and the same bf16 values to shared memory in the
-//            K-major 128-byte-swizzled layout; one thread issues the
-//            M=128 x N=E x K=16 tcgen05.mma steps into TMEM; the partial logits
-//            go TMEM -> registers (tcgen05.ld) -> workspace.  Barrier.
-//   phase 3  block c sums the G partial logits of its tokens in block order,
-//            adds the bias, and writes ids (top-k on the raw logits, ties ->
-//            lower expert) and the masked bf16 affinities.
+// Work split: thread-block clusters of CS CTAs.  A cluster owns one group of
+// tokens (64, or all T <= 128) and one group of 64 experts over the whole
+// hidden dimension; CTA j of the cluster owns the j-th K-slice (a run of
+// 64-column chunks).  CS (1..16) and the token group size are chosen per GPU
+// from how many clusters of each size it can keep resident: the fewest
+// staged bytes per CTA with every cluster resident at once.  For T=128,
+// H=7168, E=256 that is e.g. 4 clusters x 16 CTAs (448 columns each) or
+// 8 clusters x 14 CTAs (512 columns, 64 tokens).
+//
+//   stage    x chunks (tokens x 64 columns) first, then gamma, then W chunks
+//            (64 rows x 64 experts) -> shared memory by TMA, 128-byte swizzle
+//            (the canonical K-major A / MN-major B layouts of tcgen05.mma); a
+//            ring of up to 8 chunk stages, refilled when the slice is longer.
+//   sum x^2  per token over the CTA's slice (double, from the staged chunks),
+//            exchanged through distributed shared memory after a cluster
+//            barrier; every CTA adds the CS partials in rank order and forms
+//            r_t = 1/sqrt(mean + eps) in double (all CTAs get the same bits),
+//            kept as r_hi + r_lo in fp32.
+//   project  the staged chunks are normalised in place: x*gamma is exact in
+//            fp32, its product with r_hi is rounded to fp32 and then to bf16;
+//            where that fp32 value sits exactly on a bf16 rounding midpoint
+//            the sign of the remainder (x*gamma*r_hi - p + x*gamma*r_lo, from
+//            two fused multiply-adds) picks the side, so the bf16 value is the
+//            single rounding of x*gamma*r.  One cluster per chunk also stores
+//            it to out_norm; one thread issues the M=128 x N=64 x K=16 MMAs.
+//   reduce   TMEM -> registers -> shared memory; after a cluster barrier CTA j
+//            adds its tokens' partial logits over the CS ranks (rank order) and
+//            stores the fp32 logits of its (tokens, experts) tile.
+//   select   a per-(token group, rank) ticket: the last of the expert-group
+//            clusters to store its tile (no waiting) adds the bias, takes the
+//            top-k on the raw logits (ties -> lower expert) and writes ids and
+//            the masked bf16 affinities, then resets the ticket.
+// No grid-wide barrier, no cooperative launch: clusters never wait on one
+// another, so the kernel also completes when the clusters run in waves.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -36,12 +53,18 @@
 namespace moe {
 namespace {
 
-constexpr int kDecThreads = 256;
+constexpr int kDecThreads = 512;
 constexpr int kDecWarps = kDecThreads / 32;
-constexpr int kKC = 128;         // hidden columns (MMA K) per slice
-constexpr int kM = 128;          // MMA M (tokens, zero-padded)
-constexpr int kMaxE = 256;       // MMA N limit
-constexpr int kSmemMin = 120 * 1024;  // > half an SM's shared memory: one block (and TMEM user) per SM
+constexpr int kChunk = 64;       // hidden columns per staged chunk (one 128-byte swizzle atom)
+constexpr int kExpGroup = 64;    // experts per cluster (MMA N <= 64)
+constexpr int kM = 128;          // MMA M: 64 token rows + 64 zero rows
+constexpr int kMaxE = 256;       // top-k stage: 8 experts per lane
+constexpr int kMaxStages = 8;    // staged chunks in flight (fewer when shared memory is short)
+constexpr int kMaxSliceChunks = 64;  // gamma slice kept in shared memory
+constexpr int kATile = kM * 128;      // 16 KB
+constexpr int kBTile = kChunk * 128;  // 8 KB (64 K rows x 64 experts)
+constexpr int kRedStride = kExpGroup + 4;  // padded fp32 row of the partial-logit tile
+constexpr int kSmemLimit = 227 * 1024;     // opt-in shared memory per CTA
 
 struct DecodeArgs {
   const uint16_t* x;      // [T,H] bf16
@@ -52,16 +75,41 @@ struct DecodeArgs {
   uint16_t* aff;          // [T,E]
   float* dbg_logits;      // [T,E] or null
   WsHeader* hdr;
-  double* sumsq;          // [G][kM]
-  float* plogits;         // [G][kM][NP]
+  float* logits;          // [T,E] fp32 (workspace)
+  uint32_t* tickets;      // [2][16] (workspace), zero between calls
   int T, H, E, k, act;
-  int NP;                 // E rounded up to 64 (B tile columns)
-  int N;                  // MMA N = E rounded up to 16
-  int G;
-  int nslices;            // H / kKC
+  int CS;                 // CTAs per cluster (K-split)
+  int TGS;                // tokens per cluster: 64 or 128
+  int NG;                 // expert groups
+  int nch;                // H / 64
+  int S;                  // ring stages
+  int maxb;               // most chunks any CTA owns
   float eps;
   long long timeout_ns;
 };
+
+// shared-memory layout (offsets from a 1024-byte aligned base)
+struct DecLayout {
+  int a, b, red, gam, psq, rs, bars, slot, flag, total;
+};
+// red: partial logits pushed by every CTA of the cluster for the rows this CTA
+// reduces, [CS][tpb][kRedStride] fp32; psq: partial sums of squares pushed by
+// every CTA, [CS][TGS] double.
+__host__ __device__ inline int dec_tpb(int TGS, int CS) { return (TGS + CS - 1) / CS; }
+__host__ __device__ inline DecLayout dec_layout(int S, int maxb, int TGS, int CS) {
+  DecLayout L;
+  L.a = 0;
+  L.b = L.a + S * kATile;
+  L.red = L.b + S * kBTile;
+  L.gam = L.red + CS * dec_tpb(TGS, CS) * kRedStride * 4;
+  L.psq = L.gam + ((maxb * kChunk * 2 + 15) & ~15);
+  L.rs = L.psq + CS * TGS * 8;
+  L.bars = L.rs + TGS * 8;
+  L.slot = L.bars + (3 * kMaxStages + 2) * 8;
+  L.flag = L.slot + 16;
+  L.total = L.flag + 16;
+  return L;
+}
 
 // ---- tcgen05 helpers (inline PTX, sm_100a) ----
 __device__ __forceinline__ void tmem_alloc(uint32_t* smem_dst, uint32_t ncols) {
@@ -130,321 +178,467 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
 
 __device__ __forceinline__ float sigmoid_f32(float x) { return 1.0f / (1.0f + expf(-x)); }
 
-// double -> bf16 bits, one rounding to nearest-even: truncate to fp32 and set
-// the last bit if anything was cut (round to odd), then round to nearest-even
-// at bf16 precision; with >= 2 extra bits this equals direct rounding (Boldo &
-// Melquiond, "Emulation of FMA and correctly rounded sums: proved algorithms
-// using rounding to odd", IEEE Trans. Computers 2008).
-__device__ __forceinline__ uint16_t f64_to_bf16_bits(double y) {
-  float f = __double2float_rz(y);
-  if ((double)f != y) f = __uint_as_float(__float_as_uint(f) | 1u);
-  const __nv_bfloat16 h = __float2bfloat16_rn(f);
-  return *reinterpret_cast<const uint16_t*>(&h);
+// ---- thread-block cluster helpers ----
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_sync() {
+  cluster_arrive();
+  cluster_wait();
+}
+// shared::cta address -> the same offset in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+// stores into another CTA's shared memory (made visible by the next cluster barrier)
+__device__ __forceinline__ void st_cluster_f64(uint32_t addr, double v) {
+  asm volatile("st.shared::cluster.f64 [%0], %1;" ::"r"(addr), "d"(v) : "memory");
+}
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+// packed fp32 pairs (two IEEE round-to-nearest products per instruction)
+__device__ __forceinline__ unsigned long long pack2(float lo, float hi) {
+  return (unsigned long long)__float_as_uint(lo) | ((unsigned long long)__float_as_uint(hi) << 32);
+}
+__device__ __forceinline__ unsigned long long mul2(unsigned long long x, unsigned long long y) {
+  unsigned long long z;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(z) : "l"(x), "l"(y));
+  return z;
+}
+
+// bf16 of x*gamma*r with one rounding, for 8 bf16 of x (a 16-byte group) and
+// the matching gamma (as fp32); xg = x*gamma is exact in fp32 and r = rh + rl.
+// p = fl32(xg*rh) rounds to bf16 like the exact product unless p is exactly a
+// bf16 midpoint (low 16 bits 0x8000); normalize8 reports whether that happened
+// and normalize8_exact then moves such p one fp32 ulp towards the exact value,
+// by the sign of the remainder (xg*rh - p, exact by a fused multiply-add, plus
+// xg*rl), before the bf16 rounding.
+__device__ __forceinline__ bool normalize8(uint4 xv, const unsigned long long* g2, float rh, uint4* out) {
+  const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+  const unsigned long long r2 = pack2(rh, rh);
+  uint32_t ow[4];
+  uint32_t mid = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    // (x*gamma)*rh for the two bf16 of the word: x*gamma exact, one rounding to fp32
+    const unsigned long long p = mul2(mul2(pack2(__uint_as_float(xw[j] << 16), __uint_as_float(xw[j] & 0xffff0000u)), g2[j]), r2);
+    const uint32_t u0 = (uint32_t)p, u1 = (uint32_t)(p >> 32);
+    mid |= (uint32_t)(((u0 & 0xffffu) == 0x8000u) | ((u1 & 0xffffu) == 0x8000u));
+    const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(u0), __uint_as_float(u1));
+    ow[j] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  *out = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+  return mid != 0;
+}
+
+__device__ __noinline__ uint4 normalize8_exact(uint4 xv, const float* g, float rh, float rl) {
+  const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+  uint32_t ow[4];
+  for (int j = 0; j < 8; ++j) {
+    const float xg = __uint_as_float((j & 1) ? (xw[j >> 1] & 0xffff0000u) : (xw[j >> 1] << 16)) * g[j];
+    const float p = xg * rh;
+    uint32_t u = __float_as_uint(p);
+    if ((u & 0xffffu) == 0x8000u) {
+      const float c = fmaf(xg, rl, fmaf(xg, rh, -p));
+      if (c != 0.0f) u += ((__float_as_uint(c) ^ u) >> 31) ? 0xffffffffu : 1u;
+    }
+    const __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(u));
+    const uint32_t hb = *reinterpret_cast<const uint16_t*>(&h);
+    if (j & 1) ow[j >> 1] |= hb << 16;
+    else ow[j >> 1] = hb;
+  }
+  return make_uint4(ow[0], ow[1], ow[2], ow[3]);
+}
+
+__device__ __forceinline__ double sumsq8(uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  double acc = 0.0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xffff0000u);
+    acc += (double)(lo * lo);  // squares of bf16 values are exact in fp32
+    acc += (double)(hi * hi);
+  }
+  return acc;
+}
+
+// ids, affinities (and debug logits) of token t from its fp32 logits row
+__device__ void select_token(const DecodeArgs& a, int t, int lane) {
+  float lg[8];
+  uint32_t valid = 0;
+  if (lane * 8 < a.E) {
+    const float* src = a.logits + (size_t)t * a.E + lane * 8;
+    const float4 u = __ldcg(reinterpret_cast<const float4*>(src));
+    const float4 w = __ldcg(reinterpret_cast<const float4*>(src + 4));
+    lg[0] = u.x; lg[1] = u.y; lg[2] = u.z; lg[3] = u.w;
+    lg[4] = w.x; lg[5] = w.y; lg[6] = w.z; lg[7] = w.w;
+    valid = 0xffu;
+    if (a.bias) {
+      const uint4 bv = __ldg(reinterpret_cast<const uint4*>(a.bias + lane * 8));
+      const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        lg[2 * i] += __uint_as_float(bw[i] << 16);
+        lg[2 * i + 1] += __uint_as_float(bw[i] & 0xffff0000u);
+      }
+    }
+    if (a.dbg_logits) {
+      float* d = a.dbg_logits + (size_t)t * a.E + lane * 8;
+      *reinterpret_cast<float4*>(d) = make_float4(lg[0], lg[1], lg[2], lg[3]);
+      *reinterpret_cast<float4*>(d + 4) = make_float4(lg[4], lg[5], lg[6], lg[7]);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) lg[i] = 0.0f;
+  }
+  // top-k on the raw logits: k rounds of warp argmax, ties -> lower expert
+  uint32_t chosen = 0, avail = valid;
+  int my_id = 0;
+  for (int j = 0; j < a.k; ++j) {
+    unsigned long long best = 0ull;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if ((avail >> i) & 1u) {
+        const unsigned long long pk = pack_key(lg[i], lane * 8 + i);
+        best = pk > best ? pk : best;
+      }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const unsigned long long o = shfl_xor_u64(0xffffffffu, best, off);
+      best = o > best ? o : best;
+    }
+    const int win = packed_expert(best);
+    if (lane == (win >> 3)) {
+      avail &= ~(1u << (win & 7));
+      chosen |= 1u << (win & 7);
+    }
+    if (lane == j) my_id = win;
+  }
+  // activation over the selected only (ACT2): sigmoid each, or softmax over the k
+  float m = -INFINITY, ssum = 0.0f;
+  if (a.act == MOE_SOFTMAX) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if ((chosen >> i) & 1u) m = fmaxf(m, lg[i]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if ((chosen >> i) & 1u) ssum += expf(lg[i] - m);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, off);
+  }
+  if (lane < a.k) a.ids[(size_t)t * a.k + lane] = my_id;
+  if (lane * 8 < a.E) {
+    uint32_t ow[4];
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      float v0 = 0.0f, v1 = 0.0f;
+      if ((chosen >> i) & 1u) v0 = (a.act == MOE_SOFTMAX) ? expf(lg[i] - m) / ssum : sigmoid_f32(lg[i]);
+      if ((chosen >> (i + 1)) & 1u)
+        v1 = (a.act == MOE_SOFTMAX) ? expf(lg[i + 1] - m) / ssum : sigmoid_f32(lg[i + 1]);
+      const __nv_bfloat16 h0 = __float2bfloat16_rn(v0), h1 = __float2bfloat16_rn(v1);
+      ow[i / 2] = (uint32_t)(*reinterpret_cast<const uint16_t*>(&h0)) |
+                  ((uint32_t)(*reinterpret_cast<const uint16_t*>(&h1)) << 16);
+    }
+    *reinterpret_cast<uint4*>(a.aff + (size_t)t * a.E + lane * 8) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+  }
 }
 
 __global__ void __launch_bounds__(kDecThreads, 1)
-    decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap wmap) {
+    decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap xmap,
+                  const __grid_constant__ CUtensorMap wmap) {
   extern __shared__ uint8_t smem_raw[];
-  // 1024-byte aligned base for the swizzled operand tiles
   const uint32_t raw = smem_addr(smem_raw);
-  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  const int NB = a.NP / 64;                         // 64-column N boxes
-  uint8_t* sA = smem;                               // [2 K-blocks][128 rows][128 B]  = 32 KB
-  uint8_t* sB = smem + 32 * 1024;                   // [2 K-blocks][NB][64 rows][128 B] = NB * 16 KB
-  uint8_t* tail = sB + NB * 16 * 1024;
-  uint64_t* tma_bar = reinterpret_cast<uint64_t*>(tail);
-  uint64_t* mma_bar = tma_bar + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tail + 16);
-  int* flag = reinterpret_cast<int*>(tail + 32);    // [0] barrier scratch, [1] failure
-  double* r_s = reinterpret_cast<double*>(tail + 64); // [kM]
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);  // 1024-byte aligned (swizzle atoms)
+  const int TGS = a.TGS;
+  const DecLayout L = dec_layout(a.S, a.maxb, TGS, a.CS);
+  uint8_t* sA = smem + L.a;
+  uint8_t* sB = smem + L.b;
+  float* red = reinterpret_cast<float*>(smem + L.red);
+  uint16_t* gam = reinterpret_cast<uint16_t*>(smem + L.gam);
+  double* psq = reinterpret_cast<double*>(smem + L.psq);
+  float2* rs = reinterpret_cast<float2*>(smem + L.rs);
+  uint64_t* fullx = reinterpret_cast<uint64_t*>(smem + L.bars);  // x chunk landed
+  uint64_t* fullw = fullx + kMaxStages;                          // W chunk landed
+  uint64_t* empty = fullw + kMaxStages;                          // the stage's MMAs are done
+  uint64_t* mma_bar = empty + kMaxStages;
+  uint64_t* gam_bar = mma_bar + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.slot);
+  int* flag = reinterpret_cast<int*>(smem + L.flag);
 
-  const int c = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint32_t gen = barrier_generation(a.hdr);
-  const uint32_t ncols = a.N <= 32 ? 32u : (a.N <= 64 ? 64u : (a.N <= 128 ? 128u : 256u));
-  const int sl0 = (int)((long long)a.nslices * c / a.G), sl1 = (int)((long long)a.nslices * (c + 1) / a.G);
+  const uint32_t rank = cluster_rank();
+  const int cid = blockIdx.x / a.CS;
+  const int tg = cid / a.NG, ng = cid % a.NG;
+  const int row0 = tg * TGS;                       // first token of the group
+  const int e0 = ng * kExpGroup;                   // first expert of the group
+  const int N = min(kExpGroup, a.E - e0);          // multiple of 16
+  const int c0 = (int)((long long)a.nch * rank / a.CS);
+  const int nb = (int)((long long)a.nch * (rank + 1) / a.CS) - c0;  // chunks of this CTA (>= 1)
+  const int S = a.S;
+  const int nres = min(S, nb);
+  const uint32_t x_tx = (uint32_t)(TGS * 128);
 
+  int issued = 0;  // chunks whose copies have been issued (thread 0)
   if (tid == 0) {
-    mbar_init(tma_bar, 1);
+    for (int s = 0; s < kMaxStages; ++s) {
+      mbar_init(fullx + s, 1);
+      mbar_init(fullw + s, 1);
+      mbar_init(empty + s, 1);
+    }
     mbar_init(mma_bar, 1);
-    flag[1] = 0;
+    mbar_init(gam_bar, 1);
+    flag[0] = 0;
+    // x first (the sums of squares wait for it), then gamma, then W (needed by the MMAs only)
+    for (int i = 0; i < nres; ++i) {
+      mbar_arrive_expect_tx(fullx + i, x_tx);
+      tma_load_2d(sA + i * kATile, &xmap, (c0 + i) * kChunk, row0, fullx + i);
+    }
+    mbar_arrive_expect_tx(gam_bar, (uint32_t)(nb * kChunk * 2));
+    bulk_g2s(gam, a.gamma + (size_t)c0 * kChunk, (uint32_t)(nb * kChunk * 2), gam_bar);
+    for (int i = 0; i < nres; ++i) {
+      mbar_arrive_expect_tx(fullw + i, (uint32_t)kBTile);
+      tma_load_2d(sB + i * kBTile, &wmap, e0, (c0 + i) * kChunk, fullw + i);
+    }
+    issued = nres;
   }
-  if (warp == 0) tmem_alloc(tmem_slot, ncols);
-  // zero the A rows of padding tokens once (they stay zero for every slice)
-  for (int i = tid; i < (kM - a.T) * 2 * 8; i += kDecThreads) {
-    const int r = a.T + i / 16, kb = (i / 8) & 1, q = i & 7;
-    *reinterpret_cast<uint4*>(sA + kb * 16384 + r * 128 + q * 16) = make_uint4(0, 0, 0, 0);
-  }
+  if (warp == 0) tmem_alloc(tmem_slot, 64);
+  // with 64-token groups, A rows 64..127 are zero in every stage (the TMA box fills rows 0..63)
+  if (TGS < kM)
+    for (int i = tid; i < S * ((kM - TGS) * 8); i += kDecThreads) {
+      const int s = i / ((kM - TGS) * 8), off = i % ((kM - TGS) * 8);
+      *reinterpret_cast<uint4*>(sA + s * kATile + TGS * 128 + off * 16) = make_uint4(0, 0, 0, 0);
+    }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // ---------------- phase 1: partial sums of squares ----------------
-  // two threads per token, 64 columns each per slice; squares of bf16 values
-  // are exact, and are summed in double
+  // ---------------- sum of squares over the slice ----------------
+  // TPT = 512/TGS threads per token row; part p reads 16-byte groups p, p+TPT, ..
+  // of each chunk row (conflict-free under the swizzle)
   {
-    const int t = tid >> 1, half = tid & 1;
+    const int TPT = kDecThreads / TGS;  // 8 or 4
+    const int r = tid / TPT, part = tid % TPT;
     double acc = 0.0;
-    if (t < a.T) {
-      for (int sl = sl0; sl < sl1; ++sl) {
-        const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)t * a.H + sl * kKC + half * 64);
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          const uint4 q = __ldg(src + v);
-          const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xffff0000u);
-            acc += (double)(lo * lo);
-            acc += (double)(hi * hi);
-          }
-        }
-      }
-    }
-    double d = acc;
-    d += __shfl_xor_sync(0xffffffffu, d, 1);
-    if (half == 0 && t < kM) a.sumsq[(size_t)c * kM + t] = d;
-  }
-  bool ok = grid_barrier(a.hdr, (uint32_t)a.G, gen, a.timeout_ns, flag);
-
-  // ---------------- phase 2: normalise, project ----------------
-  if (ok) {
-    // warp w reduces tokens w, w+8, ...: lane l adds the partials of blocks
-    // l, l+32, ... (all loads in flight), then a fixed shuffle tree; every
-    // block computes the same r_t
-    for (int t = warp; t < a.T; t += kDecWarps) {
-      double sv[5];
-#pragma unroll
-      for (int i = 0; i < 5; ++i) {
-        const int cp = lane + 32 * i;
-        sv[i] = cp < a.G ? __ldcg(&a.sumsq[(size_t)cp * kM + t]) : 0.0;
-      }
-      double s = (sv[0] + sv[1]) + (sv[2] + sv[3]) + sv[4];
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-      if (lane == 0) r_s[t] = 1.0 / sqrt(s / (double)a.H + (double)a.eps);
-    }
-    __syncthreads();
-    const uint32_t idesc = idesc_bf16_f32(a.N);
-    uint32_t phase = 0;
-    for (int sl = sl0; sl < sl1 && ok; ++sl) {
-      if (tid == 0) {
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_arrive_expect_tx(tma_bar, (uint32_t)(NB * 16 * 1024));
-        for (int kb = 0; kb < 2; ++kb)
-          for (int nb = 0; nb < NB; ++nb)
-            tma_load_2d(sB + (kb * NB + nb) * 8192, &wmap, nb * 64, sl * kKC + kb * 64, tma_bar);
-      }
-      // normalised slice: (token, 16-byte group) pairs, 16 groups per token row;
-      // a thread's loads are all issued before any is used
-      constexpr int kPer = (kM * 16) / kDecThreads;  // pairs per thread (8)
-      uint4 xb[kPer];
-      const uint4 gv = __ldg(reinterpret_cast<const uint4*>(a.gamma + sl * kKC + (tid & 15) * 8));
-#pragma unroll
-      for (int b = 0; b < kPer; ++b) {
-        const int i = tid + b * kDecThreads;
-        const int t = i >> 4, q = i & 15;
-        xb[b] = t < a.T ? __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)t * a.H + sl * kKC + q * 8))
-                        : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int b = 0; b < kPer; ++b) {
-        const int i = tid + b * kDecThreads;
-        const int t = i >> 4, q = i & 15;
-        if (t >= a.T) continue;
-        const size_t off = (size_t)t * a.H + sl * kKC + q * 8;
-        const uint4 xv = xb[b];
-        const double r = r_s[t];
-        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
-        uint32_t ow[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float x0 = __uint_as_float(xw[j] << 16), x1 = __uint_as_float(xw[j] & 0xffff0000u);
-          const float g0 = __uint_as_float(gw[j] << 16), g1 = __uint_as_float(gw[j] & 0xffff0000u);
-          // x*gamma is exact in fp32; the product with r is formed in double and
-          // rounded once to bf16
-          ow[j] = (uint32_t)f64_to_bf16_bits((double)(x0 * g0) * r) |
-                  ((uint32_t)f64_to_bf16_bits((double)(x1 * g1) * r) << 16);
-        }
-        const uint4 o = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-        *reinterpret_cast<uint4*>(a.out_norm + off) = o;
-        const int kb = q >> 3, cq = q & 7;
-        *reinterpret_cast<uint4*>(sA + kb * 16384 + t * 128 + ((cq ^ (t & 7)) << 4)) = o;
-      }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      __syncthreads();
-      if (tid == 0) {
-        if (!mbar_wait_bounded(tma_bar, phase, a.timeout_ns)) {
-          record_timeout(a.hdr);
-          flag[1] = 1;
-        } else {
-          tc_fence_after();
-          const uint32_t aBase = smem_addr(sA), bBase = smem_addr(sB);
-#pragma unroll
-          for (int ks = 0; ks < kKC / 16; ++ks) {
-            const int kb = ks >> 2, kk = ks & 3;
-            const uint64_t ad = smem_desc_sw128(aBase + kb * 16384 + kk * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(bBase + kb * NB * 8192 + kk * 2048, 8192, 1024);
-            umma_bf16(tmem, ad, bd, idesc, (sl > sl0 || ks > 0) ? 1u : 0u);
-          }
-          umma_commit(mma_bar);
-        }
-      }
-      __syncthreads();
-      if (flag[1]) {
-        ok = false;
+    bool waited = true;
+    for (int i = 0; i < nres; ++i) {
+      if (!mbar_wait_bounded(fullx + i, 0, a.timeout_ns)) {
+        waited = false;
         break;
       }
-      // the MMAs must finish before the operand tiles are rewritten (next slice) or read out
-      if (!mbar_wait_bounded(mma_bar, phase, a.timeout_ns)) {
-        record_timeout(a.hdr);
-        flag[1] = 1;
-      }
-      phase ^= 1u;
-      __syncthreads();
-      if (flag[1]) ok = false;
+      const uint8_t* rowp = sA + i * kATile + r * 128;
+      for (int qq = part; qq < 8; qq += TPT) acc += sumsq8(*reinterpret_cast<const uint4*>(rowp + ((qq ^ (r & 7)) << 4)));
     }
-    if (ok) {
-      tc_fence_after();
-      // TMEM -> registers -> workspace: warp w reads lanes 32*(w%4).., columns half (w/4)
-      const int lb = (warp & 3) * 32;
-      const int t = lb + lane;
-      const int chalf = a.N > 128 ? 128 : a.N;  // columns per warp half
-      for (int c0 = (warp >> 2) * chalf; c0 < min(a.N, ((warp >> 2) + 1) * chalf); c0 += 32) {
-        float v[32];
-        tmem_ld32(tmem + ((uint32_t)lb << 16) + (uint32_t)c0, v);
-        if (t < a.T) {
-          float* dst = a.plogits + ((size_t)c * kM + t) * a.NP + c0;
+    if (!waited) {
+      record_timeout(a.hdr);
+      flag[0] = 1;
+    }
+    // chunks beyond the ring (long slices): straight from global memory
+    if (nb > nres && row0 + r < a.T) {
+      const uint16_t* xr = a.x + (size_t)(row0 + r) * a.H;
+      for (int i = nres; i < nb; ++i)
+        for (int qq = part; qq < 8; qq += TPT)
+          acc += sumsq8(__ldg(reinterpret_cast<const uint4*>(xr + (c0 + i) * kChunk + qq * 8)));
+    }
+    for (int off = 1; off < TPT; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    // every CTA of the cluster receives this partial in slot [rank][r]
+    const uint32_t dst = smem_addr(psq + (int)rank * TGS + r);
+    for (int j = part; j < a.CS; j += TPT) st_cluster_f64(cluster_map(dst, (uint32_t)j), acc);
+  }
+  cluster_sync();
+  if (tid < TGS) {
+    // the CS partial sums in rank order: identical bits in every CTA
+    double v[16];
 #pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            if (c0 + i < a.NP) *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+    for (int j = 0; j < 16; ++j) v[j] = j < a.CS ? psq[j * TGS + tid] : 0.0;
+    double s = 0.0;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) s += v[j];
+    const double r = 1.0 / sqrt(s / (double)a.H + (double)a.eps);
+    const float rh = (float)r;
+    rs[tid] = make_float2(rh, (float)(r - (double)rh));
+  }
+  if (!mbar_wait_bounded(gam_bar, 0, a.timeout_ns)) {
+    record_timeout(a.hdr);
+    flag[0] = 1;
+  }
+  __syncthreads();
+  bool ok = flag[0] == 0;
+
+  // ---------------- normalise in place, project (rounds of up to S chunks) ----------------
+  const uint32_t idesc = idesc_bf16_f32(N);
+  bool mma_issued = false;
+  const int q = tid & 7;  // the thread's 16-byte group in every chunk row
+  for (int i0 = 0; i0 < nb && ok; i0 += S) {
+    const int i1 = min(nb, i0 + S);
+    for (int i = i0; i < i1; ++i) {
+      const int s = i % S;
+      if (i >= nres && !mbar_wait_bounded(fullx + s, (uint32_t)(i / S) & 1u, a.timeout_ns)) {
+        record_timeout(a.hdr);
+        flag[0] = 1;
+      }
+      const int chunk = c0 + i;
+      const bool writer = (chunk % a.NG) == ng;  // one expert-group cluster stores each out_norm chunk
+      unsigned long long g2[4];
+      float g[8];
+      {
+        const uint4 gv = *reinterpret_cast<const uint4*>(gam + i * kChunk + q * 8);
+        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          g[2 * j] = __uint_as_float(gw[j] << 16);
+          g[2 * j + 1] = __uint_as_float(gw[j] & 0xffff0000u);
+          g2[j] = pack2(g[2 * j], g[2 * j + 1]);
         }
       }
+      // rows tid/8 and tid/8 + 64 of the chunk (the second only for 128-token groups)
+      const int r0 = tid >> 3, r1 = r0 + 64;
+      uint8_t* p0 = sA + s * kATile + r0 * 128 + ((q ^ (r0 & 7)) << 4);
+      uint8_t* p1 = sA + s * kATile + r1 * 128 + ((q ^ (r1 & 7)) << 4);
+      const bool two = r1 < TGS;
+      const uint4 x0 = *reinterpret_cast<const uint4*>(p0);
+      const uint4 x1 = two ? *reinterpret_cast<const uint4*>(p1) : make_uint4(0, 0, 0, 0);
+      const float2 rr0 = rs[r0], rr1 = rs[two ? r1 : r0];
+      uint4 o0, o1;
+      const bool m0 = normalize8(x0, g2, rr0.x, &o0);
+      const bool m1 = normalize8(x1, g2, rr1.x, &o1);
+      if (m0 | m1) {  // a bf16 rounding midpoint: settle it with the remainder (rare)
+        if (m0) o0 = normalize8_exact(x0, g, rr0.x, rr0.y);
+        if (m1) o1 = normalize8_exact(x1, g, rr1.x, rr1.y);
+      }
+      *reinterpret_cast<uint4*>(p0) = o0;
+      if (two) *reinterpret_cast<uint4*>(p1) = o1;
+      if (writer) {
+        const size_t col = (size_t)chunk * kChunk + q * 8;
+        if (row0 + r0 < a.T) *reinterpret_cast<uint4*>(a.out_norm + (size_t)(row0 + r0) * a.H + col) = o0;
+        if (two && row0 + r1 < a.T) *reinterpret_cast<uint4*>(a.out_norm + (size_t)(row0 + r1) * a.H + col) = o1;
+      }
     }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+    if (tid == 0 && flag[0] == 0) {
+      tc_fence_after();
+      for (int i = i0; i < i1; ++i) {
+        const int s = i % S;
+        if (!mbar_wait_bounded(fullw + s, (uint32_t)(i / S) & 1u, a.timeout_ns)) {
+          record_timeout(a.hdr);
+          flag[0] = 1;
+          break;
+        }
+        const uint32_t aBase = smem_addr(sA + s * kATile), bBase = smem_addr(sB + s * kBTile);
+#pragma unroll
+        for (int kk = 0; kk < kChunk / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(aBase + kk * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(bBase + kk * 2048, 8192, 1024);
+          umma_bf16(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(empty + s);
+        mma_issued = true;
+      }
+      // refill the round's stages with the next round's chunks once their MMAs have read them
+      for (int i = i0; i < i1 && issued < nb && flag[0] == 0; ++i) {
+        const int s = i % S;
+        if (!mbar_wait_bounded(empty + s, (uint32_t)(i / S) & 1u, a.timeout_ns)) {
+          record_timeout(a.hdr);
+          flag[0] = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(fullx + s, x_tx);
+        tma_load_2d(sA + s * kATile, &xmap, (c0 + issued) * kChunk, row0, fullx + s);
+        mbar_arrive_expect_tx(fullw + s, (uint32_t)kBTile);
+        tma_load_2d(sB + s * kBTile, &wmap, e0, (c0 + issued) * kChunk, fullw + s);
+        ++issued;
+      }
+    }
+    __syncthreads();
+    ok = flag[0] == 0;
+  }
+  if (tid == 0 && mma_issued) umma_commit(mma_bar);
+  // every thread waits for the MMAs (also on the error path: TMEM is freed below)
+  if (__syncthreads_or(tid == 0 && mma_issued)) {
+    if (!mbar_wait_bounded(mma_bar, 0, a.timeout_ns)) {
+      record_timeout(a.hdr);
+      flag[0] = 1;
+    }
+  }
+  __syncthreads();
+  ok = flag[0] == 0;
+  const int tpb = dec_tpb(TGS, a.CS);  // token rows reduced by each CTA
+  if (ok) {
+    tc_fence_after();
+    // TMEM lane = token row; warp w < 8 reads lanes 32*(w%4).. and column half w/4,
+    // and pushes the 32 partial logits to the CTA that reduces that row (slot [rank])
+    const int wq = warp & 3, ch = warp >> 2;
+    if (ch < 2 && wq * 32 < TGS && ch * 32 < N) {
+      float v[32];
+      tmem_ld32(tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)(ch * 32), v);
+      const int row = wq * 32 + lane;
+      if (row < TGS) {
+        const int owner = row / tpb;
+        const uint32_t dst =
+            cluster_map(smem_addr(red + (((int)rank * tpb) + (row - owner * tpb)) * kRedStride + ch * 32), (uint32_t)owner);
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) st_cluster_v4(dst + i * 4, v[i], v[i + 1], v[i + 2], v[i + 3]);
+      }
+    }
+  }
+  if (tid == 0 && !ok) {
+    // a wait gave up: let copies still in flight land before the CTA exits
+    for (int i = max(0, issued - S); i < issued; ++i) {
+      mbar_wait_bounded(fullx + (i % S), (uint32_t)(i / S) & 1u, a.timeout_ns);
+      mbar_wait_bounded(fullw + (i % S), (uint32_t)(i / S) & 1u, a.timeout_ns);
+    }
+    mbar_wait_bounded(gam_bar, 0, a.timeout_ns);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, ncols);
-  if (!ok) {
-    // let the other blocks pass the second barrier quickly; outputs are undefined
-    grid_barrier(a.hdr, (uint32_t)a.G, gen + 1, a.timeout_ns, flag);
-    return;
-  }
-  if (!grid_barrier(a.hdr, (uint32_t)a.G, gen + 1, a.timeout_ns, flag)) return;
+  if (warp == 0) tmem_dealloc(tmem, 64);
 
-  // ---------------- phase 3: reduce partial logits, top-k, affinities ----------------
-  // For each token of this block, warp w adds the partial logits of blocks
-  // w, w+8, ... (lane = 8 experts; all loads of a warp in flight), the 8 warp
-  // sums meet in shared memory and warp 0 adds them in warp order.
-  float* red = reinterpret_cast<float*>(sA);  // [kDecWarps][NP], the operand tiles are free now
-  const int t0 = (int)((long long)a.T * c / a.G), t1 = (int)((long long)a.T * (c + 1) / a.G);
-  for (int t = t0; t < t1; ++t) {
-    {
-      float acc[8];
+  // ---------------- cluster reduction of the partial logits ----------------
+  cluster_sync();  // all pushes have landed; no shared memory is touched across CTAs after this
+  const int rA = min(TGS, (int)rank * tpb), rB = min(TGS, rA + tpb);
+  if (ok) {
+    for (int idx = tid; idx < (rB - rA) * kExpGroup; idx += kDecThreads) {
+      const int rr = idx / kExpGroup, e = idx % kExpGroup;
+      if (e >= N || row0 + rA + rr >= a.T) continue;
+      float v[16];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-      if (lane * 8 < a.NP) {
-        constexpr int kB = 8;
-        for (int cp0 = warp; cp0 < a.G; cp0 += kDecWarps * kB) {
-          float4 u[kB], w[kB];
+      for (int j = 0; j < 16; ++j) v[j] = j < a.CS ? red[(j * tpb + rr) * kRedStride + e] : 0.0f;
+      float sum = 0.0f;  // rank order
 #pragma unroll
-          for (int b = 0; b < kB; ++b) {
-            const int cp = cp0 + b * kDecWarps;
-            if (cp < a.G) {
-              const float* src = a.plogits + ((size_t)cp * kM + t) * a.NP + lane * 8;
-              u[b] = __ldcg(reinterpret_cast<const float4*>(src));
-              w[b] = __ldcg(reinterpret_cast<const float4*>(src + 4));
-            } else {
-              u[b] = w[b] = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-          }
-#pragma unroll
-          for (int b = 0; b < kB; ++b) {
-            acc[0] += u[b].x; acc[1] += u[b].y; acc[2] += u[b].z; acc[3] += u[b].w;
-            acc[4] += w[b].x; acc[5] += w[b].y; acc[6] += w[b].z; acc[7] += w[b].w;
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) red[warp * a.NP + lane * 8 + i] = acc[i];
-      }
+      for (int j = 0; j < 16; ++j) sum += v[j];
+      a.logits[(size_t)(row0 + rA + rr) * a.E + e0 + e] = sum;
     }
-    __syncthreads();
-    if (warp != 0) {
-      __syncthreads();
-      continue;
-    }
-    float lg[8];
-    float bsum[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      lg[i] = 0.0f;
-      const int e = lane * 8 + i;
-      bsum[i] = (a.bias && e < a.E) ? bf16_bits_to_f32(a.bias[e]) : 0.0f;
-    }
-    if (lane * 8 < a.NP) {
-      for (int w = 0; w < kDecWarps; ++w)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) lg[i] += red[w * a.NP + lane * 8 + i];
-    }
-    uint32_t valid = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = lane * 8 + i;
-      lg[i] += bsum[i];
-      if (e < a.E) valid |= 1u << i;
-      if (a.dbg_logits && e < a.E) a.dbg_logits[(size_t)t * a.E + e] = lg[i];
-    }
-    // top-k on the raw logits: k rounds of warp argmax, ties -> lower expert
-    uint32_t chosen = 0, avail = valid;
-    int my_id = 0;
-    for (int j = 0; j < a.k; ++j) {
-      unsigned long long best = 0ull;
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if ((avail >> i) & 1u) {
-          const unsigned long long pk = pack_key(lg[i], lane * 8 + i);
-          best = pk > best ? pk : best;
-        }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const unsigned long long o = shfl_xor_u64(0xffffffffu, best, off);
-        best = o > best ? o : best;
-      }
-      const int win = packed_expert(best);
-      const int owner = win >> 3;
-      if (lane == owner) {
-        avail &= ~(1u << (win & 7));
-        chosen |= 1u << (win & 7);
-      }
-      if (lane == j) my_id = win;
-    }
-    // activation over the selected only (ACT2): sigmoid each, or softmax over the k
-    float m = -INFINITY, ssum = 0.0f;
-    if (a.act == MOE_SOFTMAX) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if ((chosen >> i) & 1u) m = fmaxf(m, lg[i]);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if ((chosen >> i) & 1u) ssum += expf(lg[i] - m);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, off);
-    }
-    if (lane < a.k) a.ids[(size_t)t * a.k + lane] = my_id;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = lane * 8 + i;
-      if (e < a.E) {
-        float v = 0.0f;
-        if ((chosen >> i) & 1u) v = (a.act == MOE_SOFTMAX) ? expf(lg[i] - m) / ssum : sigmoid_f32(lg[i]);
-        const __nv_bfloat16 hb = __float2bfloat16_rn(v);
-        a.aff[(size_t)t * a.E + e] = *reinterpret_cast<const uint16_t*>(&hb);
-      }
-    }
-    __syncthreads();
+  }
+  __threadfence();
+
+  // ---------------- top-k by the last expert-group cluster of each token run ----------------
+  __syncthreads();
+  if (tid == 0) {
+    const uint32_t tk = atomicAdd(&a.tickets[tg * 16 + rank], 1u);
+    const int last = tk == (uint32_t)(a.NG - 1);
+    if (last) a.tickets[tg * 16 + rank] = 0u;  // every cluster of the run has arrived: reset for the next call
+    flag[1] = last;
+  }
+  __syncthreads();
+  if (flag[1]) {
+    __threadfence();
+    if (flag[0] == 0 && a.hdr->status == MOE_OK)
+      for (int r = rA + warp; r < rB; r += kDecWarps)
+        if (row0 + r < a.T) select_token(a, row0 + r, lane);
   }
 }
 
@@ -466,28 +660,94 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-int dec_sms() {
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return sms;
+constexpr int kDecSmemMax = kSmemLimit;
+
+// Per device: kernel attributes set once, and for each cluster size 8..16 how
+// many clusters can be resident at once (one CTA per SM at these sizes).
+struct DecDevice {
+  std::once_flag once;
+  int ok = 0;
+  int active[17] = {0};
+};
+DecDevice g_dec_dev[64];
+
+int max_active_clusters(int cs) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cs * 16);
+  cfg.blockDim = dim3(kDecThreads);
+  cfg.dynamicSmemBytes = 200 * 1024;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, decode_kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
 }
 
-int dec_grid(int H) {
-  const int ns = H / kKC;
-  return std::max(1, std::min(ns, dec_sms()));
+int dec_device_setup(int dev) {
+  DecDevice& d = g_dec_dev[dev];
+  std::call_once(d.once, [&d] {
+    if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmemMax) != cudaSuccess)
+      return;
+    d.ok = 1;
+    const bool nonportable =
+        cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+    if (!nonportable) cudaGetLastError();
+    for (int cs = 1; cs <= 16; ++cs) d.active[cs] = (cs <= 8 || nonportable) ? max_active_clusters(cs) : 0;
+  });
+  return d.ok;
 }
 
-size_t dec_ws_bytes(int H, int E) {
-  const int G = dec_grid(H);
-  const int NP = (E + 63) / 64 * 64;
-  return sizeof(WsHeader) + (size_t)G * kM * sizeof(double) + (size_t)G * kM * NP * sizeof(float);
+struct DecPlan {
+  int CS, NG, TG, TGS, nch, maxb, S, smem;
+};
+
+// Choose the cluster size CS (CTAs sharing the hidden dimension) and the token
+// group size: least staged bytes per CTA, counting a second wave of clusters
+// as a second pass and a slice longer than the ring as one more pass.
+DecPlan dec_plan(int T, int H, int E, const int* active) {
+  DecPlan best = {};
+  double best_cost = 1e300;
+  const int nch = H / kChunk;
+  const int NG = (E + kExpGroup - 1) / kExpGroup;
+  for (int cs = 1; cs <= std::min(16, nch); ++cs) {
+    if (active[cs] < 1) continue;
+    for (int tgs = 64; tgs <= 128; tgs += 64) {
+      if (tgs == 128 && T <= 64) continue;
+      DecPlan p;
+      p.CS = cs;
+      p.NG = NG;
+      p.TGS = tgs;
+      p.TG = (T + tgs - 1) / tgs;
+      p.nch = nch;
+      p.maxb = (nch + cs - 1) / cs;
+      if (p.maxb > kMaxSliceChunks) continue;
+      p.S = std::min(kMaxStages, p.maxb);
+      while (p.S > 1 && 1024 + dec_layout(p.S, p.maxb, tgs, cs).total > kSmemLimit) --p.S;
+      p.smem = 1024 + dec_layout(p.S, p.maxb, tgs, cs).total;
+      if (p.smem > kSmemLimit) continue;
+      const int clusters = p.TG * p.NG;
+      const int waves = (clusters + active[cs] - 1) / active[cs];
+      const double per_cta = (double)p.maxb * (tgs * 128 + kBTile);
+      const double cost = per_cta * (waves + (p.maxb > p.S ? 1 : 0)) + 1e-3 * cs * clusters;
+      if (cost < best_cost) {
+        best_cost = cost;
+        best = p;
+      }
+    }
+  }
+  return best;
 }
 
-int dec_smem(int E) {
-  const int NB = (E + 63) / 64;
-  const int need = 1024 + 32 * 1024 + NB * 16 * 1024 + 64 + kM * 8;
-  return std::max(need, kSmemMin);
+size_t dec_ws_bytes(int T, int E) {
+  return sizeof(WsHeader) + (size_t)std::max(T, 1) * E * sizeof(float) + 2 * 16 * sizeof(uint32_t);
 }
 
 }  // namespace
@@ -497,8 +757,8 @@ using namespace moe;
 
 extern "C" int moe_rmsnorm_router_topk_workspace_bytes(int32_t T, int32_t H, int32_t E, size_t* bytes) {
   if (T < 0 || T > 128 || H <= 0 || H % 128 != 0 || E <= 0 || !bytes) return MOE_ERR_INVALID_ARG;
-  if (E % 16 != 0 || E > kMaxE) return MOE_ERR_UNSUPPORTED;
-  *bytes = dec_ws_bytes(H, E);
+  if (E % 16 != 0 || E > kMaxE || H > kMaxSliceChunks * kChunk * 8) return MOE_ERR_UNSUPPORTED;
+  *bytes = dec_ws_bytes(T, E);
   return MOE_OK;
 }
 
@@ -508,15 +768,21 @@ extern "C" int moe_rmsnorm_router_topk(int32_t T, int32_t H, int32_t E, int32_t 
                                        size_t ws_bytes, void* stream) {
   if (T < 0 || T > 128 || H <= 0 || H % 128 != 0 || E <= 0 || k <= 0 || k > E) return MOE_ERR_INVALID_ARG;
   if (act != MOE_SIGMOID && act != MOE_SOFTMAX) return MOE_ERR_INVALID_ARG;
-  if (E % 16 != 0 || E > kMaxE || k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+  if (E % 16 != 0 || E > kMaxE || k > MOE_MAX_TOPK || H > kMaxSliceChunks * kChunk * 8) return MOE_ERR_UNSUPPORTED;
   if (T == 0) return MOE_OK;
   if (!hidden || !gamma || !W || !out_norm || !ids || !affinities) return MOE_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(hidden) | reinterpret_cast<uintptr_t>(gamma) | reinterpret_cast<uintptr_t>(W) |
-       reinterpret_cast<uintptr_t>(out_norm)) & 15)
+       reinterpret_cast<uintptr_t>(out_norm) | reinterpret_cast<uintptr_t>(affinities) |
+       reinterpret_cast<uintptr_t>(bias) | reinterpret_cast<uintptr_t>(debug_logits)) & 15)
     return MOE_ERR_INVALID_ARG;
-  if (!ws || ws_bytes < dec_ws_bytes(H, E) || (reinterpret_cast<uintptr_t>(ws) & 15)) return MOE_ERR_WORKSPACE;
+  if (!ws || ws_bytes < dec_ws_bytes(T, E) || (reinterpret_cast<uintptr_t>(ws) & 15)) return MOE_ERR_WORKSPACE;
   EncodeTiledFn enc = encode_fn();
   if (!enc) return MOE_ERR_CUDA;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+  if (!dec_device_setup(dev)) return MOE_ERR_CUDA;
+  const DecPlan plan = dec_plan(T, H, E, g_dec_dev[dev].active);
+  if (plan.CS < 1) return MOE_ERR_UNSUPPORTED;
 
   DecodeArgs a = {};
   a.x = reinterpret_cast<const uint16_t*>(hidden);
@@ -527,50 +793,57 @@ extern "C" int moe_rmsnorm_router_topk(int32_t T, int32_t H, int32_t E, int32_t 
   a.aff = reinterpret_cast<uint16_t*>(affinities);
   a.dbg_logits = debug_logits;
   a.hdr = reinterpret_cast<WsHeader*>(ws);
-  a.G = dec_grid(H);
-  a.sumsq = reinterpret_cast<double*>(reinterpret_cast<uint8_t*>(ws) + sizeof(WsHeader));
-  a.plogits = reinterpret_cast<float*>(a.sumsq + (size_t)a.G * kM);
+  a.logits = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + sizeof(WsHeader));
+  a.tickets = reinterpret_cast<uint32_t*>(a.logits + (size_t)T * E);
   a.T = T;
   a.H = H;
   a.E = E;
   a.k = k;
   a.act = act;
-  a.NP = (E + 63) / 64 * 64;
-  a.N = (E + 15) / 16 * 16;
-  a.nslices = H / kKC;
+  a.CS = plan.CS;
+  a.TGS = plan.TGS;
+  a.NG = plan.NG;
+  a.nch = plan.nch;
+  a.S = plan.S;
+  a.maxb = plan.maxb;
   a.eps = eps;
   a.timeout_ns = kDefaultTimeoutNs;
 
-  // W [H][E] bf16: dim0 = E (contiguous), dim1 = H; 64 x 64 boxes, 128-byte swizzle
-  CUtensorMap wmap;
-  const cuuint64_t gdim[2] = {(cuuint64_t)E, (cuuint64_t)H};
-  const cuuint64_t gstride[1] = {(cuuint64_t)E * 2};
+  // x [T][H]: dim0 = H (contiguous), dim1 = T; 64 x TGS boxes (rows past T read as zero)
+  // W [H][E]: dim0 = E (contiguous), dim1 = H; 64 x 64 boxes (experts past E read as zero)
+  CUtensorMap xmap, wmap;
   const cuuint32_t box[2] = {64, 64};
   const cuuint32_t estr[2] = {1, 1};
-  if (enc(&wmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(W), gdim, gstride, box, estr,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return MOE_ERR_INVALID_ARG;
-
-  const int smem = dec_smem(E);
-  static bool configured[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
-    if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    configured[dev] = true;
+  {
+    const cuuint64_t gdim[2] = {(cuuint64_t)H, (cuuint64_t)T};
+    const cuuint64_t gstride[1] = {(cuuint64_t)H * 2};
+    const cuuint32_t xbox[2] = {64, (cuuint32_t)plan.TGS};
+    if (enc(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(hidden), gdim, gstride, xbox, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return MOE_ERR_INVALID_ARG;
   }
+  {
+    const cuuint64_t gdim[2] = {(cuuint64_t)E, (cuuint64_t)H};
+    const cuuint64_t gstride[1] = {(cuuint64_t)E * 2};
+    if (enc(&wmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(W), gdim, gstride, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return MOE_ERR_INVALID_ARG;
+  }
+
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.G);
+  cfg.gridDim = dim3(plan.CS * plan.NG * plan.TG);
   cfg.blockDim = dim3(kDecThreads);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = plan.smem;
   cfg.stream = reinterpret_cast<cudaStream_t>(stream);
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = plan.CS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel, a, wmap);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel, a, xmap, wmap);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
