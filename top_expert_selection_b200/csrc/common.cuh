@@ -58,34 +58,51 @@ __device__ __forceinline__ uint32_t barrier_generation(WsHeader* h) {
 }
 
 // Grid-wide barrier for a co-resident (cooperatively launched) grid of
-// `nblocks` blocks.  One 64-bit word holds generation | arrivals: a block adds
-// 1; the last arrival adds 2^32 - nblocks, which bumps the generation and
-// clears the count in the same atomic.  Waiters poll the generation.
-// Returns false (and records a timeout) if the wait exceeded timeout_ns.
-// Must be called by all threads of the block.
+// `nblocks` blocks, split into an arrival and a wait so a block can do local
+// work in between.  One 64-bit word holds generation | arrivals: a block adds
+// 1; the last arrival then adds 2^32 - nblocks (no return value needed), which
+// bumps the generation and clears the count.  Waiters are released as soon as
+// the count reads nblocks (before that reset lands) or the generation has
+// moved on, so the barrier costs one atomic round trip.  One barrier per
+// launch: a second one could see the first one's count before its reset.
+//
+// grid_arrive: thread 0 only, after the block's writes to publish.
+__device__ __forceinline__ void grid_arrive(WsHeader* h, uint32_t nblocks) {
+  __threadfence();
+  const unsigned long long old = atomicAdd(&h->barrier, 1ull);
+  if ((uint32_t)old == nblocks - 1) {
+    asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" ::"l"(&h->barrier),
+                 "l"((1ull << 32) - (unsigned long long)nblocks)
+                 : "memory");
+  }
+}
+
+// grid_wait: thread 0 only; false (and a recorded timeout) if the wait
+// exceeded timeout_ns.
+__device__ __forceinline__ bool grid_wait(WsHeader* h, uint32_t nblocks, uint32_t gen_at_entry,
+                                          long long timeout_ns) {
+  unsigned long long t0 = 0;
+  int spins = 0;
+  while (true) {
+    const unsigned long long v = ld_acquire_u64(&h->barrier);
+    if ((uint32_t)(v >> 32) != gen_at_entry || (uint32_t)v == nblocks) break;
+    if (++spins == 64) t0 = globaltimer_ns();
+    if (spins > 64 && (long long)(globaltimer_ns() - t0) > timeout_ns) {
+      record_timeout(h);
+      return false;
+    }
+  }
+  __threadfence();
+  return true;
+}
+
+// Both halves; must be called by all threads of the block.
 __device__ __forceinline__ bool grid_barrier(WsHeader* h, uint32_t nblocks, uint32_t gen_at_entry,
                                              long long timeout_ns, int* smem_flag) {
   __syncthreads();
   if (threadIdx.x == 0) {
-    int ok = 1;
-    __threadfence();
-    const unsigned long long old = atomicAdd(&h->barrier, 1ull);
-    if ((uint32_t)old == nblocks - 1) {
-      atomicAdd(&h->barrier, (1ull << 32) - (unsigned long long)nblocks);
-    } else {
-      unsigned long long t0 = 0;
-      int spins = 0;
-      while ((uint32_t)(ld_acquire_u64(&h->barrier) >> 32) == gen_at_entry) {
-        if (++spins == 64) t0 = globaltimer_ns();
-        if (spins > 64 && (long long)(globaltimer_ns() - t0) > timeout_ns) {
-          record_timeout(h);
-          ok = 0;
-          break;
-        }
-      }
-    }
-    __threadfence();
-    *smem_flag = ok;
+    grid_arrive(h, nblocks);
+    *smem_flag = grid_wait(h, nblocks, gen_at_entry, timeout_ns) ? 1 : 0;
   }
   __syncthreads();
   return *smem_flag != 0;

@@ -219,11 +219,14 @@ __device__ __forceinline__ unsigned long long mul2(unsigned long long x, unsigne
 
 // bf16 of x*gamma*r with one rounding, for 8 bf16 of x (a 16-byte group) and
 // the matching gamma (as fp32); xg = x*gamma is exact in fp32 and r = rh + rl.
-// p = fl32(xg*rh) rounds to bf16 like the exact product unless p is exactly a
-// bf16 midpoint (low 16 bits 0x8000); normalize8 reports whether that happened
-// and normalize8_exact then moves such p one fp32 ulp towards the exact value,
-// by the sign of the remainder (xg*rh - p, exact by a fused multiply-add, plus
-// xg*rl), before the bf16 rounding.
+// p = fl32(xg*rh) is within one fp32 ulp of xg*r (half an ulp from rounding,
+// at most half from dropping xg*rl), so it rounds to bf16 like the exact
+// product unless p is a bf16 midpoint m or one ulp from it (low 16 bits
+// 0x7fff, 0x8000 or 0x8001).  normalize8 reports whether that happened;
+// normalize8_exact then takes the side of m from the sign of
+// (p - m) + (xg*rh - p) + xg*rl (the middle term exact by a fused
+// multiply-add) and nudges m one fp32 ulp that way before the bf16 rounding
+// (an exact tie stays on m: round half to even).
 __device__ __forceinline__ bool normalize8(uint4 xv, const unsigned long long* g2, float rh, uint4* out) {
   const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
   const unsigned long long r2 = pack2(rh, rh);
@@ -234,7 +237,7 @@ __device__ __forceinline__ bool normalize8(uint4 xv, const unsigned long long* g
     // (x*gamma)*rh for the two bf16 of the word: x*gamma exact, one rounding to fp32
     const unsigned long long p = mul2(mul2(pack2(__uint_as_float(xw[j] << 16), __uint_as_float(xw[j] & 0xffff0000u)), g2[j]), r2);
     const uint32_t u0 = (uint32_t)p, u1 = (uint32_t)(p >> 32);
-    mid |= (uint32_t)(((u0 & 0xffffu) == 0x8000u) | ((u1 & 0xffffu) == 0x8000u));
+    mid |= (uint32_t)((((u0 + 0x8001u) & 0xffffu) < 3u) | (((u1 + 0x8001u) & 0xffffu) < 3u));
     const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(u0), __uint_as_float(u1));
     ow[j] = *reinterpret_cast<const uint32_t*>(&h);
   }
@@ -249,9 +252,12 @@ __device__ __noinline__ uint4 normalize8_exact(uint4 xv, const float* g, float r
     const float xg = __uint_as_float((j & 1) ? (xw[j >> 1] & 0xffff0000u) : (xw[j >> 1] << 16)) * g[j];
     const float p = xg * rh;
     uint32_t u = __float_as_uint(p);
-    if ((u & 0xffffu) == 0x8000u) {
-      const float c = fmaf(xg, rl, fmaf(xg, rh, -p));
-      if (c != 0.0f) u += ((__float_as_uint(c) ^ u) >> 31) ? 0xffffffffu : 1u;
+    if (((u + 0x8001u) & 0xffffu) < 3u) {
+      const uint32_t mb = (u & 0xffff0000u) | 0x8000u;  // the bf16 midpoint next to p
+      const float m = __uint_as_float(mb);
+      const float d = (p - m) + fmaf(xg, rl, fmaf(xg, rh, -p));  // p - m is exact
+      u = mb;
+      if (d != 0.0f) u += ((__float_as_uint(d) ^ mb) >> 31) ? 0xffffffffu : 1u;
     }
     const __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(u));
     const uint32_t hb = *reinterpret_cast<const uint16_t*>(&h);

@@ -81,7 +81,8 @@ struct RouteArgs {
   int score_fn, pre, grouped, n_group, topk_group, topn;
   int renorm;
   float scale;
-  int tile;
+  int tile;          // power of two
+  uint32_t kinv;     // ceil(2^32 / k): item -> token by a multiply-high
   int logits_dtype, bias_dtype, weights_dtype;
   int has_bias;
   int G;
@@ -99,7 +100,7 @@ struct RouteArgs {
 
 struct RouteSmem {
   // offsets (bytes) inside dynamic shared memory
-  int stage, cand, bias, hist_cta, hist_w, offs, cnt, bar, flag, scan, ids, lut, total;
+  int stage, cand, bias, hist_cta, hist_w, offs, cnt, bar, flag, scan, ids, lrank, lut, total;
 };
 
 // per warp: 4 tokens x kCandStride packed u64 keys, then 4 x kCandStride fp32 scores
@@ -130,6 +131,8 @@ __host__ __device__ inline RouteSmem route_smem_layout(int E, int stage_bytes, i
   L.scan = o;
   o += 32 * 4;
   L.ids = o;
+  o += (ids_bytes + 15) & ~15;
+  L.lrank = o;  // per selection: rank among the block's selections of the same expert (u16)
   o += (ids_bytes + 15) & ~15;
   L.lut = o;
   o += (lut_bytes + 15) & ~15;
@@ -828,45 +831,36 @@ __device__ void select_quad_fast(const RouteArgs& a, const uint8_t* stage, int l
   __syncwarp();
 }
 
-// Block-wide exclusive scan of padded counts into offs[0..E]; E <= 1024.
-__device__ void scan_padded_offsets(const int* cnt, int* offs, int E, int tile, int* scratch_w) {
-  // each thread takes ceil(E / blockDim) consecutive experts
-  const int per = (E + blockDim.x - 1) / blockDim.x;
-  const int e0 = threadIdx.x * per;
-  int local = 0;
-  for (int i = 0; i < per; ++i) {
-    const int e = e0 + i;
-    if (e < E) local += ((cnt[e] + tile - 1) / tile) * tile;
-  }
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = local;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int o = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += o;
-  }
-  if (lane == 31) scratch_w[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    int w = (lane < (int)(blockDim.x >> 5)) ? scratch_w[lane] : 0;
-    int wi = w;
+// Exclusive scan of padded counts into offs[0..E] (E <= 1024) by warp 0: lane
+// l takes a run of consecutive experts, then one shuffle scan over the lanes.
+// Ends with a block barrier.
+__device__ void scan_padded_offsets(const int* cnt, int* offs, int E, int tile, int* /*scratch*/) {
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int per = (E + 31) >> 5;
+    const int e0 = lane * per;
+    int local = 0;
+    const int tm = tile - 1;  // tile is a power of two
+    for (int i = 0; i < per; ++i) {
+      const int e = e0 + i;
+      if (e < E) local += (cnt[e] + tm) & ~tm;
+    }
+    int incl = local;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-      const int o = __shfl_up_sync(0xffffffffu, wi, off);
-      if (lane >= off) wi += o;
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
     }
-    if (lane < (int)(blockDim.x >> 5)) scratch_w[lane] = wi - w;
-  }
-  __syncthreads();
-  int run = scratch_w[warp] + incl - local;
-  for (int i = 0; i < per; ++i) {
-    const int e = e0 + i;
-    if (e < E) {
-      offs[e] = run;
-      run += ((cnt[e] + tile - 1) / tile) * tile;
+    int run = incl - local;
+    for (int i = 0; i < per; ++i) {
+      const int e = e0 + i;
+      if (e < E) {
+        offs[e] = run;
+        run += (cnt[e] + tm) & ~tm;
+      }
     }
+    if (lane == 31) offs[E] = incl;
   }
-  if (e0 < E && e0 + per >= E) offs[E] = run;
   __syncthreads();
 }
 
@@ -896,6 +890,7 @@ __global__ void __launch_bounds__((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneri
   int* flag = reinterpret_cast<int*>(smem + L.flag);
   int* scan_scratch = reinterpret_cast<int*>(smem + L.scan);
   uint16_t* ids_s = a.ids_in_smem ? reinterpret_cast<uint16_t*>(smem + L.ids) : nullptr;
+  uint16_t* lrank_s = a.ids_in_smem ? reinterpret_cast<uint16_t*>(smem + L.lrank) : nullptr;
 
   const uint32_t gen = barrier_generation(a.hdr);
 
@@ -982,7 +977,55 @@ __global__ void __launch_bounds__((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneri
     else if (a.cnt_bytes == 2) reinterpret_cast<uint16_t*>(trow)[e] = (uint16_t)h;
     else reinterpret_cast<uint32_t*>(trow)[e] = (uint32_t)h;
   }
-  if (!grid_barrier(a.hdr, (uint32_t)a.G, gen, a.timeout_ns, flag)) return;
+  __syncthreads();
+  if (threadIdx.x == 0) grid_arrive(a.hdr, (uint32_t)a.G);
+
+  // ---- while the other blocks finish: each selection's rank among this
+  //      block's selections of the same expert, in item order (per-warp counts
+  //      over a contiguous split of the items, their exclusive prefix over
+  //      warps, then a walk that ranks equal experts inside each 32-item chunk)
+  const long long i_begin = (long long)t_begin * a.k;
+  const int w_begin = (int)((long long)n_items * warp / kWarps);
+  const int w_end = (int)((long long)n_items * (warp + 1) / kWarps);
+  if (lrank_s) {
+    for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) hist_w[i] = 0;
+    __syncthreads();
+    for (int i = w_begin + lane; i < w_end; i += 32) {
+      const int e = ids_s[i];
+      if (e < E) atomicAdd(&hist_w[warp * E + e], 1);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      int h[kWarps];
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) h[w] = hist_w[w * E + e];
+      int run = 0;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        hist_w[w * E + e] = run;
+        run += h[w];
+      }
+    }
+    __syncthreads();
+    for (int i0 = w_begin; i0 < w_end; i0 += 32) {
+      const int i = i0 + lane;
+      const bool act = i < w_end;
+      const unsigned amask = __ballot_sync(0xffffffffu, act);
+      if (act) {
+        const int e = min((int)ids_s[i], E - 1);  // ids were range-checked when selected
+        const unsigned m = __match_any_sync(amask, e);
+        const int rank = __popc(m & ((1u << lane) - 1u));
+        const int leader = __ffs(m) - 1;
+        lrank_s[i] = (uint16_t)(hist_w[warp * E + e] + rank);
+        __syncwarp(amask);
+        if (lane == leader) hist_w[warp * E + e] += __popc(m);
+      }
+      __syncwarp();
+    }
+  }
+  if (threadIdx.x == 0) flag[0] = grid_wait(a.hdr, (uint32_t)a.G, gen, a.timeout_ns) ? 1 : 0;
+  __syncthreads();
+  if (!flag[0]) return;
   if (!staged_ok) return;  // a staging wait gave up (recorded); outputs undefined
 
   // ---------------- phase 2: totals and block base from the table ----------------
@@ -993,9 +1036,6 @@ __global__ void __launch_bounds__((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneri
   // keeps per-entry sums; the partial sums go to shared memory word-major so
   // the stores and the reduction reads hit distinct banks.  Integer sums in a
   // fixed order: deterministic, no atomics.
-  const long long i_begin = (long long)t_begin * a.k;
-  const int w_begin = (int)((long long)n_items * warp / kWarps);
-  const int w_end = (int)((long long)n_items * (warp + 1) / kWarps);
   int P = 0;
   {
     const int WPR = a.row_stride >> 2;                     // 32-bit words per row
@@ -1003,7 +1043,64 @@ __global__ void __launch_bounds__((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneri
     const int R = max(1, min((int)blockDim.x / WPR, a.G));  // row groups
     const int rg = threadIdx.x / WPR, w = threadIdx.x % WPR;
     int tot[4] = {0, 0, 0, 0}, pre[4] = {0, 0, 0, 0};
-    if (rg < R) {
+    const bool wide = a.cnt_bytes == 1 && (a.row_stride >> 4) * 16 <= (int)blockDim.x;
+    if (wide) {
+      // byte entries, 16-byte loads: thread (row group rg4 < 16, 16-byte column w4)
+      // reads rows rg4, rg4 + 16, ... (all loads in flight) and keeps two 16-bit
+      // lanes per 32-bit accumulator (a row group's sums stay below 65536)
+      const int W4 = a.row_stride >> 4;
+      const int R4 = min(16, a.G);
+      const int rg4 = threadIdx.x / W4, w4 = threadIdx.x % W4;
+      uint32_t* part_w = reinterpret_cast<uint32_t*>(stage);  // [2][R4][8][W4 + 1] packed pairs
+      const int pstride = W4 + 1;
+      if (rg4 < R4) {
+        uint32_t acc_t[8] = {0, 0, 0, 0, 0, 0, 0, 0}, acc_p[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        constexpr int kB4 = 10;
+        for (int cp0 = rg4; cp0 < a.G; cp0 += R4 * kB4) {
+          uint4 v[kB4];
+#pragma unroll
+          for (int b = 0; b < kB4; ++b) {
+            const int cp = cp0 + b * R4;
+            v[b] = cp < a.G ? __ldcg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(a.table) +
+                                                                     (size_t)cp * a.row_stride) + w4)
+                            : make_uint4(0, 0, 0, 0);
+          }
+#pragma unroll
+          for (int b = 0; b < kB4; ++b) {
+            const bool before = cp0 + b * R4 < c;
+            const uint32_t vw[4] = {v[b].x, v[b].y, v[b].z, v[b].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t e02 = vw[j] & 0x00ff00ffu, e13 = (vw[j] >> 8) & 0x00ff00ffu;
+              acc_t[2 * j] += e02;
+              acc_t[2 * j + 1] += e13;
+              if (before) {
+                acc_p[2 * j] += e02;
+                acc_p[2 * j + 1] += e13;
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          part_w[(rg4 * 8 + j) * pstride + w4] = acc_t[j];
+          part_w[((R4 + rg4) * 8 + j) * pstride + w4] = acc_p[j];
+        }
+      }
+      __syncthreads();
+      // entry e = 16*w4 + 4*j + lo/hi*2 + odd: accumulator 2*j + odd, 16-bit lane lo/hi
+      for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        const int ww = e >> 4, within = e & 15;
+        const int acc = (within >> 2) * 2 + (within & 1), sh = (within & 2) ? 16 : 0;
+        int st = 0, sp = 0;
+        for (int r = 0; r < R4; ++r) {
+          st += (int)((part_w[(r * 8 + acc) * pstride + ww] >> sh) & 0xffffu);
+          sp += (int)((part_w[((R4 + r) * 8 + acc) * pstride + ww] >> sh) & 0xffffu);
+        }
+        cnt[e] = st;
+        hist_cta[e] = sp;
+      }
+    } else if (rg < R) {
       constexpr int kBatch = 20;
       for (int cp0 = rg; cp0 < a.G; cp0 += R * kBatch) {
         uint32_t v[kBatch];
@@ -1050,7 +1147,7 @@ __global__ void __launch_bounds__((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneri
     }
     int* part_t = reinterpret_cast<int*>(stage);   // [R][EPW][WPR]
     int* part_p = part_t + R * EPW * WPR;          // [R][EPW][WPR]
-    if (rg < R) {
+    if (!wide && rg < R) {
 #pragma unroll
       for (int i = 0; i < 4; ++i)
         if (i < EPW) {
@@ -1059,7 +1156,7 @@ __global__ void __launch_bounds__((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneri
         }
     }
     __syncthreads();
-    for (int x = threadIdx.x; x < EPW * WPR; x += blockDim.x) {
+    for (int x = threadIdx.x; !wide && x < EPW * WPR; x += blockDim.x) {
       const int i = x / WPR, ww = x % WPR;
       const int e = ww * EPW + i;
       if (e < E) {
@@ -1072,7 +1169,8 @@ __global__ void __launch_bounds__((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneri
         hist_cta[e] = sp;
       }
     }
-    for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) hist_w[i] = 0;
+    if (!lrank_s)
+      for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) hist_w[i] = 0;
     __syncthreads();
     scan_padded_offsets(cnt, offs, E, a.tile, scan_scratch);
     P = offs[E];
@@ -1091,43 +1189,60 @@ __global__ void __launch_bounds__((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneri
   const int ntiles = P / a.tile;
 
   // ---------------- phase 2: slots in token order ----------------
-  // per-warp counts over a contiguous split of the block's selections, their
-  // exclusive prefix over warps, then a walk that ranks equal experts inside
-  // each 32-item chunk (match + popcount)
-  for (int i = w_begin + lane; i < w_end; i += 32) {
-    const int e = ids_s ? (int)ids_s[i] : a.ids[i_begin + i];
-    if ((unsigned)e < (unsigned)E) atomicAdd(&hist_w[warp * E + e], 1); else record_bounds(a.hdr);
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int run = offs[e] + hist_cta[e];
-    for (int w = 0; w < kWarps; ++w) {
-      const int h = hist_w[w * E + e];
-      hist_w[w * E + e] = run;
-      run += h;
-    }
-  }
-  __syncthreads();
-  for (int i0 = w_begin; i0 < w_end; i0 += 32) {
-    const int i = i0 + lane;
-    const bool act = i < w_end;
-    const unsigned amask = __ballot_sync(0xffffffffu, act);
-    if (act) {
-      int e = ids_s ? (int)ids_s[i] : a.ids[i_begin + i];
-      if ((unsigned)e >= (unsigned)E) {
+  if (lrank_s) {
+    // slot = expert offset + earlier blocks' selections of the expert + local rank
+    for (int i = threadIdx.x; i < n_items; i += blockDim.x) {
+      const int e = ids_s[i];
+      if (e >= E) {
         record_bounds(a.hdr);
-        e = 0;
+        continue;
       }
-      const unsigned m = __match_any_sync(amask, e);
-      const int rank = __popc(m & ((1u << lane) - 1u));
-      const int leader = __ffs(m) - 1;
-      const int slot = hist_w[warp * E + e] + rank;
-      __syncwarp(amask);
-      if (lane == leader) hist_w[warp * E + e] += __popc(m);
+      const int slot = offs[e] + hist_cta[e] + lrank_s[i];
       a.e2p[i_begin + i] = slot;
-      if ((unsigned)slot < (unsigned)a.max_padded) a.p2t[slot] = (int)((i_begin + i) / a.k); else record_bounds(a.hdr);
+      // token of item i: t_begin + i / k (i < 2^16, so the multiply-high is exact)
+      const int lt = a.k == 1 ? i : (int)__umulhi((uint32_t)i, a.kinv);
+      if ((unsigned)slot < (unsigned)a.max_padded) a.p2t[slot] = t_begin + lt;
+      else record_bounds(a.hdr);
     }
-    __syncwarp();
+  } else {
+    // per-warp counts over a contiguous split of the block's selections, their
+    // exclusive prefix over warps, then a walk that ranks equal experts inside
+    // each 32-item chunk (match + popcount)
+    for (int i = w_begin + lane; i < w_end; i += 32) {
+      const int e = ids_s ? (int)ids_s[i] : a.ids[i_begin + i];
+      if ((unsigned)e < (unsigned)E) atomicAdd(&hist_w[warp * E + e], 1); else record_bounds(a.hdr);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      int run = offs[e] + hist_cta[e];
+      for (int w = 0; w < kWarps; ++w) {
+        const int h = hist_w[w * E + e];
+        hist_w[w * E + e] = run;
+        run += h;
+      }
+    }
+    __syncthreads();
+    for (int i0 = w_begin; i0 < w_end; i0 += 32) {
+      const int i = i0 + lane;
+      const bool act = i < w_end;
+      const unsigned amask = __ballot_sync(0xffffffffu, act);
+      if (act) {
+        int e = ids_s ? (int)ids_s[i] : a.ids[i_begin + i];
+        if ((unsigned)e >= (unsigned)E) {
+          record_bounds(a.hdr);
+          e = 0;
+        }
+        const unsigned m = __match_any_sync(amask, e);
+        const int rank = __popc(m & ((1u << lane) - 1u));
+        const int leader = __ffs(m) - 1;
+        const int slot = hist_w[warp * E + e] + rank;
+        __syncwarp(amask);
+        if (lane == leader) hist_w[warp * E + e] += __popc(m);
+        a.e2p[i_begin + i] = slot;
+        if ((unsigned)slot < (unsigned)a.max_padded) a.p2t[slot] = (int)((i_begin + i) / a.k); else record_bounds(a.hdr);
+      }
+      __syncwarp();
+    }
   }
 
   // ---------------- tile tables and padding rows (a warp per tile) ----------------
@@ -1348,6 +1463,7 @@ extern "C" int moe_route(const moe_route_params* p, const void* logits, const vo
   a.renorm = p->renormalize ? 1 : 0;
   a.scale = p->scaling_factor;
   a.tile = p->tile_tokens_dim;
+  a.kinv = p->top_k > 1 ? (uint32_t)((0x100000000ull + (uint64_t)p->top_k - 1) / (uint64_t)p->top_k) : 0u;
   a.logits_dtype = p->logits_dtype;
   a.bias_dtype = p->bias_dtype;
   a.weights_dtype = p->weights_dtype;
