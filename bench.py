@@ -191,6 +191,27 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def rank_spec(rank: int):
+    """The workload of one rank: same shape on every rank, its own seeded batch (data-parallel, weak scaling)."""
+    from top_expert_selection_b200 import workloads as W
+    return W.DSV3_GROUPED_SIGMOID.with_(seed=W.DSV3_GROUPED_SIGMOID.seed + rank)
+
+
+def max_over_ranks(x: float, pg, device) -> float:
+    """The maximum of a per-rank number over all ranks (a no-op without a process group)."""
+    if pg is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
+    """Tokens/s over all ranks for one step of ms_per_step (max over ranks)."""
+    return world * tokens_per_rank / (ms_per_step / 1000.0)
+
+
 def workload_config():
     return {"workload": "dsv3_grouped_sigmoid_route: T=16384 E=256 top_k=8 n_group=8 topk_group=4 "
                         "(top-2 group score) bf16 logits N(0,2) fp32 bias U(-0.1,0.1) renorm scale=2.5 tile=128 "
@@ -218,7 +239,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         pg = dist
 
-    spec = W.DSV3_GROUPED_SIGMOID.with_(seed=W.DSV3_GROUPED_SIGMOID.seed + rank)
+    spec = rank_spec(rank)
     inp = W.route_inputs(spec)
     p = B.route_params(spec.T, spec.E, spec.k, score_fn=spec.score_fn, n_group=spec.n_group,
                        topk_group=spec.topk_group, group_score_topn=spec.group_score_topn, renormalize=1,
@@ -268,13 +289,9 @@ def main():
     clocks = sampler.stop()
     if pg:
         pg.barrier()
-    ms_total = e0.elapsed_time(e1)
-    if pg:
-        t = torch.tensor([ms_total], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(e0.elapsed_time(e1), pg, dev)
     ms_step = ms_total / args.steps
-    value = world * spec.T / (ms_step / 1000.0)
+    value = whole_job_rate(world, spec.T, ms_step)
 
     # correctness of what was timed: every rotated output set reports OK and the same bookkeeping
     ok = all(B.status(r.ws) == B.MOE_OK for r in routers)
@@ -319,12 +336,8 @@ def main():
                 e2e_step()
             f1.record(stream)
         torch.cuda.synchronize()
-        ms_e2e = f0.elapsed_time(f1) / n_e2e
-        if pg:
-            t = torch.tensor([ms_e2e], device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            ms_e2e = float(t.item())
-        e2e = {"value": world * spec.T / (ms_e2e / 1000.0), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+        ms_e2e = max_over_ranks(f0.elapsed_time(f1) / n_e2e, pg, dev)
+        e2e = {"value": whole_job_rate(world, spec.T, ms_e2e), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "ms_per_step": ms_e2e, "steps": n_e2e}
 
     extra = None

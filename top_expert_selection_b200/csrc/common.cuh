@@ -59,22 +59,18 @@ __device__ __forceinline__ uint32_t barrier_generation(WsHeader* h) {
 
 // Grid-wide barrier for a co-resident (cooperatively launched) grid of
 // `nblocks` blocks, split into an arrival and a wait so a block can do local
-// work in between.  One 64-bit word holds generation | arrivals: a block adds
-// 1; the last arrival then adds 2^32 - nblocks (no return value needed), which
-// bumps the generation and clears the count.  Waiters are released as soon as
-// the count reads nblocks (before that reset lands) or the generation has
-// moved on, so the barrier costs one atomic round trip.  One barrier per
-// launch: a second one could see the first one's count before its reset.
+// work in between.  One 64-bit word holds generation | arrivals.  A block's
+// arrival is a fire-and-forget add of 1 (the arriving thread does not wait
+// for it); waiters are released as soon as the count reads nblocks, and block
+// 0, once released, adds 2^32 - nblocks, which bumps the generation and clears
+// the count for the next launch (waiters that read the word after that see
+// the new generation instead).  One barrier per launch; after a wait that gave
+// up (status MOE_ERR_DEVICE_TIMEOUT) the workspace must be initialised again.
 //
 // grid_arrive: thread 0 only, after the block's writes to publish.
-__device__ __forceinline__ void grid_arrive(WsHeader* h, uint32_t nblocks) {
+__device__ __forceinline__ void grid_arrive(WsHeader* h, uint32_t /*nblocks*/) {
   __threadfence();
-  const unsigned long long old = atomicAdd(&h->barrier, 1ull);
-  if ((uint32_t)old == nblocks - 1) {
-    asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" ::"l"(&h->barrier),
-                 "l"((1ull << 32) - (unsigned long long)nblocks)
-                 : "memory");
-  }
+  asm volatile("red.relaxed.gpu.global.add.u64 [%0], 1;" ::"l"(&h->barrier) : "memory");
 }
 
 // grid_wait: thread 0 only; false (and a recorded timeout) if the wait
@@ -93,6 +89,10 @@ __device__ __forceinline__ bool grid_wait(WsHeader* h, uint32_t nblocks, uint32_
     }
   }
   __threadfence();
+  if (blockIdx.x == 0)
+    asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" ::"l"(&h->barrier),
+                 "l"((1ull << 32) - (unsigned long long)nblocks)
+                 : "memory");
   return true;
 }
 

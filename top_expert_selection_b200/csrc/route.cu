@@ -704,16 +704,30 @@ __device__ void select_quad_fast(const RouteArgs& a, const uint8_t* stage, int l
     for (int j = 0; j < V; ++j) mq[j & 3] |= (p[j] >= th ? 1u : 0u) << j;
     uint32_t m = (mq[0] | mq[1]) | (mq[2] | mq[3]);
     while (m) {
-      const int j = __ffs(m) - 1;
-      m &= m - 1;
-      const int e = slot_expert<V, ESZ>(g, rot, j);
-      const float sg = (ESZ == 2) ? sigmoid_bf16_row(lut, row, e) : sigmoid_f32(stage_val(a, row, e));
-      const float K = sg + bias_s[e];
-      if (K > K1) {
-        K2 = K1; S2 = S1; j2 = j1;
-        K1 = K; S1 = sg; j1 = j;
-      } else if (K > K2) {
-        K2 = K; S2 = sg; j2 = j;
+      // up to 4 members per pass, their exact keys evaluated side by side
+      int jb[4];
+      float kb4[4], sb4[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        jb[u] = m ? __ffs(m) - 1 : -1;
+        m &= m - 1;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = slot_expert<V, ESZ>(g, rot, max(jb[u], 0));
+        sb4[u] = (ESZ == 2) ? sigmoid_bf16_row(lut, row, e) : sigmoid_f32(stage_val(a, row, e));
+        kb4[u] = sb4[u] + bias_s[e];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (jb[u] < 0) continue;
+        const float K = kb4[u];
+        if (K > K1) {
+          K2 = K1; S2 = S1; j2 = j1;
+          K1 = K; S1 = sb4[u]; j1 = jb[u];
+        } else if (K > K2) {
+          K2 = K; S2 = sb4[u]; j2 = jb[u];
+        }
       }
     }
   }
@@ -768,22 +782,33 @@ __device__ void select_quad_fast(const RouteArgs& a, const uint8_t* stage, int l
   if (tv && !slow) {
     int pos = incl - cnt;
     uint32_t m = mask;
+    if (j1 >= 0) m &= ~(1u << j1);
+    if (j2 >= 0) m &= ~(1u << j2);
+    // the lane's top-2 (exact already), then the other candidates 4 per pass
+    if (j1 >= 0 && ((mask >> j1) & 1u)) {
+      ck[pos] = pack_key(K1, slot_expert<V, ESZ>(g, rot, j1));
+      cs[pos++] = S1;
+    }
+    if (j2 >= 0 && ((mask >> j2) & 1u)) {
+      ck[pos] = pack_key(K2, slot_expert<V, ESZ>(g, rot, j2));
+      cs[pos++] = S2;
+    }
     while (m) {
-      const int j = __ffs(m) - 1;
-      m &= m - 1;
-      const int e = slot_expert<V, ESZ>(g, rot, j);
-      float sg, K;
-      if (j == j1) {
-        sg = S1; K = K1;
-      } else if (j == j2) {
-        sg = S2; K = K2;
-      } else {
-        sg = (ESZ == 2) ? sigmoid_bf16_row(lut, row, e) : sigmoid_f32(stage_val(a, row, e));
-        K = sg + bias_s[e];
+      int jb[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        jb[u] = m ? __ffs(m) - 1 : -1;
+        m &= m - 1;
       }
-      ck[pos] = pack_key(K, e);
-      cs[pos] = sg;
-      ++pos;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = slot_expert<V, ESZ>(g, rot, max(jb[u], 0));
+        const float sg = (ESZ == 2) ? sigmoid_bf16_row(lut, row, e) : sigmoid_f32(stage_val(a, row, e));
+        if (jb[u] >= 0) {
+          ck[pos] = pack_key(sg + bias_s[e], e);
+          cs[pos++] = sg;
+        }
+      }
     }
   }
   __syncwarp();
@@ -1008,18 +1033,25 @@ __global__ void __launch_bounds__((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneri
     }
     __syncthreads();
     for (int i0 = w_begin; i0 < w_end; i0 += 32) {
+      // rank inside the 32-item chunk = earlier lanes holding the same expert
+      // (inactive lanes hold distinct negative values); the chunk's last item of
+      // each expert then raises the running count
       const int i = i0 + lane;
       const bool act = i < w_end;
-      const unsigned amask = __ballot_sync(0xffffffffu, act);
-      if (act) {
-        const int e = min((int)ids_s[i], E - 1);  // ids were range-checked when selected
-        const unsigned m = __match_any_sync(amask, e);
-        const int rank = __popc(m & ((1u << lane) - 1u));
-        const int leader = __ffs(m) - 1;
-        lrank_s[i] = (uint16_t)(hist_w[warp * E + e] + rank);
-        __syncwarp(amask);
-        if (lane == leader) hist_w[warp * E + e] += __popc(m);
+      const int e = act ? min((int)ids_s[i], E - 1) : -1 - lane;  // ids were range-checked when selected
+      int rank = 0;
+#pragma unroll
+      for (int d = 1; d < 32; ++d) {
+        const int o = __shfl_up_sync(0xffffffffu, e, d);
+        rank += (lane >= d && o == e) ? 1 : 0;
       }
+      int slot = 0;
+      if (act) {
+        slot = hist_w[warp * E + e] + rank;
+        lrank_s[i] = (uint16_t)slot;
+      }
+      __syncwarp();
+      if (act) atomicMax(&hist_w[warp * E + e], slot + 1);
       __syncwarp();
     }
   }
