@@ -52,13 +52,74 @@ __device__ __forceinline__ float sigmoid_f32(float x) { return 1.0f / (1.0f + ex
 // --------------------------------------------------------------------------
 constexpr int kScoreThreads = 512;
 
+// Top-k mask of one row held by a warp (lane l: entries [l*VPL, l*VPL+VPL)),
+// for k <= 8, by threshold and counting instead of k argmax rounds.  In each
+// 8-lane group the second-largest lane maximum is at most its group's top-2
+// lane maxima, so at least 8 >= k entries are >= tau = the smallest of the
+// four groups' second maxima.  The entries >= tau (the candidates) are ranked by
+// counting on packed (ordered key, ~index) words - larger value first, equal
+// values by lower index - and the mask keeps those at or above the k-th.
+// Returns false (warp-uniform) when the candidates exceed 32 or number fewer
+// than k (non-finite values); the caller then uses the k rounds.
+template <int VPL>
+__device__ __forceinline__ bool topk_mask_by_threshold(const float* p, uint32_t valid, int lane, int k,
+                                                       unsigned long long* list, uint32_t* chosen_out) {
+  const unsigned FULL = 0xffffffffu;
+  float mx = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i)
+    if ((valid >> i) & 1u) mx = fmaxf(mx, p[i]);
+  float a1 = mx, a2 = -INFINITY;
+#pragma unroll
+  for (int off = 1; off < 8; off <<= 1) {
+    const float o1 = __shfl_xor_sync(FULL, a1, off), o2 = __shfl_xor_sync(FULL, a2, off);
+    a2 = fmaxf(fminf(a1, o1), fmaxf(a2, o2));
+    a1 = fmaxf(a1, o1);
+  }
+  float tau = fminf(a2, __shfl_xor_sync(FULL, a2, 8));
+  tau = fminf(tau, __shfl_xor_sync(FULL, tau, 16));
+  uint32_t cm = 0;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) cm |= (((valid >> i) & 1u) && p[i] >= tau ? 1u : 0u) << i;
+  const int cnt = __popc(cm);
+  int incl = cnt;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(FULL, incl, off);
+    if (lane >= off) incl += o;
+  }
+  const int total = __shfl_sync(FULL, incl, 31);
+  if (total > 32 || total < k) return false;
+  int pos = incl - cnt;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i)
+    if ((cm >> i) & 1u) list[pos++] = pack_key(p[i], lane * VPL + i);
+  __syncwarp();
+  unsigned long long key = 0ull;
+  int rank = 32;
+  if (lane < total) {
+    key = list[lane];
+    rank = 0;
+    for (int j = 0; j < total; ++j) rank += (list[j] > key) ? 1 : 0;
+  }
+  const int src = __ffs(__ballot_sync(FULL, rank == k - 1)) - 1;  // keys are distinct: one lane
+  const unsigned long long kth = shfl_xor_u64(FULL, key, src ^ lane);
+  uint32_t chosen = 0;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i)
+    if ((cm >> i) & 1u) chosen |= (pack_key(p[i], lane * VPL + i) >= kth ? 1u : 0u) << i;
+  __syncwarp();  // the list is reused by the next row
+  *chosen_out = chosen;
+  return true;
+}
+
 template <int VPL>
 __global__ void __launch_bounds__(kScoreThreads) aux_scores_kernel(int T, int E, int k, int score_fn,
                                                                  const float* __restrict__ logits,
                                                                  float* __restrict__ probs,
                                                                  uint8_t* __restrict__ rmap,
                                                                  int32_t* __restrict__ tpe, void* ws) {
-  extern __shared__ int hist[];  // [E]
+  extern __shared__ int hist[];  // [E], then per warp 32 packed candidate keys
   const unsigned FULL = 0xffffffffu;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
@@ -67,35 +128,32 @@ __global__ void __launch_bounds__(kScoreThreads) aux_scores_kernel(int T, int E,
   __syncthreads();
 
   const int nw = blockDim.x >> 5;
-  for (long long t = (long long)blockIdx.x * nw + warp; t < T; t += (long long)gridDim.x * nw) {
+  uint32_t valid = 0;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) valid |= ((lane * VPL + i < E) ? 1u : 0u) << i;
+  // a lane's VPL experts are contiguous: 16-byte loads when the row allows it
+  const bool vec = (VPL % 4 == 0) && ((E & 3) == 0) && (lane * VPL + VPL <= E);
+  auto load_row = [&](long long t, float* x) {
     const float* row = logits + t * E;
-    float x[VPL], p[VPL];
-    uint32_t valid = 0;
-    if constexpr (VPL % 4 == 0) {
-      // a lane's VPL experts are contiguous: 16-byte loads when the row allows it
-      const bool vec = ((E & 3) == 0) && (lane * VPL + VPL <= E);
 #pragma unroll
-      for (int i = 0; i < VPL; i += 4) {
-        const int e = lane * VPL + i;
-        if (vec) {
+    for (int i = 0; i < VPL; ++i) {
+      const int e = lane * VPL + i;
+      if (vec) {
+        if ((i & 3) == 0) {
           const float4 q = __ldcs(reinterpret_cast<const float4*>(row + e));
-          x[i] = q.x; x[i + 1] = q.y; x[i + 2] = q.z; x[i + 3] = q.w;
-        } else {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) x[i + j] = (e + j < E) ? __ldcs(row + e + j) : 0.0f;
+          x[i] = q.x;
+          if (i + 1 < VPL) x[i + 1] = q.y;
+          if (i + 2 < VPL) x[i + 2] = q.z;
+          if (i + 3 < VPL) x[i + 3] = q.w;
         }
-      }
-#pragma unroll
-      for (int i = 0; i < VPL; ++i) valid |= ((lane * VPL + i < E) ? 1u : 0u) << i;
-    } else {
-#pragma unroll
-      for (int i = 0; i < VPL; ++i) {
-        const int e = lane * VPL + i;
-        const bool v = e < E;
-        x[i] = v ? __ldcs(row + e) : 0.0f;
-        valid |= (v ? 1u : 0u) << i;
+      } else {
+        x[i] = e < E ? __ldcs(row + e) : 0.0f;
       }
     }
+  };
+  for (long long t = (long long)blockIdx.x * nw + warp; t < T; t += (long long)gridDim.x * nw) {
+    float x[VPL], p[VPL];
+    load_row(t, x);
     float sum = 0.0f;
     if (score_fn == MOE_SOFTMAX) {
       float m = -INFINITY;
@@ -121,9 +179,15 @@ __global__ void __launch_bounds__(kScoreThreads) aux_scores_kernel(int T, int E,
 #pragma unroll
     for (int i = 0; i < VPL; ++i) p[i] = p[i] / sum;
 
-    // top-k mask over probs: k rounds of warp argmax, ties -> lower expert
+    // top-k mask over probs, ties -> lower expert: threshold + counting, else
+    // k rounds of warp argmax
     uint32_t avail = valid, chosen = 0;
-    for (int j = 0; j < k; ++j) {
+    bool done = false;
+    if constexpr (VPL <= 8) {
+      unsigned long long* list = reinterpret_cast<unsigned long long*>(hist + ((E + 1) & ~1)) + warp * 32;
+      if (k <= 8) done = topk_mask_by_threshold<VPL>(p, valid, lane, k, list, &chosen);
+    }
+    for (int j = 0; j < k && !done; ++j) {
       unsigned long long best = 0ull;
 #pragma unroll
       for (int i = 0; i < VPL; ++i)
@@ -195,7 +259,7 @@ __global__ void __launch_bounds__(kScoreThreads) aux_scores_kernel(int T, int E,
 // --------------------------------------------------------------------------
 // loss forward: one pass over probs; fixed grid; deterministic reduction
 // --------------------------------------------------------------------------
-__global__ void __launch_bounds__(kAuxThreads) aux_loss_fwd_kernel(long long n, int E, double C,
+__global__ void __launch_bounds__(kAuxThreads, 2) aux_loss_fwd_kernel(long long n, int E, double C,
                                                                    const float* __restrict__ probs,
                                                                    const int32_t* __restrict__ tpe, float* loss,
                                                                    void* ws) {
@@ -212,24 +276,29 @@ __global__ void __launch_bounds__(kAuxThreads) aux_loss_fwd_kernel(long long n, 
   float acc = 0.0f;
   if ((E & 3) == 0 && (b0 & 3) == 0) {
     const long long q1 = b1 >> 2;
-    constexpr int kB = 8;  // independent 16-byte loads in flight per thread
-    for (long long q0 = (b0 >> 2) + threadIdx.x; q0 < q1; q0 += (long long)blockDim.x * kB) {
+    const float4* base = reinterpret_cast<const float4*>(probs) + (b0 >> 2);
+    const int nq = (int)(q1 - (b0 >> 2));  // float4s of this block (< 2^31)
+    constexpr int kB = 16;                 // independent 16-byte loads in flight per thread
+    // column of a float4: advances by step (mod E) from one load to the next,
+    // so the only division is the first one
+    const int step = (int)((blockDim.x * 4) % (unsigned)E);
+    int e = (int)((((b0 >> 2) + threadIdx.x) << 2) % E);
+    for (int l0 = threadIdx.x; l0 < nq; l0 += blockDim.x * kB) {
       float4 v[kB];
 #pragma unroll
       for (int b = 0; b < kB; ++b) {
-        const long long q = q0 + (long long)b * blockDim.x;
-        v[b] = q < q1 ? __ldcs(reinterpret_cast<const float4*>(probs) + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const int l = l0 + b * (int)blockDim.x;
+        v[b] = l < nq ? __ldcs(base + l) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
       for (int b = 0; b < kB; ++b) {
-        const long long q = q0 + (long long)b * blockDim.x;
-        const int e = (int)((q << 2) % E);
-        if (q < q1) {
-          acc = fmaf(v[b].x, tpe_s[e], acc);
-          acc = fmaf(v[b].y, tpe_s[e + 1], acc);
-          acc = fmaf(v[b].z, tpe_s[e + 2], acc);
-          acc = fmaf(v[b].w, tpe_s[e + 3], acc);
-        }
+        // entries past the block's range load as zeros and add nothing
+        acc = fmaf(v[b].x, tpe_s[e], acc);
+        acc = fmaf(v[b].y, tpe_s[e + 1], acc);
+        acc = fmaf(v[b].z, tpe_s[e + 2], acc);
+        acc = fmaf(v[b].w, tpe_s[e + 3], acc);
+        e += step;
+        if (e >= E) e -= E;
       }
     }
     for (long long i = (q1 << 2) + threadIdx.x; i < b1; i += blockDim.x) acc = fmaf(probs[i], tpe_s[i % E], acc);
@@ -371,7 +440,8 @@ extern "C" int moe_aux_scores(int32_t T, int32_t E, int32_t k, int32_t score_fn,
   const int vpl = pick_vpl(E);
   const int grid = std::max(1, std::min((T + 15) / 16, sm_count() * 2));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const size_t smem = (size_t)E * sizeof(int);
+  // histogram, then 32 packed candidate keys per warp
+  const size_t smem = (size_t)((E + 1) & ~1) * sizeof(int) + (size_t)(kScoreThreads / 32) * 32 * 8;
   MOE_VPL_SWITCH(vpl, (aux_scores_kernel<V><<<grid, kScoreThreads, smem, st>>>(T, E, k, score_fn, logits, probs,
                                                                             routing_map, tokens_per_expert, ws)));
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
