@@ -50,7 +50,7 @@ namespace {
 
 // threads per block: the sigmoid fast path keeps few registers and runs 24
 // warps per SM; the generic paths keep larger per-thread arrays and run 16
-constexpr int kThreadsFast = 768;
+constexpr int kThreadsFast = 896;
 constexpr int kThreadsGeneric = 512;
 constexpr int kWarpsMax = kThreadsFast / 32;
 constexpr int kStageBytesMax = 96 * 1024;
