@@ -174,6 +174,38 @@ def test_repeated_calls_are_deterministic():
         assert torch.equal(first[n], views[n]), n
 
 
+def test_one_workspace_across_shapes_and_paths():
+    """One workspace reused by calls of different shapes, in both count-table
+    formats (byte counts: tagged rows, no grid barrier; wider counts: the grid
+    barrier), must give what a fresh workspace gives, call after call."""
+    big = B.route_params(16384, 256, 8)
+    ws = B.make_workspace(max(B.route_workspace_bytes(big),
+                              B.route_workspace_bytes(B.route_params(65536, 8, 2))), "cuda")
+    seq = [W.DSV3_GROUPED_SIGMOID, W.DSV3_GROUPED_SIGMOID.with_(T=3000, seed=5), W.MIXTRAL_ROUTE,
+           W.DSV3_GROUPED_SIGMOID.with_(seed=6), W.DSV3_GROUPED_SIGMOID.with_(T=500, seed=7),
+           W.DSV3_GROUPED_SIGMOID.with_(seed=6), W.MIXTRAL_ROUTE.with_(T=20000, seed=8)]
+    for spec in seq:
+        inp = W.route_inputs(spec)
+        kw = dict(score_fn=spec.score_fn, n_group=spec.n_group, topk_group=spec.topk_group,
+                  group_score_topn=spec.group_score_topn, renormalize=spec.renormalize,
+                  softmax_before_topk=spec.softmax_before_topk, scaling_factor=spec.scaling_factor,
+                  tile_tokens_dim=spec.tile_tokens_dim, logits_dtype=spec.logits_dtype, bias_dtype=spec.bias_dtype,
+                  weights_dtype=spec.weights_dtype)
+        p = B.route_params(spec.T, spec.E, spec.k, **kw)
+        lg = inp["logits"].cuda()
+        b = inp["bias"].cuda() if inp["bias"] is not None else None
+        fresh = B.Router(p)
+        ref = fresh(lg, b)
+        shared = B.Router(p)
+        B.route_into(p, lg, b, shared.out, ws)
+        torch.cuda.synchronize()
+        assert B.status(ws) == B.MOE_OK and B.status(fresh.ws) == B.MOE_OK
+        P = int(ref["totals"][0])
+        for n in ("ids", "weights", "counts", "offsets", "e2p", "totals"):
+            assert torch.equal(ref[n], shared.out[n]), (spec, n)
+        assert torch.equal(ref["p2t"][:P], shared.out["p2t"][:P]), spec
+
+
 def test_zero_tokens():
     p = B.route_params(0, 16, 2, tile_tokens_dim=4)
     dev = torch.device("cuda")
