@@ -917,6 +917,13 @@ __global__ void __launch_bounds__((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneri
   uint16_t* ids_s = a.ids_in_smem ? reinterpret_cast<uint16_t*>(smem + L.ids) : nullptr;
   uint16_t* lrank_s = a.ids_in_smem ? reinterpret_cast<uint16_t*>(smem + L.lrank) : nullptr;
 
+  // Programmatic dependent launch: the next grid in the stream may be scheduled
+  // at once (its blocks start as this grid's blocks retire), and this grid
+  // touches no global memory before the previous one has completed and its
+  // writes are visible.  Without the launch attribute both are no-ops.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
   const uint32_t gen = barrier_generation(a.hdr);
 
   // the first round's logits start streaming before anything else: thread 0
@@ -1416,12 +1423,21 @@ cudaError_t launch_route(const RouteArgs& a, int smem, cudaStream_t st) {
   cfg.blockDim = dim3((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneric);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, route_kernel<VPL, FAST_ESZ>, a);
+  cfg.numAttrs = 2;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, route_kernel<VPL, FAST_ESZ>, a);
+  if (e != cudaSuccess) {
+    // the pair of attributes was refused: a plain cooperative launch
+    cudaGetLastError();
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, route_kernel<VPL, FAST_ESZ>, a);
+  }
+  return e;
 }
 
 }  // namespace
