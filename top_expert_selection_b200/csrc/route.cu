@@ -922,6 +922,16 @@ __global__ void __launch_bounds__((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneri
   // touches no global memory before the previous one has completed and its
   // writes are visible.  Without the launch attribute both are no-ops.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // bf16 fast path: the exact-sigmoid table needs no global memory, so all
+  // threads but thread 0 (which waits first and starts the logits copies)
+  // fill it before waiting
+  float* lut = nullptr;
+  if constexpr (FAST_ESZ == 2) {
+    lut = reinterpret_cast<float*>(smem + L.lut);
+    if (threadIdx.x > 0)
+      for (int i = threadIdx.x - 1; i < kLutEntries; i += blockDim.x - 1)
+        lut[i] = sigmoid_f32(bf16_bits_to_f32((uint16_t)lut_bits(i)));
+  }
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
   const uint32_t gen = barrier_generation(a.hdr);
@@ -952,14 +962,6 @@ __global__ void __launch_bounds__((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneri
     __syncthreads();
   }
   float* cand = reinterpret_cast<float*>(smem + L.cand + warp * cand_bytes_per_warp());
-  // bf16 fast path: exact-sigmoid table, filled while the logits stream in
-  float* lut = nullptr;
-  if constexpr (FAST_ESZ == 2) {
-    lut = reinterpret_cast<float*>(smem + L.lut);
-    for (int i = threadIdx.x; i < kLutEntries; i += blockDim.x)
-      lut[i] = sigmoid_f32(bf16_bits_to_f32((uint16_t)lut_bits(i)));
-    __syncthreads();
-  }
 
   // ---------------- phase 1: select ----------------
   uint32_t round = 0;
