@@ -121,6 +121,7 @@ __global__ void __launch_bounds__(kScoreThreads) aux_scores_kernel(int T, int E,
                                                                  int32_t* __restrict__ tpe, void* ws) {
   extern __shared__ int hist[];  // [E], then per warp 32 packed candidate keys
   const unsigned FULL = 0xffffffffu;
+  pdl_entry();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
   AuxWs w = aux_ws(ws, E);
@@ -265,6 +266,7 @@ __global__ void __launch_bounds__(kAuxThreads, 2) aux_loss_fwd_kernel(long long 
                                                                    void* ws) {
   extern __shared__ float tpe_s[];  // [E]
   __shared__ double red[kAuxWarps];
+  pdl_entry();
   __shared__ int last;
   WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
   AuxWs w = aux_ws(ws, E);
@@ -344,6 +346,7 @@ __global__ void __launch_bounds__(kAuxThreads) aux_loss_bwd_kernel(int T, int E,
                                                                    float* __restrict__ grad_probs,
                                                                    float* __restrict__ grad_logits) {
   extern __shared__ float gp_s[];  // [E] = g * C * tpe[e]
+  pdl_entry();
   const float g = *grad_loss;
   for (int e = threadIdx.x; e < E; e += blockDim.x) gp_s[e] = g * C * (float)tpe[e];
   __syncthreads();
@@ -442,9 +445,10 @@ extern "C" int moe_aux_scores(int32_t T, int32_t E, int32_t k, int32_t score_fn,
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   // histogram, then 32 packed candidate keys per warp
   const size_t smem = (size_t)((E + 1) & ~1) * sizeof(int) + (size_t)(kScoreThreads / 32) * 32 * 8;
-  MOE_VPL_SWITCH(vpl, (aux_scores_kernel<V><<<grid, kScoreThreads, smem, st>>>(T, E, k, score_fn, logits, probs,
-                                                                            routing_map, tokens_per_expert, ws)));
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  cudaError_t err = cudaSuccess;
+  MOE_VPL_SWITCH(vpl, (err = launch_pdl(aux_scores_kernel<V>, dim3(grid), dim3(kScoreThreads), smem, st, T, E, k,
+                                        score_fn, logits, probs, routing_map, tokens_per_expert, ws)));
+  return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 extern "C" int moe_aux_loss_fwd(int32_t T_rows, int32_t T_total, int32_t E, int32_t k, float coeff,
@@ -457,9 +461,10 @@ extern "C" int moe_aux_loss_fwd(int32_t T_rows, int32_t T_total, int32_t E, int3
   if (reinterpret_cast<uintptr_t>(probs) & 15) return MOE_ERR_INVALID_ARG;
   const double C = (double)coeff * (double)E / ((double)T_total * (double)k);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  aux_loss_fwd_kernel<<<kLossBlocks, kAuxThreads, (size_t)E * sizeof(float), st>>>((long long)T_rows * E, E, C, probs,
-                                                                                 tokens_per_expert, loss, ws);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  const cudaError_t err = launch_pdl(aux_loss_fwd_kernel, dim3(kLossBlocks), dim3(kAuxThreads),
+                                     (size_t)E * sizeof(float), st, (long long)T_rows * E, E, C, probs,
+                                     tokens_per_expert, loss, ws);
+  return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 extern "C" int moe_aux_loss_bwd(int32_t T_rows, int32_t T_total, int32_t E, int32_t k, float coeff,
@@ -474,8 +479,8 @@ extern "C" int moe_aux_loss_bwd(int32_t T_rows, int32_t T_total, int32_t E, int3
   const int grid = std::max(1, std::min((T_rows + kAuxWarps - 1) / kAuxWarps, sm_count() * 8));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const size_t smem = (size_t)E * sizeof(float);
-  MOE_VPL_SWITCH(vpl, (aux_loss_bwd_kernel<V><<<grid, kAuxThreads, smem, st>>>(T_rows, E, C, grad_loss, probs,
-                                                                               tokens_per_expert, grad_probs,
-                                                                               grad_logits)));
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  cudaError_t err = cudaSuccess;
+  MOE_VPL_SWITCH(vpl, (err = launch_pdl(aux_loss_bwd_kernel<V>, dim3(grid), dim3(kAuxThreads), smem, st, T_rows, E,
+                                        C, grad_loss, probs, tokens_per_expert, grad_probs, grad_logits)));
+  return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -386,6 +386,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t rank = cluster_rank();
+  pdl_entry();
   const int cid = blockIdx.x / a.CS;
   const int tg = cid / a.NG, ng = cid % a.NG;
   const int row0 = tg * TGS;                       // first token of the group
@@ -843,13 +844,20 @@ extern "C" int moe_rmsnorm_router_topk(int32_t T, int32_t H, int32_t E, int32_t 
   cfg.blockDim = dim3(kDecThreads);
   cfg.dynamicSmemBytes = plan.smem;
   cfg.stream = reinterpret_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = plan.CS;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel, a, xmap, wmap);
+  cfg.numAttrs = 2;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel, a, xmap, wmap);
+  if (e != cudaSuccess) {  // the pair of attributes was refused: a plain cluster launch
+    cudaGetLastError();
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, decode_kernel, a, xmap, wmap);
+  }
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -35,6 +35,7 @@ struct DispatchArgs {
 
 template <int KMAX>
 __global__ void __launch_bounds__(kDcThreads) dispatch_kernel(DispatchArgs a) {
+  pdl_entry();
   const int lane = threadIdx.x & 31;
   const long long warp_g = ((long long)blockIdx.x * kDcThreads + threadIdx.x) >> 5;
   const long long nwarps = ((long long)gridDim.x * kDcThreads) >> 5;
@@ -121,6 +122,7 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float* f) {
 // ELEMS = elements per 16-byte vector: 8 for bf16, 4 for fp32; KMAX bounds k
 template <int ELEMS, int KMAX>
 __global__ void __launch_bounds__(kDcThreads) combine_kernel(CombineArgs a) {
+  pdl_entry();
   const int lane = threadIdx.x & 31;
   const long long warp_g = ((long long)blockIdx.x * kDcThreads + threadIdx.x) >> 5;
   const long long nwarps = ((long long)gridDim.x * kDcThreads) >> 5;
@@ -223,13 +225,14 @@ extern "C" int moe_dispatch(int32_t T, int32_t H, int32_t k, int32_t dtype, cons
   a.max_padded = max_padded;
   const int grid = dc_grid(std::max<long long>(T, (max_padded + 31) / 32));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t err;
   if (k <= 2)
-    dispatch_kernel<2><<<grid, kDcThreads, 0, st>>>(a);
+    err = launch_pdl(dispatch_kernel<2>, dim3(grid), dim3(kDcThreads), 0, st, a);
   else if (k <= 8)
-    dispatch_kernel<8><<<grid, kDcThreads, 0, st>>>(a);
+    err = launch_pdl(dispatch_kernel<8>, dim3(grid), dim3(kDcThreads), 0, st, a);
   else
-    dispatch_kernel<32><<<grid, kDcThreads, 0, st>>>(a);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    err = launch_pdl(dispatch_kernel<32>, dim3(grid), dim3(kDcThreads), 0, st, a);
+  return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 extern "C" int moe_combine(int32_t T, int32_t H, int32_t k, int32_t dtype, const void* expert_out,
@@ -254,14 +257,15 @@ extern "C" int moe_combine(int32_t T, int32_t H, int32_t k, int32_t dtype, const
   a.vec_per_row = (int)(row_bytes / 16);
   const int grid = dc_grid(T);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t err;
   if (dtype == MOE_BF16) {
-    if (k <= 2) combine_kernel<8, 2><<<grid, kDcThreads, 0, st>>>(a);
-    else if (k <= 8) combine_kernel<8, 8><<<grid, kDcThreads, 0, st>>>(a);
-    else combine_kernel<8, 32><<<grid, kDcThreads, 0, st>>>(a);
+    if (k <= 2) err = launch_pdl(combine_kernel<8, 2>, dim3(grid), dim3(kDcThreads), 0, st, a);
+    else if (k <= 8) err = launch_pdl(combine_kernel<8, 8>, dim3(grid), dim3(kDcThreads), 0, st, a);
+    else err = launch_pdl(combine_kernel<8, 32>, dim3(grid), dim3(kDcThreads), 0, st, a);
   } else {
-    if (k <= 2) combine_kernel<4, 2><<<grid, kDcThreads, 0, st>>>(a);
-    else if (k <= 8) combine_kernel<4, 8><<<grid, kDcThreads, 0, st>>>(a);
-    else combine_kernel<4, 32><<<grid, kDcThreads, 0, st>>>(a);
+    if (k <= 2) err = launch_pdl(combine_kernel<4, 2>, dim3(grid), dim3(kDcThreads), 0, st, a);
+    else if (k <= 8) err = launch_pdl(combine_kernel<4, 8>, dim3(grid), dim3(kDcThreads), 0, st, a);
+    else err = launch_pdl(combine_kernel<4, 32>, dim3(grid), dim3(kDcThreads), 0, st, a);
   }
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
