@@ -301,44 +301,77 @@ def main():
     hbm, tflops, peak_kind = load_peaks()
     achieved = alg / (ms_step / 1000.0) / 1e9
 
-    # end to end through host buffers: pinned inputs -> device, route, outputs -> pinned host, every step
+    # end to end through host buffers, every step: pinned inputs -> device, route, outputs -> pinned host.
+    # The inputs (logits, bias) and the outputs (all nine) each live in one buffer, so a step is one
+    # host-to-device copy, one moe_route and one device-to-host copy.  Two slots on two streams (each with
+    # its own buffers and workspace), as a serving loop would run them: step i+1's host-to-device copy
+    # overlaps step i's route and its device-to-host copy; each slot's steps stay in order on its stream.
     e2e = None
     if rank == 0 or True:
-        h_logits = inp["logits"].pin_memory()
-        h_bias = inp["bias"].pin_memory()
-        r0 = routers[0]
         out_names = ("ids", "weights", "counts", "offsets", "e2p", "p2t", "tile_expert", "tile_mn_limit", "totals")
-        h_out = {n: torch.empty_like(r0.out[n], device="cpu").pin_memory() for n in out_names}
-        d_logits = logits[0]
-        d_bias = torch.empty_like(bias)
+        in_layout = [("logits", inp["logits"]), ("bias", inp["bias"])]
+        out_layout = [(n, routers[0].out[n]) for n in out_names]
+
+        def carve(buf, layout):
+            views, off = {}, 0
+            for name, like in layout:
+                nb = like.numel() * like.element_size()
+                views[name] = buf[off:off + nb].view(like.dtype).view(like.shape)
+                off = (off + nb + 255) // 256 * 256
+            return views
+
+        def nbytes(layout):
+            off = 0
+            for _, like in layout:
+                off = (off + like.numel() * like.element_size() + 255) // 256 * 256
+            return off
+
+        h_in = torch.empty(nbytes(in_layout), dtype=torch.uint8).pin_memory()
+        for name, t in carve(h_in, in_layout).items():
+            t.copy_(dict(in_layout)[name])
+        slots = []
+        for si in range(2):
+            d_in = torch.empty(nbytes(in_layout), dtype=torch.uint8, device=dev)
+            d_out = torch.empty(nbytes(out_layout), dtype=torch.uint8, device=dev)
+            slots.append({"stream": torch.cuda.Stream(dev), "ws": B.make_workspace(B.route_workspace_bytes(p), dev),
+                          "d_in": d_in, "in": carve(d_in, in_layout), "d_out": d_out, "out": carve(d_out, out_layout),
+                          "h_out": torch.empty(nbytes(out_layout), dtype=torch.uint8).pin_memory()})
         n_e2e = max(20, min(2000, args.steps // 10))
-        h2d = h_logits.numel() * h_logits.element_size() + h_bias.numel() * h_bias.element_size()
-        d2h = sum(h_out[n].numel() * h_out[n].element_size() for n in out_names)
+        h2d = sum(t.numel() * t.element_size() for _, t in in_layout)
+        d2h = sum(t.numel() * t.element_size() for _, t in out_layout)
 
-        def e2e_step():
-            d_logits.copy_(h_logits, non_blocking=True)
-            d_bias.copy_(h_bias, non_blocking=True)
-            o = r0(d_logits, d_bias)
-            for n in out_names:
-                h_out[n].copy_(o[n], non_blocking=True)
+        def e2e_step(i):
+            sl = slots[i & 1]
+            with torch.cuda.stream(sl["stream"]):
+                sl["d_in"].copy_(h_in, non_blocking=True)
+                B.route_into(p, sl["in"]["logits"], sl["in"]["bias"], sl["out"], sl["ws"], stream=sl["stream"])
+                sl["h_out"].copy_(sl["d_out"], non_blocking=True)
 
-        with torch.cuda.stream(stream):
-            for _ in range(5):
-                e2e_step()
+        main = torch.cuda.current_stream(dev)
+        for i in range(6):
+            e2e_step(i)
         torch.cuda.synchronize()
         if pg:
             pg.barrier()
         f0 = torch.cuda.Event(enable_timing=True)
         f1 = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            f0.record(stream)
-            for _ in range(n_e2e):
-                e2e_step()
-            f1.record(stream)
+        f0.record(main)
+        for sl in slots:
+            sl["stream"].wait_event(f0)
+        for i in range(n_e2e):
+            e2e_step(i)
+        for sl in slots:
+            main.wait_stream(sl["stream"])
+        f1.record(main)
         torch.cuda.synchronize()
         ms_e2e = max_over_ranks(f0.elapsed_time(f1) / n_e2e, pg, dev)
+        # the last step's outputs, read back on the host, are the device's
+        h_views = carve(slots[(n_e2e - 1) & 1]["h_out"], out_layout)
+        e2e_ok = all(torch.equal(h_views[n], routers[0].out[n].cpu()) for n in ("ids", "counts", "offsets", "totals"))
         e2e = {"value": whole_job_rate(world, spec.T, ms_e2e), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h), "ms_per_step": ms_e2e, "steps": n_e2e}
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": ms_e2e, "steps": n_e2e, "outputs_match": e2e_ok,
+               "pipeline": "2 slots on 2 streams; each step: 1 host-to-device copy of the inputs, moe_route, "
+                           "1 device-to-host copy of all outputs"}
 
     extra = None
     if rank == 0 and not args.no_extra:
