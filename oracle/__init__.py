@@ -54,6 +54,7 @@ def _lib():
         L.oracle_aux_scores.argtypes = [i32, i32, i32, i32, P, P, P, P]
         L.oracle_aux_loss_fwd.argtypes = [i32, i32, i32, i32, f32, P, P, P]
         L.oracle_aux_loss_bwd.argtypes = [i32, i32, i32, i32, f32, f32, P, P, P, P]
+        L.oracle_aux_scores_bwd.argtypes = [i32, i32, i32, P, P, P]
         L.oracle_dispatch.argtypes = [i32, i32, i32, P, P, P, i32, P]
         L.oracle_combine.argtypes = [i32, i32, i32, P, P, P, i32, P]
         L.oracle_rmsnorm_router_topk.argtypes = [i32, i32, i32, i32, f32, i32, P, P, P, P, P, P, P, P]
@@ -66,7 +67,7 @@ def _lib():
         L.oracle_f64_to_bf16.argtypes = [ctypes.c_double]
         L.oracle_f64_to_bf16.restype = ctypes.c_uint16
         for name in ("oracle_route_select", "oracle_route_capacity", "oracle_route_bookkeeping",
-                     "oracle_aux_scores", "oracle_aux_loss_fwd", "oracle_aux_loss_bwd",
+                     "oracle_aux_scores", "oracle_aux_loss_fwd", "oracle_aux_loss_bwd", "oracle_aux_scores_bwd",
                      "oracle_dispatch", "oracle_combine", "oracle_rmsnorm_router_topk"):
             getattr(L, name).restype = i32
         _lib_handle = L
@@ -207,6 +208,16 @@ def aux_loss_bwd(probs, tokens_per_expert, T_total: int, k: int, coeff: float, g
                                     _ptr(gp), _ptr(gl))
     _check(rc, "aux_loss_bwd")
     return {"grad_probs": gp, "grad_logits": gl}
+
+
+def aux_scores_bwd(probs, grad_probs, score_fn: int = 0) -> np.ndarray:
+    """dL/dlogits of the softmax aux scores given dL/dprobs (rows of probs sum to 1)."""
+    p = np.ascontiguousarray(as_numpy(probs), dtype=np.float32)
+    g = np.ascontiguousarray(as_numpy(grad_probs), dtype=np.float32)
+    T, E = p.shape
+    gl = np.zeros((T, E), np.float32)
+    _check(_lib().oracle_aux_scores_bwd(T, E, int(score_fn), _ptr(p), _ptr(g), _ptr(gl)), "aux_scores_bwd")
+    return gl
 
 
 def dispatch(hidden, e2p, p2t, P: int, max_padded: int, fill: int = 0xFFFF) -> np.ndarray:

@@ -408,6 +408,29 @@ int oracle_aux_loss_bwd(int T_rows, int T_total, int E, int k, float coeff, floa
 }
 
 /*
+ * Backward of the aux scores [TE: Description, fused_compute_score_for_moe_aux_loss
+ * forward and backward]: given dL/dprobs, dL/dlogits for the softmax scores
+ * probs = softmax(logits) per row:
+ *   grad_logits[t,e] = p[t,e] * (g[t,e] - sum_j p[t,j] * g[t,j])
+ * (the softmax Jacobian, written out); the sum and the product in double,
+ * rounded once.  score_fn SIGMOID: -2 (READING: the sigmoid scores normalised by
+ * their row sum need that sum, which the probs alone do not give).
+ */
+int oracle_aux_scores_bwd(int T, int E, int score_fn, const float* probs, const float* grad_probs,
+                          float* grad_logits) {
+  if (T < 0 || E <= 0) return -1;
+  if (score_fn != ORC_SOFTMAX) return -2;
+  for (int t = 0; t < T; ++t) {
+    const float* p = probs + (size_t)t * E;
+    const float* g = grad_probs + (size_t)t * E;
+    double dot = 0.0;
+    for (int e = 0; e < E; ++e) dot += (double)p[e] * (double)g[e];
+    for (int e = 0; e < E; ++e) grad_logits[(size_t)t * E + e] = (float)((double)p[e] * ((double)g[e] - dot));
+  }
+  return 0;
+}
+
+/*
  * Dispatch [LMD: invokeMoeDispatch]: copy each token's hidden row to each of
  * its k permuted rows; padding rows below P (p2t == -1) are zero (READING);
  * rows at or past P are left untouched.  Rows are raw 16-bit elements.

@@ -346,6 +346,48 @@ def test_aux_backward_finite_differences():
     np.testing.assert_allclose(gr["grad_logits"], fd, rtol=2e-5, atol=1e-7)
 
 
+def test_aux_scores_backward_finite_differences():
+    """aux_scores_bwd is the vector-Jacobian product of the softmax scores: for a fixed upstream
+    gradient G, grad_logits = d/dlogits of sum_t sum_e softmax(l_t)_e * G[t,e] (central differences of a
+    float64 softmax)."""
+    T, E = 5, 12
+    rng = np.random.default_rng(3)
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    G = rng.standard_normal((T, E)).astype(np.float32)
+    probs = oracle.aux_scores(lg, 2)["probs"]
+    gl = oracle.aux_scores_bwd(probs, G)
+
+    def f64(x):
+        z = np.exp(x - x.max(1, keepdims=True))
+        return float(((z / z.sum(1, keepdims=True)) * G.astype(np.float64)).sum())
+
+    x0 = lg.astype(np.float64)
+    h = 1e-6
+    fd = np.zeros_like(x0)
+    for t in range(T):
+        for e in range(E):
+            xp = x0.copy(); xp[t, e] += h
+            xm = x0.copy(); xm[t, e] -= h
+            fd[t, e] = (f64(xp) - f64(xm)) / (2 * h)
+    np.testing.assert_allclose(gl, fd, rtol=2e-5, atol=2e-7)
+
+
+def test_aux_scores_backward_special_cases():
+    """A constant upstream gradient moves no logit (softmax is shift-invariant); a one-hot upstream
+    gradient on expert j gives p_j * (1 - p_j) at j; sigmoid scores are refused."""
+    rng = np.random.default_rng(4)
+    lg = rng.standard_normal((4, 9)).astype(np.float32)
+    probs = oracle.aux_scores(lg, 2)["probs"]
+    z = oracle.aux_scores_bwd(probs, np.full_like(probs, 2.5))
+    assert np.all(np.abs(z) <= 1e-6 * probs)
+    onehot = np.zeros_like(probs)
+    onehot[:, 3] = 1.0
+    g1 = oracle.aux_scores_bwd(probs, onehot)
+    np.testing.assert_allclose(g1[:, 3], probs[:, 3].astype(np.float64) * (1 - probs[:, 3]), rtol=1e-6)
+    with pytest.raises(ValueError):
+        oracle.aux_scores_bwd(probs, onehot, score_fn=W.SIGMOID)
+
+
 def test_aux_sigmoid_scores_closed_forms():
     E = 8
     sc = oracle.aux_scores(np.zeros((2, E), np.float32), 2, score_fn=W.SIGMOID)
