@@ -473,7 +473,7 @@ def secondary_rows(dev, hbm):
         lg = alg.clone()
         ws = B.aux_workspace(a.T, a.E, dev)
         sc = B.aux_scores(lg, a.k, ws=ws)
-        sets.append((lg, ws, sc, torch.empty(1, device=dev), torch.empty_like(lg)))
+        sets.append((lg, ws, sc, torch.empty(1, device=dev), torch.empty_like(lg), torch.empty_like(lg)))
     gl = torch.ones(1, device=dev)
     rows["aux_scores_us"] = _time_calls(
         [(lambda z=z: B.aux_scores_into(z[0], a.k, z[2]["probs"], z[2]["routing_map"], z[2]["tokens_per_expert"],
@@ -484,6 +484,8 @@ def secondary_rows(dev, hbm):
     rows["aux_loss_bwd_us"] = _time_calls(
         [(lambda z=z: B.aux_loss_bwd_into(gl, z[2]["probs"], z[2]["tokens_per_expert"], a.T, a.k, a.coeff, None,
                                           z[4])) for z in sets], 20, stream)
+    rows["aux_scores_bwd_us"] = _time_calls(
+        [(lambda z=z: B.aux_scores_bwd_into(z[2]["probs"], z[4], z[5])) for z in sets], 20, stream)
     del sets
     # decode fused (T=128, H=7168, E=256, k=8): 24 rotated sets of hidden states and router weights
     d = W.DECODE_FUSED

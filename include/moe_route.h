@@ -213,6 +213,19 @@ int moe_aux_loss_fwd(int32_t T_rows, int32_t T_total, int32_t E, int32_t k, floa
                      size_t ws_bytes, void* stream);
 
 /*
+ * moe_aux_scores_bwd -- backward of the aux scores [TE: Description,
+ * fused_compute_score_for_moe_aux_loss, forward and backward]: given the
+ * upstream gradient with respect to the softmax probs,
+ *   grad_logits[t,e] = p[t,e] * (grad_probs[t,e] - sum_j p[t,j] grad_probs[t,j])
+ * probs, grad_probs, grad_logits [T,E] fp32 (probs as moe_aux_scores wrote
+ * them).  score_fn MOE_SIGMOID returns MOE_ERR_UNSUPPORTED: the sigmoid scores
+ * normalised by their row sum need that sum, which the probs do not carry.
+ * No workspace; returns MOE_ERR_INVALID_ARG for bad sizes or null pointers.
+ */
+int moe_aux_scores_bwd(int32_t T, int32_t E, int32_t score_fn, const float* probs, const float* grad_probs,
+                       float* grad_logits, void* stream);
+
+/*
  * moe_aux_loss_bwd -- gradient of the loss [TE: Description, forward and
  * backward].  With C = coeff * E / (T_total * k) and g = *grad_loss (device):
  *   grad_probs[t,e]  = g * C * tpe[e]                       (optional, may be NULL)

@@ -120,3 +120,28 @@ def test_aux_repeated_calls_reuse_workspace():
     l2 = B.aux_loss_fwd(a["probs"], a["tokens_per_expert"], 2000, 8, 0.01, ws=ws)
     assert torch.equal(l1, l2)
     assert B.status(ws) == B.MOE_OK
+
+
+@pytest.mark.parametrize("T,E", [(1, 8), (77, 33), (1000, 128), (32768, 128), (129, 1024)])
+def test_aux_scores_backward(T, E):
+    """moe_aux_scores_bwd against the oracle's vector-Jacobian product of the softmax, relative to the
+    terms before cancellation: |p_e*g_e| + |p_e| * sum_j |p_j*g_j| (the dot of a signed upstream
+    gradient cancels, so its fp32 rounding scales with the sum of the magnitudes of its terms)."""
+    g = torch.Generator().manual_seed(T * 7 + E)
+    lg = torch.randn(T, E, generator=g) * 1.5
+    G = torch.randn(T, E, generator=g)
+    probs = oracle.aux_scores(lg, 2)["probs"]
+    got = to_np(B.aux_scores_bwd(torch.from_numpy(probs).cuda(), G.cuda()))
+    torch.cuda.synchronize()
+    ref = oracle.aux_scores_bwd(probs, G)
+    p64 = probs.astype(np.float64)
+    terms = np.abs(p64 * G.double().numpy())
+    scale = terms + p64 * terms.sum(1, keepdims=True)
+    err = np.abs(got.astype(np.float64) - ref.astype(np.float64))
+    assert np.all(err <= RTOL * scale + 1e-30), f"err/scale max {np.max(err / (scale + 1e-30))}"
+
+
+def test_aux_scores_backward_sigmoid_unsupported():
+    p = torch.full((4, 8), 0.125, device="cuda")
+    with pytest.raises(Exception):
+        B.aux_scores_bwd(p, p, score_fn=W.SIGMOID)

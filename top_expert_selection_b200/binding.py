@@ -35,7 +35,7 @@ _TORCH = {F32: torch.float32, BF16: torch.bfloat16}
 # every symbol the C header declares (checked by the CPU test suite)
 EXPORTED = (
     "moe_error_string", "moe_workspace_init", "moe_status", "moe_route_capacity",
-    "moe_route_workspace_bytes", "moe_route", "moe_aux_workspace_bytes", "moe_aux_scores",
+    "moe_route_workspace_bytes", "moe_route", "moe_aux_workspace_bytes", "moe_aux_scores", "moe_aux_scores_bwd",
     "moe_aux_loss_fwd", "moe_aux_loss_bwd", "moe_dispatch", "moe_combine",
     "moe_rmsnorm_router_topk_workspace_bytes", "moe_rmsnorm_router_topk", "moe_debug_barrier_wait",
     "moe_debug_sigmoid_proxy_error", "moe_route_no_alloc",
@@ -87,6 +87,7 @@ def lib() -> ctypes.CDLL:
             "moe_aux_scores": ([i32, i32, i32, i32, P, P, P, P, P, sz, P], ctypes.c_int),
             "moe_aux_loss_fwd": ([i32, i32, i32, i32, f32, P, P, P, P, sz, P], ctypes.c_int),
             "moe_aux_loss_bwd": ([i32, i32, i32, i32, f32, P, P, P, P, P, P], ctypes.c_int),
+            "moe_aux_scores_bwd": ([i32, i32, i32, P, P, P, P], ctypes.c_int),
             "moe_dispatch": ([i32, i32, i32, i32, P, P, P, P, i64, P, P], ctypes.c_int),
             "moe_combine": ([i32, i32, i32, i32, P, P, P, i32, P, P], ctypes.c_int),
             "moe_rmsnorm_router_topk_workspace_bytes": ([i32, i32, i32, ctypes.POINTER(sz)], ctypes.c_int),
@@ -294,6 +295,20 @@ def aux_loss_bwd(grad_loss: torch.Tensor, probs: torch.Tensor, tokens_per_expert
     gl = torch.empty_like(probs)
     aux_loss_bwd_into(grad_loss, probs, tokens_per_expert, T_total, k, coeff, gp, gl)
     return {"grad_probs": gp, "grad_logits": gl}
+
+
+def aux_scores_bwd_into(probs: torch.Tensor, grad_probs: torch.Tensor, grad_logits: torch.Tensor,
+                        score_fn: int = SOFTMAX, stream=None) -> None:
+    T, E = probs.shape
+    _check(lib().moe_aux_scores_bwd(T, E, score_fn, _p(probs), _p(grad_probs), _p(grad_logits), _stream(stream)),
+           "moe_aux_scores_bwd")
+
+
+def aux_scores_bwd(probs: torch.Tensor, grad_probs: torch.Tensor, score_fn: int = SOFTMAX) -> torch.Tensor:
+    """dL/dlogits of the aux scores given dL/dprobs."""
+    gl = torch.empty_like(probs)
+    aux_scores_bwd_into(probs, grad_probs, gl, score_fn)
+    return gl
 
 
 # ---------------------------------------------------------------------------- dispatch / combine

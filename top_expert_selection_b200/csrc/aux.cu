@@ -392,6 +392,58 @@ __global__ void __launch_bounds__(kAuxThreads) aux_loss_bwd_kernel(int T, int E,
   }
 }
 
+// --------------------------------------------------------------------------
+// backward of the softmax scores: warp per row, dot = sum_j p_j g_j (fp32,
+// fixed order: lane partials then a shuffle tree), grad = p * (g - dot)
+// --------------------------------------------------------------------------
+template <int VPL>
+__global__ void __launch_bounds__(kAuxThreads) aux_scores_bwd_kernel(int T, int E, const float* __restrict__ probs,
+                                                                     const float* __restrict__ grad_probs,
+                                                                     float* __restrict__ grad_logits) {
+  pdl_entry();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const bool vec = (VPL % 4 == 0) && ((E & 3) == 0) && (lane * VPL + VPL <= E);
+  for (long long t = (long long)blockIdx.x * kAuxWarps + warp; t < T; t += (long long)gridDim.x * kAuxWarps) {
+    const float* prow = probs + t * E;
+    const float* grow = grad_probs + t * E;
+    float p[VPL], g[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int e = lane * VPL + i;
+      if (vec) {
+        if ((i & 3) == 0) {
+          const float4 a = __ldcs(reinterpret_cast<const float4*>(prow + e));
+          const float4 b = __ldcs(reinterpret_cast<const float4*>(grow + e));
+          p[i] = a.x; g[i] = b.x;
+          if (i + 1 < VPL) { p[i + 1] = a.y; g[i + 1] = b.y; }
+          if (i + 2 < VPL) { p[i + 2] = a.z; g[i + 2] = b.z; }
+          if (i + 3 < VPL) { p[i + 3] = a.w; g[i + 3] = b.w; }
+        }
+      } else {
+        p[i] = e < E ? __ldcs(prow + e) : 0.0f;
+        g[i] = e < E ? __ldcs(grow + e) : 0.0f;
+      }
+    }
+    float dot = 0.0f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) dot = fmaf(p[i], g[i], dot);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int e = lane * VPL + i;
+      if (vec) {
+        if ((i & 3) == 0 && i + 3 < VPL)
+          __stcs(reinterpret_cast<float4*>(grad_logits + t * E + e),
+                 make_float4(p[i] * (g[i] - dot), p[i + 1] * (g[i + 1] - dot), p[i + 2] * (g[i + 2] - dot),
+                             p[i + 3] * (g[i + 3] - dot)));
+      } else if (e < E) {
+        __stcs(grad_logits + t * E + e, p[i] * (g[i] - dot));
+      }
+    }
+  }
+}
+
 int sm_count() {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -464,6 +516,22 @@ extern "C" int moe_aux_loss_fwd(int32_t T_rows, int32_t T_total, int32_t E, int3
   const cudaError_t err = launch_pdl(aux_loss_fwd_kernel, dim3(kLossBlocks), dim3(kAuxThreads),
                                      (size_t)E * sizeof(float), st, (long long)T_rows * E, E, C, probs,
                                      tokens_per_expert, loss, ws);
+  return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+extern "C" int moe_aux_scores_bwd(int32_t T, int32_t E, int32_t score_fn, const float* probs,
+                                  const float* grad_probs, float* grad_logits, void* stream) {
+  if (T < 0 || E <= 0) return MOE_ERR_INVALID_ARG;
+  if (score_fn != MOE_SOFTMAX && score_fn != MOE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (score_fn != MOE_SOFTMAX || E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (!probs || !grad_probs || !grad_logits) return MOE_ERR_INVALID_ARG;
+  const int vpl = pick_vpl(E);
+  const int grid = std::max(1, std::min((T + kAuxWarps - 1) / kAuxWarps, sm_count() * 8));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t err = cudaSuccess;
+  MOE_VPL_SWITCH(vpl, (err = launch_pdl(aux_scores_bwd_kernel<V>, dim3(grid), dim3(kAuxThreads), 0, st, T, E, probs,
+                                        grad_probs, grad_logits)));
   return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
