@@ -55,6 +55,7 @@ def _lib():
         L.oracle_aux_loss_fwd.argtypes = [i32, i32, i32, i32, f32, P, P, P]
         L.oracle_aux_loss_bwd.argtypes = [i32, i32, i32, i32, f32, f32, P, P, P, P]
         L.oracle_aux_scores_bwd.argtypes = [i32, i32, i32, P, P, P]
+        L.oracle_route_weights_bwd.argtypes = [i32, i32, i32, i32, i32, i32, f32, P, P, P, P]
         L.oracle_dispatch.argtypes = [i32, i32, i32, P, P, P, i32, P]
         L.oracle_combine.argtypes = [i32, i32, i32, P, P, P, i32, P]
         L.oracle_rmsnorm_router_topk.argtypes = [i32, i32, i32, i32, f32, i32, P, P, P, P, P, P, P, P]
@@ -67,7 +68,7 @@ def _lib():
         L.oracle_f64_to_bf16.argtypes = [ctypes.c_double]
         L.oracle_f64_to_bf16.restype = ctypes.c_uint16
         for name in ("oracle_route_select", "oracle_route_capacity", "oracle_route_bookkeeping",
-                     "oracle_aux_scores", "oracle_aux_loss_fwd", "oracle_aux_loss_bwd", "oracle_aux_scores_bwd",
+                     "oracle_aux_scores", "oracle_aux_loss_fwd", "oracle_aux_loss_bwd", "oracle_aux_scores_bwd", "oracle_route_weights_bwd",
                      "oracle_dispatch", "oracle_combine", "oracle_rmsnorm_router_topk"):
             getattr(L, name).restype = i32
         _lib_handle = L
@@ -208,6 +209,21 @@ def aux_loss_bwd(probs, tokens_per_expert, T_total: int, k: int, coeff: float, g
                                     _ptr(gp), _ptr(gl))
     _check(rc, "aux_loss_bwd")
     return {"grad_probs": gp, "grad_logits": gl}
+
+
+def route_weights_bwd(logits, ids, grad_weights, *, score_fn: int, softmax_before_topk: int = 1,
+                      renormalize: int = 1, scaling_factor: float = 1.0) -> np.ndarray:
+    """dL/dlogits [T,E] for the routed weights of the given selection (fp32 logits)."""
+    lg = np.ascontiguousarray(as_numpy(logits), dtype=np.float32)
+    idv = np.ascontiguousarray(as_numpy(ids), dtype=np.int32)
+    gw = np.ascontiguousarray(as_numpy(grad_weights), dtype=np.float32)
+    T, E = lg.shape
+    k = idv.shape[1]
+    gl = np.zeros((T, E), np.float32)
+    _check(_lib().oracle_route_weights_bwd(T, E, k, int(score_fn), int(softmax_before_topk), int(renormalize),
+                                           float(scaling_factor), _ptr(lg), _ptr(idv), _ptr(gw), _ptr(gl)),
+           "route_weights_bwd")
+    return gl
 
 
 def aux_scores_bwd(probs, grad_probs, score_fn: int = 0) -> np.ndarray:

@@ -408,6 +408,81 @@ int oracle_aux_loss_bwd(int T_rows, int T_total, int E, int k, float coeff, floa
 }
 
 /*
+ * Backward of the routed weights [TE: Description, FusedTopkScoreFunction /
+ * fused_topk_with_score_function, forward and backward]: dL/dlogits given
+ * dL/dweights for the selection ids (the selection and the bias carry no
+ * gradient).  The forward, per token, with s_e = sigmoid(l_e) or p = softmax(l):
+ *   v_j = s_{e_j}                         (SIGMOID)
+ *   v_j = p_{e_j}                         (SOFTMAX, softmax before top-k)
+ *   v_j = softmax over the k selected l   (SOFTMAX, top-k on logits first)
+ *   w_j = scale * v_j / sum_i v_i (renormalize) or scale * v_j.
+ * Backward, written out in double and rounded once:
+ *   gv_i = scale * gw_i                                   (no renorm)
+ *   gv_i = scale / S * (gw_i - sum_j gw_j v_j / S)         (renorm, S = sum v)
+ *   SIGMOID:       gl_{e_j} += gv_j * v_j * (1 - v_j)
+ *   SOFTMAX pre:   gl_e = p_e * (sum_{j: e_j = e} gv_j - sum_j v_j gv_j)
+ *   SOFTMAX post:  gl_{e_j} = v_j * (gv_j - sum_i v_i gv_i)
+ * other entries 0.
+ */
+int oracle_route_weights_bwd(int T, int E, int k, int score_fn, int pre, int renorm, float scale,
+                             const float* logits, const int32_t* ids, const float* grad_w, float* grad_logits) {
+  if (T < 0 || E <= 0 || k <= 0 || k > E) return -1;
+  double* v = (double*)malloc(sizeof(double) * (size_t)k);
+  double* gv = (double*)malloc(sizeof(double) * (size_t)k);
+  double* p = (double*)malloc(sizeof(double) * (size_t)E);
+  double* gl = (double*)malloc(sizeof(double) * (size_t)E);
+  for (int t = 0; t < T; ++t) {
+    const float* l = logits + (size_t)t * E;
+    const int32_t* id = ids + (size_t)t * k;
+    const float* gw = grad_w + (size_t)t * k;
+    for (int j = 0; j < k; ++j)
+      if (id[j] < 0 || id[j] >= E) {
+        free(v); free(gv); free(p); free(gl);
+        return -1;
+      }
+    if (score_fn == ORC_SIGMOID) {
+      for (int j = 0; j < k; ++j) v[j] = 1.0 / (1.0 + exp(-(double)l[id[j]]));
+    } else if (pre) {
+      double m = l[0];
+      for (int e = 1; e < E; ++e) if (l[e] > m) m = l[e];
+      double z = 0.0;
+      for (int e = 0; e < E; ++e) { p[e] = exp((double)l[e] - m); z += p[e]; }
+      for (int e = 0; e < E; ++e) p[e] /= z;
+      for (int j = 0; j < k; ++j) v[j] = p[id[j]];
+    } else {
+      double m = l[id[0]];
+      for (int j = 1; j < k; ++j) if (l[id[j]] > m) m = l[id[j]];
+      double z = 0.0;
+      for (int j = 0; j < k; ++j) { v[j] = exp((double)l[id[j]] - m); z += v[j]; }
+      for (int j = 0; j < k; ++j) v[j] /= z;
+    }
+    if (renorm) {
+      double S = 0.0, dot = 0.0;
+      for (int j = 0; j < k; ++j) { S += v[j]; dot += (double)gw[j] * v[j]; }
+      for (int j = 0; j < k; ++j) gv[j] = (double)scale / S * ((double)gw[j] - dot / S);
+    } else {
+      for (int j = 0; j < k; ++j) gv[j] = (double)scale * (double)gw[j];
+    }
+    for (int e = 0; e < E; ++e) gl[e] = 0.0;
+    if (score_fn == ORC_SIGMOID) {
+      for (int j = 0; j < k; ++j) gl[id[j]] += gv[j] * v[j] * (1.0 - v[j]);
+    } else if (pre) {
+      double d = 0.0;
+      for (int j = 0; j < k; ++j) d += v[j] * gv[j];
+      for (int j = 0; j < k; ++j) gl[id[j]] += gv[j];
+      for (int e = 0; e < E; ++e) gl[e] = p[e] * (gl[e] - d);
+    } else {
+      double d = 0.0;
+      for (int j = 0; j < k; ++j) d += v[j] * gv[j];
+      for (int j = 0; j < k; ++j) gl[id[j]] = v[j] * (gv[j] - d);
+    }
+    for (int e = 0; e < E; ++e) grad_logits[(size_t)t * E + e] = (float)gl[e];
+  }
+  free(v); free(gv); free(p); free(gl);
+  return 0;
+}
+
+/*
  * Backward of the aux scores [TE: Description, fused_compute_score_for_moe_aux_loss
  * forward and backward]: given dL/dprobs, dL/dlogits for the softmax scores
  * probs = softmax(logits) per row:

@@ -372,6 +372,63 @@ def test_aux_scores_backward_finite_differences():
     np.testing.assert_allclose(gl, fd, rtol=2e-5, atol=2e-7)
 
 
+@pytest.mark.parametrize("score_fn,pre,renorm", [(W.SIGMOID, 1, 1), (W.SIGMOID, 1, 0), (W.SOFTMAX, 1, 1),
+                                                 (W.SOFTMAX, 1, 0), (W.SOFTMAX, 0, 1), (W.SOFTMAX, 0, 0)])
+def test_route_weights_backward_finite_differences(score_fn, pre, renorm):
+    """route_weights_bwd is d/dlogits of sum_t sum_j G[t,j] * w[t,j] for a fixed selection, where the
+    weights follow the forward's definition (score of the selected, optional renorm, times the scale);
+    central differences of a float64 forward written here from that definition."""
+    T, E, k, scale = 4, 10, 3, 2.5
+    rng = np.random.default_rng(11 + score_fn + 2 * pre + 4 * renorm)
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    ids = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    G = rng.standard_normal((T, k)).astype(np.float32)
+    got = oracle.route_weights_bwd(lg, ids, G, score_fn=score_fn, softmax_before_topk=pre, renormalize=renorm,
+                                   scaling_factor=scale)
+
+    def f64(x):
+        tot = 0.0
+        for t in range(T):
+            if score_fn == W.SIGMOID:
+                v = 1.0 / (1.0 + np.exp(-x[t, ids[t]]))
+            elif pre:
+                z = np.exp(x[t] - x[t].max())
+                v = (z / z.sum())[ids[t]]
+            else:
+                z = np.exp(x[t, ids[t]] - x[t, ids[t]].max())
+                v = z / z.sum()
+            w = scale * v / v.sum() if renorm else scale * v
+            tot += float((G[t].astype(np.float64) * w).sum())
+        return tot
+
+    x0 = lg.astype(np.float64)
+    h = 1e-6
+    fd = np.zeros_like(x0)
+    for t in range(T):
+        for e in range(E):
+            xp = x0.copy(); xp[t, e] += h
+            xm = x0.copy(); xm[t, e] -= h
+            fd[t, e] = (f64(xp) - f64(xm)) / (2 * h)
+    np.testing.assert_allclose(got, fd, rtol=2e-5, atol=2e-7)
+
+
+def test_route_weights_backward_zero_off_selection():
+    """Sigmoid and post-softmax weights depend only on the selected logits: the gradient is zero
+    elsewhere; renormalised post-softmax weights are the softmax itself (sum 1), so renorm changes nothing."""
+    rng = np.random.default_rng(5)
+    lg = rng.standard_normal((3, 8)).astype(np.float32)
+    ids = np.array([[1, 5], [0, 7], [6, 2]], np.int32)
+    G = rng.standard_normal((3, 2)).astype(np.float32)
+    for sf, pre in ((W.SIGMOID, 1), (W.SOFTMAX, 0)):
+        g = oracle.route_weights_bwd(lg, ids, G, score_fn=sf, softmax_before_topk=pre, renormalize=0)
+        mask = np.zeros_like(g, dtype=bool)
+        np.put_along_axis(mask, ids.astype(np.int64), True, axis=1)
+        assert np.all(g[~mask] == 0)
+    a = oracle.route_weights_bwd(lg, ids, G, score_fn=W.SOFTMAX, softmax_before_topk=0, renormalize=1)
+    b = oracle.route_weights_bwd(lg, ids, G, score_fn=W.SOFTMAX, softmax_before_topk=0, renormalize=0)
+    np.testing.assert_allclose(a, b, rtol=1e-6, atol=1e-9)
+
+
 def test_aux_scores_backward_special_cases():
     """A constant upstream gradient moves no logit (softmax is shift-invariant); a one-hot upstream
     gradient on expert j gives p_j * (1 - p_j) at j; sigmoid scores are refused."""
