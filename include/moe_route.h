@@ -213,6 +213,27 @@ int moe_aux_loss_fwd(int32_t T_rows, int32_t T_total, int32_t E, int32_t k, floa
                      size_t ws_bytes, void* stream);
 
 /*
+ * moe_route_weights_bwd -- backward of the routed weights [TE: Description,
+ * FusedTopkScoreFunction / fused_topk_with_score_function, forward and
+ * backward]: dL/dlogits [T,E] fp32 given dL/dweights [T,k] fp32 for the
+ * selection topk_ids [T,k] that moe_route returned with the same params
+ * (score_fn, softmax_before_topk, renormalize, scaling_factor; logits in
+ * logits_dtype).  The selection, the groups and the bias carry no gradient.
+ * With v_j the score of slot j (sigmoid of its logit; its softmax probability
+ * over all E; or the softmax over the k selected logits when top-k comes
+ * first), w_j = scale*v_j (/ sum_i v_i when renormalising):
+ *   gv_i = scale*gw_i, or scale/S*(gw_i - sum_j gw_j v_j / S) with S = sum v
+ *   sigmoid:       grad[e_j] = gv_j * v_j * (1 - v_j)
+ *   softmax first: grad[e]   = p_e * (gv at e - sum_j v_j gv_j), every e
+ *   top-k first:   grad[e_j] = v_j * (gv_j - sum_i v_i gv_i)
+ * and 0 elsewhere.  k <= 32.  ws (optional, >= 64 bytes) receives
+ * MOE_ERR_DEVICE_BOUNDS for an id outside [0, E).  Returns
+ * MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED for bad parameters.
+ */
+int moe_route_weights_bwd(const moe_route_params* p, const void* logits, const int32_t* topk_ids,
+                          const float* grad_weights, float* grad_logits, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * moe_aux_scores_bwd -- backward of the aux scores [TE: Description,
  * fused_compute_score_for_moe_aux_loss, forward and backward]: given the
  * upstream gradient with respect to the softmax probs,

@@ -264,3 +264,67 @@ def test_fast_path_group_ties_and_fallbacks():
     run_route(base.with_(n_group=0, topk_group=0, k=8, seed=25))
     # saturated sigmoids: many keys equal 1 + bias exactly
     run_route(base.with_(logit_std=40.0, seed=26))
+
+
+def _weights_bwd_magnitude(lg64, ids, G, score_fn, pre, renorm, scale):
+    """Error scale for the routed-weight backward: the same chain with every difference replaced by a
+    sum of magnitudes (the terms before cancellation), float64."""
+    T, E = lg64.shape
+    k = ids.shape[1]
+    mag = np.zeros((T, E))
+    for t in range(T):
+        x = lg64[t]
+        if score_fn == W.SIGMOID:
+            v = 1.0 / (1.0 + np.exp(-x[ids[t]]))
+        elif pre:
+            z = np.exp(x - x.max()); p = z / z.sum(); v = p[ids[t]]
+        else:
+            z = np.exp(x[ids[t]] - x[ids[t]].max()); v = z / z.sum()
+        g = np.abs(G[t].astype(np.float64))
+        gv = scale / v.sum() * (g + (g * v).sum() / v.sum()) if renorm else scale * g
+        D = (v * gv).sum()
+        if score_fn == W.SIGMOID:
+            mag[t, ids[t]] = gv * v * (1 - v)
+        elif pre:
+            gp = np.zeros(E); gp[ids[t]] = gv
+            mag[t] = p * (gp + D)
+        else:
+            mag[t, ids[t]] = v * (gv + D)
+    return mag
+
+
+@pytest.mark.parametrize("score_fn,pre,renorm,dtype,E,k", [
+    (W.SIGMOID, 1, 1, W.BF16, 256, 8), (W.SIGMOID, 1, 0, W.F32, 64, 6), (W.SOFTMAX, 1, 1, W.F32, 128, 8),
+    (W.SOFTMAX, 1, 0, W.BF16, 96, 4), (W.SOFTMAX, 0, 1, W.BF16, 8, 2), (W.SOFTMAX, 0, 0, W.F32, 33, 3),
+    (W.SIGMOID, 1, 1, W.F32, 1024, 32)])
+def test_route_weights_backward(score_fn, pre, renorm, dtype, E, k):
+    """moe_route_weights_bwd against the oracle, relative to the terms before cancellation."""
+    T, scale = 777, 2.5
+    g = torch.Generator().manual_seed(E + k + 10 * pre + renorm)
+    lg = torch.randn(T, E, generator=g) * 1.5
+    lg = lg.to(torch.bfloat16) if dtype == W.BF16 else lg
+    ids = torch.stack([torch.randperm(E, generator=g)[:k] for _ in range(T)]).to(torch.int32)
+    G = torch.randn(T, k, generator=g)
+    p = B.route_params(T, E, k, score_fn=score_fn, softmax_before_topk=pre, renormalize=renorm,
+                       scaling_factor=scale, logits_dtype=dtype)
+    ws = B.make_workspace(64, "cuda")
+    got = to_np(B.route_weights_bwd(p, lg.cuda(), ids.cuda(), G.cuda(), ws=ws))
+    torch.cuda.synchronize()
+    assert B.status(ws) == B.MOE_OK
+    lg32 = lg.float().numpy()
+    ref = oracle.route_weights_bwd(lg32, ids.numpy(), G.numpy(), score_fn=score_fn, softmax_before_topk=pre,
+                                   renormalize=renorm, scaling_factor=scale)
+    mag = _weights_bwd_magnitude(lg32.astype(np.float64), ids.numpy(), G.numpy(), score_fn, pre, renorm, scale)
+    err = np.abs(got.astype(np.float64) - ref.astype(np.float64))
+    assert np.all(err <= 1e-5 * mag + 1e-30), f"err/mag max {np.max(err / (mag + 1e-30))}"
+
+
+def test_route_weights_backward_bad_id_recorded():
+    """An id outside [0, E) is caught by the kernel's bounds check (clamped, status set)."""
+    p = B.route_params(4, 16, 2, score_fn=W.SIGMOID)
+    lg = torch.randn(4, 16, device="cuda")
+    ids = torch.tensor([[0, 1], [2, 3], [4, 16], [5, 6]], dtype=torch.int32, device="cuda")
+    ws = B.make_workspace(64, "cuda")
+    B.route_weights_bwd(p, lg, ids, torch.ones(4, 2, device="cuda"), ws=ws)
+    torch.cuda.synchronize()
+    assert B.status(ws) == B.MOE_ERR_DEVICE_BOUNDS

@@ -35,7 +35,7 @@ _TORCH = {F32: torch.float32, BF16: torch.bfloat16}
 # every symbol the C header declares (checked by the CPU test suite)
 EXPORTED = (
     "moe_error_string", "moe_workspace_init", "moe_status", "moe_route_capacity",
-    "moe_route_workspace_bytes", "moe_route", "moe_aux_workspace_bytes", "moe_aux_scores", "moe_aux_scores_bwd",
+    "moe_route_workspace_bytes", "moe_route", "moe_aux_workspace_bytes", "moe_aux_scores", "moe_aux_scores_bwd", "moe_route_weights_bwd",
     "moe_aux_loss_fwd", "moe_aux_loss_bwd", "moe_dispatch", "moe_combine",
     "moe_rmsnorm_router_topk_workspace_bytes", "moe_rmsnorm_router_topk", "moe_debug_barrier_wait",
     "moe_debug_sigmoid_proxy_error", "moe_route_no_alloc",
@@ -88,6 +88,7 @@ def lib() -> ctypes.CDLL:
             "moe_aux_loss_fwd": ([i32, i32, i32, i32, f32, P, P, P, P, sz, P], ctypes.c_int),
             "moe_aux_loss_bwd": ([i32, i32, i32, i32, f32, P, P, P, P, P, P], ctypes.c_int),
             "moe_aux_scores_bwd": ([i32, i32, i32, P, P, P, P], ctypes.c_int),
+            "moe_route_weights_bwd": ([RP, P, P, P, P, P, sz, P], ctypes.c_int),
             "moe_dispatch": ([i32, i32, i32, i32, P, P, P, P, i64, P, P], ctypes.c_int),
             "moe_combine": ([i32, i32, i32, i32, P, P, P, i32, P, P], ctypes.c_int),
             "moe_rmsnorm_router_topk_workspace_bytes": ([i32, i32, i32, ctypes.POINTER(sz)], ctypes.c_int),
@@ -224,6 +225,17 @@ def route_into(p: RouteParams, logits: torch.Tensor, bias: Optional[torch.Tensor
     rc = lib().moe_route(ctypes.byref(p), _p(logits), _p(bias), *[_p(out[n]) for n in names], _p(ws),
                          ctypes.c_size_t(ws.numel()), _stream(stream))
     _check(rc, "moe_route")
+
+
+def route_weights_bwd(p: RouteParams, logits: torch.Tensor, ids: torch.Tensor, grad_weights: torch.Tensor,
+                      ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """moe_route_weights_bwd: dL/dlogits [T,E] fp32 from dL/dweights [T,k] fp32 for the given selection."""
+    T, E = logits.shape
+    gl = torch.empty((T, E), dtype=torch.float32, device=logits.device)
+    _check(lib().moe_route_weights_bwd(ctypes.byref(p), _p(logits), _p(ids), _p(grad_weights), _p(gl), _p(ws),
+                                       ctypes.c_size_t(ws.numel() if ws is not None else 0), _stream(stream)),
+           "moe_route_weights_bwd")
+    return gl
 
 
 def route_workspace_bytes(p: RouteParams) -> int:

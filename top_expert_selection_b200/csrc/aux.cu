@@ -477,6 +477,109 @@ int pick_vpl(int E) {
 
 using namespace moe;
 
+// --------------------------------------------------------------------------
+// backward of the routed weights: warp per token; lane j < k holds slot j
+// (expert, upstream gradient, score); lane l writes row entries
+// [l*VPL, l*VPL + VPL).  fp32, fixed reduction orders.
+// --------------------------------------------------------------------------
+template <int VPL>
+__global__ void __launch_bounds__(kAuxThreads) route_weights_bwd_kernel(int T, int E, int k, int score_fn, int pre,
+                                                                        int renorm, float scale, const void* logits,
+                                                                        int logits_dtype, const int32_t* ids,
+                                                                        const float* grad_w, float* grad_logits,
+                                                                        WsHeader* hdr) {
+  pdl_entry();
+  const unsigned FULL = 0xffffffffu;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (long long t = (long long)blockIdx.x * kAuxWarps + warp; t < T; t += (long long)gridDim.x * kAuxWarps) {
+    const bool slot = lane < k;
+    int e = slot ? ids[t * k + lane] : 0;
+    if (slot && (unsigned)e >= (unsigned)E) {
+      if (hdr) record_bounds(hdr);
+      e = 0;
+    }
+    const float gw = slot ? grad_w[t * k + lane] : 0.0f;
+    const float xj = slot ? load_as_f32(logits, logits_dtype, (size_t)t * E + e) : -INFINITY;
+    // scores of the selected (v) and, for softmax before top-k, of the lane's row entries (p)
+    float v = 0.0f, pr[VPL];
+    float m = 0.0f, z = 0.0f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) pr[i] = 0.0f;
+    if (score_fn == MOE_SIGMOID) {
+      v = slot ? sigmoid_f32(xj) : 0.0f;
+    } else if (pre) {
+      float x[VPL];
+      m = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const int ee = lane * VPL + i;
+        x[i] = ee < E ? load_as_f32(logits, logits_dtype, (size_t)t * E + ee) : -INFINITY;
+        m = fmaxf(m, x[i]);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, off));
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        pr[i] = lane * VPL + i < E ? expf(x[i] - m) : 0.0f;
+        z += pr[i];
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(FULL, z, off);
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) pr[i] = pr[i] / z;
+      v = slot ? expf(xj - m) / z : 0.0f;
+    } else {
+      m = xj;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, off));
+      const float ex = slot ? expf(xj - m) : 0.0f;
+      z = ex;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(FULL, z, off);
+      v = slot ? ex / z : 0.0f;
+    }
+    // renormalisation and scale
+    float gv;
+    if (renorm) {
+      float S = v, dot = gw * v;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        S += __shfl_xor_sync(FULL, S, off);
+        dot += __shfl_xor_sync(FULL, dot, off);
+      }
+      gv = slot ? scale / S * (gw - dot / S) : 0.0f;
+    } else {
+      gv = slot ? scale * gw : 0.0f;
+    }
+    float D = v * gv;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) D += __shfl_xor_sync(FULL, D, off);
+    // per-slot contributions (the selected experts of a token are distinct)
+    float g;
+    if (score_fn == MOE_SIGMOID) g = gv * v * (1.0f - v);
+    else if (pre) g = gv;  // gp at the selected expert; the row entries add p * (gp - D) below
+    else g = v * (gv - D);
+    float acc[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) acc[i] = 0.0f;
+    for (int j = 0; j < k; ++j) {
+      const int ej = __shfl_sync(FULL, e, j);
+      const float gj = __shfl_sync(FULL, g, j);
+      if (ej / VPL == lane) {
+#pragma unroll
+        for (int i = 0; i < VPL; ++i)
+          if (ej - lane * VPL == i) acc[i] = gj;
+      }
+    }
+    float* grow = grad_logits + t * E;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int ee = lane * VPL + i;
+      if (ee < E) __stcs(grow + ee, (score_fn != MOE_SIGMOID && pre) ? pr[i] * (acc[i] - D) : acc[i]);
+    }
+  }
+}
+
 extern "C" int moe_aux_workspace_bytes(int32_t num_tokens, int32_t num_experts, size_t* bytes) {
   if (num_tokens < 0 || num_experts <= 0 || !bytes) return MOE_ERR_INVALID_ARG;
   if (num_experts > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
@@ -532,6 +635,29 @@ extern "C" int moe_aux_scores_bwd(int32_t T, int32_t E, int32_t score_fn, const 
   cudaError_t err = cudaSuccess;
   MOE_VPL_SWITCH(vpl, (err = launch_pdl(aux_scores_bwd_kernel<V>, dim3(grid), dim3(kAuxThreads), 0, st, T, E, probs,
                                         grad_probs, grad_logits)));
+  return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+extern "C" int moe_route_weights_bwd(const moe_route_params* p, const void* logits, const int32_t* topk_ids,
+                                     const float* grad_weights, float* grad_logits, void* ws, size_t ws_bytes,
+                                     void* stream) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  const int T = p->num_tokens, E = p->num_experts, k = p->top_k;
+  if (T < 0 || E <= 0 || k <= 0 || k > E) return MOE_ERR_INVALID_ARG;
+  if (p->score_fn != MOE_SOFTMAX && p->score_fn != MOE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (p->logits_dtype != MOE_F32 && p->logits_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (E > MOE_MAX_EXPERTS || k > 32) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (!logits || !topk_ids || !grad_weights || !grad_logits) return MOE_ERR_INVALID_ARG;
+  if (ws && ws_bytes < sizeof(WsHeader)) return MOE_ERR_WORKSPACE;
+  const int vpl = pick_vpl(E);
+  const int grid = std::max(1, std::min((T + kAuxWarps - 1) / kAuxWarps, sm_count() * 8));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t err = cudaSuccess;
+  MOE_VPL_SWITCH(vpl, (err = launch_pdl(route_weights_bwd_kernel<V>, dim3(grid), dim3(kAuxThreads), 0, st, T, E, k,
+                                        p->score_fn, p->softmax_before_topk ? 1 : 0, p->renormalize ? 1 : 0,
+                                        p->scaling_factor, logits, p->logits_dtype, topk_ids, grad_weights,
+                                        grad_logits, reinterpret_cast<WsHeader*>(ws))));
   return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
