@@ -308,10 +308,11 @@ int moe_rmsnorm_router_topk_workspace_bytes(int32_t T, int32_t H, int32_t E, siz
  * affinities [T,E] -- bf16; ids [T,k] int32; debug_logits [T,E] fp32 or NULL
  * (receives the logits when given).  T <= 128 and H % 128 == 0 [NKI: Notes];
  * this build also needs E % 16 == 0, E <= 256 and H <= 32768, and every
- * pointer 16-byte aligned.  The launch is a grid of thread-block clusters
- * (16 CTAs each where the GPU can place them, else 8) that never wait on one
- * another; device-side waits are bounded and a wait that gives up leaves
- * MOE_ERR_DEVICE_TIMEOUT in the workspace status word (outputs undefined).
+ * pointer 16-byte aligned.  Two launches: a row-parallel RMSNorm writing
+ * out_norm, then the projection + top-k on thread-block clusters (sized per
+ * GPU) that read out_norm and never wait on one another; device-side waits are
+ * bounded and a wait that gives up leaves MOE_ERR_DEVICE_TIMEOUT in the
+ * workspace status word (outputs undefined).
  * Returns MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED / MOE_ERR_WORKSPACE for
  * bad arguments, MOE_ERR_CUDA when the launch fails.  Calls sharing one
  * workspace must not overlap in time.

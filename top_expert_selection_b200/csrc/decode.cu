@@ -8,40 +8,40 @@
 // Returns, Notes (T <= 128; H % 128 == 0; ACT2: top-K on raw logits, then the
 // activation on the selected experts only).
 //
-// Work split: thread-block clusters of CS CTAs.  A cluster owns one group of
-// tokens (64, or all T <= 128) and one group of 64 experts over the whole
-// hidden dimension; CTA j of the cluster owns the j-th K-slice (a run of
-// 64-column chunks).  CS (1..16) and the token group size are chosen per GPU
-// from how many clusters of each size it can keep resident: the fewest
-// staged bytes per CTA with every cluster resident at once.  For T=128,
-// H=7168, E=256 that is e.g. 4 clusters x 16 CTAs (448 columns each) or
-// 8 clusters x 14 CTAs (512 columns, 64 tokens).
+// Two launches.
 //
-//   stage    x chunks (tokens x 64 columns) first, then gamma, then W chunks
-//            (64 rows x 64 experts) -> shared memory by TMA, 128-byte swizzle
-//            (the canonical K-major A / MN-major B layouts of tcgen05.mma); a
-//            ring of up to 8 chunk stages, refilled when the slice is longer.
-//   sum x^2  per token over the CTA's slice (double, from the staged chunks),
-//            exchanged through distributed shared memory after a cluster
-//            barrier; every CTA adds the CS partials in rank order and forms
-//            r_t = 1/sqrt(mean + eps) in double (all CTAs get the same bits),
-//            kept as r_hi + r_lo in fp32.
-//   project  the staged chunks are normalised in place: x*gamma is exact in
-//            fp32, its product with r_hi is rounded to fp32 and then to bf16;
-//            where that fp32 value sits exactly on a bf16 rounding midpoint
-//            the sign of the remainder (x*gamma*r_hi - p + x*gamma*r_lo, from
-//            two fused multiply-adds) picks the side, so the bf16 value is the
-//            single rounding of x*gamma*r.  One cluster per chunk also stores
-//            it to out_norm; one thread issues the M=128 x N=64 x K=16 MMAs.
-//   reduce   TMEM -> registers -> shared memory; after a cluster barrier CTA j
-//            adds its tokens' partial logits over the CS ranks (rank order) and
-//            stores the fp32 logits of its (tokens, experts) tile.
-//   select   a per-(token group, rank) ticket: the last of the expert-group
-//            clusters to store its tile (no waiting) adds the bias, takes the
-//            top-k on the raw logits (ties -> lower expert) and writes ids and
-//            the masked bf16 affinities, then resets the ticket.
+//   K1 rmsnorm_kernel, a block per token: the sum of exact squares of the row
+//   in double, r_t = 1/sqrt(mean + eps) in double (kept as r_hi + r_lo in
+//   fp32), then each x*gamma*r rounded once to bf16: x*gamma is exact in fp32,
+//   its product with r_hi is rounded to fp32 and then to bf16; where that fp32
+//   value is a bf16 rounding midpoint or one fp32 ulp from one, the side is
+//   taken from the remainder (x*gamma*r_hi - p + x*gamma*r_lo, two fused
+//   multiply-adds), so the bf16 value is the single rounding of x*gamma*r.
+//   The result is out_norm.
+//
+//   K2 decode_kernel (programmatic dependent launch after K1), thread-block
+//   clusters of CS CTAs.  A cluster owns one group of tokens (64, or all
+//   T <= 128) and one group of 64 experts over the whole hidden dimension; CTA
+//   j owns the j-th K-slice (a run of 64-column chunks).  CS (1..16) and the
+//   token group size are chosen per GPU from how many clusters of each size it
+//   can keep resident: the fewest staged bytes per CTA with every cluster
+//   resident at once (T=128, H=7168, E=256: 4 clusters x 16 CTAs).
+//     stage    out_norm chunks (tokens x 64 columns) and W chunks (64 rows x
+//              64 experts) -> shared memory by 2-D TMA, 128-byte swizzle (the
+//              canonical K-major A / MN-major B layouts of tcgen05.mma); a
+//              ring of up to 8 chunk stages, refilled when the slice is longer.
+//     project  one thread issues each chunk's M=128 x N=64 x K=16 MMAs into
+//              TMEM as soon as the chunk has landed.
+//     reduce   TMEM -> registers -> pushed into the shared memory of the CTA
+//              that reduces those rows (st.shared::cluster); after one cluster
+//              barrier CTA j adds the CS partials of its rows in rank order and
+//              stores the fp32 logits of its (tokens, experts) tile.
+//     select   a per-(token group, rank) ticket: the last of the expert-group
+//              clusters to store its tile (no waiting) adds the bias, takes
+//              the top-k on the raw logits (ties -> lower expert) and writes
+//              ids and the masked bf16 affinities, then resets the ticket.
 // No grid-wide barrier, no cooperative launch: clusters never wait on one
-// another, so the kernel also completes when the clusters run in waves.
+// another, so K2 also completes when the clusters run in waves.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -93,18 +93,15 @@ struct DecLayout {
   int a, b, red, gam, psq, rs, bars, slot, flag, total;
 };
 // red: partial logits pushed by every CTA of the cluster for the rows this CTA
-// reduces, [CS][tpb][kRedStride] fp32; psq: partial sums of squares pushed by
-// every CTA, [CS][TGS] double.
+// reduces, [CS][tpb][kRedStride] fp32.
 __host__ __device__ inline int dec_tpb(int TGS, int CS) { return (TGS + CS - 1) / CS; }
-__host__ __device__ inline DecLayout dec_layout(int S, int maxb, int TGS, int CS) {
+__host__ __device__ inline DecLayout dec_layout(int S, int /*maxb*/, int TGS, int CS) {
   DecLayout L;
   L.a = 0;
   L.b = L.a + S * kATile;
   L.red = L.b + S * kBTile;
-  L.gam = L.red + CS * dec_tpb(TGS, CS) * kRedStride * 4;
-  L.psq = L.gam + ((maxb * kChunk * 2 + 15) & ~15);
-  L.rs = L.psq + CS * TGS * 8;
-  L.bars = L.rs + TGS * 8;
+  L.gam = L.psq = L.rs = 0;  // (unused)
+  L.bars = L.red + CS * dec_tpb(TGS, CS) * kRedStride * 4;
   L.slot = L.bars + (3 * kMaxStages + 2) * 8;
   L.flag = L.slot + 16;
   L.total = L.flag + 16;
@@ -199,9 +196,6 @@ __device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
   return r;
 }
 // stores into another CTA's shared memory (made visible by the next cluster barrier)
-__device__ __forceinline__ void st_cluster_f64(uint32_t addr, double v) {
-  asm volatile("st.shared::cluster.f64 [%0], %1;" ::"r"(addr), "d"(v) : "memory");
-}
 __device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
   asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                : "memory");
@@ -362,6 +356,70 @@ __device__ void select_token(const DecodeArgs& a, int t, int lane) {
   }
 }
 
+// K1: RMSNorm, a block per token row.  Sum of exact squares in double (a fixed
+// order: thread partials, a shuffle tree, warps in order), r = 1/sqrt(mean +
+// eps) in double kept as r_hi + r_lo, then x*gamma*r rounded once to bf16
+// (normalize8 / normalize8_exact) into out_norm.
+constexpr int kNormThreads = 256;
+constexpr int kNormKeep = 4;  // 16-byte groups a thread keeps in registers (H <= 8192)
+
+__global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const DecodeArgs a) {
+  __shared__ double red[kNormThreads / 32];
+  __shared__ float2 rr;
+  pdl_entry();
+  const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nq = a.H / 8;  // 16-byte groups in a row
+  const uint16_t* xr = a.x + (size_t)t * a.H;
+  uint4 keep[kNormKeep];
+  double acc = 0.0;
+#pragma unroll
+  for (int j = 0; j < kNormKeep; ++j) {
+    const int qq = tid + j * kNormThreads;
+    keep[j] = qq < nq ? __ldg(reinterpret_cast<const uint4*>(xr) + qq) : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int j = 0; j < kNormKeep; ++j) acc += sumsq8(keep[j]);
+  for (int qq = tid + kNormKeep * kNormThreads; qq < nq; qq += kNormThreads)
+    acc += sumsq8(__ldg(reinterpret_cast<const uint4*>(xr) + qq));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) red[warp] = acc;
+  __syncthreads();
+  if (tid == 0) {
+    double ss = 0.0;
+    for (int w = 0; w < kNormThreads / 32; ++w) ss += red[w];
+    const double r = 1.0 / sqrt(ss / (double)a.H + (double)a.eps);
+    const float rh = (float)r;
+    rr = make_float2(rh, (float)(r - (double)rh));
+  }
+  __syncthreads();
+  const float2 r2 = rr;
+  uint16_t* orow = a.out_norm + (size_t)t * a.H;
+  auto normalise = [&](int qq, uint4 xv) {
+    const uint4 gv = __ldg(reinterpret_cast<const uint4*>(a.gamma) + qq);
+    const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+    float g[8];
+    unsigned long long g2[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      g[2 * i] = __uint_as_float(gw[i] << 16);
+      g[2 * i + 1] = __uint_as_float(gw[i] & 0xffff0000u);
+      g2[i] = pack2(g[2 * i], g[2 * i + 1]);
+    }
+    uint4 o;
+    if (normalize8(xv, g2, r2.x, &o)) o = normalize8_exact(xv, g, r2.x, r2.y);  // a bf16 midpoint (rare)
+    reinterpret_cast<uint4*>(orow)[qq] = o;
+  };
+#pragma unroll
+  for (int j = 0; j < kNormKeep; ++j)
+    if (tid + j * kNormThreads < nq) normalise(tid + j * kNormThreads, keep[j]);
+  for (int qq = tid + kNormKeep * kNormThreads; qq < nq; qq += kNormThreads)
+    normalise(qq, __ldg(reinterpret_cast<const uint4*>(xr) + qq));
+}
+
+// K2: router projection + top-k on thread-block clusters (see the file head):
+// staged out_norm and W chunks, M=128 x N=64 x K=16 MMAs per chunk as soon as
+// both land, partial logits pushed to the reducing CTA, the ticketed top-k.
 __global__ void __launch_bounds__(kDecThreads, 1)
     decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap xmap,
                   const __grid_constant__ CUtensorMap wmap) {
@@ -373,14 +431,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   uint8_t* sA = smem + L.a;
   uint8_t* sB = smem + L.b;
   float* red = reinterpret_cast<float*>(smem + L.red);
-  uint16_t* gam = reinterpret_cast<uint16_t*>(smem + L.gam);
-  double* psq = reinterpret_cast<double*>(smem + L.psq);
-  float2* rs = reinterpret_cast<float2*>(smem + L.rs);
-  uint64_t* fullx = reinterpret_cast<uint64_t*>(smem + L.bars);  // x chunk landed
+  uint64_t* fullx = reinterpret_cast<uint64_t*>(smem + L.bars);  // normalised rows landed
   uint64_t* fullw = fullx + kMaxStages;                          // W chunk landed
   uint64_t* empty = fullw + kMaxStages;                          // the stage's MMAs are done
   uint64_t* mma_bar = empty + kMaxStages;
-  uint64_t* gam_bar = mma_bar + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.slot);
   int* flag = reinterpret_cast<int*>(smem + L.flag);
 
@@ -396,30 +450,21 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const int nb = (int)((long long)a.nch * (rank + 1) / a.CS) - c0;  // chunks of this CTA (>= 1)
   const int S = a.S;
   const int nres = min(S, nb);
-  const uint32_t x_tx = (uint32_t)(TGS * 128);
+  const uint32_t stage_tx = (uint32_t)(TGS * 128 + kBTile);
 
   int issued = 0;  // chunks whose copies have been issued (thread 0)
   if (tid == 0) {
     for (int s = 0; s < kMaxStages; ++s) {
       mbar_init(fullx + s, 1);
-      mbar_init(fullw + s, 1);
       mbar_init(empty + s, 1);
     }
     mbar_init(mma_bar, 1);
-    mbar_init(gam_bar, 1);
     flag[0] = 0;
-    // x first (the sums of squares wait for it), then gamma, then W (needed by the MMAs only)
-    for (int i = 0; i < nres; ++i) {
-      mbar_arrive_expect_tx(fullx + i, x_tx);
-      tma_load_2d(sA + i * kATile, &xmap, (c0 + i) * kChunk, row0, fullx + i);
+    for (; issued < nres; ++issued) {
+      mbar_arrive_expect_tx(fullx + issued, stage_tx);
+      tma_load_2d(sA + issued * kATile, &xmap, (c0 + issued) * kChunk, row0, fullx + issued);
+      tma_load_2d(sB + issued * kBTile, &wmap, e0, (c0 + issued) * kChunk, fullx + issued);
     }
-    mbar_arrive_expect_tx(gam_bar, (uint32_t)(nb * kChunk * 2));
-    bulk_g2s(gam, a.gamma + (size_t)c0 * kChunk, (uint32_t)(nb * kChunk * 2), gam_bar);
-    for (int i = 0; i < nres; ++i) {
-      mbar_arrive_expect_tx(fullw + i, (uint32_t)kBTile);
-      tma_load_2d(sB + i * kBTile, &wmap, e0, (c0 + i) * kChunk, fullw + i);
-    }
-    issued = nres;
   }
   if (warp == 0) tmem_alloc(tmem_slot, 64);
   // with 64-token groups, A rows 64..127 are zero in every stage (the TMA box fills rows 0..63)
@@ -428,162 +473,67 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       const int s = i / ((kM - TGS) * 8), off = i % ((kM - TGS) * 8);
       *reinterpret_cast<uint4*>(sA + s * kATile + TGS * 128 + off * 16) = make_uint4(0, 0, 0, 0);
     }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // every CTA of the cluster must be running before any CTA writes into its
+  // shared memory: arrive now, wait before the first push
+  cluster_arrive();
 
-  // ---------------- sum of squares over the slice ----------------
-  // TPT = 512/TGS threads per token row; part p reads 16-byte groups p, p+TPT, ..
-  // of each chunk row (conflict-free under the swizzle)
-  {
-    const int TPT = kDecThreads / TGS;  // 8 or 4
-    const int r = tid / TPT, part = tid % TPT;
-    double acc = 0.0;
-    bool waited = true;
-    for (int i = 0; i < nres; ++i) {
-      if (!mbar_wait_bounded(fullx + i, 0, a.timeout_ns)) {
-        waited = false;
-        break;
-      }
-      const uint8_t* rowp = sA + i * kATile + r * 128;
-      for (int qq = part; qq < 8; qq += TPT) acc += sumsq8(*reinterpret_cast<const uint4*>(rowp + ((qq ^ (r & 7)) << 4)));
-    }
-    if (!waited) {
-      record_timeout(a.hdr);
-      flag[0] = 1;
-    }
-    // chunks beyond the ring (long slices): straight from global memory
-    if (nb > nres && row0 + r < a.T) {
-      const uint16_t* xr = a.x + (size_t)(row0 + r) * a.H;
-      for (int i = nres; i < nb; ++i)
-        for (int qq = part; qq < 8; qq += TPT)
-          acc += sumsq8(__ldg(reinterpret_cast<const uint4*>(xr + (c0 + i) * kChunk + qq * 8)));
-    }
-    for (int off = 1; off < TPT; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    // every CTA of the cluster receives this partial in slot [rank][r]
-    const uint32_t dst = smem_addr(psq + (int)rank * TGS + r);
-    for (int j = part; j < a.CS; j += TPT) st_cluster_f64(cluster_map(dst, (uint32_t)j), acc);
-  }
-  cluster_sync();
-  if (tid < TGS) {
-    // the CS partial sums in rank order: identical bits in every CTA
-    double v[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] = j < a.CS ? psq[j * TGS + tid] : 0.0;
-    double s = 0.0;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) s += v[j];
-    const double r = 1.0 / sqrt(s / (double)a.H + (double)a.eps);
-    const float rh = (float)r;
-    rs[tid] = make_float2(rh, (float)(r - (double)rh));
-  }
-  if (!mbar_wait_bounded(gam_bar, 0, a.timeout_ns)) {
-    record_timeout(a.hdr);
-    flag[0] = 1;
-  }
-  __syncthreads();
-  bool ok = flag[0] == 0;
-
-  // ---------------- normalise in place, project (rounds of up to S chunks) ----------------
-  const uint32_t idesc = idesc_bf16_f32(N);
-  bool mma_issued = false;
-  const int q = tid & 7;  // the thread's 16-byte group in every chunk row
-  for (int i0 = 0; i0 < nb && ok; i0 += S) {
-    const int i1 = min(nb, i0 + S);
-    for (int i = i0; i < i1; ++i) {
+  // ---------------- project: one thread issues each chunk's MMAs as it lands ----------------
+  if (tid == 0) {
+    const uint32_t idesc = idesc_bf16_f32(N);
+    bool mma_issued = false;
+    for (int i = 0; i < nb; ++i) {
       const int s = i % S;
-      if (i >= nres && !mbar_wait_bounded(fullx + s, (uint32_t)(i / S) & 1u, a.timeout_ns)) {
+      const uint32_t ph = (uint32_t)(i / S) & 1u;
+      if (!mbar_wait_bounded(fullx + s, ph, a.timeout_ns)) {
         record_timeout(a.hdr);
         flag[0] = 1;
+        break;
       }
-      const int chunk = c0 + i;
-      const bool writer = (chunk % a.NG) == ng;  // one expert-group cluster stores each out_norm chunk
-      unsigned long long g2[4];
-      float g[8];
-      {
-        const uint4 gv = *reinterpret_cast<const uint4*>(gam + i * kChunk + q * 8);
-        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          g[2 * j] = __uint_as_float(gw[j] << 16);
-          g[2 * j + 1] = __uint_as_float(gw[j] & 0xffff0000u);
-          g2[j] = pack2(g[2 * j], g[2 * j + 1]);
-        }
-      }
-      // rows tid/8 and tid/8 + 64 of the chunk (the second only for 128-token groups)
-      const int r0 = tid >> 3, r1 = r0 + 64;
-      uint8_t* p0 = sA + s * kATile + r0 * 128 + ((q ^ (r0 & 7)) << 4);
-      uint8_t* p1 = sA + s * kATile + r1 * 128 + ((q ^ (r1 & 7)) << 4);
-      const bool two = r1 < TGS;
-      const uint4 x0 = *reinterpret_cast<const uint4*>(p0);
-      const uint4 x1 = two ? *reinterpret_cast<const uint4*>(p1) : make_uint4(0, 0, 0, 0);
-      const float2 rr0 = rs[r0], rr1 = rs[two ? r1 : r0];
-      uint4 o0, o1;
-      const bool m0 = normalize8(x0, g2, rr0.x, &o0);
-      const bool m1 = normalize8(x1, g2, rr1.x, &o1);
-      if (m0 | m1) {  // a bf16 rounding midpoint: settle it with the remainder (rare)
-        if (m0) o0 = normalize8_exact(x0, g, rr0.x, rr0.y);
-        if (m1) o1 = normalize8_exact(x1, g, rr1.x, rr1.y);
-      }
-      *reinterpret_cast<uint4*>(p0) = o0;
-      if (two) *reinterpret_cast<uint4*>(p1) = o1;
-      if (writer) {
-        const size_t col = (size_t)chunk * kChunk + q * 8;
-        if (row0 + r0 < a.T) *reinterpret_cast<uint4*>(a.out_norm + (size_t)(row0 + r0) * a.H + col) = o0;
-        if (two && row0 + r1 < a.T) *reinterpret_cast<uint4*>(a.out_norm + (size_t)(row0 + r1) * a.H + col) = o1;
-      }
-    }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    __syncthreads();
-    if (tid == 0 && flag[0] == 0) {
       tc_fence_after();
-      for (int i = i0; i < i1; ++i) {
-        const int s = i % S;
-        if (!mbar_wait_bounded(fullw + s, (uint32_t)(i / S) & 1u, a.timeout_ns)) {
-          record_timeout(a.hdr);
-          flag[0] = 1;
-          break;
-        }
-        const uint32_t aBase = smem_addr(sA + s * kATile), bBase = smem_addr(sB + s * kBTile);
+      const uint32_t aBase = smem_addr(sA + s * kATile), bBase = smem_addr(sB + s * kBTile);
 #pragma unroll
-        for (int kk = 0; kk < kChunk / 16; ++kk) {
-          const uint64_t ad = smem_desc_sw128(aBase + kk * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(bBase + kk * 2048, 8192, 1024);
-          umma_bf16(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(empty + s);
-        mma_issued = true;
+      for (int kk = 0; kk < kChunk / 16; ++kk) {
+        const uint64_t ad = smem_desc_sw128(aBase + kk * 32, 16, 1024);
+        const uint64_t bd = smem_desc_sw128(bBase + kk * 2048, 8192, 1024);
+        umma_bf16(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
       }
-      // refill the round's stages with the next round's chunks once their MMAs have read them
-      for (int i = i0; i < i1 && issued < nb && flag[0] == 0; ++i) {
-        const int s = i % S;
-        if (!mbar_wait_bounded(empty + s, (uint32_t)(i / S) & 1u, a.timeout_ns)) {
+      umma_commit(empty + s);
+      mma_issued = true;
+      if (issued < nb) {
+        // refill this stage with chunk i + S once its MMAs have read it
+        if (!mbar_wait_bounded(empty + s, ph, a.timeout_ns)) {
           record_timeout(a.hdr);
           flag[0] = 1;
           break;
         }
-        mbar_arrive_expect_tx(fullx + s, x_tx);
+        mbar_arrive_expect_tx(fullx + s, stage_tx);
         tma_load_2d(sA + s * kATile, &xmap, (c0 + issued) * kChunk, row0, fullx + s);
-        mbar_arrive_expect_tx(fullw + s, (uint32_t)kBTile);
-        tma_load_2d(sB + s * kBTile, &wmap, e0, (c0 + issued) * kChunk, fullw + s);
+        tma_load_2d(sB + s * kBTile, &wmap, e0, (c0 + issued) * kChunk, fullx + s);
         ++issued;
       }
     }
-    __syncthreads();
-    ok = flag[0] == 0;
-  }
-  if (tid == 0 && mma_issued) umma_commit(mma_bar);
-  // every thread waits for the MMAs (also on the error path: TMEM is freed below)
-  if (__syncthreads_or(tid == 0 && mma_issued)) {
-    if (!mbar_wait_bounded(mma_bar, 0, a.timeout_ns)) {
-      record_timeout(a.hdr);
-      flag[0] = 1;
+    if (mma_issued) {
+      umma_commit(mma_bar);
+      if (!mbar_wait_bounded(mma_bar, 0, a.timeout_ns)) {
+        record_timeout(a.hdr);
+        flag[0] = 1;
+      }
+    }
+    if (flag[0]) {
+      // a wait gave up: let copies still in flight land before the CTA exits
+      for (int i = max(0, issued - S); i < issued; ++i)
+        mbar_wait_bounded(fullx + (i % S), (uint32_t)(i / S) & 1u, a.timeout_ns);
     }
   }
   __syncthreads();
-  ok = flag[0] == 0;
+  const bool ok = flag[0] == 0;
   const int tpb = dec_tpb(TGS, a.CS);  // token rows reduced by each CTA
+  cluster_wait();
   if (ok) {
     tc_fence_after();
     // TMEM lane = token row; warp w < 8 reads lanes 32*(w%4).. and column half w/4,
@@ -601,14 +551,6 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         for (int i = 0; i < 32; i += 4) st_cluster_v4(dst + i * 4, v[i], v[i + 1], v[i + 2], v[i + 3]);
       }
     }
-  }
-  if (tid == 0 && !ok) {
-    // a wait gave up: let copies still in flight land before the CTA exits
-    for (int i = max(0, issued - S); i < issued; ++i) {
-      mbar_wait_bounded(fullx + (i % S), (uint32_t)(i / S) & 1u, a.timeout_ns);
-      mbar_wait_bounded(fullw + (i % S), (uint32_t)(i / S) & 1u, a.timeout_ns);
-    }
-    mbar_wait_bounded(gam_bar, 0, a.timeout_ns);
   }
   tc_fence_before();
   __syncthreads();
@@ -825,7 +767,7 @@ extern "C" int moe_rmsnorm_router_topk(int32_t T, int32_t H, int32_t E, int32_t 
     const cuuint64_t gdim[2] = {(cuuint64_t)H, (cuuint64_t)T};
     const cuuint64_t gstride[1] = {(cuuint64_t)H * 2};
     const cuuint32_t xbox[2] = {64, (cuuint32_t)plan.TGS};
-    if (enc(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(hidden), gdim, gstride, xbox, estr,
+    if (enc(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out_norm, gdim, gstride, xbox, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return MOE_ERR_INVALID_ARG;
@@ -839,11 +781,14 @@ extern "C" int moe_rmsnorm_router_topk(int32_t T, int32_t H, int32_t E, int32_t 
       return MOE_ERR_INVALID_ARG;
   }
 
+  // K1: the normalised rows (out_norm), then K2 projects them
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (launch_pdl(rmsnorm_kernel, dim3(T), dim3(kNormThreads), 0, st, a) != cudaSuccess) return MOE_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(plan.CS * plan.NG * plan.TG);
   cfg.blockDim = dim3(kDecThreads);
   cfg.dynamicSmemBytes = plan.smem;
-  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cfg.stream = st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = plan.CS;
