@@ -97,9 +97,10 @@ struct DecLayout {
 __host__ __device__ inline int dec_tpb(int TGS, int CS) { return (TGS + CS - 1) / CS; }
 __host__ __device__ inline DecLayout dec_layout(int S, int /*maxb*/, int TGS, int CS) {
   DecLayout L;
+  const int stg_bytes = TGS * kRedStride * 4;  // partial-logit staging rows, in the stage buffers once free
   L.a = 0;
   L.b = L.a + S * kATile;
-  L.red = L.b + S * kBTile;
+  L.red = L.b + S * kBTile > stg_bytes ? L.b + S * kBTile : stg_bytes;
   L.gam = L.psq = L.rs = 0;  // (unused)
   L.bars = L.red + CS * dec_tpb(TGS, CS) * kRedStride * 4;
   L.slot = L.bars + (3 * kMaxStages + 2) * 8;
@@ -273,8 +274,11 @@ __device__ __forceinline__ double sumsq8(uint4 v) {
   return acc;
 }
 
-// ids, affinities (and debug logits) of token t from its fp32 logits row
+// ids, affinities (and debug logits) of token t from its fp32 logits row.
+// Outputs are written only while the workspace status is MOE_OK (its load
+// is issued with the logits').
 __device__ void select_token(const DecodeArgs& a, int t, int lane) {
+  const int status = *reinterpret_cast<const volatile int32_t*>(&a.hdr->status);
   float lg[8];
   uint32_t valid = 0;
   if (lane * 8 < a.E) {
@@ -293,37 +297,46 @@ __device__ void select_token(const DecodeArgs& a, int t, int lane) {
         lg[2 * i + 1] += __uint_as_float(bw[i] & 0xffff0000u);
       }
     }
-    if (a.dbg_logits) {
-      float* d = a.dbg_logits + (size_t)t * a.E + lane * 8;
-      *reinterpret_cast<float4*>(d) = make_float4(lg[0], lg[1], lg[2], lg[3]);
-      *reinterpret_cast<float4*>(d + 4) = make_float4(lg[4], lg[5], lg[6], lg[7]);
-    }
   } else {
 #pragma unroll
     for (int i = 0; i < 8; ++i) lg[i] = 0.0f;
   }
-  // top-k on the raw logits: k rounds of warp argmax, ties -> lower expert
+  // top-k on the raw logits: k rounds of (warp max of the order-preserving
+  // key, then the lowest expert holding it), ties -> lower expert
+  uint32_t key[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) key[i] = ordered_key(lg[i]);
   uint32_t chosen = 0, avail = valid;
   int my_id = 0;
-  for (int j = 0; j < a.k; ++j) {
-    unsigned long long best = 0ull;
+  uint32_t bk = 0u;
+  int bi = 8;  // this lane's best remaining (key, slot); slot 8 = none
+  auto lane_best = [&]() {
+    bk = 0u;
+    bi = 8;
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if ((avail >> i) & 1u) {
-        const unsigned long long pk = pack_key(lg[i], lane * 8 + i);
-        best = pk > best ? pk : best;
+    for (int i = 7; i >= 0; --i)
+      if (((avail >> i) & 1u) && key[i] >= bk) {
+        bk = key[i];
+        bi = i;
       }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const unsigned long long o = shfl_xor_u64(0xffffffffu, best, off);
-      best = o > best ? o : best;
+  };
+  lane_best();
+  for (int j = 0; j < a.k; ++j) {
+    const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+    const uint32_t win =
+        __reduce_min_sync(0xffffffffu, (bi < 8 && bk == m) ? (uint32_t)(lane * 8 + bi) : 0xffffffffu);
+    if (bi < 8 && (uint32_t)(lane * 8 + bi) == win) {
+      avail &= ~(1u << bi);
+      chosen |= 1u << bi;
+      lane_best();
     }
-    const int win = packed_expert(best);
-    if (lane == (win >> 3)) {
-      avail &= ~(1u << (win & 7));
-      chosen |= 1u << (win & 7);
-    }
-    if (lane == j) my_id = win;
+    if (lane == j) my_id = (int)win;
+  }
+  if (status != MOE_OK) return;
+  if (a.dbg_logits && lane * 8 < a.E) {
+    float* d = a.dbg_logits + (size_t)t * a.E + lane * 8;
+    *reinterpret_cast<float4*>(d) = make_float4(lg[0], lg[1], lg[2], lg[3]);
+    *reinterpret_cast<float4*>(d + 4) = make_float4(lg[4], lg[5], lg[6], lg[7]);
   }
   // activation over the selected only (ACT2): sigmoid each, or softmax over the k
   float m = -INFINITY, ssum = 0.0f;
@@ -440,7 +453,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t rank = cluster_rank();
-  pdl_entry();
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int cid = blockIdx.x / a.CS;
   const int tg = cid / a.NG, ng = cid % a.NG;
   const int row0 = tg * TGS;                       // first token of the group
@@ -454,16 +467,19 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
   int issued = 0;  // chunks whose copies have been issued (thread 0)
   if (tid == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&wmap)) : "memory");
     for (int s = 0; s < kMaxStages; ++s) {
       mbar_init(fullx + s, 1);
       mbar_init(empty + s, 1);
     }
     mbar_init(mma_bar, 1);
     flag[0] = 0;
-    for (; issued < nres; ++issued) {
-      mbar_arrive_expect_tx(fullx + issued, stage_tx);
-      tma_load_2d(sA + issued * kATile, &xmap, (c0 + issued) * kChunk, row0, fullx + issued);
-      tma_load_2d(sB + issued * kBTile, &wmap, e0, (c0 + issued) * kChunk, fullx + issued);
+    // before the dependency wait, only the router weights (not written by the
+    // preceding kernel); each stage's barrier expects both of its copies
+    for (int s = 0; s < nres; ++s) {
+      mbar_arrive_expect_tx(fullx + s, stage_tx);
+      tma_load_2d(sB + s * kBTile, &wmap, e0, (c0 + s) * kChunk, fullx + s);
     }
   }
   if (warp == 0) tmem_alloc(tmem_slot, 64);
@@ -481,6 +497,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   // every CTA of the cluster must be running before any CTA writes into its
   // shared memory: arrive now, wait before the first push
   cluster_arrive();
+  // the normalised rows are the preceding kernel's (K1's) output
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (tid == 0)
+    for (; issued < nres; ++issued)
+      tma_load_2d(sA + issued * kATile, &xmap, (c0 + issued) * kChunk, row0, fullx + issued);
 
   // ---------------- project: one thread issues each chunk's MMAs as it lands ----------------
   if (tid == 0) {
@@ -533,28 +554,35 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   __syncthreads();
   const bool ok = flag[0] == 0;
   const int tpb = dec_tpb(TGS, a.CS);  // token rows reduced by each CTA
-  cluster_wait();
-  if (ok) {
-    tc_fence_after();
-    // TMEM lane = token row; warp w < 8 reads lanes 32*(w%4).. and column half w/4,
-    // and pushes the 32 partial logits to the CTA that reduces that row (slot [rank])
+  // partial logits: TMEM -> staging rows in the (now free) stage buffers ->
+  // one contiguous run per owning CTA.  Warp w < 8 reads TMEM lanes
+  // 32*(w%4).. (token rows) and column half w/4.
+  float* stg = reinterpret_cast<float*>(sA);  // [TGS][kRedStride] fp32
+  {
     const int wq = warp & 3, ch = warp >> 2;
-    if (ch < 2 && wq * 32 < TGS && ch * 32 < N) {
+    if (ok && ch < 2 && wq * 32 < TGS && ch * 32 < N) {
+      tc_fence_after();
       float v[32];
       tmem_ld32(tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)(ch * 32), v);
-      const int row = wq * 32 + lane;
-      if (row < TGS) {
-        const int owner = row / tpb;
-        const uint32_t dst =
-            cluster_map(smem_addr(red + (((int)rank * tpb) + (row - owner * tpb)) * kRedStride + ch * 32), (uint32_t)owner);
+      float4* d = reinterpret_cast<float4*>(stg + (wq * 32 + lane) * kRedStride + ch * 32);
 #pragma unroll
-        for (int i = 0; i < 32; i += 4) st_cluster_v4(dst + i * 4, v[i], v[i + 1], v[i + 2], v[i + 3]);
-      }
+      for (int i = 0; i < 8; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 64);
+  cluster_wait();
+  // warp d sends rows [d*tpb, (d+1)*tpb) to CTA d, slot [rank]
+  if (ok && warp < a.CS) {
+    const int dA = min(TGS, warp * tpb), dB = min(TGS, dA + tpb);
+    const float4* src = reinterpret_cast<const float4*>(stg + dA * kRedStride);
+    const uint32_t dst = cluster_map(smem_addr(red + (int)rank * tpb * kRedStride), (uint32_t)warp);
+    for (int j = lane; j < (dB - dA) * (kRedStride / 4); j += 32) {
+      const float4 v = src[j];
+      st_cluster_v4(dst + j * 16, v.x, v.y, v.z, v.w);
+    }
+  }
 
   // ---------------- cluster reduction of the partial logits ----------------
   cluster_sync();  // all pushes have landed; no shared memory is touched across CTAs after this
@@ -572,23 +600,26 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       a.logits[(size_t)(row0 + rA + rr) * a.E + e0 + e] = sum;
     }
   }
-  __threadfence();
 
   // ---------------- top-k by the last expert-group cluster of each token run ----------------
+  // The block's logit stores are ordered before thread 0's fence by the
+  // barrier; the last arriver's fence orders the other clusters' stores
+  // before its block's reads (L2 reads, after the second barrier).
   __syncthreads();
   if (tid == 0) {
+    __threadfence();
     const uint32_t tk = atomicAdd(&a.tickets[tg * 16 + rank], 1u);
     const int last = tk == (uint32_t)(a.NG - 1);
-    if (last) a.tickets[tg * 16 + rank] = 0u;  // every cluster of the run has arrived: reset for the next call
+    if (last) {
+      a.tickets[tg * 16 + rank] = 0u;  // every cluster of the run has arrived: reset for the next call
+      __threadfence();
+    }
     flag[1] = last;
   }
   __syncthreads();
-  if (flag[1]) {
-    __threadfence();
-    if (flag[0] == 0 && a.hdr->status == MOE_OK)
-      for (int r = rA + warp; r < rB; r += kDecWarps)
-        if (row0 + r < a.T) select_token(a, row0 + r, lane);
-  }
+  if (flag[1] && flag[0] == 0)
+    for (int r = rA + warp; r < rB; r += kDecWarps)
+      if (row0 + r < a.T) select_token(a, row0 + r, lane);
 }
 
 // ---- host ----
