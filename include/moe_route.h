@@ -288,9 +288,9 @@ int moe_combine(int32_t T, int32_t H, int32_t k, int32_t dtype, const void* expe
                 void* out, void* stream);
 
 /*
- * Workspace bytes of moe_rmsnorm_router_topk (header, fp32 logits [T,E] and
- * per-token-run tickets).  The workspace must be zero before its first use
- * (moe_workspace_init); each call leaves its tickets at zero again.
+ * Workspace bytes of moe_rmsnorm_router_topk (header and the fp32 partial
+ * logits of the K-split projection; depends on T, H and E).  The workspace
+ * must be zero before its first use (moe_workspace_init).
  */
 int moe_rmsnorm_router_topk_workspace_bytes(int32_t T, int32_t H, int32_t E, size_t* bytes);
 
@@ -308,11 +308,15 @@ int moe_rmsnorm_router_topk_workspace_bytes(int32_t T, int32_t H, int32_t E, siz
  * affinities [T,E] -- bf16; ids [T,k] int32; debug_logits [T,E] fp32 or NULL
  * (receives the logits when given).  T <= 128 and H % 128 == 0 [NKI: Notes];
  * this build also needs E % 16 == 0, E <= 256 and H <= 32768, and every
- * pointer 16-byte aligned.  Two launches: a row-parallel RMSNorm writing
- * out_norm, then the projection + top-k on thread-block clusters (sized per
- * GPU) that read out_norm and never wait on one another; device-side waits are
- * bounded and a wait that gives up leaves MOE_ERR_DEVICE_TIMEOUT in the
- * workspace status word (outputs undefined).
+ * pointer 16-byte aligned.  Three launches chained by programmatic dependent
+ * launch: a row-parallel RMSNorm writing out_norm; the projection split over
+ * K-slices (one CTA per token group x 64 experts x slice, all resident at
+ * once) writing fp32 partial logits to the workspace; a block per token that
+ * adds the partials in slice order and takes the top-k.  Each launch reads
+ * W, gamma and bias before waiting on its predecessor: a preceding kernel
+ * that lets dependents start early must not write them.  Device-side waits
+ * are bounded and a wait that gives up leaves MOE_ERR_DEVICE_TIMEOUT in the
+ * workspace status word (outputs are then left unwritten).
  * Returns MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED / MOE_ERR_WORKSPACE for
  * bad arguments, MOE_ERR_CUDA when the launch fails.  Calls sharing one
  * workspace must not overlap in time.

@@ -8,7 +8,10 @@
 // Returns, Notes (T <= 128; H % 128 == 0; ACT2: top-K on raw logits, then the
 // activation on the selected experts only).
 //
-// Two launches.
+// Three launches chained by programmatic dependent launch: each kernel lets
+// the next one be scheduled at its entry, and the next one does everything
+// that does not read its predecessor's output (the router weights, gamma,
+// barriers, TMEM) before waiting on it.
 //
 //   K1 rmsnorm_kernel, a block per token: the sum of exact squares of the row
 //   in double, r_t = 1/sqrt(mean + eps) in double (kept as r_hi + r_lo in
@@ -19,29 +22,22 @@
 //   multiply-adds), so the bf16 value is the single rounding of x*gamma*r.
 //   The result is out_norm.
 //
-//   K2 decode_kernel (programmatic dependent launch after K1), thread-block
-//   clusters of CS CTAs.  A cluster owns one group of tokens (64, or all
-//   T <= 128) and one group of 64 experts over the whole hidden dimension; CTA
-//   j owns the j-th K-slice (a run of 64-column chunks).  CS (1..16) and the
-//   token group size are chosen per GPU from how many clusters of each size it
-//   can keep resident: the fewest staged bytes per CTA with every cluster
-//   resident at once (T=128, H=7168, E=256: 4 clusters x 16 CTAs).
-//     stage    out_norm chunks (tokens x 64 columns) and W chunks (64 rows x
-//              64 experts) -> shared memory by 2-D TMA, 128-byte swizzle (the
-//              canonical K-major A / MN-major B layouts of tcgen05.mma); a
-//              ring of up to 8 chunk stages, refilled when the slice is longer.
-//     project  one thread issues each chunk's M=128 x N=64 x K=16 MMAs into
-//              TMEM as soon as the chunk has landed.
-//     reduce   TMEM -> registers -> pushed into the shared memory of the CTA
-//              that reduces those rows (st.shared::cluster); after one cluster
-//              barrier CTA j adds the CS partials of its rows in rank order and
-//              stores the fp32 logits of its (tokens, experts) tile.
-//     select   a per-(token group, rank) ticket: the last of the expert-group
-//              clusters to store its tile (no waiting) adds the bias, takes
-//              the top-k on the raw logits (ties -> lower expert) and writes
-//              ids and the masked bf16 affinities, then resets the ticket.
-// No grid-wide barrier, no cooperative launch: clusters never wait on one
-// another, so K2 also completes when the clusters run in waves.
+//   K2 project_kernel, one CTA per (token group, expert group of 64, K-slice):
+//   the slice's W chunks (64 rows x 64 experts) staged by 2-D TMA before the
+//   wait, its out_norm chunks (tokens x 64 columns) after it, both with the
+//   128-byte swizzle (the canonical K-major A / MN-major B layouts of
+//   tcgen05.mma); one thread issues each chunk's M=128 x N=64 x K=16 MMAs into
+//   TMEM as it lands; the fp32 partial logits go from TMEM to the workspace.
+//   The K-split KS is chosen so that every CTA is resident at once with the
+//   fewest post-wait staged bytes per CTA (T=128, H=7168, E=256: 4 expert
+//   groups x 28 slices of 4 chunks = 112 CTAs).
+//
+//   K3 select_kernel, a block per token: the logit of expert e is the sum of
+//   its KS partials in slice order (fp32), then the bias, the top-k on the raw
+//   logits (ties -> lower expert), ids and the masked bf16 affinities.
+//
+// No kernel waits on another's blocks: no grid-wide barrier, no cluster, no
+// cooperative launch.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -53,18 +49,18 @@
 namespace moe {
 namespace {
 
-constexpr int kDecThreads = 512;
-constexpr int kDecWarps = kDecThreads / 32;
-constexpr int kChunk = 64;       // hidden columns per staged chunk (one 128-byte swizzle atom)
-constexpr int kExpGroup = 64;    // experts per cluster (MMA N <= 64)
-constexpr int kM = 128;          // MMA M: 64 token rows + 64 zero rows
-constexpr int kMaxE = 256;       // top-k stage: 8 experts per lane
-constexpr int kMaxStages = 8;    // staged chunks in flight (fewer when shared memory is short)
-constexpr int kMaxSliceChunks = 64;  // gamma slice kept in shared memory
+constexpr int kProjThreads = 256;  // 8 warps: 4 TMEM lane quarters x 2 column halves
+constexpr int kChunk = 64;         // hidden columns per staged chunk (one 128-byte swizzle atom)
+constexpr int kExpGroup = 64;      // experts per CTA (MMA N <= 64)
+constexpr int kM = 128;            // MMA M: token rows (a 64-token group pads with zero rows)
+constexpr int kMaxE = 256;         // top-k stage: 8 experts per lane
+constexpr int kMaxStages = 8;      // staged chunks in flight
+constexpr int kMaxKS = 48;         // K-slices (bounds the partial-logit workspace)
 constexpr int kATile = kM * 128;      // 16 KB
 constexpr int kBTile = kChunk * 128;  // 8 KB (64 K rows x 64 experts)
-constexpr int kRedStride = kExpGroup + 4;  // padded fp32 row of the partial-logit tile
-constexpr int kSmemLimit = 227 * 1024;     // opt-in shared memory per CTA
+constexpr int kSmemLimit = 227 * 1024;  // opt-in shared memory per CTA
+constexpr int kSelThreads = 256;        // K3: one thread per expert
+constexpr int kMaxH = 32768;            // hidden size limit
 
 struct DecodeArgs {
   const uint16_t* x;      // [T,H] bf16
@@ -75,35 +71,28 @@ struct DecodeArgs {
   uint16_t* aff;          // [T,E]
   float* dbg_logits;      // [T,E] or null
   WsHeader* hdr;
-  float* logits;          // [T,E] fp32 (workspace)
-  uint32_t* tickets;      // [2][16] (workspace), zero between calls
+  float* part;            // [KS][TG*TGS][NG*64] fp32 partial logits (workspace)
   int T, H, E, k, act;
-  int CS;                 // CTAs per cluster (K-split)
-  int TGS;                // tokens per cluster: 64 or 128
+  int KS;                 // K-slices
+  int TGS;                // tokens per group: 64 or 128
+  int TG;                 // token groups
   int NG;                 // expert groups
   int nch;                // H / 64
   int S;                  // ring stages
-  int maxb;               // most chunks any CTA owns
   float eps;
   long long timeout_ns;
 };
 
-// shared-memory layout (offsets from a 1024-byte aligned base)
+// K2 shared-memory layout (offsets from a 1024-byte aligned base)
 struct DecLayout {
-  int a, b, red, gam, psq, rs, bars, slot, flag, total;
+  int a, b, bars, slot, flag, total;
 };
-// red: partial logits pushed by every CTA of the cluster for the rows this CTA
-// reduces, [CS][tpb][kRedStride] fp32.
-__host__ __device__ inline int dec_tpb(int TGS, int CS) { return (TGS + CS - 1) / CS; }
-__host__ __device__ inline DecLayout dec_layout(int S, int /*maxb*/, int TGS, int CS) {
+__host__ __device__ inline DecLayout dec_layout(int S) {
   DecLayout L;
-  const int stg_bytes = TGS * kRedStride * 4;  // partial-logit staging rows, in the stage buffers once free
   L.a = 0;
   L.b = L.a + S * kATile;
-  L.red = L.b + S * kBTile > stg_bytes ? L.b + S * kBTile : stg_bytes;
-  L.gam = L.psq = L.rs = 0;  // (unused)
-  L.bars = L.red + CS * dec_tpb(TGS, CS) * kRedStride * 4;
-  L.slot = L.bars + (3 * kMaxStages + 2) * 8;
+  L.bars = L.b + S * kBTile;
+  L.slot = L.bars + (2 * kMaxStages + 1) * 8;
   L.flag = L.slot + 16;
   L.total = L.flag + 16;
   return L;
@@ -175,32 +164,6 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
 }
 
 __device__ __forceinline__ float sigmoid_f32(float x) { return 1.0f / (1.0f + expf(-x)); }
-
-// ---- thread-block cluster helpers ----
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cluster_arrive() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
-__device__ __forceinline__ void cluster_sync() {
-  cluster_arrive();
-  cluster_wait();
-}
-// shared::cta address -> the same offset in CTA `rank` of the cluster
-__device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-  return r;
-}
-// stores into another CTA's shared memory (made visible by the next cluster barrier)
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
 
 // packed fp32 pairs (two IEEE round-to-nearest products per instruction)
 __device__ __forceinline__ unsigned long long pack2(float lo, float hi) {
@@ -274,22 +237,19 @@ __device__ __forceinline__ double sumsq8(uint4 v) {
   return acc;
 }
 
-// ids, affinities (and debug logits) of token t from its fp32 logits row.
-// Outputs are written only while the workspace status is MOE_OK (its load
-// is issued with the logits').
-__device__ void select_token(const DecodeArgs& a, int t, int lane) {
-  const int status = *reinterpret_cast<const volatile int32_t*>(&a.hdr->status);
+// K3: ids, affinities (and debug logits) of one token from its logits row in
+// shared memory; outputs are written only while the workspace status is
+// MOE_OK.
+__device__ void select_row(const DecodeArgs& a, int t, int lane, const float* row, int status, uint4 bv) {
   float lg[8];
   uint32_t valid = 0;
   if (lane * 8 < a.E) {
-    const float* src = a.logits + (size_t)t * a.E + lane * 8;
-    const float4 u = __ldcg(reinterpret_cast<const float4*>(src));
-    const float4 w = __ldcg(reinterpret_cast<const float4*>(src + 4));
+    const float4 u = reinterpret_cast<const float4*>(row + lane * 8)[0];
+    const float4 w = reinterpret_cast<const float4*>(row + lane * 8)[1];
     lg[0] = u.x; lg[1] = u.y; lg[2] = u.z; lg[3] = u.w;
     lg[4] = w.x; lg[5] = w.y; lg[6] = w.z; lg[7] = w.w;
     valid = 0xffu;
     if (a.bias) {
-      const uint4 bv = __ldg(reinterpret_cast<const uint4*>(a.bias + lane * 8));
       const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -372,28 +332,36 @@ __device__ void select_token(const DecodeArgs& a, int t, int lane) {
 // K1: RMSNorm, a block per token row.  Sum of exact squares in double (a fixed
 // order: thread partials, a shuffle tree, warps in order), r = 1/sqrt(mean +
 // eps) in double kept as r_hi + r_lo, then x*gamma*r rounded once to bf16
-// (normalize8 / normalize8_exact) into out_norm.
+// (normalize8 / normalize8_exact) into out_norm.  gamma is read before the
+// dependency wait (a weight, not written by the preceding kernel).
 constexpr int kNormThreads = 256;
 constexpr int kNormKeep = 4;  // 16-byte groups a thread keeps in registers (H <= 8192)
 
 __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const DecodeArgs a) {
   __shared__ double red[kNormThreads / 32];
   __shared__ float2 rr;
-  pdl_entry();
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nq = a.H / 8;  // 16-byte groups in a row
+  uint4 gkeep[kNormKeep];
+#pragma unroll
+  for (int j = 0; j < kNormKeep; ++j) {
+    const int qq = tid + j * kNormThreads;
+    gkeep[j] = qq < nq ? __ldg(reinterpret_cast<const uint4*>(a.gamma) + qq) : make_uint4(0, 0, 0, 0);
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the hidden states are the preceding kernel's output
   const uint16_t* xr = a.x + (size_t)t * a.H;
   uint4 keep[kNormKeep];
   double acc = 0.0;
 #pragma unroll
   for (int j = 0; j < kNormKeep; ++j) {
     const int qq = tid + j * kNormThreads;
-    keep[j] = qq < nq ? __ldg(reinterpret_cast<const uint4*>(xr) + qq) : make_uint4(0, 0, 0, 0);
+    keep[j] = qq < nq ? __ldcg(reinterpret_cast<const uint4*>(xr) + qq) : make_uint4(0, 0, 0, 0);
   }
 #pragma unroll
   for (int j = 0; j < kNormKeep; ++j) acc += sumsq8(keep[j]);
   for (int qq = tid + kNormKeep * kNormThreads; qq < nq; qq += kNormThreads)
-    acc += sumsq8(__ldg(reinterpret_cast<const uint4*>(xr) + qq));
+    acc += sumsq8(__ldcg(reinterpret_cast<const uint4*>(xr) + qq));
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (lane == 0) red[warp] = acc;
@@ -408,8 +376,7 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const DecodeArgs 
   __syncthreads();
   const float2 r2 = rr;
   uint16_t* orow = a.out_norm + (size_t)t * a.H;
-  auto normalise = [&](int qq, uint4 xv) {
-    const uint4 gv = __ldg(reinterpret_cast<const uint4*>(a.gamma) + qq);
+  auto normalise = [&](int qq, uint4 xv, uint4 gv) {
     const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
     float g[8];
     unsigned long long g2[4];
@@ -425,43 +392,37 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const DecodeArgs 
   };
 #pragma unroll
   for (int j = 0; j < kNormKeep; ++j)
-    if (tid + j * kNormThreads < nq) normalise(tid + j * kNormThreads, keep[j]);
+    if (tid + j * kNormThreads < nq) normalise(tid + j * kNormThreads, keep[j], gkeep[j]);
   for (int qq = tid + kNormKeep * kNormThreads; qq < nq; qq += kNormThreads)
-    normalise(qq, __ldg(reinterpret_cast<const uint4*>(xr) + qq));
+    normalise(qq, __ldcg(reinterpret_cast<const uint4*>(xr) + qq), __ldg(reinterpret_cast<const uint4*>(a.gamma) + qq));
 }
 
-// K2: router projection + top-k on thread-block clusters (see the file head):
-// staged out_norm and W chunks, M=128 x N=64 x K=16 MMAs per chunk as soon as
-// both land, partial logits pushed to the reducing CTA, the ticketed top-k.
-__global__ void __launch_bounds__(kDecThreads, 1)
-    decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap xmap,
-                  const __grid_constant__ CUtensorMap wmap) {
+// K2: the partial logits of one (token group, expert group, K-slice).
+__global__ void __launch_bounds__(kProjThreads, 1)
+    project_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap xmap,
+                   const __grid_constant__ CUtensorMap wmap) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);  // 1024-byte aligned (swizzle atoms)
-  const int TGS = a.TGS;
-  const DecLayout L = dec_layout(a.S, a.maxb, TGS, a.CS);
+  const int TGS = a.TGS, S = a.S;
+  const DecLayout L = dec_layout(S);
   uint8_t* sA = smem + L.a;
   uint8_t* sB = smem + L.b;
-  float* red = reinterpret_cast<float*>(smem + L.red);
-  uint64_t* fullx = reinterpret_cast<uint64_t*>(smem + L.bars);  // normalised rows landed
-  uint64_t* fullw = fullx + kMaxStages;                          // W chunk landed
-  uint64_t* empty = fullw + kMaxStages;                          // the stage's MMAs are done
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);  // both copies of the stage landed
+  uint64_t* empty = full + kMaxStages;                          // the stage's MMAs are done
   uint64_t* mma_bar = empty + kMaxStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.slot);
-  int* flag = reinterpret_cast<int*>(smem + L.flag);
+  volatile int* flag = reinterpret_cast<volatile int*>(smem + L.flag);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint32_t rank = cluster_rank();
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int cid = blockIdx.x / a.CS;
-  const int tg = cid / a.NG, ng = cid % a.NG;
-  const int row0 = tg * TGS;                       // first token of the group
-  const int e0 = ng * kExpGroup;                   // first expert of the group
-  const int N = min(kExpGroup, a.E - e0);          // multiple of 16
-  const int c0 = (int)((long long)a.nch * rank / a.CS);
-  const int nb = (int)((long long)a.nch * (rank + 1) / a.CS) - c0;  // chunks of this CTA (>= 1)
-  const int S = a.S;
+  const int ks = blockIdx.x % a.KS, rest = blockIdx.x / a.KS;
+  const int ng = rest % a.NG, tg = rest / a.NG;
+  const int row0 = tg * TGS;               // first token of the group
+  const int e0 = ng * kExpGroup;           // first expert of the group
+  const int N = min(kExpGroup, a.E - e0);  // multiple of 16
+  const int c0 = (int)((long long)a.nch * ks / a.KS);
+  const int nb = (int)((long long)a.nch * (ks + 1) / a.KS) - c0;  // chunks of this CTA (>= 1)
   const int nres = min(S, nb);
   const uint32_t stage_tx = (uint32_t)(TGS * 128 + kBTile);
 
@@ -470,7 +431,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&wmap)) : "memory");
     for (int s = 0; s < kMaxStages; ++s) {
-      mbar_init(fullx + s, 1);
+      mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
     }
     mbar_init(mma_bar, 1);
@@ -478,14 +439,14 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     // before the dependency wait, only the router weights (not written by the
     // preceding kernel); each stage's barrier expects both of its copies
     for (int s = 0; s < nres; ++s) {
-      mbar_arrive_expect_tx(fullx + s, stage_tx);
-      tma_load_2d(sB + s * kBTile, &wmap, e0, (c0 + s) * kChunk, fullx + s);
+      mbar_arrive_expect_tx(full + s, stage_tx);
+      tma_load_2d(sB + s * kBTile, &wmap, e0, (c0 + s) * kChunk, full + s);
     }
   }
   if (warp == 0) tmem_alloc(tmem_slot, 64);
   // with 64-token groups, A rows 64..127 are zero in every stage (the TMA box fills rows 0..63)
   if (TGS < kM)
-    for (int i = tid; i < S * ((kM - TGS) * 8); i += kDecThreads) {
+    for (int i = tid; i < S * ((kM - TGS) * 8); i += kProjThreads) {
       const int s = i / ((kM - TGS) * 8), off = i % ((kM - TGS) * 8);
       *reinterpret_cast<uint4*>(sA + s * kATile + TGS * 128 + off * 16) = make_uint4(0, 0, 0, 0);
     }
@@ -494,23 +455,19 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // every CTA of the cluster must be running before any CTA writes into its
-  // shared memory: arrive now, wait before the first push
-  cluster_arrive();
-  // the normalised rows are the preceding kernel's (K1's) output
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  if (tid == 0)
-    for (; issued < nres; ++issued)
-      tma_load_2d(sA + issued * kATile, &xmap, (c0 + issued) * kChunk, row0, fullx + issued);
 
-  // ---------------- project: one thread issues each chunk's MMAs as it lands ----------------
+  // the normalised rows are K1's output
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   if (tid == 0) {
+    for (; issued < nres; ++issued)
+      tma_load_2d(sA + issued * kATile, &xmap, (c0 + issued) * kChunk, row0, full + issued);
+    // ---------------- project: each chunk's MMAs as soon as it has landed ----------------
     const uint32_t idesc = idesc_bf16_f32(N);
     bool mma_issued = false;
     for (int i = 0; i < nb; ++i) {
       const int s = i % S;
       const uint32_t ph = (uint32_t)(i / S) & 1u;
-      if (!mbar_wait_bounded(fullx + s, ph, a.timeout_ns)) {
+      if (!mbar_wait_bounded(full + s, ph, a.timeout_ns)) {
         record_timeout(a.hdr);
         flag[0] = 1;
         break;
@@ -532,13 +489,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           flag[0] = 1;
           break;
         }
-        mbar_arrive_expect_tx(fullx + s, stage_tx);
-        tma_load_2d(sA + s * kATile, &xmap, (c0 + issued) * kChunk, row0, fullx + s);
-        tma_load_2d(sB + s * kBTile, &wmap, e0, (c0 + issued) * kChunk, fullx + s);
+        mbar_arrive_expect_tx(full + s, stage_tx);
+        tma_load_2d(sA + s * kATile, &xmap, (c0 + issued) * kChunk, row0, full + s);
+        tma_load_2d(sB + s * kBTile, &wmap, e0, (c0 + issued) * kChunk, full + s);
         ++issued;
       }
     }
-    if (mma_issued) {
+    if (mma_issued && flag[0] == 0) {
       umma_commit(mma_bar);
       if (!mbar_wait_bounded(mma_bar, 0, a.timeout_ns)) {
         record_timeout(a.hdr);
@@ -546,25 +503,23 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       }
     }
     if (flag[0]) {
-      // a wait gave up: let copies still in flight land before the CTA exits
+      // a wait gave up: let the copies still in flight land before the CTA exits
       for (int i = max(0, issued - S); i < issued; ++i)
-        mbar_wait_bounded(fullx + (i % S), (uint32_t)(i / S) & 1u, a.timeout_ns);
+        mbar_wait_bounded(full + (i % S), (uint32_t)(i / S) & 1u, a.timeout_ns);
     }
   }
   __syncthreads();
-  const bool ok = flag[0] == 0;
-  const int tpb = dec_tpb(TGS, a.CS);  // token rows reduced by each CTA
-  // partial logits: TMEM -> staging rows in the (now free) stage buffers ->
-  // one contiguous run per owning CTA.  Warp w < 8 reads TMEM lanes
-  // 32*(w%4).. (token rows) and column half w/4.
-  float* stg = reinterpret_cast<float*>(sA);  // [TGS][kRedStride] fp32
-  {
+  // ---------------- partial logits: TMEM -> the workspace ----------------
+  // warp w reads TMEM lanes 32*(w%4).. (token rows) and column half w/4; each
+  // thread stores its row's 32 fp32 (128 contiguous bytes)
+  if (flag[0] == 0) {
     const int wq = warp & 3, ch = warp >> 2;
-    if (ok && ch < 2 && wq * 32 < TGS && ch * 32 < N) {
+    if (wq * 32 < TGS && ch * 32 < N) {
       tc_fence_after();
       float v[32];
       tmem_ld32(tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)(ch * 32), v);
-      float4* d = reinterpret_cast<float4*>(stg + (wq * 32 + lane) * kRedStride + ch * 32);
+      const int row = wq * 32 + lane;
+      float4* d = reinterpret_cast<float4*>(a.part + ((size_t)ks * (a.TG * TGS) + row0 + row) * (a.NG * kExpGroup) + e0 + ch * 32);
 #pragma unroll
       for (int i = 0; i < 8; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
     }
@@ -572,54 +527,28 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 64);
-  cluster_wait();
-  // warp d sends rows [d*tpb, (d+1)*tpb) to CTA d, slot [rank]
-  if (ok && warp < a.CS) {
-    const int dA = min(TGS, warp * tpb), dB = min(TGS, dA + tpb);
-    const float4* src = reinterpret_cast<const float4*>(stg + dA * kRedStride);
-    const uint32_t dst = cluster_map(smem_addr(red + (int)rank * tpb * kRedStride), (uint32_t)warp);
-    for (int j = lane; j < (dB - dA) * (kRedStride / 4); j += 32) {
-      const float4 v = src[j];
-      st_cluster_v4(dst + j * 16, v.x, v.y, v.z, v.w);
-    }
-  }
+}
 
-  // ---------------- cluster reduction of the partial logits ----------------
-  cluster_sync();  // all pushes have landed; no shared memory is touched across CTAs after this
-  const int rA = min(TGS, (int)rank * tpb), rB = min(TGS, rA + tpb);
-  if (ok) {
-    for (int idx = tid; idx < (rB - rA) * kExpGroup; idx += kDecThreads) {
-      const int rr = idx / kExpGroup, e = idx % kExpGroup;
-      if (e >= N || row0 + rA + rr >= a.T) continue;
-      float v[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) v[j] = j < a.CS ? red[(j * tpb + rr) * kRedStride + e] : 0.0f;
-      float sum = 0.0f;  // rank order
-#pragma unroll
-      for (int j = 0; j < 16; ++j) sum += v[j];
-      a.logits[(size_t)(row0 + rA + rr) * a.E + e0 + e] = sum;
-    }
-  }
-
-  // ---------------- top-k by the last expert-group cluster of each token run ----------------
-  // The block's logit stores are ordered before thread 0's fence by the
-  // barrier; the last arriver's fence orders the other clusters' stores
-  // before its block's reads (L2 reads, after the second barrier).
-  __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    const uint32_t tk = atomicAdd(&a.tickets[tg * 16 + rank], 1u);
-    const int last = tk == (uint32_t)(a.NG - 1);
-    if (last) {
-      a.tickets[tg * 16 + rank] = 0u;  // every cluster of the run has arrived: reset for the next call
-      __threadfence();
-    }
-    flag[1] = last;
+// K3: the logits of one token (its partials summed in slice order) and its top-k.
+__global__ void __launch_bounds__(kSelThreads) select_kernel(const DecodeArgs a) {
+  __shared__ __align__(16) float row[kMaxE];
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int t = blockIdx.x, e = threadIdx.x;
+  uint4 bv = make_uint4(0, 0, 0, 0);  // the bias of lane l's experts 8l..8l+7 (warp 0), a weight
+  if (e < 32 && a.bias && e * 8 < a.E) bv = __ldg(reinterpret_cast<const uint4*>(a.bias + e * 8));
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the partial logits are K2's output
+  int status = MOE_OK;
+  if (e < 32) status = *reinterpret_cast<const volatile int32_t*>(&a.hdr->status);
+  const int tp = a.TG * a.TGS, ep = a.NG * kExpGroup;
+  if (e < a.E) {
+    const float* p = a.part + (size_t)t * ep + e;
+    float sum = 0.0f;  // slice order (a deeper unroll measured slower)
+#pragma unroll 4
+    for (int s = 0; s < a.KS; ++s) sum += __ldcg(p + (size_t)s * tp * ep);
+    row[e] = sum;
   }
   __syncthreads();
-  if (flag[1] && flag[0] == 0)
-    for (int r = rA + warp; r < rB; r += kDecWarps)
-      if (row0 + r < a.T) select_token(a, row0 + r, lane);
+  if (e < 32) select_row(a, t, e, row, status, bv);
 }
 
 // ---- host ----
@@ -642,81 +571,55 @@ EncodeTiledFn encode_fn() {
 
 constexpr int kDecSmemMax = kSmemLimit;
 
-// Per device: kernel attributes set once, and for each cluster size 8..16 how
-// many clusters can be resident at once (one CTA per SM at these sizes).
+// Per device: the kernel attribute set once, and the SM count.
 struct DecDevice {
   std::once_flag once;
   int ok = 0;
-  int active[17] = {0};
+  int sms = 0;
 };
 DecDevice g_dec_dev[64];
 
-int max_active_clusters(int cs) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(cs * 16);
-  cfg.blockDim = dim3(kDecThreads);
-  cfg.dynamicSmemBytes = 200 * 1024;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = cs;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, decode_kernel, &cfg) != cudaSuccess) {
-    cudaGetLastError();
-    return 0;
-  }
-  return n;
-}
-
 int dec_device_setup(int dev) {
   DecDevice& d = g_dec_dev[dev];
-  std::call_once(d.once, [&d] {
-    if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmemMax) != cudaSuccess)
+  std::call_once(d.once, [&d, dev] {
+    if (cudaFuncSetAttribute(project_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmemMax) !=
+        cudaSuccess)
       return;
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || d.sms < 1) return;
     d.ok = 1;
-    const bool nonportable =
-        cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
-    if (!nonportable) cudaGetLastError();
-    for (int cs = 1; cs <= 16; ++cs) d.active[cs] = (cs <= 8 || nonportable) ? max_active_clusters(cs) : 0;
   });
   return d.ok;
 }
 
 struct DecPlan {
-  int CS, NG, TG, TGS, nch, maxb, S, smem;
+  int KS, NG, TG, TGS, nch, S, smem;
 };
 
-// Choose the cluster size CS (CTAs sharing the hidden dimension) and the token
-// group size: least staged bytes per CTA, counting a second wave of clusters
-// as a second pass and a slice longer than the ring as one more pass.
-DecPlan dec_plan(int T, int H, int E, const int* active) {
+// Choose the token group size and the K-split: every CTA resident at once
+// (one per SM), least cost = post-wait staged bytes per CTA (the normalised
+// rows) + the partial logits K3 reads per token.
+DecPlan dec_plan(int T, int H, int E, int sms) {
   DecPlan best = {};
   double best_cost = 1e300;
   const int nch = H / kChunk;
   const int NG = (E + kExpGroup - 1) / kExpGroup;
-  for (int cs = 1; cs <= std::min(16, nch); ++cs) {
-    if (active[cs] < 1) continue;
-    for (int tgs = 64; tgs <= 128; tgs += 64) {
-      if (tgs == 128 && T <= 64) continue;
+  for (int tgs = 64; tgs <= 128; tgs += 64) {
+    if (tgs == 128 && T <= 64) continue;
+    const int TG = (T + tgs - 1) / tgs;
+    for (int ks = 1; ks <= std::min(nch, kMaxKS); ++ks) {
+      if (TG * NG * ks > sms && ks > 1) break;
       DecPlan p;
-      p.CS = cs;
+      p.KS = ks;
       p.NG = NG;
+      p.TG = TG;
       p.TGS = tgs;
-      p.TG = (T + tgs - 1) / tgs;
       p.nch = nch;
-      p.maxb = (nch + cs - 1) / cs;
-      if (p.maxb > kMaxSliceChunks) continue;
-      p.S = std::min(kMaxStages, p.maxb);
-      while (p.S > 1 && 1024 + dec_layout(p.S, p.maxb, tgs, cs).total > kSmemLimit) --p.S;
-      p.smem = 1024 + dec_layout(p.S, p.maxb, tgs, cs).total;
-      if (p.smem > kSmemLimit) continue;
-      const int clusters = p.TG * p.NG;
-      const int waves = (clusters + active[cs] - 1) / active[cs];
-      const double per_cta = (double)p.maxb * (tgs * 128 + kBTile);
-      const double cost = per_cta * (waves + (p.maxb > p.S ? 1 : 0)) + 1e-3 * cs * clusters;
+      const int maxb = (nch + ks - 1) / ks;
+      p.S = std::min(kMaxStages, maxb);
+      p.smem = 1024 + dec_layout(p.S).total;
+      // post-wait staged bytes per CTA (a ring stages the rows a second
+      // time) + the partial logits K3 reads per token
+      const double cost = (double)maxb * tgs * 128 * (maxb > p.S ? 2.0 : 1.0) + (double)ks * NG * kExpGroup * 4;
       if (cost < best_cost) {
         best_cost = cost;
         best = p;
@@ -726,8 +629,10 @@ DecPlan dec_plan(int T, int H, int E, const int* active) {
   return best;
 }
 
-size_t dec_ws_bytes(int T, int E) {
-  return sizeof(WsHeader) + (size_t)std::max(T, 1) * E * sizeof(float) + 2 * 16 * sizeof(uint32_t);
+size_t dec_ws_bytes(int T, int H, int E) {
+  const int NG = (E + kExpGroup - 1) / kExpGroup;
+  const int tp = T <= 64 ? 64 : 128;
+  return sizeof(WsHeader) + (size_t)std::min(H / kChunk, kMaxKS) * tp * NG * kExpGroup * sizeof(float);
 }
 
 }  // namespace
@@ -737,8 +642,8 @@ using namespace moe;
 
 extern "C" int moe_rmsnorm_router_topk_workspace_bytes(int32_t T, int32_t H, int32_t E, size_t* bytes) {
   if (T < 0 || T > 128 || H <= 0 || H % 128 != 0 || E <= 0 || !bytes) return MOE_ERR_INVALID_ARG;
-  if (E % 16 != 0 || E > kMaxE || H > kMaxSliceChunks * kChunk * 8) return MOE_ERR_UNSUPPORTED;
-  *bytes = dec_ws_bytes(T, E);
+  if (E % 16 != 0 || E > kMaxE || H > kMaxH) return MOE_ERR_UNSUPPORTED;
+  *bytes = dec_ws_bytes(T, H, E);
   return MOE_OK;
 }
 
@@ -748,21 +653,21 @@ extern "C" int moe_rmsnorm_router_topk(int32_t T, int32_t H, int32_t E, int32_t 
                                        size_t ws_bytes, void* stream) {
   if (T < 0 || T > 128 || H <= 0 || H % 128 != 0 || E <= 0 || k <= 0 || k > E) return MOE_ERR_INVALID_ARG;
   if (act != MOE_SIGMOID && act != MOE_SOFTMAX) return MOE_ERR_INVALID_ARG;
-  if (E % 16 != 0 || E > kMaxE || k > MOE_MAX_TOPK || H > kMaxSliceChunks * kChunk * 8) return MOE_ERR_UNSUPPORTED;
+  if (E % 16 != 0 || E > kMaxE || k > MOE_MAX_TOPK || H > kMaxH) return MOE_ERR_UNSUPPORTED;
   if (T == 0) return MOE_OK;
   if (!hidden || !gamma || !W || !out_norm || !ids || !affinities) return MOE_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(hidden) | reinterpret_cast<uintptr_t>(gamma) | reinterpret_cast<uintptr_t>(W) |
        reinterpret_cast<uintptr_t>(out_norm) | reinterpret_cast<uintptr_t>(affinities) |
        reinterpret_cast<uintptr_t>(bias) | reinterpret_cast<uintptr_t>(debug_logits)) & 15)
     return MOE_ERR_INVALID_ARG;
-  if (!ws || ws_bytes < dec_ws_bytes(T, E) || (reinterpret_cast<uintptr_t>(ws) & 15)) return MOE_ERR_WORKSPACE;
+  if (!ws || ws_bytes < dec_ws_bytes(T, H, E) || (reinterpret_cast<uintptr_t>(ws) & 15)) return MOE_ERR_WORKSPACE;
   EncodeTiledFn enc = encode_fn();
   if (!enc) return MOE_ERR_CUDA;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
   if (!dec_device_setup(dev)) return MOE_ERR_CUDA;
-  const DecPlan plan = dec_plan(T, H, E, g_dec_dev[dev].active);
-  if (plan.CS < 1) return MOE_ERR_UNSUPPORTED;
+  const DecPlan plan = dec_plan(T, H, E, g_dec_dev[dev].sms);
+  if (plan.KS < 1) return MOE_ERR_UNSUPPORTED;
 
   DecodeArgs a = {};
   a.x = reinterpret_cast<const uint16_t*>(hidden);
@@ -773,23 +678,22 @@ extern "C" int moe_rmsnorm_router_topk(int32_t T, int32_t H, int32_t E, int32_t 
   a.aff = reinterpret_cast<uint16_t*>(affinities);
   a.dbg_logits = debug_logits;
   a.hdr = reinterpret_cast<WsHeader*>(ws);
-  a.logits = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + sizeof(WsHeader));
-  a.tickets = reinterpret_cast<uint32_t*>(a.logits + (size_t)T * E);
+  a.part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + sizeof(WsHeader));
   a.T = T;
   a.H = H;
   a.E = E;
   a.k = k;
   a.act = act;
-  a.CS = plan.CS;
+  a.KS = plan.KS;
   a.TGS = plan.TGS;
+  a.TG = plan.TG;
   a.NG = plan.NG;
   a.nch = plan.nch;
   a.S = plan.S;
-  a.maxb = plan.maxb;
   a.eps = eps;
   a.timeout_ns = kDefaultTimeoutNs;
 
-  // x [T][H]: dim0 = H (contiguous), dim1 = T; 64 x TGS boxes (rows past T read as zero)
+  // out_norm [T][H]: dim0 = H (contiguous), dim1 = T; 64 x TGS boxes (rows past T read as zero)
   // W [H][E]: dim0 = E (contiguous), dim1 = H; 64 x 64 boxes (experts past E read as zero)
   CUtensorMap xmap, wmap;
   const cuuint32_t box[2] = {64, 64};
@@ -812,28 +716,11 @@ extern "C" int moe_rmsnorm_router_topk(int32_t T, int32_t H, int32_t E, int32_t 
       return MOE_ERR_INVALID_ARG;
   }
 
-  // K1: the normalised rows (out_norm), then K2 projects them
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (launch_pdl(rmsnorm_kernel, dim3(T), dim3(kNormThreads), 0, st, a) != cudaSuccess) return MOE_ERR_CUDA;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(plan.CS * plan.NG * plan.TG);
-  cfg.blockDim = dim3(kDecThreads);
-  cfg.dynamicSmemBytes = plan.smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = plan.CS;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel, a, xmap, wmap);
-  if (e != cudaSuccess) {  // the pair of attributes was refused: a plain cluster launch
-    cudaGetLastError();
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, decode_kernel, a, xmap, wmap);
-  }
-  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  if (launch_pdl(project_kernel, dim3(plan.KS * plan.NG * plan.TG), dim3(kProjThreads), (size_t)plan.smem, st, a,
+                 xmap, wmap) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (launch_pdl(select_kernel, dim3(T), dim3(kSelThreads), 0, st, a) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
 }
