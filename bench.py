@@ -487,6 +487,26 @@ def secondary_rows(dev, hbm):
     rows["aux_scores_bwd_us"] = _time_calls(
         [(lambda z=z: B.aux_scores_bwd_into(z[2]["probs"], z[4], z[5])) for z in sets], 20, stream)
     del sets
+    # routed-weight backward of the headline workload (T=16384, E=256, k=8): 8 rotated sets of bf16 logits,
+    # ids and weight gradients -> fp32 logit gradients (26.2 MB per call, 210 MB over the sets)
+    g = W.DSV3_GROUPED_SIGMOID
+    gi = W.route_inputs(g)
+    gp = B.route_params(g.T, g.E, g.k, score_fn=g.score_fn, n_group=g.n_group, topk_group=g.topk_group,
+                        group_score_topn=g.group_score_topn, renormalize=1, scaling_factor=g.scaling_factor,
+                        tile_tokens_dim=g.tile_tokens_dim, logits_dtype=g.logits_dtype, bias_dtype=g.bias_dtype,
+                        weights_dtype=g.weights_dtype)
+    rr = B.Router(gp, dev)
+    go = rr(gi["logits"].to(dev), gi["bias"].to(dev))
+    gsets = []
+    for _ in range(8):
+        gsets.append((gi["logits"].to(dev), go["ids"].clone(), torch.randn((g.T, g.k), device=dev),
+                      torch.empty((g.T, g.E), dtype=torch.float32, device=dev),
+                      torch.zeros(64, dtype=torch.uint8, device=dev)))
+    rw_bytes = g.T * g.E * 2 + g.T * g.k * 4 * 2 + g.T * g.E * 4
+    us_rw = _time_calls([(lambda z=z: B.route_weights_bwd_into(gp, z[0], z[1], z[2], z[3], z[4])) for z in gsets],
+                        20, stream)
+    rows["route_weights_bwd"] = {"us": us_rw, "GBps": rw_bytes / us_rw / 1e3, "frac": rw_bytes / us_rw / 1e3 / hbm}
+    del gsets, rr, go
     # decode fused (T=128, H=7168, E=256, k=8): 24 rotated sets of hidden states and router weights
     d = W.DECODE_FUSED
     di = W.decode_inputs(d)

@@ -227,14 +227,20 @@ def route_into(p: RouteParams, logits: torch.Tensor, bias: Optional[torch.Tensor
     _check(rc, "moe_route")
 
 
+def route_weights_bwd_into(p: RouteParams, logits: torch.Tensor, ids: torch.Tensor, grad_weights: torch.Tensor,
+                           grad_logits: torch.Tensor, ws: Optional[torch.Tensor] = None, stream=None) -> None:
+    _check(lib().moe_route_weights_bwd(ctypes.byref(p), _p(logits), _p(ids), _p(grad_weights), _p(grad_logits),
+                                       _p(ws), ctypes.c_size_t(ws.numel() if ws is not None else 0),
+                                       _stream(stream)),
+           "moe_route_weights_bwd")
+
+
 def route_weights_bwd(p: RouteParams, logits: torch.Tensor, ids: torch.Tensor, grad_weights: torch.Tensor,
                       ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """moe_route_weights_bwd: dL/dlogits [T,E] fp32 from dL/dweights [T,k] fp32 for the given selection."""
     T, E = logits.shape
     gl = torch.empty((T, E), dtype=torch.float32, device=logits.device)
-    _check(lib().moe_route_weights_bwd(ctypes.byref(p), _p(logits), _p(ids), _p(grad_weights), _p(gl), _p(ws),
-                                       ctypes.c_size_t(ws.numel() if ws is not None else 0), _stream(stream)),
-           "moe_route_weights_bwd")
+    route_weights_bwd_into(p, logits, ids, grad_weights, gl, ws, stream)
     return gl
 
 

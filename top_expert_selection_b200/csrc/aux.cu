@@ -17,6 +17,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 
@@ -491,15 +492,63 @@ __global__ void __launch_bounds__(kAuxThreads) route_weights_bwd_kernel(int T, i
   pdl_entry();
   const unsigned FULL = 0xffffffffu;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (long long t = (long long)blockIdx.x * kAuxWarps + warp; t < T; t += (long long)gridDim.x * kAuxWarps) {
-    const bool slot = lane < k;
-    int e = slot ? ids[t * k + lane] : 0;
+  const bool vec = (VPL % 4 == 0) && ((E & 3) == 0) && (lane * VPL + VPL <= E) &&
+                   ((reinterpret_cast<uintptr_t>(grad_logits) & 15) == 0);
+  const bool xvec = (VPL % 8 == 0) && logits_dtype == MOE_BF16 && ((E & 7) == 0) && (lane * VPL + VPL <= E) &&
+                    ((reinterpret_cast<uintptr_t>(logits) & 15) == 0);
+  const bool slot = lane < k;
+  // a row's inputs: the slot lanes' ids and weight gradients, and the lane's
+  // logits (experts lane*VPL + i); a slot lane later takes its selected
+  // logit from the owning lane
+  auto load_row = [&](long long t, int& e, float& gw, float* x) {
+    e = slot ? ids[t * k + lane] : 0;
+    gw = slot ? grad_w[t * k + lane] : 0.0f;
+    if (xvec) {
+      const uint16_t* xr = reinterpret_cast<const uint16_t*>(logits) + (size_t)t * E + lane * VPL;
+#pragma unroll
+      for (int i = 0; i < VPL; i += 8) {
+        const uint4 u = __ldcs(reinterpret_cast<const uint4*>(xr + i));
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          x[i + 2 * h] = __uint_as_float(w[h] << 16);
+          x[i + 2 * h + 1] = __uint_as_float(w[h] & 0xffff0000u);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const int ee = lane * VPL + i;
+        x[i] = ee < E ? load_as_f32(logits, logits_dtype, (size_t)t * E + ee) : -INFINITY;
+      }
+    }
+  };
+  const long long stride = (long long)gridDim.x * kAuxWarps;
+  long long t = (long long)blockIdx.x * kAuxWarps + warp;
+  int e_next = 0;
+  float gw_next = 0.0f, x_next[VPL];
+  if (t < T) load_row(t, e_next, gw_next, x_next);
+  for (; t < T; t += stride) {
+    int e = e_next;
+    const float gw = gw_next;
+    float x[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) x[i] = x_next[i];
+    if (t + stride < T) load_row(t + stride, e_next, gw_next, x_next);  // in flight during this row
     if (slot && (unsigned)e >= (unsigned)E) {
       if (hdr) record_bounds(hdr);
       e = 0;
     }
-    const float gw = slot ? grad_w[t * k + lane] : 0.0f;
-    const float xj = slot ? load_as_f32(logits, logits_dtype, (size_t)t * E + e) : -INFINITY;
+    float xj = -INFINITY;
+    {
+      const int src = e / VPL, sub = e - src * VPL;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const float o = __shfl_sync(FULL, x[i], src);
+        if (i == sub) xj = o;
+      }
+      if (!slot) xj = -INFINITY;
+    }
     // scores of the selected (v) and, for softmax before top-k, of the lane's row entries (p)
     float v = 0.0f, pr[VPL];
     float m = 0.0f, z = 0.0f;
@@ -508,14 +557,9 @@ __global__ void __launch_bounds__(kAuxThreads) route_weights_bwd_kernel(int T, i
     if (score_fn == MOE_SIGMOID) {
       v = slot ? sigmoid_f32(xj) : 0.0f;
     } else if (pre) {
-      float x[VPL];
       m = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < VPL; ++i) {
-        const int ee = lane * VPL + i;
-        x[i] = ee < E ? load_as_f32(logits, logits_dtype, (size_t)t * E + ee) : -INFINITY;
-        m = fmaxf(m, x[i]);
-      }
+      for (int i = 0; i < VPL; ++i) m = fmaxf(m, x[i]);
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, off));
 #pragma unroll
@@ -554,28 +598,32 @@ __global__ void __launch_bounds__(kAuxThreads) route_weights_bwd_kernel(int T, i
     float D = v * gv;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) D += __shfl_xor_sync(FULL, D, off);
-    // per-slot contributions (the selected experts of a token are distinct)
-    float g;
-    if (score_fn == MOE_SIGMOID) g = gv * v * (1.0f - v);
-    else if (pre) g = gv;  // gp at the selected expert; the row entries add p * (gp - D) below
-    else g = v * (gv - D);
-    float acc[VPL];
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) acc[i] = 0.0f;
-    for (int j = 0; j < k; ++j) {
-      const int ej = __shfl_sync(FULL, e, j);
-      const float gj = __shfl_sync(FULL, g, j);
-      if (ej / VPL == lane) {
-#pragma unroll
-        for (int i = 0; i < VPL; ++i)
-          if (ej - lane * VPL == i) acc[i] = gj;
-      }
-    }
+    // the row in two stores: every element as if unselected (softmax before
+    // top-k: p * (0 - D); otherwise 0) by its owner lane, 16 bytes at a time,
+    // then after __syncwarp (which orders the warp's memory operations) each
+    // slot lane overwrites its selected expert (the selected experts of a
+    // token are distinct)
+    const bool prerow = score_fn != MOE_SIGMOID && pre;
     float* grow = grad_logits + t * E;
+    float val[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) val[i] = prerow ? pr[i] * (0.0f - D) : 0.0f;
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       const int ee = lane * VPL + i;
-      if (ee < E) __stcs(grow + ee, (score_fn != MOE_SIGMOID && pre) ? pr[i] * (acc[i] - D) : acc[i]);
+      if (vec) {
+        if ((i & 3) == 0 && i + 3 < VPL)
+          __stcs(reinterpret_cast<float4*>(grow + ee), make_float4(val[i], val[i + 1], val[i + 2], val[i + 3]));
+      } else if (ee < E) {
+        __stcs(grow + ee, val[i]);
+      }
+    }
+    __syncwarp();
+    if (slot) {
+      float gs;
+      if (score_fn == MOE_SIGMOID) gs = gv * v * (1.0f - v);
+      else gs = v * (gv - D);  // softmax before top-k: p_e * (gp_e - D) with p_e = v; after: v * (gv - D)
+      grow[e] = gs;
     }
   }
 }
@@ -638,6 +686,22 @@ extern "C" int moe_aux_scores_bwd(int32_t T, int32_t E, int32_t score_fn, const 
   return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// blocks of route_weights_bwd_kernel<V> resident per SM (queried once per V)
+template <int V>
+int rw_resident_blocks() {
+  static int n = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, route_weights_bwd_kernel<V>, kAuxThreads, 0) !=
+            cudaSuccess ||
+        n < 1) {
+      cudaGetLastError();
+      n = 1;
+    }
+  });
+  return n;
+}
+
 extern "C" int moe_route_weights_bwd(const moe_route_params* p, const void* logits, const int32_t* topk_ids,
                                      const float* grad_weights, float* grad_logits, void* ws, size_t ws_bytes,
                                      void* stream) {
@@ -651,10 +715,13 @@ extern "C" int moe_route_weights_bwd(const moe_route_params* p, const void* logi
   if (!logits || !topk_ids || !grad_weights || !grad_logits) return MOE_ERR_INVALID_ARG;
   if (ws && ws_bytes < sizeof(WsHeader)) return MOE_ERR_WORKSPACE;
   const int vpl = pick_vpl(E);
-  const int grid = std::max(1, std::min((T + kAuxWarps - 1) / kAuxWarps, sm_count() * 8));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t err = cudaSuccess;
-  MOE_VPL_SWITCH(vpl, (err = launch_pdl(route_weights_bwd_kernel<V>, dim3(grid), dim3(kAuxThreads), 0, st, T, E, k,
+  // one resident wave (the rows are grid-strided)
+  MOE_VPL_SWITCH(vpl, (err = launch_pdl(route_weights_bwd_kernel<V>,
+                                        dim3(std::max(1, std::min((T + kAuxWarps - 1) / kAuxWarps,
+                                                                  sm_count() * rw_resident_blocks<V>()))),
+                                        dim3(kAuxThreads), 0, st, T, E, k,
                                         p->score_fn, p->softmax_before_topk ? 1 : 0, p->renormalize ? 1 : 0,
                                         p->scaling_factor, logits, p->logits_dtype, topk_ids, grad_weights,
                                         grad_logits, reinterpret_cast<WsHeader*>(ws))));
