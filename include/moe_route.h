@@ -153,8 +153,10 @@ int moe_route_workspace_bytes(const moe_route_params* p, size_t* bytes);
  * Errors: MOE_ERR_INVALID_ARG (sizes, k > E, tile not a power of two, groups
  * not dividing E, k > topk_group * E / n_group, NULL outputs),
  * MOE_ERR_UNSUPPORTED (E or k past the build limits, a group layout the
- * kernels do not map), MOE_ERR_WORKSPACE, MOE_ERR_CUDA; device timeout via
- * moe_status.
+ * kernels do not map: with groups, a lane holds v in {2,3,4,5,6,8,12,16,24,32}
+ * experts (the least with 32v >= E) and a group must span a power of two of
+ * whole lanes or a lane whole groups), MOE_ERR_WORKSPACE, MOE_ERR_CUDA;
+ * device timeout via moe_status.
  */
 int moe_route(const moe_route_params* p, const void* logits, const void* bias, int32_t* topk_ids,
               void* topk_weights, int32_t* expert_counts, int32_t* padded_offsets,

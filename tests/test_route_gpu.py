@@ -103,13 +103,13 @@ for T in (1, 31, 33, 4097):
     EDGE.append(W.RouteSpec(T=T, E=256, k=8, score_fn=W.SIGMOID, n_group=8, topk_group=4, renormalize=1,
                             scaling_factor=2.5, tile_tokens_dim=128, logits_dtype=W.BF16, weights_dtype=W.BF16,
                             has_bias=True, logit_std=2.0, seed=T + 1))
-for E, k in ((4, 1), (16, 6), (64, 8), (72, 6), (128, 8), (384, 8), (1024, 32), (33, 2), (100, 3)):
+for E, k in ((4, 1), (16, 6), (64, 8), (72, 6), (128, 8), (160, 6), (384, 8), (1024, 32), (33, 2), (100, 3)):
     EDGE.append(W.RouteSpec(T=257, E=E, k=k, tile_tokens_dim=8, seed=E))
     EDGE.append(W.RouteSpec(T=257, E=E, k=k, score_fn=W.SIGMOID, has_bias=True, renormalize=0,
                             scaling_factor=1.5, tile_tokens_dim=1, seed=E + 7))
     EDGE.append(W.RouteSpec(T=129, E=E, k=k, softmax_before_topk=0, renormalize=0, logits_dtype=W.BF16,
                             tile_tokens_dim=4, seed=E + 9))
-for E, ng, tg, k in ((64, 8, 4, 8), (128, 4, 2, 6), (256, 16, 4, 8), (16, 4, 2, 3), (384, 8, 3, 8),
+for E, ng, tg, k in ((64, 8, 4, 8), (128, 4, 2, 6), (160, 8, 3, 6), (256, 16, 4, 8), (16, 4, 2, 3), (384, 8, 3, 8),
                      (64, 32, 8, 4), (256, 8, 8, 8)):
     EDGE.append(W.RouteSpec(T=300, E=E, k=k, score_fn=W.SIGMOID, n_group=ng, topk_group=tg, has_bias=True,
                             logits_dtype=W.BF16, logit_std=2.0, tile_tokens_dim=8, seed=E + ng))

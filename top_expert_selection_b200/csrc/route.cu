@@ -1371,7 +1371,7 @@ bool group_layout_ok(const moe_route_params* p, int vpl) {
 // Experts per lane for the warp-per-token path (0 = thread per token): the
 // smallest supported width that covers E in one warp and maps every group onto
 // whole lanes (or whole groups onto one lane).  -1 if none does.
-constexpr int kVplChoices[] = {2, 3, 4, 6, 8, 12, 16, 24, 32};
+constexpr int kVplChoices[] = {2, 3, 4, 5, 6, 8, 12, 16, 24, 32};
 
 int pick_mode(const moe_route_params* p) {
   const int E = p->num_experts;
@@ -1559,6 +1559,7 @@ extern "C" int moe_route(const moe_route_params* p, const void* logits, const vo
       case 2: err = launch_route<2, 0>(a, smem, st); break;
       case 3: err = launch_route<3, 0>(a, smem, st); break;
       case 4: err = launch_route<4, 0>(a, smem, st); break;
+      case 5: err = launch_route<5, 0>(a, smem, st); break;  // e.g. 160 experts in groups of 20
       case 6: err = launch_route<6, 0>(a, smem, st); break;
       case 8: err = launch_route<8, 0>(a, smem, st); break;
       case 12: err = launch_route<12, 0>(a, smem, st); break;
