@@ -50,7 +50,7 @@ def _lib():
         L.oracle_route_select.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32, f32,
                                           P, i32, P, i32, P, P, P, P, P]
         L.oracle_route_capacity.argtypes = [i32, i32, i32, i32, P, P]
-        L.oracle_route_bookkeeping.argtypes = [i32, i32, i32, i32, P, P, P, P, P, P, P, P]
+        L.oracle_route_bookkeeping.argtypes = [i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P]
         L.oracle_aux_scores.argtypes = [i32, i32, i32, i32, P, P, P, P]
         L.oracle_aux_loss_fwd.argtypes = [i32, i32, i32, i32, f32, P, P, P]
         L.oracle_aux_loss_bwd.argtypes = [i32, i32, i32, i32, f32, f32, P, P, P, P]
@@ -157,18 +157,23 @@ def route_capacity(T: int, E: int, k: int, tile: int):
     return int(mp.value), int(mt.value)
 
 
-def route_bookkeeping(ids, E: int, tile: int) -> dict:
+def route_bookkeeping(ids, E: int, tile: int, local_expert_offset: int = 0,
+                      local_num_experts: Optional[int] = None) -> dict:
+    """Bookkeeping of the experts [local_expert_offset, local_expert_offset + local_num_experts)
+    (all E by default); counts/offsets/tile_expert are indexed by the local expert."""
     ids = as_numpy(ids).astype(np.int32, copy=False)
     T, k = ids.shape
+    nl = E if local_num_experts is None else int(local_num_experts)
     max_padded, max_tiles = route_capacity(T, E, k, tile)
-    counts = np.zeros(E, np.int32)
-    offsets = np.zeros(E + 1, np.int32)
+    counts = np.zeros(nl, np.int32)
+    offsets = np.zeros(nl + 1, np.int32)
     e2p = np.zeros(T * k, np.int32)
     p2t = np.full(max(max_padded, 1), -7, np.int32)
     te = np.full(max(max_tiles, 1), -7, np.int32)
     tl = np.full(max(max_tiles, 1), -7, np.int32)
     totals = np.zeros(2, np.int32)
-    rc = _lib().oracle_route_bookkeeping(T, E, k, tile, _ptr(np.ascontiguousarray(ids)), _ptr(counts),
+    rc = _lib().oracle_route_bookkeeping(T, E, k, tile, int(local_expert_offset), nl,
+                                         _ptr(np.ascontiguousarray(ids)), _ptr(counts),
                                          _ptr(offsets), _ptr(e2p), _ptr(p2t), _ptr(te), _ptr(tl),
                                          _ptr(totals))
     _check(rc, "route_bookkeeping")

@@ -263,43 +263,55 @@ int oracle_route_capacity(int T, int E, int k, int tile, int64_t* max_padded, in
 
 /*
  * Permutation bookkeeping for a grouped GEMM [TRT: Returns; Notes; LMD:
- * invokeMoeGate_V2 offsets and maps].
- *   counts[e]      = number of (t, j) with ids[t,j] == e
- *   padded_e       = ceil(counts[e] / tile) * tile        (tile a power of two)
- *   offsets[0] = 0, offsets[e+1] = offsets[e] + padded_e;  P = offsets[E]
- *   e2p[t*k + j]   = offsets[e] + (number of earlier (t', j') in token-major
- *                    order routed to the same e)  -- slots follow token order
+ * invokeMoeGate_V2 offsets and maps], for the experts of one expert-parallel
+ * shard [TRT: Parameters, local_expert_offset / local_num_experts; Notes: a
+ * tile's expert is its batch index + local_expert_offset].  Expert e is local
+ * when off <= e < off + nl; its local index is le = e - off (off = 0, nl = E:
+ * every expert, the single-GPU case).
+ *   counts[le]     = number of (t, j) with ids[t,j] == off + le
+ *   padded_le      = ceil(counts[le] / tile) * tile        (tile a power of two)
+ *   offsets[0] = 0, offsets[le+1] = offsets[le] + padded_le;  P = offsets[nl]
+ *   e2p[t*k + j]   = offsets[le] + (number of earlier (t', j') in token-major
+ *                    order routed to the same expert)  -- slots follow token
+ *                    order; -1 when ids[t,j] is not local (READING)
  *   p2t[p]         = t for every filled slot, -1 on padding (READING)
- *   for tile c in [0, P / tile): tile_expert[c] = the e whose padded range
- *                    holds row c*tile; tile_mn_limit[c] = min((c+1)*tile,
- *                    offsets[e] + counts[e])  (READING: exclusive end row)
+ *   for tile c in [0, P / tile): tile_expert[c] = the le whose padded range
+ *                    holds row c*tile (the batch index); tile_mn_limit[c] =
+ *                    min((c+1)*tile, offsets[le] + counts[le])  (READING:
+ *                    exclusive end row)
  *   totals = {P, P / tile}
  * Entries of p2t at or past P and of the tile tables at or past P/tile are
  * left as the caller filled them.
  */
-int oracle_route_bookkeeping(int T, int E, int k, int tile, const int32_t* ids,
+int oracle_route_bookkeeping(int T, int E, int k, int tile, int off, int nl, const int32_t* ids,
                              int32_t* counts, int32_t* offsets, int32_t* e2p, int32_t* p2t,
                              int32_t* tile_expert, int32_t* tile_mn_limit, int32_t* totals) {
   if (T < 0 || E <= 0 || k <= 0 || !is_pow2(tile)) return -1;
-  for (int e = 0; e < E; ++e) counts[e] = 0;
+  if (off < 0 || nl <= 0 || off + nl > E) return -1;
+  for (int le = 0; le < nl; ++le) counts[le] = 0;
   for (int64_t i = 0; i < (int64_t)T * k; ++i) {
     int e = ids[i];
     if (e < 0 || e >= E) return -1;
-    counts[e] += 1;
+    if (e >= off && e < off + nl) counts[e - off] += 1;
   }
   offsets[0] = 0;
-  for (int e = 0; e < E; ++e) {
-    int32_t padded = ((counts[e] + tile - 1) / tile) * tile;
-    offsets[e + 1] = offsets[e] + padded;
+  for (int le = 0; le < nl; ++le) {
+    int32_t padded = ((counts[le] + tile - 1) / tile) * tile;
+    offsets[le + 1] = offsets[le] + padded;
   }
-  int32_t P = offsets[E];
+  int32_t P = offsets[nl];
   for (int32_t p = 0; p < P; ++p) p2t[p] = -1;
-  int32_t* running = (int32_t*)calloc((size_t)E, sizeof(int32_t));
+  int32_t* running = (int32_t*)calloc((size_t)nl, sizeof(int32_t));
   for (int t = 0; t < T; ++t) {
     for (int j = 0; j < k; ++j) {
       int e = ids[(size_t)t * k + j];
-      int32_t slot = offsets[e] + running[e];
-      running[e] += 1;
+      if (e < off || e >= off + nl) {
+        e2p[(size_t)t * k + j] = -1;
+        continue;
+      }
+      int le = e - off;
+      int32_t slot = offsets[le] + running[le];
+      running[le] += 1;
       e2p[(size_t)t * k + j] = slot;
       p2t[slot] = t;
     }
@@ -308,11 +320,11 @@ int oracle_route_bookkeeping(int T, int E, int k, int tile, const int32_t* ids,
   int32_t ntiles = P / tile;
   for (int32_t c = 0; c < ntiles; ++c) {
     int32_t row = c * tile;
-    int e = 0;
-    while (!(offsets[e] <= row && row < offsets[e + 1])) ++e;
+    int le = 0;
+    while (!(offsets[le] <= row && row < offsets[le + 1])) ++le;
     int32_t lim = (c + 1) * tile;
-    int32_t valid_end = offsets[e] + counts[e];
-    tile_expert[c] = e;
+    int32_t valid_end = offsets[le] + counts[le];
+    tile_expert[c] = le;
     tile_mn_limit[c] = lim < valid_end ? lim : valid_end;
   }
   totals[0] = P;

@@ -73,9 +73,39 @@ def test_f64_to_bf16_single_rounding_brute_force():
 @pytest.mark.parametrize("case", read_golden("bookkeeping_handworked.txt"), ids=lambda c: c["case"])
 def test_bookkeeping_handworked(case):
     ids = np.array([ints(r) for r in case["ids"].split("|")], np.int32)
-    out = oracle.route_bookkeeping(ids, int(case["E"]), int(case["tile"]))
+    out = oracle.route_bookkeeping(ids, int(case["E"]), int(case["tile"]), int(case.get("local_offset", 0)),
+                                   int(case["local_num"]) if "local_num" in case else None)
     for key in ("counts", "offsets", "e2p", "p2t", "tile_expert", "tile_mn_limit", "totals"):
         assert out[key].tolist() == ints(case[key]), key
+
+
+@pytest.mark.parametrize("tile", [1, 4, 128])
+@pytest.mark.parametrize("shards", [[(0, 4), (4, 4), (8, 4), (12, 4)], [(0, 5), (5, 6), (11, 5)], [(3, 1)]])
+def test_bookkeeping_shards_match_the_global_bookkeeping(tile, shards):
+    # an expert-parallel shard's bookkeeping is the global bookkeeping restricted to its experts
+    # and shifted by the global offset of its first expert (slots, token map, tiles)
+    rng = np.random.default_rng(tile + len(shards))
+    T, E, k = 203, 16, 3
+    ids = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    g = oracle.route_bookkeeping(ids, E, tile)
+    owned = np.zeros(T * k, np.int32)
+    for off, nl in shards:
+        s = oracle.route_bookkeeping(ids, E, tile, off, nl)
+        base = int(g["offsets"][off])
+        assert np.array_equal(s["counts"], g["counts"][off:off + nl])
+        assert np.array_equal(s["offsets"], g["offsets"][off:off + nl + 1] - base)
+        loc = (ids.ravel() >= off) & (ids.ravel() < off + nl)
+        owned += loc
+        assert np.all(s["e2p"][~loc] == -1)
+        assert np.array_equal(s["e2p"][loc], g["e2p"][loc] - base)
+        P = int(s["totals"][0])
+        assert P == int(g["offsets"][off + nl]) - base
+        assert np.array_equal(s["p2t"], g["p2t"][base:base + P])
+        t0, t1 = base // tile, (base + P) // tile
+        assert np.array_equal(s["tile_expert"] + off, g["tile_expert"][t0:t1])
+        assert np.array_equal(s["tile_mn_limit"], g["tile_mn_limit"][t0:t1] - base)
+    if sum(nl for _, nl in shards) == E:
+        assert np.all(owned == 1)  # every selection has exactly one owning shard
 
 
 def _check_bookkeeping_invariants(ids, E, tile, bk):
