@@ -85,6 +85,14 @@ typedef struct moe_route_params {
   int32_t logits_dtype;        /* MOE_F32 | MOE_BF16 [TRT: routing_logits] */
   int32_t bias_dtype;          /* MOE_F32 | MOE_BF16 [TRT: routing_bias] */
   int32_t weights_dtype;       /* MOE_F32 | MOE_BF16 [TRT: Notes, topk_weights dtype] */
+  int32_t local_expert_offset; /* expert-parallel shard: the experts [local_expert_offset,   */
+  int32_t local_num_experts;   /* local_expert_offset + local_num_experts) are local; 0 (with
+                                  offset 0) = all E [TRT: local_expert_offset, local_num_experts].
+                                  Selection and weights stay global; counts, offsets, slots and
+                                  tiles cover the local experts only (tile_expert = local index,
+                                  global expert = it + local_expert_offset [TRT: Notes]); a
+                                  selection of another shard's expert gets
+                                  expanded_to_permuted = -1 */
 } moe_route_params;
 
 /* Human-readable name of a status code (static string). */
@@ -128,14 +136,18 @@ int moe_route_workspace_bytes(const moe_route_params* p, size_t* bytes);
  *   weight  w_j = v_j / sum(v) * scale (renormalize) or v_j * scale, where v_j
  *           is the selected expert's unbiased score (softmax_before_topk == 0:
  *           the score function applied to the k selected logits)
- * Bookkeeping over all T*k selections (token-major order):
- *   expert_counts[e]          rows routed to e
- *   padded_offsets[e]         exclusive prefix of ceil(count/tile)*tile; [E] = P
+ * Bookkeeping over all T*k selections (token-major order), for the local
+ * experts e = local_expert_offset + le, le < L = local_num_experts (all E
+ * when local_num_experts == 0):
+ *   expert_counts[le]         rows routed to e
+ *   padded_offsets[le]        exclusive prefix of ceil(count/tile)*tile; [L] = P
  *   expanded_to_permuted[i]   row of selection i = t*k + j in the expert-
  *                             contiguous padded layout; rows of one expert
- *                             follow token order
+ *                             follow token order; -1 when the selected
+ *                             expert is not local
  *   permuted_to_token[p]      source token of row p, -1 on padding rows (p < P)
- *   tile_expert[c]            expert of tile c (rows c*tile .. c*tile+tile-1)
+ *   tile_expert[c]            local expert le of tile c (rows c*tile ..
+ *                             c*tile+tile-1)
  *   tile_mn_limit[c]          exclusive end of tile c's valid rows
  *   totals[0] = P (total_num_padded_tokens), totals[1] = P / tile
  *                             (num_non_exiting_ctas); device-resident, so a
@@ -146,12 +158,13 @@ int moe_route_workspace_bytes(const moe_route_params* p, size_t* bytes);
  * Device pointers (caller-owned):
  *   logits [T,E] (logits_dtype), bias [E] (bias_dtype) or NULL,
  *   topk_ids [T,k] int32, topk_weights [T,k] (weights_dtype),
- *   expert_counts [E], padded_offsets [E+1], expanded_to_permuted [T*k],
+ *   expert_counts [L], padded_offsets [L+1], expanded_to_permuted [T*k],
  *   permuted_to_token [max_padded], tile_expert [max_tiles],
  *   tile_mn_limit [max_tiles], totals [2] -- all int32,
  *   ws [ws_bytes] from moe_route_workspace_bytes (zero-filled before first use).
  * Errors: MOE_ERR_INVALID_ARG (sizes, k > E, tile not a power of two, groups
- * not dividing E, k > topk_group * E / n_group, NULL outputs),
+ * not dividing E, k > topk_group * E / n_group, a local expert range outside
+ * [0, E), NULL outputs),
  * MOE_ERR_UNSUPPORTED (E or k past the build limits, a group layout the
  * kernels do not map: with groups, a lane holds v in {2,3,4,5,6,8,12,16,24,32}
  * experts (the least with 32v >= E) and a group must span a power of two of

@@ -128,16 +128,18 @@ def compare_route(spec: dict, gpu: dict, orc: dict, *, max_flip_frac: float = 1e
         err = np.abs(w[same].astype(np.float64) - ref) - F32_RTOL * np.abs(ref)
         assert err.max(initial=-1) <= 0, f"fp32 weights rel err {np.max(np.abs(w[same] - ref) / np.abs(ref))}"
 
-    # bookkeeping: bit-exact vs the oracle re-run on the GPU's ids
-    bk = oracle.route_bookkeeping(g_ids, E, tile)
+    # bookkeeping (of the local experts, all E by default): bit-exact vs the oracle re-run on the GPU's ids
+    off = spec.get("local_expert_offset", 0)
+    nl = spec.get("local_num_experts", 0) or E
+    bk = oracle.route_bookkeeping(g_ids, E, tile, off, nl)
     P, nt = int(bk["totals"][0]), int(bk["totals"][1])
     got_totals = to_np(gpu["totals"]).tolist()
     assert got_totals == [P, nt], f"totals {got_totals} vs {[P, nt]}"
-    for name, n in (("counts", E), ("offsets", E + 1), ("e2p", T * k), ("p2t", P), ("tile_expert", nt),
+    for name, n in (("counts", nl), ("offsets", nl + 1), ("e2p", T * k), ("p2t", P), ("tile_expert", nt),
                     ("tile_mn_limit", nt)):
         got = to_np(gpu[name])[:n]
         assert np.array_equal(got, bk[name][:n]), f"{name} differs from the oracle on the GPU's ids"
     if not flips:
-        bk0 = oracle.route_bookkeeping(o_ids, E, tile)
+        bk0 = oracle.route_bookkeeping(o_ids, E, tile, off, nl)
         assert np.array_equal(bk0["e2p"], bk["e2p"]) and np.array_equal(bk0["p2t"], bk["p2t"])
     return {"tokens": T, "flips": len(flips), "flip_tokens": flips[:10], "P": P, "tiles": nt}

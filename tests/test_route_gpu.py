@@ -48,12 +48,14 @@ def run_route(spec: W.RouteSpec, logits=None, bias=None):
                        n_group=spec.n_group, topk_group=spec.topk_group, group_score_topn=spec.group_score_topn,
                        renormalize=spec.renormalize, scaling_factor=spec.scaling_factor,
                        tile_tokens_dim=spec.tile_tokens_dim, logits_dtype=spec.logits_dtype,
-                       bias_dtype=spec.bias_dtype, weights_dtype=spec.weights_dtype)
+                       bias_dtype=spec.bias_dtype, weights_dtype=spec.weights_dtype,
+                       local_expert_offset=spec.local_expert_offset, local_num_experts=spec.local_num_experts)
     max_padded, max_tiles = B.route_capacity(p)
     T, E, k = spec.T, spec.E, spec.k
+    nl = spec.local_num_experts or E
     wdt = torch.bfloat16 if spec.weights_dtype == W.BF16 else torch.float32
-    sizes = {"ids": (T * k, torch.int32), "weights": (T * k, wdt), "counts": (E, torch.int32),
-             "offsets": (E + 1, torch.int32), "e2p": (T * k, torch.int32), "p2t": (max_padded, torch.int32),
+    sizes = {"ids": (T * k, torch.int32), "weights": (T * k, wdt), "counts": (nl, torch.int32),
+             "offsets": (nl + 1, torch.int32), "e2p": (T * k, torch.int32), "p2t": (max_padded, torch.int32),
              "tile_expert": (max_tiles, torch.int32), "tile_mn_limit": (max_tiles, torch.int32),
              "totals": (2, torch.int32)}
     fulls, views = {}, {}
@@ -77,7 +79,8 @@ def run_route(spec: W.RouteSpec, logits=None, bias=None):
                               n_group=spec.n_group, topk_group=spec.topk_group,
                               group_score_topn=spec.group_score_topn, renormalize=spec.renormalize,
                               scaling_factor=spec.scaling_factor, bias=bias)
-    sp = {"k": k, "E": E, "tile": spec.tile_tokens_dim, "n_group": spec.n_group, "topk_group": spec.topk_group}
+    sp = {"k": k, "E": E, "tile": spec.tile_tokens_dim, "n_group": spec.n_group, "topk_group": spec.topk_group,
+          "local_expert_offset": spec.local_expert_offset, "local_num_experts": spec.local_num_experts}
     rep = compare_route(sp, gpu, orc)
     return rep, gpu, (p, lg_d, b_d, ws, views)
 
@@ -328,3 +331,30 @@ def test_route_weights_backward_bad_id_recorded():
     B.route_weights_bwd(p, lg, ids, torch.ones(4, 2, device="cuda"), ws=ws)
     torch.cuda.synchronize()
     assert B.status(ws) == B.MOE_ERR_DEVICE_BOUNDS
+
+
+# expert-parallel shards: selection global, bookkeeping of the local experts only
+@pytest.mark.parametrize("spec", [
+    W.DSV3_GROUPED_SIGMOID.with_(T=4096, local_expert_offset=64, local_num_experts=64),
+    W.DSV3_GROUPED_SIGMOID.with_(T=777, local_expert_offset=0, local_num_experts=32),
+    W.DSV3_GROUPED_SIGMOID.with_(T=777, local_expert_offset=255, local_num_experts=1),
+    W.RouteSpec(T=5000, E=8, k=2, softmax_before_topk=0, renormalize=0, logits_dtype=W.BF16, tile_tokens_dim=128,
+                local_expert_offset=2, local_num_experts=4, seed=3),
+    W.RouteSpec(T=300, E=160, k=6, score_fn=W.SOFTMAX, n_group=8, topk_group=3, tile_tokens_dim=8,
+                local_expert_offset=40, local_num_experts=40, seed=11),
+    W.RouteSpec(T=129, E=16, k=3, tile_tokens_dim=4, local_expert_offset=5, local_num_experts=7, seed=12),
+], ids=lambda s: f"T{s.T}-E{s.E}-local{s.local_expert_offset}+{s.local_num_experts}")
+def test_route_expert_parallel_shard(spec):
+    rep, gpu, _ = run_route(spec)
+    e2p = to_np(gpu["e2p"]).reshape(spec.T, spec.k)
+    ids = to_np(gpu["ids"])
+    loc = (ids >= spec.local_expert_offset) & (ids < spec.local_expert_offset + spec.local_num_experts)
+    assert np.all(e2p[~loc] == -1) and np.all(e2p[loc] >= 0)
+    print(rep)
+
+
+def test_route_expert_parallel_shard_bad_range():
+    for off, nl in ((-1, 4), (6, 4), (3, -2), (2, 0)):
+        p = B.route_params(16, 8, 2, local_expert_offset=off, local_num_experts=nl)
+        with pytest.raises(B.MoeError):
+            B.Router(p)(torch.randn(16, 8, device="cuda"))

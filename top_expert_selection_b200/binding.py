@@ -56,6 +56,7 @@ class RouteParams(ctypes.Structure):
         ("renormalize", ctypes.c_int32), ("scaling_factor", ctypes.c_float),
         ("tile_tokens_dim", ctypes.c_int32), ("logits_dtype", ctypes.c_int32), ("bias_dtype", ctypes.c_int32),
         ("weights_dtype", ctypes.c_int32),
+        ("local_expert_offset", ctypes.c_int32), ("local_num_experts", ctypes.c_int32),
     ]
 
 
@@ -148,9 +149,12 @@ def status(ws: torch.Tensor, clear: bool = True, stream=None) -> int:
 def route_params(T: int, E: int, k: int, *, score_fn: int = SOFTMAX, softmax_before_topk: int = 1,
                  n_group: int = 0, topk_group: int = 0, group_score_topn: int = 2, renormalize: int = 1,
                  scaling_factor: float = 1.0, tile_tokens_dim: int = 8, logits_dtype: int = F32,
-                 bias_dtype: int = F32, weights_dtype: int = F32) -> RouteParams:
+                 bias_dtype: int = F32, weights_dtype: int = F32, local_expert_offset: int = 0,
+                 local_num_experts: int = 0) -> RouteParams:
+    """local_num_experts == 0: every expert is local (single GPU)."""
     return RouteParams(T, E, k, score_fn, softmax_before_topk, n_group, topk_group, group_score_topn,
-                       renormalize, scaling_factor, tile_tokens_dim, logits_dtype, bias_dtype, weights_dtype)
+                       renormalize, scaling_factor, tile_tokens_dim, logits_dtype, bias_dtype, weights_dtype,
+                       local_expert_offset, local_num_experts)
 
 
 def route_capacity(p: RouteParams):
@@ -172,12 +176,13 @@ class Router:
             _check(L.moe_route_workspace_bytes(ctypes.byref(p), ctypes.byref(nb)), "moe_route_workspace_bytes")
         dev = self.device
         T, E, k = p.num_tokens, p.num_experts, p.top_k
+        L_e = p.local_num_experts if p.local_num_experts > 0 else E  # the local experts' bookkeeping
         self.ws = make_workspace(nb.value, dev)
         self.out = {
             "ids": torch.empty((T, k), dtype=torch.int32, device=dev),
             "weights": torch.empty((T, k), dtype=_TORCH[p.weights_dtype], device=dev),
-            "counts": torch.empty(E, dtype=torch.int32, device=dev),
-            "offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
+            "counts": torch.empty(L_e, dtype=torch.int32, device=dev),
+            "offsets": torch.empty(L_e + 1, dtype=torch.int32, device=dev),
             "e2p": torch.empty(T * k, dtype=torch.int32, device=dev),
             "p2t": torch.empty(max(self.max_padded, 1), dtype=torch.int32, device=dev),
             "tile_expert": torch.empty(max(self.max_tiles, 1), dtype=torch.int32, device=dev),

@@ -88,6 +88,7 @@ struct RouteArgs {
   int G;
   int max_padded;
   int max_tiles;
+  int loc_off, loc_n;  // the local experts [loc_off, loc_off + loc_n): only they get slots and tiles
   int chunk_tokens;
   int stage_bytes;  // stage region: >= chunk_tokens * row_bytes and >= phase 2's partials
   int row_bytes;
@@ -223,6 +224,11 @@ __device__ __forceinline__ float sigmoid_bf16_row(const float* lut, const uint8_
 // -------------------------------------------------------------------------
 // keep a copy of a selection in the block's shared-memory id list (phase 2
 // reads it instead of global memory)
+// expert e belongs to this shard: it is counted and gets slots
+__device__ __forceinline__ bool is_local(const RouteArgs& a, int e) {
+  return (unsigned)(e - a.loc_off) < (unsigned)a.loc_n;
+}
+
 __device__ __forceinline__ void keep_id(uint16_t* ids_s, int local_item, int e) {
   if (ids_s) ids_s[local_item] = (uint16_t)e;
 }
@@ -410,7 +416,11 @@ __device__ void select_token_warp(const RouteArgs& a, const uint8_t* row, int t,
     a.ids[o] = my_id;
     keep_id(ids_s, (t - t_base) * a.k + lane, my_id);
     store_from_f32(a.weights, a.weights_dtype, o, v);
-    if ((unsigned)my_id < (unsigned)E) atomicAdd(&hist_cta[my_id], 1); else record_bounds(a.hdr);
+    if ((unsigned)my_id < (unsigned)E) {
+      if (is_local(a, my_id)) atomicAdd(&hist_cta[my_id], 1);
+    } else {
+      record_bounds(a.hdr);
+    }
   }
 }
 
@@ -538,7 +548,11 @@ __device__ void select_token_thread(const RouteArgs& a, const uint8_t* row, int 
       a.ids[o] = sel[j];
       keep_id(ids_s, (t - t_base) * a.k + j, sel[j]);
       store_from_f32(a.weights, a.weights_dtype, o, w);
-      if ((unsigned)sel[j] < (unsigned)E) atomicAdd(&hist_cta[sel[j]], 1); else record_bounds(a.hdr);
+      if ((unsigned)sel[j] < (unsigned)E) {
+        if (is_local(a, sel[j])) atomicAdd(&hist_cta[sel[j]], 1);
+      } else {
+        record_bounds(a.hdr);
+      }
     }
   }
 }
@@ -624,7 +638,11 @@ __device__ __noinline__ void select_token_exact8(const RouteArgs& a, const uint8
       a.ids[(size_t)t * a.k + jr] = win;
       keep_id(ids_s, (int)(t - t_base) * a.k + jr, win);
       ssum = ssum + sg;
-      if ((unsigned)win < (unsigned)a.E) atomicAdd(&hist_cta[win], 1); else record_bounds(a.hdr);
+      if ((unsigned)win < (unsigned)a.E) {
+        if (is_local(a, win)) atomicAdd(&hist_cta[win], 1);
+      } else {
+        record_bounds(a.hdr);
+      }
     }
   }
   if (g == 0) {
@@ -844,7 +862,7 @@ __device__ void select_quad_fast(const RouteArgs& a, const uint8_t* stage, int l
         a.ids[o] = my_e[r];
         keep_id(ids_s, (int)(t - t_base) * a.k + my_rank[r], my_e[r]);
         store_from_f32(a.weights, a.weights_dtype, o, wv);
-        atomicAdd(&hist_cta[my_e[r]], 1);
+        if (is_local(a, my_e[r])) atomicAdd(&hist_cta[my_e[r]], 1);
       }
     }
   }
@@ -1216,12 +1234,13 @@ __global__ void __launch_bounds__((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneri
     scan_padded_offsets(cnt, offs, E, a.tile, scan_scratch);
     P = offs[E];
     if (c == 0) {
-      for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        a.counts[e] = cnt[e];
-        a.offsets[e] = offs[e];
+      // the shard's experts (those before it have no rows: offs[loc_off] == 0)
+      for (int le = threadIdx.x; le < a.loc_n; le += blockDim.x) {
+        a.counts[le] = cnt[a.loc_off + le];
+        a.offsets[le] = offs[a.loc_off + le];
       }
       if (threadIdx.x == 0) {
-        a.offsets[E] = P;
+        a.offsets[a.loc_n] = P;
         a.totals[0] = P;
         a.totals[1] = P / a.tile;
       }
@@ -1236,6 +1255,10 @@ __global__ void __launch_bounds__((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneri
       const int e = ids_s[i];
       if (e >= E) {
         record_bounds(a.hdr);
+        continue;
+      }
+      if (!is_local(a, e)) {  // another shard's expert: no slot
+        a.e2p[i_begin + i] = -1;
         continue;
       }
       const int slot = offs[e] + hist_cta[e] + lrank_s[i];
@@ -1279,8 +1302,12 @@ __global__ void __launch_bounds__((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneri
         const int slot = hist_w[warp * E + e] + rank;
         __syncwarp(amask);
         if (lane == leader) hist_w[warp * E + e] += __popc(m);
-        a.e2p[i_begin + i] = slot;
-        if ((unsigned)slot < (unsigned)a.max_padded) a.p2t[slot] = (int)((i_begin + i) / a.k); else record_bounds(a.hdr);
+        if (is_local(a, e)) {
+          a.e2p[i_begin + i] = slot;
+          if ((unsigned)slot < (unsigned)a.max_padded) a.p2t[slot] = (int)((i_begin + i) / a.k); else record_bounds(a.hdr);
+        } else {
+          a.e2p[i_begin + i] = -1;  // another shard's expert: no slot
+        }
       }
       __syncwarp();
     }
@@ -1301,7 +1328,7 @@ __global__ void __launch_bounds__((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneri
     }
     const int lim = min(row + a.tile, offs[lo] + cnt[lo]);
     if (lane == 0) {
-      a.tile_expert[tc] = lo;
+      a.tile_expert[tc] = lo - a.loc_off;  // the local expert (batch index)
       a.tile_mn[tc] = lim;
     }
     for (int r = lim + lane; r < row + a.tile; r += 32) a.p2t[r] = -1;
@@ -1339,6 +1366,10 @@ int validate(const moe_route_params* p) {
   if (p->num_tokens < 0 || p->num_experts <= 0 || p->top_k <= 0 || p->top_k > p->num_experts)
     return MOE_ERR_INVALID_ARG;
   if (p->score_fn != MOE_SOFTMAX && p->score_fn != MOE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (p->local_expert_offset < 0 || p->local_num_experts < 0 ||
+      (long long)p->local_expert_offset + (p->local_num_experts > 0 ? p->local_num_experts : 1) > p->num_experts ||
+      (p->local_num_experts == 0 && p->local_expert_offset != 0))
+    return MOE_ERR_INVALID_ARG;
   if ((p->logits_dtype != MOE_F32 && p->logits_dtype != MOE_BF16) ||
       (p->bias_dtype != MOE_F32 && p->bias_dtype != MOE_BF16) ||
       (p->weights_dtype != MOE_F32 && p->weights_dtype != MOE_BF16))
@@ -1525,6 +1556,8 @@ extern "C" int moe_route(const moe_route_params* p, const void* logits, const vo
     a.max_padded = (int)mp;
     a.max_tiles = (int)mt;
   }
+  a.loc_off = p->local_expert_offset;
+  a.loc_n = p->local_num_experts > 0 ? p->local_num_experts : p->num_experts;
   a.row_bytes = p->num_experts * esize(p->logits_dtype);
   const int per_block = (T + a.G - 1) / a.G;
   a.chunk_tokens = std::max(1, std::min(per_block, kStageBytesMax / a.row_bytes));

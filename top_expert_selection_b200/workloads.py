@@ -66,6 +66,8 @@ class RouteSpec:
     logits_dtype: int = F32
     bias_dtype: int = F32
     weights_dtype: int = F32
+    local_expert_offset: int = 0  # expert-parallel shard (local_num_experts 0: all experts local)
+    local_num_experts: int = 0
     has_bias: bool = False
     # distributions
     logit_mean: float = 0.0
