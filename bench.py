@@ -487,6 +487,19 @@ def secondary_rows(dev, hbm):
     rows["aux_scores_bwd_us"] = _time_calls(
         [(lambda z=z: B.aux_scores_bwd_into(z[2]["probs"], z[4], z[5])) for z in sets], 20, stream)
     del sets
+    # the headline workload routed for one expert-parallel shard of four (experts 64..127): selection of
+    # all 256 experts, bookkeeping of the shard's 64 (24 rotated logit sets, as the headline)
+    g = W.DSV3_GROUPED_SIGMOID
+    gi = W.route_inputs(g)
+    sp = B.route_params(g.T, g.E, g.k, score_fn=g.score_fn, n_group=g.n_group, topk_group=g.topk_group,
+                        group_score_topn=g.group_score_topn, renormalize=1, scaling_factor=g.scaling_factor,
+                        tile_tokens_dim=g.tile_tokens_dim, logits_dtype=g.logits_dtype, bias_dtype=g.bias_dtype,
+                        weights_dtype=g.weights_dtype, local_expert_offset=64, local_num_experts=64)
+    srs = [B.Router(sp, dev) for _ in range(24)]
+    slg = [gi["logits"].to(dev) for _ in range(24)]
+    sb = gi["bias"].to(dev)
+    rows["ep_shard_route_us"] = _time_calls([(lambda i=i: srs[i](slg[i], sb)) for i in range(24)], 20, stream)
+    del srs, slg
     # routed-weight backward of the headline workload (T=16384, E=256, k=8): 8 rotated sets of bf16 logits,
     # ids and weight gradients -> fp32 logit gradients (26.2 MB per call, 210 MB over the sets)
     g = W.DSV3_GROUPED_SIGMOID
