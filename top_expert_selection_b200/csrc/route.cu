@@ -224,7 +224,8 @@ __device__ __forceinline__ float sigmoid_bf16_row(const float* lut, const uint8_
 // -------------------------------------------------------------------------
 // keep a copy of a selection in the block's shared-memory id list (phase 2
 // reads it instead of global memory)
-// expert e belongs to this shard: it is counted and gets slots
+// expert e belongs to this shard: it gets rows, slots and tiles (phase 1
+// counts every expert; phase 2 gives the others zero width)
 __device__ __forceinline__ bool is_local(const RouteArgs& a, int e) {
   return (unsigned)(e - a.loc_off) < (unsigned)a.loc_n;
 }
@@ -416,11 +417,7 @@ __device__ void select_token_warp(const RouteArgs& a, const uint8_t* row, int t,
     a.ids[o] = my_id;
     keep_id(ids_s, (t - t_base) * a.k + lane, my_id);
     store_from_f32(a.weights, a.weights_dtype, o, v);
-    if ((unsigned)my_id < (unsigned)E) {
-      if (is_local(a, my_id)) atomicAdd(&hist_cta[my_id], 1);
-    } else {
-      record_bounds(a.hdr);
-    }
+    if ((unsigned)my_id < (unsigned)E) atomicAdd(&hist_cta[my_id], 1); else record_bounds(a.hdr);
   }
 }
 
@@ -548,11 +545,7 @@ __device__ void select_token_thread(const RouteArgs& a, const uint8_t* row, int 
       a.ids[o] = sel[j];
       keep_id(ids_s, (t - t_base) * a.k + j, sel[j]);
       store_from_f32(a.weights, a.weights_dtype, o, w);
-      if ((unsigned)sel[j] < (unsigned)E) {
-        if (is_local(a, sel[j])) atomicAdd(&hist_cta[sel[j]], 1);
-      } else {
-        record_bounds(a.hdr);
-      }
+      if ((unsigned)sel[j] < (unsigned)E) atomicAdd(&hist_cta[sel[j]], 1); else record_bounds(a.hdr);
     }
   }
 }
@@ -638,11 +631,7 @@ __device__ __noinline__ void select_token_exact8(const RouteArgs& a, const uint8
       a.ids[(size_t)t * a.k + jr] = win;
       keep_id(ids_s, (int)(t - t_base) * a.k + jr, win);
       ssum = ssum + sg;
-      if ((unsigned)win < (unsigned)a.E) {
-        if (is_local(a, win)) atomicAdd(&hist_cta[win], 1);
-      } else {
-        record_bounds(a.hdr);
-      }
+      if ((unsigned)win < (unsigned)a.E) atomicAdd(&hist_cta[win], 1); else record_bounds(a.hdr);
     }
   }
   if (g == 0) {
@@ -862,7 +851,7 @@ __device__ void select_quad_fast(const RouteArgs& a, const uint8_t* stage, int l
         a.ids[o] = my_e[r];
         keep_id(ids_s, (int)(t - t_base) * a.k + my_rank[r], my_e[r]);
         store_from_f32(a.weights, a.weights_dtype, o, wv);
-        if (is_local(a, my_e[r])) atomicAdd(&hist_cta[my_e[r]], 1);
+        atomicAdd(&hist_cta[my_e[r]], 1);
       }
     }
   }
@@ -1156,7 +1145,7 @@ __global__ void __launch_bounds__((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneri
           st += (int)((part_w[(r * 8 + acc) * pstride + ww] >> sh) & 0xffffu);
           sp += (int)((part_w[((R4 + r) * 8 + acc) * pstride + ww] >> sh) & 0xffffu);
         }
-        cnt[e] = st;
+        cnt[e] = is_local(a, e) ? st : 0;  // another shard's expert: zero width
         hist_cta[e] = sp;
       }
     } else if (rg < R) {
@@ -1224,7 +1213,7 @@ __global__ void __launch_bounds__((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneri
           st += part_t[(r * EPW + i) * WPR + ww];
           sp += part_p[(r * EPW + i) * WPR + ww];
         }
-        cnt[e] = st;
+        cnt[e] = is_local(a, e) ? st : 0;  // another shard's expert: zero width
         hist_cta[e] = sp;
       }
     }
