@@ -54,6 +54,12 @@ def _p(**kw):
     (_p(E=2048, k=2), B.MOE_ERR_UNSUPPORTED),
     (_p(E=64, k=40), B.MOE_ERR_UNSUPPORTED),
     (_p(logits_dtype=5), B.MOE_ERR_INVALID_ARG),
+    # expert-parallel shard ranges outside [0, E), or an offset without a count
+    (_p(local_expert_offset=-1, local_num_experts=4), B.MOE_ERR_INVALID_ARG),
+    (_p(local_expert_offset=6, local_num_experts=4), B.MOE_ERR_INVALID_ARG),
+    (_p(local_expert_offset=0, local_num_experts=-2), B.MOE_ERR_INVALID_ARG),
+    (_p(local_expert_offset=3, local_num_experts=0), B.MOE_ERR_INVALID_ARG),
+    (_p(local_expert_offset=8, local_num_experts=1), B.MOE_ERR_INVALID_ARG),
 ])
 def test_route_validation_rejects_before_any_launch(params, code):
     L = B.lib()
@@ -63,6 +69,13 @@ def test_route_validation_rejects_before_any_launch(params, code):
     assert rc == code
     mp, mt = ctypes.c_int64(), ctypes.c_int64()
     assert L.moe_route_capacity(ctypes.byref(params), ctypes.byref(mp), ctypes.byref(mt)) == code
+
+
+@pytest.mark.parametrize("off,nl", [(0, 0), (0, 8), (4, 4), (7, 1), (2, 3)])
+def test_route_shard_ranges_accepted(off, nl):
+    # a valid shard has the single-GPU capacity bound (it never has more rows)
+    p = _p(local_expert_offset=off, local_num_experts=nl)
+    assert B.route_capacity(p) == B.route_capacity(_p())
 
 
 def test_route_capacity_formula():
