@@ -28,9 +28,10 @@
 //   128-byte swizzle (the canonical K-major A / MN-major B layouts of
 //   tcgen05.mma); one thread issues each chunk's M=128 x N=64 x K=16 MMAs into
 //   TMEM as it lands; the fp32 partial logits go from TMEM to the workspace.
-//   The K-split KS is chosen so that every CTA is resident at once with the
-//   fewest post-wait staged bytes per CTA (T=128, H=7168, E=256: 4 expert
-//   groups x 28 slices of 4 chunks = 112 CTAs).
+//   The token group size and the K-split KS are chosen so that every CTA is
+//   resident at once with the fewest post-wait staged bytes per CTA plus
+//   partial-logit bytes K3 reads per token (T=128, H=7168, E=256: two 64-token
+//   groups x 4 expert groups x 16 slices of 7 chunks = 128 CTAs).
 //
 //   K3 select_kernel, a block per token: the logit of expert e is the sum of
 //   its KS partials in slice order (fp32), then the bias, the top-k on the raw
