@@ -85,3 +85,33 @@ def test_dispatch_combine_shapes(T, H, E, k, tile):
 def test_dispatch_combine_fp32_and_bf16_weights():
     run_dispatch_combine(300, 256, 8, 2, 8, dtype=torch.float32, seed=5)
     run_dispatch_combine(300, 256, 8, 2, 8, wdtype=torch.bfloat16, seed=6)
+
+
+@pytest.mark.parametrize("off,nl", [(2, 4), (0, 1), (7, 1)])
+def test_dispatch_combine_expert_parallel_shard(off, nl):
+    # one shard's route -> dispatch -> combine: only the local experts' rows are moved and summed;
+    # the other shards' selections (expanded_to_permuted = -1) contribute nothing here
+    T, H, E, k, tile = 700, 256, 8, 2, 16
+    g = torch.Generator().manual_seed(off * 10 + nl)
+    logits = torch.randn(T, E, generator=g).to(torch.bfloat16)
+    hidden = torch.randn(T, H, generator=g).to(torch.bfloat16)
+    p = B.route_params(T, E, k, score_fn=W.SOFTMAX, softmax_before_topk=0, renormalize=0, tile_tokens_dim=tile,
+                       logits_dtype=W.BF16, weights_dtype=W.F32, local_expert_offset=off, local_num_experts=nl)
+    r = B.Router(p)
+    out = r(logits.cuda())
+    torch.cuda.synchronize()
+    bk = oracle.route_bookkeeping(to_np(out["ids"]), E, tile, off, nl)
+    assert np.array_equal(to_np(out["e2p"]), bk["e2p"])
+    P, maxp = int(bk["totals"][0]), r.max_padded
+    dev_out = torch.empty((maxp, H), dtype=torch.bfloat16, device="cuda")
+    dev_out.view(torch.int16).fill_(FILL)
+    B.dispatch_into(hidden.cuda(), out["e2p"], out["p2t"], out["totals"], k, dev_out)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_np(dev_out), oracle.dispatch(hidden, bk["e2p"], bk["p2t"], P, maxp, fill=FILL))
+    rows = torch.randn(int((bk["e2p"] >= 0).sum()), H, generator=g).to(torch.bfloat16)
+    eo = W.place_expert_rows(rows, torch.from_numpy(bk["p2t"]), P, maxp)
+    res = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    B.combine_into(eo.cuda(), out["e2p"], out["weights"].contiguous(), k, res)
+    torch.cuda.synchronize()
+    ref = oracle.combine(eo, bk["e2p"], to_np(out["weights"]), k)
+    assert bf16_ulp_dist(to_np(res), ref).max() <= 1

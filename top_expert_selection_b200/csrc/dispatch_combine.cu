@@ -53,6 +53,11 @@ __global__ void __launch_bounds__(kDcThreads) dispatch_kernel(DispatchArgs a) {
         dst[j] = (p >= 0 && p < P) ? (int)p : -1;
       }
     }
+    // a token with no row here (every selection another shard's) is not read
+    bool any = false;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) any |= (j < k && dst[j] >= 0);
+    if (!any) continue;
     const uint4* src = a.hidden + t * V;
     for (int v0 = 0; v0 < V; v0 += 32 * kUnroll) {
       uint4 buf[kUnroll];
