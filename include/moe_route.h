@@ -278,7 +278,9 @@ int moe_aux_loss_bwd(int32_t T_rows, int32_t T_total, int32_t E, int32_t k, floa
  * [LMD: invokeMoeDispatch].
  *   out[expanded_to_permuted[t*k+j], :] = hidden[t, :]
  *   out[p, :] = 0 for padding rows p < P (permuted_to_token[p] == -1)
- * Rows at or past P (= totals[0], read on the device) are not written.
+ * Rows at or past P (= totals[0], read on the device) are not written.  Slots
+ * whose expanded_to_permuted is negative (another expert-parallel shard's
+ * selection) are skipped, and a token with no slot here is not read.
  * hidden [T,H], out [max_padded,H] (dtype MOE_BF16 or MOE_F32),
  * expanded_to_permuted [T*k], permuted_to_token [max_padded], totals [2]: the
  * outputs of moe_route.  H * element size must be a multiple of 16 bytes and
@@ -293,7 +295,8 @@ int moe_dispatch(int32_t T, int32_t H, int32_t k, int32_t dtype, const void* hid
  * order [LMD: invokeMoeCombine, routing scales]:
  *   out[t, :] = round( sum_j w[t,j] * expert_out[expanded_to_permuted[t*k+j], :] )
  * accumulated in fp32 in slot order, stored in `dtype` (bf16: round to
- * nearest even).  Slots whose expanded_to_permuted is negative are skipped.
+ * nearest even).  Slots whose expanded_to_permuted is negative (another
+ * expert-parallel shard's selection) are skipped: they add nothing here.
  * expert_out [max_padded,H], out [T,H] (dtype MOE_BF16 or MOE_F32), weights
  * [T,k] (weights_dtype).  Padding rows of expert_out are never read.
  * H * element size must be a multiple of 16 bytes and rows 16-byte aligned.
