@@ -525,6 +525,26 @@ def test_combine_closed_forms():
     assert np.array_equal(oracle.combine(eo, np.array([1], np.int32), np.array([[1.0]], np.float32), 1), eo[1:2])
     wb = _bf([0.5, 0.5]).reshape(1, 2)
     assert oracle.combine(eo, e2p, wb, 2)[0, :2].tolist() == _bf([2.0, 3.0]).tolist()
+    # another shard's selections (slot -1) add nothing: with the other slot weighted 1 the
+    # result is that row; with every slot -1 it is zero
+    w = np.array([[1.0, 0.75]], np.float32)
+    assert np.array_equal(oracle.combine(eo, np.array([0, -1], np.int32), w, 2), eo[0:1])
+    assert np.all(oracle.combine(eo, np.array([-1, -1], np.int32), w, 2) == 0)
+
+
+def test_dispatch_skips_other_shards_selections():
+    # dispatch of a shard: rows only for local slots; tokens whose selections are all elsewhere are
+    # copied nowhere; padding rows zero; rows past P untouched
+    hidden = np.stack([_bf([1.0, 2.0]), _bf([3.0, 4.0]), _bf([5.0, 6.0])])
+    ids = np.array([[1, 0], [1, 2], [3, 0]], np.int32)  # experts 1, 2 local (offset 1, two experts)
+    bk = oracle.route_bookkeeping(ids, 4, 4, 1, 2)
+    P = int(bk["totals"][0])
+    out = oracle.dispatch(hidden, bk["e2p"], bk["p2t"], P, P + 4, fill=0x7FBF)
+    assert P == 8 and bk["e2p"].tolist() == [0, -1, 1, 4, -1, -1]
+    assert out[0].tolist() == hidden[0].tolist() and out[1].tolist() == hidden[1].tolist()
+    assert out[4].tolist() == hidden[1].tolist()
+    assert np.all(out[[2, 3, 5, 6, 7]] == 0)
+    assert np.all(out[P:] == 0x7FBF)
 
 
 # --------------------------------------------------------------------------- decode fused
