@@ -20,7 +20,8 @@
  *
  * Readings where the pages are silent are marked READING and listed in the
  * design notes.  "parity unpinned": the sigmoid branch of the aux scores
- * (normalised sigmoid) has no closed form beyond the uniform case.
+ * (normalised sigmoid) is pinned only by closed forms (uniform rows, and rows
+ * whose sigmoids are exact: 0, 1/2, 1).
  *
  * Return codes: 0 ok, -1 invalid argument.
  */
@@ -336,8 +337,8 @@ int oracle_route_bookkeeping(int T, int E, int k, int tile, int off, int nl, con
  * Scores and routing map for the load-balancing loss [TE: Description,
  * fused_compute_score_for_moe_aux_loss; Signature].
  *   probs = softmax(logits) over E (fp32, as above); READING for sigmoid:
- *           s = sigmoid(logit), probs = s / sum_e s (parity unpinned beyond the
- *           uniform case)
+ *           s = sigmoid(logit), probs = s / sum_e s (parity unpinned beyond
+ *           closed forms: uniform rows, rows of exact sigmoids 0, 1/2, 1)
  *   routing_map[t,e] = 1 for the k best probs of the token (ties -> lower e)
  *   tokens_per_expert[e] = sum_t routing_map[t,e]
  */

@@ -483,6 +483,12 @@ def test_aux_sigmoid_scores_closed_forms():
     lg[0, 3] = 1.0
     sc = oracle.aux_scores(lg, 1, score_fn=W.SIGMOID)
     assert sc["probs"][0].tolist() == [0, 0, 0, 1.0, 0, 0, 0, 0]
+    # exact sigmoids 1/2, 1, 0, 1/2 (saturated at +-100) normalise to 1/4, 1/2, 0, 1/4; the top-2
+    # map takes expert 1, then expert 0 of the tied 1/4s (lower index)
+    sc = oracle.aux_scores(np.array([[0.0, 100.0, -100.0, 0.0]], np.float32), 2, score_fn=W.SIGMOID)
+    assert sc["probs"][0].tolist() == [0.25, 0.5, 0.0, 0.25]
+    assert sc["routing_map"][0].tolist() == [1, 1, 0, 0]
+    assert sc["tokens_per_expert"].tolist() == [1, 1, 0, 0]
 
 
 # --------------------------------------------------------------------------- dispatch / combine
