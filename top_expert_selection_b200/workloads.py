@@ -20,7 +20,7 @@ aux-loss batch, and a decode-size fused RMSNorm + router + top-k batch.
 """
 from __future__ import annotations
 
-from dataclasses import dataclass, field, replace
+from dataclasses import dataclass, replace
 from typing import Dict, Optional
 
 import torch
