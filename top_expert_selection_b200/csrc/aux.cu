@@ -115,7 +115,7 @@ __device__ __forceinline__ bool topk_mask_by_threshold(const float* p, uint32_t 
 }
 
 template <int VPL>
-__global__ void __launch_bounds__(kScoreThreads) aux_scores_kernel(int T, int E, int k, int score_fn,
+__global__ void __launch_bounds__(kScoreThreads, 3) aux_scores_kernel(int T, int E, int k, int score_fn,
                                                                  const float* __restrict__ logits,
                                                                  float* __restrict__ probs,
                                                                  uint8_t* __restrict__ rmap,
@@ -644,7 +644,7 @@ extern "C" int moe_aux_scores(int32_t T, int32_t E, int32_t k, int32_t score_fn,
   if (!tokens_per_expert || (T > 0 && (!logits || !probs || !routing_map))) return MOE_ERR_INVALID_ARG;
   if (!ws || ws_bytes < aux_ws_bytes(E)) return MOE_ERR_WORKSPACE;
   const int vpl = pick_vpl(E);
-  const int grid = std::max(1, std::min((T + 15) / 16, sm_count() * 2));
+  const int grid = std::max(1, std::min((T + 15) / 16, sm_count() * 3));  // 3 blocks per SM (40 registers)
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   // histogram, then 32 packed candidate keys per warp
   const size_t smem = (size_t)((E + 1) & ~1) * sizeof(int) + (size_t)(kScoreThreads / 32) * 32 * 8;
