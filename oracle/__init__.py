@@ -58,6 +58,7 @@ def _lib():
         L.oracle_route_weights_bwd.argtypes = [i32, i32, i32, i32, i32, i32, f32, P, P, P, P]
         L.oracle_dispatch.argtypes = [i32, i32, i32, P, P, P, i32, P]
         L.oracle_combine.argtypes = [i32, i32, i32, P, P, P, i32, P]
+        L.oracle_combine_f32.argtypes = [i32, i32, i32, P, P, P, i32, P]
         L.oracle_rmsnorm_router_topk.argtypes = [i32, i32, i32, i32, f32, i32, P, P, P, P, P, P, P, P]
         L.oracle_router_logits.argtypes = [i32, i32, i32, P, P, P, P]
         L.oracle_router_logits.restype = i32
@@ -69,7 +70,7 @@ def _lib():
         L.oracle_f64_to_bf16.restype = ctypes.c_uint16
         for name in ("oracle_route_select", "oracle_route_capacity", "oracle_route_bookkeeping",
                      "oracle_aux_scores", "oracle_aux_loss_fwd", "oracle_aux_loss_bwd", "oracle_aux_scores_bwd", "oracle_route_weights_bwd",
-                     "oracle_dispatch", "oracle_combine", "oracle_rmsnorm_router_topk"):
+                     "oracle_dispatch", "oracle_combine", "oracle_combine_f32", "oracle_rmsnorm_router_topk"):
             getattr(L, name).restype = i32
         _lib_handle = L
     return _lib_handle
@@ -256,15 +257,16 @@ def dispatch(hidden, e2p, p2t, P: int, max_padded: int, fill: int = 0xFFFF) -> n
 
 
 def combine(expert_out, e2p, weights, k: int) -> np.ndarray:
+    """Weighted sum of each token's k expert rows: bf16 rows -> bf16 tokens, fp32 rows -> fp32 tokens."""
     eo = as_numpy(expert_out)
-    assert eo.dtype == np.uint16
+    assert eo.dtype in (np.uint16, np.float32)
     w = as_numpy(weights)
     e2p = np.ascontiguousarray(as_numpy(e2p), dtype=np.int32).ravel()
     T = e2p.size // k
     H = eo.shape[1]
-    out = np.zeros((T, H), np.uint16)
-    rc = _lib().oracle_combine(T, H, k, _ptr(eo), _ptr(e2p), _ptr(np.ascontiguousarray(w)), _dtype_code(w),
-                               _ptr(out))
+    out = np.zeros((T, H), eo.dtype)
+    fn = _lib().oracle_combine if eo.dtype == np.uint16 else _lib().oracle_combine_f32
+    rc = fn(T, H, k, _ptr(eo), _ptr(e2p), _ptr(np.ascontiguousarray(w)), _dtype_code(w), _ptr(out))
     _check(rc, "combine")
     return out
 

@@ -568,6 +568,33 @@ int oracle_combine(int T, int H, int k, const uint16_t* expert_out, const int32_
 }
 
 /*
+ * Combine of fp32 expert rows into fp32 token rows [LMD: invokeMoeCombine,
+ * routing scales]: the same READING as the bf16 combine (fp32 accumulation in
+ * slot order, acc = acc + w_j * x with a rounded product and a rounded add,
+ * starting from 0; weights in their stored dtype; slots with e2p < 0 skipped),
+ * and the fp32 sum is the result (no further rounding).
+ */
+int oracle_combine_f32(int T, int H, int k, const float* expert_out, const int32_t* e2p,
+                       const void* weights, int weights_dtype, float* out) {
+  if (T < 0 || H <= 0 || k <= 0) return -1;
+  for (int t = 0; t < T; ++t) {
+    float* acc = out + (size_t)t * H;
+    for (int h = 0; h < H; ++h) acc[h] = 0.0f;
+    for (int j = 0; j < k; ++j) {
+      int32_t p = e2p[(size_t)t * k + j];
+      if (p < 0) continue;
+      float w = load_elem(weights, weights_dtype, (size_t)t * k + j);
+      const float* row = expert_out + (size_t)p * H;
+      for (int h = 0; h < H; ++h) {
+        float prod = w * row[h];
+        acc[h] = acc[h] + prod;
+      }
+    }
+  }
+  return 0;
+}
+
+/*
  * Fused RMSNorm + router + top-k for small decode batches [NKI: Background;
  * Parameters; Returns; Notes].
  *   r_t       = 1 / sqrt( mean_h x[t,h]^2 + eps )                 (double)

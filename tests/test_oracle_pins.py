@@ -527,6 +527,9 @@ def test_combine_closed_forms():
     eo2 = np.stack([x, x])
     w = np.array([[np.float32(1.0 + 2 ** -23), -1.0]], np.float32)
     assert oracle.combine(eo2, e2p, w, 2)[0, 0] == _bf([2.0 ** -23])[0]
+    # exact product second: a fused multiply-add would leave 2^-23 + 2^-30 = 2^-23 (1 + 2^-7), a bf16 value
+    w = np.array([[-1.0, np.float32(1.0 + 2 ** -23)]], np.float32)
+    assert oracle.combine(eo2, e2p, w, 2)[0, 0] == _bf([2.0 ** -23])[0]
     # k=1 with weight 1 is a copy; bf16 weights are read as bf16
     assert np.array_equal(oracle.combine(eo, np.array([1], np.int32), np.array([[1.0]], np.float32), 1), eo[1:2])
     wb = _bf([0.5, 0.5]).reshape(1, 2)
@@ -551,6 +554,36 @@ def test_dispatch_skips_other_shards_selections():
     assert out[4].tolist() == hidden[1].tolist()
     assert np.all(out[[2, 3, 5, 6, 7]] == 0)
     assert np.all(out[P:] == 0x7FBF)
+
+
+def test_combine_f32_rows_closed_forms():
+    """fp32 expert rows -> fp32 token rows: the same slot-order fp32 accumulation (rounded product, rounded
+    add), with no final rounding."""
+    eo = np.array([[1.0, 2.0, -3.0], [3.0, 4.0, 0.5]], np.float32)
+    e2p = np.array([0, 1], np.int32)
+    out = oracle.combine(eo, e2p, np.array([[0.25, 0.75]], np.float32), 2)
+    assert out.dtype == np.float32 and out[0].tolist() == [2.5, 3.5, -0.375]
+    # a rounded product then a rounded add: (1 + 2^-23)(1 + 2^-7) rounds to 1 + 2^-7 + 2^-23, minus
+    # (1 + 2^-7) leaves 2^-23; a fused multiply-add or an exact sum gives 2^-23 + 2^-30
+    x = np.float32(1.0 + 2 ** -7)
+    eo2 = np.array([[x], [x]], np.float32)
+    w = np.array([[np.float32(1.0 + 2 ** -23), -1.0]], np.float32)
+    assert oracle.combine(eo2, e2p, w, 2)[0, 0] == np.float32(2.0 ** -23)
+    # the same with the exact product second, where a fused multiply-add would keep the 2^-30
+    w = np.array([[-1.0, np.float32(1.0 + 2 ** -23)]], np.float32)
+    assert oracle.combine(eo2, e2p, w, 2)[0, 0] == np.float32(2.0 ** -23)
+    # slot order: 1 + 2^-24 + 2^-24 in slot order stays 1 (each add ties to even); the reverse order
+    # would give 1 + 2^-23
+    ones = np.ones((3, 1), np.float32)
+    w3 = np.array([[1.0, 2 ** -24, 2 ** -24]], np.float32)
+    assert oracle.combine(ones, np.array([0, 1, 2], np.int32), w3, 3)[0, 0] == np.float32(1.0)
+    w3r = np.array([[2 ** -24, 2 ** -24, 1.0]], np.float32)
+    assert oracle.combine(ones, np.array([0, 1, 2], np.int32), w3r, 3)[0, 0] == np.float32(1.0 + 2 ** -23)
+    # bf16 weights read as bf16; another shard's slot adds nothing
+    wb = _bf([0.5, 0.5]).reshape(1, 2)
+    assert oracle.combine(eo, e2p, wb, 2)[0].tolist() == [2.0, 3.0, -1.25]
+    assert oracle.combine(eo, np.array([-1, 1], np.int32), np.array([[9.0, 2.0]], np.float32), 2)[0].tolist() == \
+        [6.0, 8.0, 1.0]
 
 
 # --------------------------------------------------------------------------- decode fused
@@ -579,6 +612,69 @@ def test_decode_rmsnorm_special_cases():
     a = oracle.rmsnorm_router_topk(xa, ones, Wm, None, k=2, eps=0.0)
     b = oracle.rmsnorm_router_topk(xa * 4, ones, Wm, None, k=2, eps=0.0)
     assert np.array_equal(a["out_norm"], b["out_norm"])
+
+
+def _bf16_round_fraction(y: Fraction) -> float:
+    """The bf16 value nearest to the exact rational y (ties to even), as a float."""
+    if y == 0:
+        return 0.0
+    f = np.float32(float(y))
+    base = int(np.array(f, np.float32).view(np.uint32)) >> 16
+    best = None
+    for cand in range(max(base - 2, 0), base + 3):
+        v = Fraction(float(np.array(cand << 16, np.uint32).view(np.float32)))
+        key = (abs(v - y), cand & 1)
+        if best is None or key < best[0]:
+            best = (key, float(v))
+    return best[1]
+
+
+def _near_bf16_midpoint(y: Fraction, rel: float) -> bool:
+    """True if y lies within rel (relative) of a point halfway between two bf16 values."""
+    if y == 0:
+        return False
+    f = np.float32(float(y))
+    base = int(np.array(f, np.float32).view(np.uint32)) >> 16
+    for cand in range(max(base - 2, 0), base + 2):
+        lo = Fraction(float(np.array(cand << 16, np.uint32).view(np.float32)))
+        hi = Fraction(float(np.array((cand + 1) << 16, np.uint32).view(np.float32)))
+        if abs((lo + hi) / 2 - y) <= abs(y) * Fraction(rel):
+            return True
+    return False
+
+
+def test_decode_rmsnorm_gamma_per_hidden_index_exact():
+    """out_norm[t,h] = bf16(x[t,h] * gamma[h] / sqrt(mean_h x[t,h]^2 + eps)) against exact rationals (the
+    square root to 60 significant digits), with a gamma that differs on every h and has negative and zero
+    entries: dropping gamma, indexing it by the token, or applying it twice fails this pin (NKI page,
+    Parameters: gamma [1, H], and Background: RMSNorm before the router)."""
+    import decimal
+    T, H = 3, 256
+    g = torch.Generator().manual_seed(11)
+    x = torch.randn(T, H, generator=g).to(torch.bfloat16)
+    gam = torch.randn(H, generator=g) * 0.7 + 0.2
+    gam[::17] = 0.0
+    gam[5::23] *= -3.0
+    gam = gam.to(torch.bfloat16)
+    eps = 1e-6
+    out = oracle.rmsnorm_router_topk(x, gam, np.zeros((H, 8), np.uint16), None, k=2, eps=eps)
+    xn = oracle.bf16_to_f32(out["out_norm"])
+    xf, gf = x.float().numpy(), gam.float().numpy()
+    assert len(set(gf.tolist())) > H // 2 and (gf < 0).any() and (gf == 0).any()
+    ctx = decimal.Context(prec=60)
+    eps_q = Fraction(float(np.float32(eps)))
+    checked = 0
+    for t in range(T):
+        ms = sum(Fraction(float(v)) ** 2 for v in xf[t]) / H + eps_q
+        root = ctx.sqrt(ctx.divide(decimal.Decimal(ms.numerator), decimal.Decimal(ms.denominator)))
+        r = 1 / Fraction(root)  # 1/sqrt to ~60 digits
+        for h in range(H):
+            y = Fraction(float(xf[t, h])) * Fraction(float(gf[h])) * r
+            if _near_bf16_midpoint(y, 1e-12):
+                continue
+            assert xn[t, h] == _bf16_round_fraction(y), (t, h, float(y), xn[t, h])
+            checked += 1
+    assert checked >= T * H - 4
 
 
 def test_decode_one_hot_projection_and_affinity():
