@@ -37,6 +37,8 @@ sys.path.insert(0, ROOT)
 METRIC = "routed tokens/s (moe_route, grouped sigmoid top-8 of 256 + permutation bookkeeping)"
 UNIT = "tokens/s"
 ROTATE = 24
+SLEEP_CYCLES = 2_000_000  # ~1 ms at 1.9 GHz: longer than the host needs to queue a graph replay
+ROUTE_LAUNCHES_PER_CALL = 1  # kernels of one moe_route call at the headline workload
 
 
 def parse():
@@ -151,8 +153,20 @@ def algorithmic_bytes(T, E, k, P, ntiles, logits_bytes=2, bias_bytes=4, w_bytes=
             + 2 * ntiles * 4)                                 # tile expert, tile row limit
 
 
-def cpu_baseline(budget_s: float = 12.0):
-    """The CPU oracle (single thread, as it stands) on the same workload, repeated up to ~budget_s."""
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_baseline(budget_s: float = 12.0, return_outputs: bool = False):
+    """The CPU oracle (single thread, as it stands) on the same workload, repeated up to ~budget_s.
+    With return_outputs, also the oracle's selection and bookkeeping of the batch (for the parity report)."""
     import oracle
     from top_expert_selection_b200 import workloads as W
     spec = W.DSV3_GROUPED_SIGMOID
@@ -164,14 +178,81 @@ def cpu_baseline(budget_s: float = 12.0):
         sel = oracle.route_select(lg, k=spec.k, score_fn=spec.score_fn, n_group=spec.n_group,
                                   topk_group=spec.topk_group, renormalize=1, scaling_factor=spec.scaling_factor, bias=b)
         oracle.f32_to_bf16(sel["weights"][:1])
-        oracle.route_bookkeeping(sel["ids"], spec.E, spec.tile_tokens_dim)
+        bk = oracle.route_bookkeeping(sel["ids"], spec.E, spec.tile_tokens_dim)
         n += 1
         el = time.perf_counter() - t0
         if el >= budget_s or n >= 50:
             break
-    return {"value": spec.T * n / el, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"the full {spec.T}-token batch routed {n}x (selection, weights, bookkeeping) "
-                      f"by the single-threaded C oracle, {el:.1f} s"}
+    cb = {"value": spec.T * n / el, "unit": UNIT, "cores": 1, "kind": "oracle", "cpu_model": cpu_model(),
+          "host_threads_available": os.cpu_count(),
+          "sample": f"the full {spec.T}-token batch routed {n}x (selection, weights, bookkeeping) "
+                    f"by the single-threaded C oracle, {el:.1f} s"}
+    if return_outputs:
+        return cb, {"sel": sel, "bk": bk}
+    return cb
+
+
+def _ordered(x):
+    import numpy as np
+    u = np.asarray(x, np.float32).view(np.int32).astype(np.int64)
+    return np.where(u < 0, -(u & 0x7FFFFFFF), u)
+
+
+def _id_flips(gpu_ids, orc_ids, keys):
+    """Tokens whose GPU ids differ from the oracle's, and the largest oracle-key gap (fp32 ulp) between the
+    two choices at a differing position."""
+    import numpy as np
+    diff = np.nonzero((gpu_ids != orc_ids).any(1))[0]
+    gap = 0
+    for t in diff:
+        kk = _ordered(keys[t])
+        gap = max(gap, int(np.abs(kk[gpu_ids[t]] - kk[orc_ids[t]]).max()))
+    return int(diff.size), gap
+
+
+def route_parity(orc, gpu_out, spec):
+    """The CPU-oracle leg's comparison of the timed route's outputs with the oracle's (the oracle ran on the
+    same seeded batch): near-tie id flips counted and reported, bookkeeping re-run on the GPU's ids."""
+    import numpy as np
+    import oracle
+    g_ids = gpu_out["ids"].cpu().numpy()
+    flips, gap = _id_flips(g_ids, orc["sel"]["ids"], orc["sel"]["keys"])
+    bk = oracle.route_bookkeeping(g_ids, spec.E, spec.tile_tokens_dim)
+    P, nt = int(bk["totals"][0]), int(bk["totals"][1])
+    exact = (gpu_out["totals"].cpu().tolist() == [P, nt]
+             and all(np.array_equal(gpu_out[n].cpu().numpy().reshape(-1)[:m], bk[n].reshape(-1)[:m])
+                     for n, m in (("counts", spec.E), ("offsets", spec.E + 1), ("e2p", spec.T * spec.k),
+                                  ("p2t", P), ("tile_expert", nt), ("tile_mn_limit", nt))))
+    return {"tokens": spec.T, "id_flips": flips, "max_flip_key_gap_ulp": gap,
+            "bookkeeping_bit_exact_on_gpu_ids": bool(exact)}
+
+
+def other_parity(dev):
+    """The same report for the Mixtral route (near-tie flips of the top-2) and the aux scores (routing-map
+    rows that differ from the oracle's), run by the CPU-oracle leg on the seeded workloads."""
+    import numpy as np
+    import oracle
+    from top_expert_selection_b200 import binding as B
+    from top_expert_selection_b200 import workloads as W
+    rep = {}
+    spec = W.MIXTRAL_ROUTE
+    lg = W.mixtral_inputs()["logits"]
+    p = B.route_params(spec.T, spec.E, spec.k, score_fn=W.SOFTMAX, softmax_before_topk=0, renormalize=0,
+                       tile_tokens_dim=128, logits_dtype=W.BF16, weights_dtype=W.F32)
+    out = B.Router(p, dev)(lg.to(dev))
+    sel = oracle.route_select(lg, k=spec.k, score_fn=W.SOFTMAX, softmax_before_topk=0, renormalize=0)
+    flips, gap = _id_flips(out["ids"].cpu().numpy(), sel["ids"], sel["keys"])
+    rep["mixtral_route"] = {"tokens": spec.T, "id_flips": flips, "max_flip_key_gap_ulp": gap}
+    a = W.QWEN3_AUX
+    alg = W.aux_inputs(a)["logits"]
+    sc = B.aux_scores(alg.to(dev), a.k)
+    ref = oracle.aux_scores(alg, a.k)
+    gm = sc["routing_map"].cpu().numpy().astype(np.uint8)
+    rows = np.nonzero((gm != ref["routing_map"]).any(1))[0]
+    rep["qwen3_aux_scores"] = {"tokens": a.T, "routing_map_row_flips": int(rows.size),
+                               "tokens_per_expert_equal": bool(np.array_equal(
+                                   sc["tokens_per_expert"].cpu().numpy(), ref["tokens_per_expert"]))}
+    return rep
 
 
 def run_reference(args):
@@ -217,7 +298,8 @@ def workload_config():
                         "(top-2 group score) bf16 logits N(0,2) fp32 bias U(-0.1,0.1) renorm scale=2.5 tile=128 "
                         "bf16 weights",
             "global_batch": 16384, "parallelism": "data-parallel replicas (one batch per GPU)",
-            "l2": f"inputs/outputs rotated over {ROTATE} sets (> 126 MB L2); launches replayed from a CUDA graph"}
+            "l2": f"inputs/outputs rotated over min(steps, {ROTATE}) sets (>= 20 sets of 8.4 MB, > 126 MB L2); "
+                  "every timed call replayed from a CUDA graph"}
 
 
 def main():
@@ -254,19 +336,34 @@ def main():
             routers[i](logits[i], bias)
     torch.cuda.synchronize()
 
-    chunk = ROTATE
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        for i in range(chunk):
-            routers[i](logits[i], bias)
-    torch.cuda.synchronize()
+    # Every timed step is one moe_route call replayed from a CUDA graph: a graph of `chunk` calls over the
+    # rotated sets (chunk = min(steps, ROTATE)) replayed whole, plus one graph of the remaining calls, so
+    # exactly `steps` calls run in the timed region whatever the step count.
+    chunk = max(1, min(args.steps, ROTATE))
+    graphs = {}
+
+    def graph_of(n):
+        if n not in graphs:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(n):
+                    routers[i](logits[i], bias)
+            graphs[n] = g
+        return graphs[n]
 
     def run_steps(n):
         full, rest = divmod(n, chunk)
         for _ in range(full):
-            graph.replay()
-        for i in range(rest):
-            routers[i](logits[i], bias)
+            graph_of(chunk).replay()
+        if rest:
+            graph_of(rest).replay()
+
+    graph_of(chunk)
+    if args.steps % chunk:
+        graph_of(args.steps % chunk)
+    if args.warmup % chunk:
+        graph_of(args.warmup % chunk)
+    torch.cuda.synchronize()
 
     # warm-up
     with torch.cuda.stream(stream):
@@ -282,6 +379,9 @@ def main():
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
+        # a short device-side delay first, so that the replays are queued behind the start event and the
+        # timed region holds device time, not the host's first submission
+        torch.cuda._sleep(SLEEP_CYCLES)
         e0.record(stream)
         run_steps(args.steps)
         e1.record(stream)
@@ -292,6 +392,19 @@ def main():
     ms_total = max_over_ranks(e0.elapsed_time(e1), pg, dev)
     ms_step = ms_total / args.steps
     value = whole_job_rate(world, spec.T, ms_step)
+
+    # for context: the same calls launched eagerly one by one through the C ABI (host launch rate)
+    n_eager = min(max(args.steps, 24), 2000)
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(SLEEP_CYCLES)
+        x0 = torch.cuda.Event(enable_timing=True)
+        x1 = torch.cuda.Event(enable_timing=True)
+        x0.record(stream)
+        for i in range(n_eager):
+            routers[i % ROTATE](logits[i % ROTATE], bias)
+        x1.record(stream)
+    torch.cuda.synchronize()
+    eager_us = x0.elapsed_time(x1) * 1000.0 / n_eager
 
     # correctness of what was timed: every rotated output set reports OK and the same bookkeeping
     ok = all(B.status(r.ws) == B.MOE_OK for r in routers)
@@ -367,7 +480,10 @@ def main():
         ms_e2e = max_over_ranks(f0.elapsed_time(f1) / n_e2e, pg, dev)
         # the last step's outputs, read back on the host, are the device's
         h_views = carve(slots[(n_e2e - 1) & 1]["h_out"], out_layout)
-        e2e_ok = all(torch.equal(h_views[n], routers[0].out[n].cpu()) for n in ("ids", "counts", "offsets", "totals"))
+        ref_out = {n: routers[0].out[n].cpu() for n in out_names}
+        valid = {"p2t": P, "tile_expert": ntiles, "tile_mn_limit": ntiles}  # entries past these are not written
+        e2e_ok = all(torch.equal(h_views[n][:valid.get(n, h_views[n].numel())].reshape(-1),
+                                 ref_out[n].reshape(-1)[:valid.get(n, ref_out[n].numel())]) for n in out_names)
         e2e = {"value": whole_job_rate(world, spec.T, ms_e2e), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "ms_per_step": ms_e2e, "steps": n_e2e, "outputs_match": e2e_ok,
                "pipeline": "2 slots on 2 streams; each step: 1 host-to-device copy of the inputs, moe_route, "
@@ -380,6 +496,12 @@ def main():
         except Exception as exc:  # reported, never hides the headline
             extra = {"error": repr(exc)}
 
+    cb, parity = None, None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cb, orc = cpu_baseline(return_outputs=True)
+        parity = {"dsv3_grouped_sigmoid_route": route_parity(orc, routers[0].out, spec)}
+        if not args.no_extra:
+            parity.update(other_parity(dev))
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -392,9 +514,11 @@ def main():
                          "algorithmic_bytes_per_launch": alg, "peak_kind": f"{peak_kind} HBM copy bandwidth",
                          "kernel": "route_kernel (selection + bookkeeping, one launch)",
                          "frac_of_8TBps": achieved / 8000.0},
-            "e2e": e2e, "gpu_launches": args.steps, "status_ok": ok,
+            "e2e": e2e, "gpu_launches": args.steps * ROUTE_LAUNCHES_PER_CALL, "status_ok": ok,
+            "eager_us_per_call": eager_us,
             "clocks": clocks,
-            "cpu_baseline": cpu_baseline() if (world == 1 and not args.no_cpu) else None,
+            "cpu_baseline": cb,
+            "parity": parity,
             "other_rows": extra,
         }
         print(json.dumps(line), flush=True)

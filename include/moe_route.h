@@ -188,17 +188,29 @@ int moe_route(const moe_route_params* p, const void* logits, const void* bias, i
  * workspace is a library-owned __device__ array of 512 KB that every GPU loading
  * the library holds until the process exits.  Calls needing more (the workspace
  * grows with E and the SM count; moe_route_workspace_bytes reports it) return
- * MOE_ERR_WORKSPACE.  The first call on a device looks up the array's device
- * address (cudaGetSymbolAddress); later calls reuse it.  Each call clears the
- * array's 64-byte header on `stream` before launching.  All calls share the one
+ * MOE_ERR_WORKSPACE.  The first call on a device (or the first
+ * moe_route_no_alloc_status) does the set-up: it looks up the array's device
+ * address (cudaGetSymbolAddress) and zero-fills its 64-byte header on `stream`;
+ * make that first call before any stream capture.  A failed set-up returns
+ * MOE_ERR_CUDA and is tried again by the next call.  All calls share the one
  * array: calls that may overlap on the GPU (different streams, or several host
  * threads) race and must be serialised by the caller.  The call allocates no
- * device memory.  Device-side status (timeouts, bounds) is not reported.
+ * device memory.  Device-side status (a bounds check) lands in the array's
+ * status word, which later calls keep (sticky, first error wins): read it with
+ * moe_route_no_alloc_status.
  */
 int moe_route_no_alloc(const moe_route_params* p, const void* logits, const void* bias, int32_t* topk_ids,
                        void* topk_weights, int32_t* expert_counts, int32_t* padded_offsets,
                        int32_t* expanded_to_permuted, int32_t* permuted_to_token, int32_t* tile_expert,
                        int32_t* tile_mn_limit, int32_t* totals, void* stream);
+
+/*
+ * moe_route_no_alloc_status -- read the status word of moe_route_no_alloc's
+ * library-owned workspace on the current device (MOE_OK or the first
+ * MOE_ERR_DEVICE_* recorded since it was last cleared).  Synchronises
+ * `stream`; clear != 0 resets it to MOE_OK.  (No counterpart on the pages.)
+ */
+int moe_route_no_alloc_status(void* stream, int32_t* status, int clear);
 
 /* Workspace bytes of the aux-loss entry points (scores, loss forward). */
 int moe_aux_workspace_bytes(int32_t num_tokens, int32_t num_experts, size_t* bytes);
@@ -298,12 +310,15 @@ int moe_dispatch(int32_t T, int32_t H, int32_t k, int32_t dtype, const void* hid
  * nearest even).  Slots whose expanded_to_permuted is negative (another
  * expert-parallel shard's selection) are skipped: they add nothing here.
  * expert_out [max_padded,H], out [T,H] (dtype MOE_BF16 or MOE_F32), weights
- * [T,k] (weights_dtype).  Padding rows of expert_out are never read.
+ * [T,k] (weights_dtype).  Padding rows of expert_out are never read.  A slot
+ * whose expanded_to_permuted is max_padded or more (a stale or mismatched map)
+ * is skipped, and when ws (optional, >= 64 bytes, zero-filled before first use)
+ * is given MOE_ERR_DEVICE_BOUNDS is recorded in its status word (moe_status).
  * H * element size must be a multiple of 16 bytes and rows 16-byte aligned.
  */
-int moe_combine(int32_t T, int32_t H, int32_t k, int32_t dtype, const void* expert_out,
+int moe_combine(int32_t T, int32_t H, int32_t k, int32_t dtype, const void* expert_out, int64_t max_padded,
                 const int32_t* expanded_to_permuted, const void* weights, int32_t weights_dtype,
-                void* out, void* stream);
+                void* out, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Workspace bytes of moe_rmsnorm_router_topk (header and the fp32 partial
@@ -362,6 +377,13 @@ int moe_debug_barrier_wait(int32_t blocks, int32_t extra_arrivals, int64_t timeo
  * and keeps a 2^-10 margin.  x and out are device arrays of n floats.
  */
 int moe_debug_sigmoid_proxy_error(const float* x, int64_t n, float* out, void* stream);
+
+/*
+ * Test hook for moe_route_no_alloc_status: records `code` (negative) in the
+ * status word of the no-alloc workspace on the current device, as a kernel's
+ * bounds check would (first error wins), without running a route.
+ */
+int moe_debug_no_alloc_record(int32_t code, void* stream);
 
 #ifdef __cplusplus
 }

@@ -96,8 +96,11 @@ def test_other_entry_points_validate():
     assert L.moe_rmsnorm_router_topk(4, 128, 16, 17, 1e-6, 1, d, d, d, None, d, d, d, None, d, sz, None) == -1
     # dispatch / combine: rows must be 16-byte multiples
     assert L.moe_dispatch(4, 3, 2, 1, d, d, d, d, 16, d, None) == -1
-    assert L.moe_combine(4, 12, 2, 1, d, d, d, 0, d, None) == -1
-    assert L.moe_combine(4, 8, 0, 1, d, d, d, 0, d, None) == -1
+    assert L.moe_combine(4, 12, 2, 1, d, 16, d, d, 0, d, None, 0, None) == -1
+    assert L.moe_combine(4, 8, 0, 1, d, 16, d, d, 0, d, None, 0, None) == -1
+    assert L.moe_combine(4, 8, 2, 1, d, -1, d, d, 0, d, None, 0, None) == -1
+    # a status workspace, when given, holds at least the 64-byte header
+    assert L.moe_combine(4, 8, 2, 1, d, 16, d, d, 0, d, d, ctypes.c_size_t(8), None) == B.MOE_ERR_WORKSPACE
     # aux
     assert L.moe_aux_scores(4, 8, 9, 0, d, d, d, d, d, sz, None) == -1
     assert L.moe_aux_loss_fwd(4, 0, 8, 2, 0.1, d, d, d, d, sz, None) == -1

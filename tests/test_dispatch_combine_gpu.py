@@ -59,16 +59,27 @@ def run_dispatch_combine(T, H, E, k, tile, dtype=torch.bfloat16, wdtype=torch.fl
     eo = W.place_expert_rows(rows, torch.from_numpy(bk["p2t"]), P, maxp)
     w = out["weights"] if wdtype == torch.float32 else out["weights"].to(torch.bfloat16)
     res = torch.empty((T, H), dtype=dtype, device="cuda")
-    B.combine_into(eo.cuda(), out["e2p"], w.contiguous(), k, res)
+    ws = B.make_workspace(64, "cuda")
+    B.combine_into(eo.cuda(), out["e2p"], w.contiguous(), k, res, ws=ws)
     torch.cuda.synchronize()
+    assert B.status(ws) == B.MOE_OK
     got = to_np(res)
     assert np.all(np.isfinite(res.float().cpu().numpy())), "combine read a padding row"
+    ref = oracle.combine(eo, bk["e2p"], to_np(w), k)
     if dtype == torch.bfloat16:
-        ref = oracle.combine(eo, bk["e2p"], to_np(w), k)
         d = bf16_ulp_dist(got, ref)
         assert d.max() <= 1, f"combine off by {d.max()} bf16 ulp"
         return int((d > 0).sum())
-    return 0
+    # fp32 rows: the same slot-order fp32 sum, compared within 1e-5 of the terms before cancellation
+    ew = np.abs(np.asarray(to_np(w), np.float64)).reshape(T, k)
+    mag = np.zeros((T, H))
+    for j in range(k):
+        p = bk["e2p"].reshape(T, k)[:, j]
+        v = p >= 0
+        mag[v] += ew[v, j:j + 1] * np.abs(eo.numpy()[p[v]].astype(np.float64))
+    err = np.abs(got.astype(np.float64) - ref.astype(np.float64))
+    assert np.all(err <= 1e-5 * mag), f"fp32 combine off by {(err / np.maximum(mag, 1e-30)).max()} (relative)"
+    return int((got != ref).sum())
 
 
 def test_mixtral_dispatch_combine_full_size():
@@ -83,8 +94,31 @@ def test_dispatch_combine_shapes(T, H, E, k, tile):
 
 
 def test_dispatch_combine_fp32_and_bf16_weights():
-    run_dispatch_combine(300, 256, 8, 2, 8, dtype=torch.float32, seed=5)
+    n = run_dispatch_combine(300, 256, 8, 2, 8, dtype=torch.float32, seed=5)
+    assert n == 0, f"{n} fp32 combine elements differ from the oracle's fp32 sum"
     run_dispatch_combine(300, 256, 8, 2, 8, wdtype=torch.bfloat16, seed=6)
+
+
+def test_combine_fp32_mixtral_shape():
+    # fp32 rows at a Mixtral-like shape (several tiles, a ragged tail): T=4099, H=4096, top-2 of 8
+    n = run_dispatch_combine(4099, 4096, 8, 2, 128, dtype=torch.float32, seed=9)
+    assert n == 0
+
+
+def test_combine_skips_rows_past_the_buffer():
+    # a stale map pointing past expert_out is skipped and recorded, never read
+    T, H, k = 64, 64, 2
+    eo = torch.randn(16, H, device="cuda")
+    e2p = torch.tensor([[j % 16, 16 + j] if j % 3 == 0 else [j % 16, (j + 1) % 16] for j in range(T)],
+                       dtype=torch.int32, device="cuda").reshape(-1)
+    w = torch.ones(T, k, device="cuda")
+    res = torch.empty(T, H, device="cuda")
+    ws = B.make_workspace(64, "cuda")
+    B.combine_into(eo, e2p, w, k, res, ws=ws)
+    torch.cuda.synchronize()
+    assert B.status(ws) == B.MOE_ERR_DEVICE_BOUNDS
+    ref = oracle.combine(eo.cpu().numpy(), np.where(to_np(e2p) >= 16, -1, to_np(e2p)), w.cpu().numpy(), k)
+    assert np.array_equal(to_np(res), ref)
 
 
 @pytest.mark.parametrize("off,nl", [(2, 4), (0, 1), (7, 1)])

@@ -1,7 +1,8 @@
 """moe_route_no_alloc: the allocation-free variant of moe_route for callers that cannot allocate device
 memory (a serving runtime whose memory manager owns the GPU, a plugin interface that provides no workspace,
 a plain C caller without a device allocator).  Its workspace is a static array inside the library; this
-checks, through the C ABI, that two calls in a row give exactly what moe_route gives on the same inputs.
+checks, through the C ABI, that two calls in a row give exactly what moe_route gives on the same inputs,
+and that the static workspace's status word reports a recorded device-side error instead of losing it.
 
 Collected last (file name) so that a run stopping at the first failure has run every other test first."""
 import pytest
@@ -42,6 +43,7 @@ def test_no_alloc_route_matches_route_on_two_calls_in_a_row():
             g_ = got[n] if lim is None else got[n][:lim]
             # deterministic kernels: identical results (stricter than the parity tolerances)
             assert torch.equal(a_, g_), f"{n} differs between moe_route_no_alloc and moe_route"
+        assert B.route_no_alloc_status() == B.MOE_OK
 
 
 def test_no_alloc_route_rejects_a_workspace_it_cannot_hold():
@@ -51,3 +53,22 @@ def test_no_alloc_route_rejects_a_workspace_it_cannot_hold():
     with pytest.raises(B.MoeError) as ei:
         B.route_no_alloc_into(p, torch.zeros(64, 1024, device=dev), None, out)
     assert ei.value.code == B.MOE_ERR_WORKSPACE
+
+
+def test_no_alloc_status_survives_the_next_call():
+    # a device-side error recorded in the static workspace (here by the test hook, as a kernel's bounds
+    # check would) is still there after another moe_route_no_alloc call, and clears when read with clear=1
+    spec = W.TINY_SOFTMAX
+    p = _params(spec)
+    lg = W.route_inputs(spec)["logits"].cuda()
+    ref = B.Router(p)(lg)
+    got = {n: torch.empty_like(v) for n, v in ref.items()}
+    assert B.route_no_alloc_status() == B.MOE_OK
+    B._check(B.lib().moe_debug_no_alloc_record(B.MOE_ERR_DEVICE_BOUNDS, B._stream(None)), "record")
+    B.route_no_alloc_into(p, lg, None, got)
+    assert B.route_no_alloc_status(clear=False) == B.MOE_ERR_DEVICE_BOUNDS
+    assert B.route_no_alloc_status(clear=True) == B.MOE_ERR_DEVICE_BOUNDS
+    assert B.route_no_alloc_status() == B.MOE_OK
+    B.route_no_alloc_into(p, lg, None, got)
+    torch.cuda.synchronize()
+    assert torch.equal(got["ids"], ref["ids"]) and B.route_no_alloc_status() == B.MOE_OK

@@ -38,7 +38,8 @@ EXPORTED = (
     "moe_route_workspace_bytes", "moe_route", "moe_aux_workspace_bytes", "moe_aux_scores", "moe_aux_scores_bwd", "moe_route_weights_bwd",
     "moe_aux_loss_fwd", "moe_aux_loss_bwd", "moe_dispatch", "moe_combine",
     "moe_rmsnorm_router_topk_workspace_bytes", "moe_rmsnorm_router_topk", "moe_debug_barrier_wait",
-    "moe_debug_sigmoid_proxy_error", "moe_route_no_alloc",
+    "moe_debug_sigmoid_proxy_error", "moe_route_no_alloc", "moe_route_no_alloc_status",
+    "moe_debug_no_alloc_record",
 )
 
 
@@ -84,6 +85,8 @@ def lib() -> ctypes.CDLL:
             "moe_route_workspace_bytes": ([RP, ctypes.POINTER(sz)], ctypes.c_int),
             "moe_route": ([RP, P, P, P, P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
             "moe_route_no_alloc": ([RP, P, P, P, P, P, P, P, P, P, P, P, P], ctypes.c_int),
+            "moe_route_no_alloc_status": ([P, ctypes.POINTER(i32), ctypes.c_int], ctypes.c_int),
+            "moe_debug_no_alloc_record": ([i32, P], ctypes.c_int),
             "moe_aux_workspace_bytes": ([i32, i32, ctypes.POINTER(sz)], ctypes.c_int),
             "moe_aux_scores": ([i32, i32, i32, i32, P, P, P, P, P, sz, P], ctypes.c_int),
             "moe_aux_loss_fwd": ([i32, i32, i32, i32, f32, P, P, P, P, sz, P], ctypes.c_int),
@@ -91,7 +94,7 @@ def lib() -> ctypes.CDLL:
             "moe_aux_scores_bwd": ([i32, i32, i32, P, P, P, P], ctypes.c_int),
             "moe_route_weights_bwd": ([RP, P, P, P, P, P, sz, P], ctypes.c_int),
             "moe_dispatch": ([i32, i32, i32, i32, P, P, P, P, i64, P, P], ctypes.c_int),
-            "moe_combine": ([i32, i32, i32, i32, P, P, P, i32, P, P], ctypes.c_int),
+            "moe_combine": ([i32, i32, i32, i32, P, i64, P, P, i32, P, P, sz, P], ctypes.c_int),
             "moe_rmsnorm_router_topk_workspace_bytes": ([i32, i32, i32, ctypes.POINTER(sz)], ctypes.c_int),
             "moe_rmsnorm_router_topk": ([i32, i32, i32, i32, f32, i32, P, P, P, P, P, P, P, P, P, sz, P],
                                         ctypes.c_int),
@@ -344,10 +347,11 @@ def dispatch_into(hidden: torch.Tensor, e2p: torch.Tensor, p2t: torch.Tensor, to
 
 
 def combine_into(expert_out: torch.Tensor, e2p: torch.Tensor, weights: torch.Tensor, k: int, out: torch.Tensor,
-                 stream=None) -> None:
+                 ws: Optional[torch.Tensor] = None, stream=None) -> None:
     T, H = out.shape
-    _check(lib().moe_combine(T, H, k, _DT[expert_out.dtype], _p(expert_out), _p(e2p), _p(weights),
-                             _DT[weights.dtype], _p(out), _stream(stream)), "moe_combine")
+    _check(lib().moe_combine(T, H, k, _DT[expert_out.dtype], _p(expert_out), expert_out.shape[0], _p(e2p),
+                             _p(weights), _DT[weights.dtype], _p(out), _p(ws),
+                             ctypes.c_size_t(0 if ws is None else ws.numel()), _stream(stream)), "moe_combine")
 
 
 # ---------------------------------------------------------------------------- decode fused
@@ -389,3 +393,10 @@ def route_no_alloc_into(p: RouteParams, logits: torch.Tensor, bias: Optional[tor
     rc = lib().moe_route_no_alloc(ctypes.byref(p), _p(logits), _p(bias), *[_p(out[n]) for n in names],
                                   _stream(stream))
     _check(rc, "moe_route_no_alloc")
+
+
+def route_no_alloc_status(clear: bool = True, stream=None) -> int:
+    """The status word of moe_route_no_alloc's static workspace (sticky until cleared)."""
+    st = ctypes.c_int32(0)
+    _check(lib().moe_route_no_alloc_status(_stream(stream), ctypes.byref(st), int(clear)), "moe_route_no_alloc_status")
+    return int(st.value)

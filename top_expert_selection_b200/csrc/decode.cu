@@ -496,15 +496,22 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         ++issued;
       }
     }
-    if (mma_issued && flag[0] == 0) {
+    // one commit tracks every MMA this thread issued: its arrival means they
+    // have all finished reading shared memory and writing TMEM
+    bool drained = !mma_issued;
+    if (mma_issued) {
       umma_commit(mma_bar);
-      if (!mbar_wait_bounded(mma_bar, 0, a.timeout_ns)) {
+      drained = mbar_wait_bounded(mma_bar, 0, a.timeout_ns);
+      if (!drained) {
         record_timeout(a.hdr);
         flag[0] = 1;
       }
     }
     if (flag[0]) {
-      // a wait gave up: let the copies still in flight land before the CTA exits
+      // a wait gave up: let the MMAs (if their commit has not arrived yet, wait
+      // once more, bounded) and the copies still in flight finish before the
+      // CTA frees its TMEM and exits
+      if (!drained) mbar_wait_bounded(mma_bar, 0, a.timeout_ns);
       for (int i = max(0, issued - S); i < issued; ++i)
         mbar_wait_bounded(full + (i % S), (uint32_t)(i / S) & 1u, a.timeout_ns);
     }

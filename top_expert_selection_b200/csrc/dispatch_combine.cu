@@ -97,6 +97,8 @@ __global__ void __launch_bounds__(kDcThreads) dispatch_kernel(DispatchArgs a) {
 
 struct CombineArgs {
   const uint4* eo;
+  long long eo_rows;  // rows of expert_out: a slot at or past it is skipped and recorded
+  WsHeader* hdr;      // optional status word (NULL: not recorded)
   const int32_t* e2p;
   const void* weights;
   int weights_dtype;
@@ -141,6 +143,10 @@ __global__ void __launch_bounds__(kDcThreads) combine_kernel(CombineArgs a) {
       if (j < k) {
         src[j] = __ldg(&a.e2p[t * k + j]);
         w[j] = load_as_f32(a.weights, a.weights_dtype, (size_t)(t * k + j));
+        if (src[j] >= a.eo_rows) {  // out of range: skipped (another shard's slots are -1)
+          if (a.hdr && lane == 0) record_bounds(a.hdr);
+          src[j] = -1;
+        }
       }
     }
     for (int v0 = 0; v0 < V; v0 += 32 * kUnroll) {
@@ -241,18 +247,21 @@ extern "C" int moe_dispatch(int32_t T, int32_t H, int32_t k, int32_t dtype, cons
 }
 
 extern "C" int moe_combine(int32_t T, int32_t H, int32_t k, int32_t dtype, const void* expert_out,
-                           const int32_t* expanded_to_permuted, const void* weights, int32_t weights_dtype,
-                           void* out, void* stream) {
-  if (T < 0 || H <= 0 || k <= 0 || k > MOE_MAX_TOPK) return MOE_ERR_INVALID_ARG;
+                           int64_t max_padded, const int32_t* expanded_to_permuted, const void* weights,
+                           int32_t weights_dtype, void* out, void* ws, size_t ws_bytes, void* stream) {
+  if (T < 0 || H <= 0 || k <= 0 || k > MOE_MAX_TOPK || max_padded < 0) return MOE_ERR_INVALID_ARG;
+  if (ws && ws_bytes < sizeof(WsHeader)) return MOE_ERR_WORKSPACE;
   if (dtype != MOE_BF16 && dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
   if (weights_dtype != MOE_BF16 && weights_dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
   const long long row_bytes = (long long)H * (dtype == MOE_BF16 ? 2 : 4);
   if (row_bytes % 16 != 0) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
-  if (!expert_out || !expanded_to_permuted || !weights || !out) return MOE_ERR_INVALID_ARG;
+  if ((max_padded > 0 && !expert_out) || !expanded_to_permuted || !weights || !out) return MOE_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(expert_out) | reinterpret_cast<uintptr_t>(out)) & 15) return MOE_ERR_INVALID_ARG;
   CombineArgs a;
   a.eo = reinterpret_cast<const uint4*>(expert_out);
+  a.eo_rows = max_padded;
+  a.hdr = reinterpret_cast<WsHeader*>(ws);
   a.e2p = expanded_to_permuted;
   a.weights = weights;
   a.weights_dtype = weights_dtype;

@@ -40,6 +40,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -1374,8 +1375,8 @@ int validate(const moe_route_params* p) {
     if (p->group_score_topn > 2) return MOE_ERR_UNSUPPORTED;
   }
   if (p->num_experts > MOE_MAX_EXPERTS || p->top_k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
-  if ((long long)p->num_tokens * p->top_k + (long long)std::min(p->num_experts, p->num_tokens * p->top_k) *
-          (p->tile_tokens_dim - 1) > 0x7fffffffLL)
+  const long long items = (long long)p->num_tokens * p->top_k;
+  if (items + std::min<long long>(p->num_experts, items) * (p->tile_tokens_dim - 1) > 0x7fffffffLL)
     return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
@@ -1671,12 +1672,40 @@ namespace {
 constexpr size_t kStaticScratchBytes = 512 * 1024;  // the route workspace for E up to a few hundred experts
 __device__ __align__(256) uint8_t g_route_scratch[kStaticScratchBytes];
 
+// The array's device address, looked up once per device with that device
+// current.  A failed lookup is not cached: the next call tries again.  The
+// first successful set-up also zero-fills the array's 64-byte header on the
+// caller's stream; after that the status word is sticky across calls (a
+// recorded error stays until moe_route_no_alloc_status clears it).
 struct ScratchSlot {
-  std::once_flag once;
-  void* ptr = nullptr;
-  cudaError_t err = cudaSuccess;
+  std::mutex m;
+  std::atomic<void*> ptr{nullptr};
 };
 ScratchSlot g_scratch_slot[64];
+
+void* scratch_address(int dev, cudaStream_t st) {
+  ScratchSlot& slot = g_scratch_slot[dev];
+  void* p = slot.ptr.load(std::memory_order_acquire);
+  if (p) return p;
+  std::lock_guard<std::mutex> lock(slot.m);
+  p = slot.ptr.load(std::memory_order_relaxed);
+  if (p) return p;
+  if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || p == nullptr) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (cudaMemsetAsync(p, 0, sizeof(WsHeader), st) != cudaSuccess) return nullptr;
+  slot.ptr.store(p, std::memory_order_release);
+  return p;
+}
+
+int current_device(int* dev) {
+  return (cudaGetDevice(dev) == cudaSuccess && *dev >= 0 && *dev < 64) ? MOE_OK : MOE_ERR_CUDA;
+}
+
+__global__ void no_alloc_record_kernel(int32_t code) {
+  atomicCAS(&reinterpret_cast<WsHeader*>(g_route_scratch)->status, MOE_OK, code);
+}
 
 }  // namespace
 }  // namespace moe
@@ -1692,15 +1721,28 @@ extern "C" int moe_route_no_alloc(const moe_route_params* p, const void* logits,
   if (d.sms <= 0) return MOE_ERR_CUDA;
   if (ws_bytes_for(p->num_experts, d.sms) > kStaticScratchBytes) return MOE_ERR_WORKSPACE;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
-  ScratchSlot& slot = g_scratch_slot[dev];
-  // set-up, once per device, with that device current: the array's device address
-  std::call_once(slot.once, [&slot] { slot.err = cudaGetSymbolAddress(&slot.ptr, g_route_scratch); });
-  if (slot.err != cudaSuccess || slot.ptr == nullptr) return MOE_ERR_CUDA;
-  // the array keeps the previous call's contents: its header (status word and
-  // barrier state) must start at zero
-  if (cudaMemsetAsync(slot.ptr, 0, sizeof(WsHeader), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  if (current_device(&dev) != MOE_OK) return MOE_ERR_CUDA;
+  void* ws = scratch_address(dev, reinterpret_cast<cudaStream_t>(stream));
+  if (!ws) return MOE_ERR_CUDA;
   return moe_route(p, logits, bias, topk_ids, topk_weights, expert_counts, padded_offsets, expanded_to_permuted,
-                   permuted_to_token, tile_expert, tile_mn_limit, totals, slot.ptr, kStaticScratchBytes, stream);
+                   permuted_to_token, tile_expert, tile_mn_limit, totals, ws, kStaticScratchBytes, stream);
+}
+
+extern "C" int moe_route_no_alloc_status(void* stream, int32_t* status, int clear) {
+  if (!status) return MOE_ERR_INVALID_ARG;
+  int dev = 0;
+  if (current_device(&dev) != MOE_OK) return MOE_ERR_CUDA;
+  void* ws = scratch_address(dev, reinterpret_cast<cudaStream_t>(stream));
+  if (!ws) return MOE_ERR_CUDA;
+  return moe_status(ws, stream, status, clear);
+}
+
+extern "C" int moe_debug_no_alloc_record(int32_t code, void* stream) {
+  if (code >= 0) return MOE_ERR_INVALID_ARG;
+  int dev = 0;
+  if (current_device(&dev) != MOE_OK) return MOE_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (!scratch_address(dev, st)) return MOE_ERR_CUDA;
+  no_alloc_record_kernel<<<1, 1, 0, st>>>(code);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
