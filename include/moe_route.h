@@ -19,12 +19,11 @@
  *   - Arguments are validated before any launch; a failed check returns a
  *     negative MOE_ERR_* code and launches nothing.  MOE_ERR_CUDA reports a
  *     launch failure (cudaGetLastError after the launch).
- *   - Kernels that wait on other thread blocks (a grid barrier, a
- *     last-block reduction) wait at most a bounded time; on expiry they record
- *     MOE_ERR_DEVICE_TIMEOUT in the status word at the start of their
- *     workspace and return, leaving outputs undefined.  Read it with
- *     moe_status().  After a timeout the workspace must be zero-filled again
- *     before its next use.
+ *   - Every device-side wait (on a kernel's own bulk copies or tensor-core
+ *     operations) is bounded; on expiry the kernel records
+ *     MOE_ERR_DEVICE_TIMEOUT in the status word at the start of its
+ *     workspace and returns, leaving outputs undefined.  Read it with
+ *     moe_status().  No kernel waits on another thread block.
  *   - A workspace must be zero-filled once before its first use
  *     (moe_workspace_init or any memset); the library leaves it consistent
  *     for the next call.  One workspace serves one stream at a time: calls
@@ -162,6 +161,17 @@ int moe_route_workspace_bytes(const moe_route_params* p, size_t* bytes);
  *   permuted_to_token [max_padded], tile_expert [max_tiles],
  *   tile_mn_limit [max_tiles], totals [2] -- all int32,
  *   ws [ws_bytes] from moe_route_workspace_bytes (zero-filled before first use).
+ * Two launches chained by programmatic dependent launch: a selection kernel
+ * (one block per contiguous token segment) writes ids and weights, a count
+ * table row per segment and each selection's rank in its segment; a
+ * bookkeeping kernel turns them into slots, offsets and tile tables.  The
+ * bias is read before waiting on the preceding kernel: a preceding kernel that
+ * lets its dependents start early must not write it (the logits are read after
+ * the wait).  The sigmoid fast path (E = 8 * {8, 16, 32} bf16 or {8, 16} fp32
+ * logits, 16-byte aligned, k <= 8, ungrouped or 8 groups with 2 * topk_group
+ * >= k) chooses candidates with an approximate key whose error bound is
+ * checked exhaustively by the test suite, and computes every key that can
+ * decide the result with the stated fp32 formula.
  * Errors: MOE_ERR_INVALID_ARG (sizes, k > E, tile not a power of two, groups
  * not dividing E, k > topk_group * E / n_group, a local expert range outside
  * [0, E), NULL outputs),
@@ -360,23 +370,30 @@ int moe_rmsnorm_router_topk(int32_t T, int32_t H, int32_t E, int32_t k, float ep
                             void* ws, size_t ws_bytes, void* stream);
 
 /*
- * Test hook for the bounded grid barrier used by moe_route: launches
- * `blocks` co-resident blocks that wait for `blocks + extra_arrivals`
- * arrivals, giving up after timeout_ns.  With extra_arrivals > 0 the wait
- * cannot complete, so the status word must read MOE_ERR_DEVICE_TIMEOUT
- * afterwards; the kernel returns normally either way.  ws needs 64 bytes.
+ * Test hook for the bounded waits of the kernels (a wait on a shared-memory
+ * barrier, as the kernels wait on their bulk copies): one thread arms a
+ * barrier and waits on it for at most timeout_ns.  With never_complete != 0
+ * the barrier expects bytes that never arrive, so the wait gives up and the
+ * status word of ws (64 bytes) must read MOE_ERR_DEVICE_TIMEOUT afterwards;
+ * with 0 it completes at once.  The kernel returns normally either way.
  */
-int moe_debug_barrier_wait(int32_t blocks, int32_t extra_arrivals, int64_t timeout_ns, void* ws,
-                           size_t ws_bytes, void* stream);
+int moe_debug_wait_timeout(int32_t never_complete, int64_t timeout_ns, void* ws, size_t ws_bytes, void* stream);
 
 /*
- * Test hook for the sigmoid fast path of moe_route: for each x[i] writes
- * proxy(x) - sigmoid(x), where proxy(x) = 0.5 * tanh.approx(x / 2) + 0.5 is
- * the approximate key that chooses candidates and sigmoid(x) = 1 / (1 +
- * exp(-x)) in fp32 is the exact one.  moe_route assumes |difference| <= 2^-12
- * and keeps a 2^-10 margin.  x and out are device arrays of n floats.
+ * Test hook for the sigmoid fast path of moe_route: for each i writes
+ *   err[i]   = proxy(x[i], b[i]) - (sigmoid(x[i]) + b[i])
+ *   delta[i] = the error bound the fast path assumes for a block whose
+ *              largest |0.5 + bias| is |0.5 + b[i]|
+ * where proxy(x, b) = 0.5 * tanh.approx(x / 2) + (0.5 + b) in packed f16 (x
+ * rounded to f16, the tanh and the fused multiply-add in f16) is the
+ * approximate key that chooses candidates, and sigmoid(x) + b = 1 / (1 +
+ * exp(-x)) + b in fp32 is the exact key.  f32_logits selects the bound for
+ * fp32 logits (whose rounding to f16 adds to the error).  moe_route assumes
+ * |err| <= delta; the tests check |err| <= delta / 2.  x, b, err, delta are
+ * device arrays of n floats.
  */
-int moe_debug_sigmoid_proxy_error(const float* x, int64_t n, float* out, void* stream);
+int moe_debug_sigmoid_proxy_error(const float* x, const float* b, int64_t n, int32_t f32_logits, float* err,
+                                  float* delta, void* stream);
 
 /*
  * Test hook for moe_route_no_alloc_status: records `code` (negative) in the

@@ -107,9 +107,10 @@ def test_other_entry_points_validate():
     assert L.moe_aux_loss_bwd(4, 4, 8, 0, 0.1, d, d, d, d, d, None) == -1
     # workspace too small
     assert L.moe_aux_scores(4, 8, 2, 0, d, d, d, d, d, ctypes.c_size_t(8), None) == B.MOE_ERR_WORKSPACE
-    # barrier hook
-    assert L.moe_debug_barrier_wait(0, 1, 1000, d, sz, None) == -1
-    assert L.moe_debug_barrier_wait(2, 1, 10 ** 10, d, sz, None) == -1
+    # wait hook
+    assert L.moe_debug_wait_timeout(1, 0, d, sz, None) == -1
+    assert L.moe_debug_wait_timeout(1, 10 ** 10, d, sz, None) == -1
+    assert L.moe_debug_wait_timeout(1, 1000, d, ctypes.c_size_t(8), None) == B.MOE_ERR_WORKSPACE
 
 
 def test_binding_refuses_cpu_tensors():

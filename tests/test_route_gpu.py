@@ -223,32 +223,51 @@ def test_zero_tokens():
     assert views["totals"].tolist() == [0, 0]
 
 
-def test_bounded_barrier_times_out_cleanly():
-    """A grid barrier asked for one arrival more than it has blocks gives up after its limit and
-    records a timeout in the status word; the context stays usable."""
+def test_bounded_wait_times_out_cleanly():
+    """A bounded wait on a barrier that nothing completes (the kind of wait the kernels use for their
+    bulk copies) gives up after its limit and records a timeout in the status word; the context stays
+    usable and a wait that completes records nothing."""
     dev = torch.device("cuda")
     ws = B.make_workspace(64, dev)
-    B.debug_barrier_wait(4, 1, 20_000_000, ws)
+    B.debug_wait_timeout(True, 20_000_000, ws)
     torch.cuda.synchronize()
     assert B.status(ws, clear=True) == B.MOE_ERR_DEVICE_TIMEOUT
-    ws.zero_()
-    B.debug_barrier_wait(4, 0, 20_000_000, ws)
+    assert B.status(ws) == B.MOE_OK
+    B.debug_wait_timeout(False, 20_000_000, ws)
     torch.cuda.synchronize()
     assert B.status(ws) == B.MOE_OK
     run_route(W.TINY_SOFTMAX)
 
 
 def test_sigmoid_proxy_error_bound_exhaustive_bf16():
-    """The fast path's proxy key is within 2^-12 of the exact fp32 sigmoid for every finite bf16
-    input (it assumes that bound and keeps a 2^-10 margin); also checked on random fp32 inputs."""
+    """The fast path's half-precision proxy key 0.5 tanh(x/2) + (0.5 + b) is within the error bound it
+    assumes of the exact fp32 key sigmoid(x) + b, for every finite bf16 logit under a sweep of biases
+    (small ones like the grouped workload's, and large ones where f16 rounding grows); and for fp32
+    logits (rounded to f16 first) at every f16 input of the tanh and on random inputs."""
     bits = torch.arange(0, 1 << 16, dtype=torch.int32).to(torch.int16)
     x = bits.view(torch.bfloat16).float()
     x = x[torch.isfinite(x)]
+    biases = [float(v) for v in torch.linspace(-0.1, 0.1, 11)] + [-0.5, -0.49, 0.3, 0.7, -1.0, 1.0, -3.0, 3.0,
+                                                                  10.0, -10.0, 100.0, 700.0]
+    worst = 0.0
+    for b in biases:
+        err, delta = B.debug_sigmoid_proxy_error(x.cuda(), torch.full_like(x, b).cuda())
+        ratio = (err.abs() / delta).max().item()
+        worst = max(worst, ratio)
+        assert ratio <= 1.0, f"bias {b}: |proxy - key| reaches {ratio:.3f} of the assumed bound"
+    # fp32 logits: x = 2h for every finite f16 h reaches tanh.approx.f16 at every input it can see, plus
+    # random fp32 logits (rounded to f16 first)
+    h = torch.arange(0, 1 << 16, dtype=torch.int32).to(torch.int16).view(torch.float16).float()
+    h = h[torch.isfinite(h)]
     g = torch.Generator().manual_seed(0)
-    x = torch.cat([x, torch.randn(1 << 20, generator=g) * 8, torch.rand(1 << 20, generator=g) * 60 - 30])
-    err = B.debug_sigmoid_proxy_error(x.cuda()).abs().max().item()
-    print("max |proxy - sigmoid| =", err)
-    assert err <= 2.0 ** -12
+    xf = torch.cat([2.0 * h, torch.randn(1 << 20, generator=g) * 8, torch.rand(1 << 20, generator=g) * 60 - 30])
+    worst32 = 0.0
+    for b in (-0.1, 0.0, 0.07, 0.5, -2.0, 30.0):
+        err, delta = B.debug_sigmoid_proxy_error(xf.cuda(), torch.full_like(xf, b).cuda(), f32_logits=True)
+        ratio = (err.abs() / delta).max().item()
+        worst32 = max(worst32, ratio)
+        assert ratio <= 1.0, f"fp32 logits, bias {b}: |proxy - key| reaches {ratio:.3f} of the assumed bound"
+    print("worst |proxy - key| / bound: bf16", worst, "fp32", worst32)
 
 
 def test_fast_path_group_ties_and_fallbacks():

@@ -47,7 +47,9 @@ def test_no_alloc_route_matches_route_on_two_calls_in_a_row():
 
 
 def test_no_alloc_route_rejects_a_workspace_it_cannot_hold():
-    p = B.route_params(64, 1024, 8, tile_tokens_dim=8)
+    # 65536 tokens of 1024 experts: 256 segments of 256 tokens, 2-byte counts -> a 512 KB table plus the
+    # header, past the static array (rejected before anything is launched)
+    p = B.route_params(65536, 1024, 8, tile_tokens_dim=8)
     dev = torch.device("cuda")
     out = {n: torch.zeros(1 << 16, dtype=torch.int32, device=dev) for n in NAMES}
     with pytest.raises(B.MoeError) as ei:

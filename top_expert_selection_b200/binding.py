@@ -37,7 +37,7 @@ EXPORTED = (
     "moe_error_string", "moe_workspace_init", "moe_status", "moe_route_capacity",
     "moe_route_workspace_bytes", "moe_route", "moe_aux_workspace_bytes", "moe_aux_scores", "moe_aux_scores_bwd", "moe_route_weights_bwd",
     "moe_aux_loss_fwd", "moe_aux_loss_bwd", "moe_dispatch", "moe_combine",
-    "moe_rmsnorm_router_topk_workspace_bytes", "moe_rmsnorm_router_topk", "moe_debug_barrier_wait",
+    "moe_rmsnorm_router_topk_workspace_bytes", "moe_rmsnorm_router_topk", "moe_debug_wait_timeout",
     "moe_debug_sigmoid_proxy_error", "moe_route_no_alloc", "moe_route_no_alloc_status",
     "moe_debug_no_alloc_record",
 )
@@ -98,8 +98,8 @@ def lib() -> ctypes.CDLL:
             "moe_rmsnorm_router_topk_workspace_bytes": ([i32, i32, i32, ctypes.POINTER(sz)], ctypes.c_int),
             "moe_rmsnorm_router_topk": ([i32, i32, i32, i32, f32, i32, P, P, P, P, P, P, P, P, P, sz, P],
                                         ctypes.c_int),
-            "moe_debug_barrier_wait": ([i32, i32, i64, P, sz, P], ctypes.c_int),
-            "moe_debug_sigmoid_proxy_error": ([P, i64, P, P], ctypes.c_int),
+            "moe_debug_wait_timeout": ([i32, i64, P, sz, P], ctypes.c_int),
+            "moe_debug_sigmoid_proxy_error": ([P, P, i64, i32, P, P, P], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name, None)
@@ -221,9 +221,9 @@ def route(logits: torch.Tensor, bias: Optional[torch.Tensor] = None, *, k: int, 
     return out
 
 
-def debug_barrier_wait(blocks: int, extra_arrivals: int, timeout_ns: int, ws: torch.Tensor, stream=None):
-    _check(lib().moe_debug_barrier_wait(blocks, extra_arrivals, timeout_ns, _p(ws), ctypes.c_size_t(ws.numel()),
-                                        _stream(stream)), "moe_debug_barrier_wait")
+def debug_wait_timeout(never_complete: bool, timeout_ns: int, ws: torch.Tensor, stream=None):
+    _check(lib().moe_debug_wait_timeout(int(never_complete), timeout_ns, _p(ws), ctypes.c_size_t(ws.numel()),
+                                        _stream(stream)), "moe_debug_wait_timeout")
 
 
 def route_into(p: RouteParams, logits: torch.Tensor, bias: Optional[torch.Tensor], out: Dict[str, torch.Tensor],
@@ -258,11 +258,13 @@ def route_workspace_bytes(p: RouteParams) -> int:
     return int(nb.value)
 
 
-def debug_sigmoid_proxy_error(x: torch.Tensor, stream=None) -> torch.Tensor:
-    out = torch.empty_like(x)
-    _check(lib().moe_debug_sigmoid_proxy_error(_p(x), x.numel(), _p(out), _stream(stream)),
-           "moe_debug_sigmoid_proxy_error")
-    return out
+def debug_sigmoid_proxy_error(x: torch.Tensor, b: torch.Tensor, f32_logits: bool = False, stream=None):
+    """(proxy - exact key, the assumed bound) per element, for logits x and biases b (fp32 device tensors)."""
+    err = torch.empty_like(x)
+    delta = torch.empty_like(x)
+    _check(lib().moe_debug_sigmoid_proxy_error(_p(x), _p(b), x.numel(), int(f32_logits), _p(err), _p(delta),
+                                               _stream(stream)), "moe_debug_sigmoid_proxy_error")
+    return err, delta
 
 
 # ---------------------------------------------------------------------------- aux loss

@@ -22,8 +22,7 @@ constexpr long long kDefaultTimeoutNs = 1000LL * 1000 * 1000;  // 1 s; a healthy
 struct WsHeader {
   int32_t status;              // MOE_OK or a MOE_ERR_DEVICE_* code
   uint32_t ticket;             // last-block-done counter (reductions)
-  unsigned long long barrier;  // grid barrier: generation (high 32 bits) | arrivals (low 32 bits)
-  uint32_t pad[12];            // keeps the header 64 bytes
+  uint32_t pad[14];            // keeps the header 64 bytes
 };
 static_assert(sizeof(WsHeader) == 64, "workspace header is 64 bytes");
 
@@ -51,63 +50,6 @@ __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long
   unsigned long long v;
   asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
-}
-
-// The barrier generation a block must pass: read before the block arrives
-// (the generation only moves once every block has arrived).
-__device__ __forceinline__ uint32_t barrier_generation(WsHeader* h) {
-  return (uint32_t)(ld_acquire_u64(&h->barrier) >> 32);
-}
-
-// Grid-wide barrier for a co-resident (cooperatively launched) grid of
-// `nblocks` blocks, split into an arrival and a wait so a block can do local
-// work in between.  One 64-bit word holds generation | arrivals.  A block's
-// arrival is a fire-and-forget add of 1 (the arriving thread does not wait
-// for it); waiters are released as soon as the count reads nblocks, and block
-// 0, once released, adds 2^32 - nblocks, which bumps the generation and clears
-// the count for the next launch (waiters that read the word after that see
-// the new generation instead).  One barrier per launch; after a wait that gave
-// up (status MOE_ERR_DEVICE_TIMEOUT) the workspace must be initialised again.
-//
-// grid_arrive: thread 0 only, after the block's writes to publish.
-__device__ __forceinline__ void grid_arrive(WsHeader* h, uint32_t /*nblocks*/) {
-  __threadfence();
-  asm volatile("red.relaxed.gpu.global.add.u64 [%0], 1;" ::"l"(&h->barrier) : "memory");
-}
-
-// grid_wait: thread 0 only; false (and a recorded timeout) if the wait
-// exceeded timeout_ns.
-__device__ __forceinline__ bool grid_wait(WsHeader* h, uint32_t nblocks, uint32_t gen_at_entry,
-                                          long long timeout_ns) {
-  unsigned long long t0 = 0;
-  int spins = 0;
-  while (true) {
-    const unsigned long long v = ld_acquire_u64(&h->barrier);
-    if ((uint32_t)(v >> 32) != gen_at_entry || (uint32_t)v == nblocks) break;
-    if (++spins == 64) t0 = globaltimer_ns();
-    if (spins > 64 && (long long)(globaltimer_ns() - t0) > timeout_ns) {
-      record_timeout(h);
-      return false;
-    }
-  }
-  __threadfence();
-  if (blockIdx.x == 0)
-    asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" ::"l"(&h->barrier),
-                 "l"((1ull << 32) - (unsigned long long)nblocks)
-                 : "memory");
-  return true;
-}
-
-// Both halves; must be called by all threads of the block.
-__device__ __forceinline__ bool grid_barrier(WsHeader* h, uint32_t nblocks, uint32_t gen_at_entry,
-                                             long long timeout_ns, int* smem_flag) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    grid_arrive(h, nblocks);
-    *smem_flag = grid_wait(h, nblocks, gen_at_entry, timeout_ns) ? 1 : 0;
-  }
-  __syncthreads();
-  return *smem_flag != 0;
 }
 
 // ---- ordered keys: float -> uint32 whose unsigned order is the float order ----

@@ -1,5 +1,5 @@
 // moe_route: expert selection, routing weights and permutation bookkeeping in
-// one cooperative launch.
+// two launches chained by programmatic dependent launch.
 //
 // Sources (by page title and section):
 //   Implementation:NVIDIA TransformerEngine Fused Router -- Description
@@ -12,31 +12,38 @@
 //   Implementation:InternLM Lmdeploy Gemm MoeUtils -- invokeMoeGate_V2 (maps
 //     and per-expert offsets).
 //
-// Kernel structure (one block per SM, all blocks co-resident):
-//   phase 1  each block owns a contiguous token range; its logits arrive in
-//            shared memory by up to 8 1-D bulk copies (TMA), each with its own
-//            mbarrier, all issued up front so compute starts on the first one
-//            while the rest stream in; each token is scored and selected, its
-//            ids/weights written, and a block histogram of expert counts kept
-//            in shared memory.  Selection paths:
-//              - sigmoid fast path (E = 8*V): 8 lanes per token, a lane per
-//                V experts (one expert group when n_group = 8), 4 tokens per
-//                warp.  A proxy key from tanh.approx (error <= delta) bounds
-//                where the exact keys can matter: exact fp32 keys (the stated
-//                formula) are computed only for each lane's top-2 region (exact
-//                group scores) and for the candidate set of the top-k, which is
-//                then ranked by counting.  Tokens whose candidate set overflows
-//                fall back to exact keys for all their experts (slow path);
-//              - generic: a warp per token (E > 32) or a thread per token
-//                (E <= 32) with exact keys and k rounds of argmax;
-//   publish  the block's histogram row goes to the workspace table and is
-//            added to the global counts (integer atomics, order-free);
-//   barrier  one bounded grid barrier;
-//   phase 2  every block derives the padded offsets from the counts, its own
-//            base per expert from the earlier blocks' rows, then walks its
-//            selections in token order (warp match + popcount) to assign slots
-//            deterministically; it also writes its share of the tile tables
-//            and of the padding rows of permuted_to_token.
+// The tokens are split into G contiguous segments of at most B tokens; block c
+// of both kernels owns segment c.
+//
+// route_select_kernel (one block per segment)
+//   Each token is scored and its top-k selected; ids and weights are written.
+//   Every selection also sets bit lt (the token's index in the segment) in a
+//   shared-memory bitmask of its expert.  After the block's selections, the
+//   rank of selection (t, e) among the segment's selections of e in token
+//   order is the number of bits of e's mask below lt (popcounts), and e's
+//   count is the number of all its bits.  The block writes the counts as its
+//   row of a table in the workspace and parks (expert, rank) of every
+//   selection in expanded_to_permuted.  Selection paths:
+//     - sigmoid fast path (E = 8*V): 8 lanes per token, a lane per V experts
+//       (one expert group when n_group = 8), 4 tokens per warp; each warp
+//       stages its 4 token rows in shared memory with one bulk copy (TMA),
+//       double-buffered.  A proxy key from tanh.approx (error <= delta)
+//       bounds where the exact keys can matter: exact fp32 keys (the stated
+//       formula) are computed only for each lane's top-2 region (exact group
+//       scores) and for the candidates of the top-k, which are ranked by
+//       counting.  A token whose candidates overflow falls back to exact keys
+//       for all its experts;
+//     - generic: a warp per token (E > 32) or a thread per token (E <= 32)
+//       with exact keys and k rounds of argmax, logits read from global memory.
+// route_permute_kernel (one block per segment, launched as the dependent)
+//   Every block sums all rows of the table (the expert counts) and the rows of
+//   the segments before its own (its base per expert), scans the tile-padded
+//   offsets, and turns each parked (expert, rank) into the slot offset + base +
+//   rank (deterministic, token order, no atomics); it also writes its share of
+//   the tile tables and of the padding rows of permuted_to_token.
+// Neither kernel waits on another block, so no device-side wait can time out
+// (the only bounded waits are on the block's own bulk copies).
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -49,20 +56,10 @@ namespace moe {
 
 namespace {
 
-// threads per block: the sigmoid fast path keeps few registers and runs 24
-// warps per SM; the generic paths keep larger per-thread arrays and run 16
-constexpr int kThreadsFast = 896;
-constexpr int kThreadsGeneric = 512;
-constexpr int kWarpsMax = kThreadsFast / 32;
-constexpr int kStageBytesMax = 96 * 1024;
-constexpr int kMaxSub = 8;         // bulk copies (and mbarriers) per staged round
-constexpr int kCandMax = 32;       // fast path: candidate slots per token
-constexpr int kCandStride = 33;    // padded so the 4 tokens of a warp hit different banks
-// |proxy key - exact key| bound used by the fast path.  The proxy is
-// 0.5*tanh.approx(x/2) + (0.5 + b); tanh.approx.f32 has a relative error of
-// about 2^-11, i.e. <= 2^-12 on the sigmoid; 2^-10 leaves a 4x margin (the
-// margin is checked exhaustively over all bf16 inputs by the test suite).
-constexpr float kProxyDelta = 1.0f / 1024.0f;
+constexpr int kFastWarpsMax = 28;        // fast path: up to 28 warps of 4 tokens (72 registers a thread)
+constexpr int kGenericThreads = 512;     // generic paths
+constexpr int kPermThreads = 1024;       // bookkeeping kernel
+constexpr int kMaxSegment = 256;         // tokens per segment (8 mask words)
 
 struct RouteArgs {
   const void* logits;
@@ -77,7 +74,8 @@ struct RouteArgs {
   int32_t* tile_mn;
   int32_t* totals;
   WsHeader* hdr;
-  uint32_t* table;   // [G][row_stride bytes]: per-block expert counts
+  uint8_t* table;    // [G][row_stride]: per-segment expert counts (cnt_bytes wide)
+  uint32_t* gtot;    // [NG][E]: per-group expert counts (groups of GS segments), zero between calls
   int T, E, k;
   int score_fn, pre, grouped, n_group, topk_group, topn;
   int renorm;
@@ -86,104 +84,57 @@ struct RouteArgs {
   uint32_t kinv;     // ceil(2^32 / k): item -> token by a multiply-high
   int logits_dtype, bias_dtype, weights_dtype;
   int has_bias;
-  int G;
+  int G, B;          // segments, tokens per segment (segment c: [c*B, min(T, (c+1)*B)))
+  int MW;            // 32-bit mask words per expert: ceil(B / 32)
+  int GS, NG;        // segments per group, groups
   int max_padded;
   int max_tiles;
   int loc_off, loc_n;  // the local experts [loc_off, loc_off + loc_n): only they get slots and tiles
-  int chunk_tokens;
-  int stage_bytes;  // stage region: >= chunk_tokens * row_bytes and >= phase 2's partials
-  int row_bytes;
-  int cnt_bytes;   // width of a block's histogram entry in the table: 1, 2 or 4
-  int row_stride;  // bytes per table row (16-byte multiple)
-  int fast;        // 1: sigmoid fast path
-  int ids_in_smem; // 1: the block's selections also kept in shared memory (u16)
+  int row_bytes;     // bytes per logits row
+  int cnt_bytes;     // width of a table entry: 1 (B <= 255) or 2
+  int row_stride;    // bytes per table row (16-byte multiple)
   long long timeout_ns;
 };
 
-struct RouteSmem {
-  // offsets (bytes) inside dynamic shared memory
-  int stage, cand, bias, hist_cta, hist_w, offs, cnt, bar, flag, scan, ids, lrank, lut, total;
+// ---------------------------------------------------------------------------
+// shared-memory layout of the selection kernel
+// ---------------------------------------------------------------------------
+struct SelSmem {
+  int masks, ids, bias, cb, delta, warp0, warp_bytes, total;
+  int stage_bytes;  // per staging slot (fast path)
 };
 
-// per warp: 4 tokens x kCandStride packed u64 keys, then 4 x kCandStride fp32 scores
-__host__ __device__ inline int cand_bytes_per_warp() { return 4 * kCandStride * 12; }
+constexpr int kCandSlotsPerToken = 32;  // fast path: candidates ranked per token
+// fast path: a warp's tokens left to the exact path; a segment holds at most
+// 256 tokens = 64 quads over at least 28 warps (or one quad per warp), so a
+// warp runs at most 3 rounds of 4 tokens
+constexpr int kPendMax = 12;
+constexpr int kCandBytes = 4 * kCandSlotsPerToken * 14 + 2 * kPendMax + 8;
 
-__host__ __device__ inline RouteSmem route_smem_layout(int E, int stage_bytes, int ids_bytes, int nwarps,
-                                                       int lut_bytes) {
-  RouteSmem L;
+// per warp (fast path): 2 staging slots of 4 rows; 4 tokens x 32 packed u64
+// candidate keys, 4 x 32 fp32 scores and 4 x 32 u16 expert ids; the warp's
+// pending exact-path tokens; 2 mbarriers
+__host__ __device__ inline SelSmem sel_smem_layout(int E, int MW, int B, int k, int fast, int V, int row_bytes,
+                                                   int nwarps) {
+  SelSmem L;
   int o = 0;
-  L.stage = o;
-  o += (stage_bytes + 127) & ~127;
-  L.cand = o;
-  o += nwarps * cand_bytes_per_warp() + 8 * (32 + 4) * 4;  // + the fast path's per-lane bias table
+  L.masks = o;
+  o += E * MW * 4;
+  L.ids = o;
+  o += ((B * k * 2) + 15) & ~15;
   L.bias = o;
   o += ((E * 4) + 15) & ~15;
-  L.hist_cta = o;
-  o += ((E * 4) + 15) & ~15;
-  L.hist_w = o;
-  o += ((nwarps * E * 4) + 15) & ~15;
-  L.offs = o;
-  o += (((E + 1) * 4) + 15) & ~15;
-  L.cnt = o;
-  o += ((E * 4) + 15) & ~15;
-  L.bar = o;
-  o += 8 * kMaxSub;
-  L.flag = o;
-  o += 16;
-  L.scan = o;
-  o += 32 * 4;
-  L.ids = o;
-  o += (ids_bytes + 15) & ~15;
-  L.lrank = o;  // per selection: rank among the block's selections of the same expert (u16)
-  o += (ids_bytes + 15) & ~15;
-  L.lut = o;
-  o += (lut_bytes + 15) & ~15;
+  L.cb = o;  // fast path: 8 rows of V f16 constants 0.5 + b, 16 bytes of padding each
+  o += fast ? 8 * (V * 2 + 16) : 0;
+  L.delta = o;  // fast path: the block's proxy error bound
+  o += fast ? 16 : 0;
+  o = (o + 127) & ~127;
+  L.warp0 = o;
+  L.stage_bytes = fast ? ((4 * row_bytes + 127) & ~127) : 0;
+  L.warp_bytes = fast ? ((2 * L.stage_bytes + kCandBytes + 16 + 127) & ~127) : 0;
+  o += L.warp_bytes * nwarps;
   L.total = o;
   return L;
-}
-
-// -------------------------------------------------------------------------
-// staging: tokens [t0, t0+n) of logits into shared memory
-// -------------------------------------------------------------------------
-// Issues up to kMaxSub bulk copies, sub-copy s completing on bar[s].  Returns
-// their number; 0 means the rows were copied with plain loads instead
-// (unaligned source or rows that are not 16-byte multiples) and are ready.
-__device__ int stage_issue(const RouteArgs& a, uint8_t* stage, uint64_t* bar, int t0, int n) {
-  const uint8_t* src = reinterpret_cast<const uint8_t*>(a.logits) + (size_t)t0 * a.row_bytes;
-  const bool bulk = ((reinterpret_cast<uintptr_t>(src) & 15) == 0) && (a.row_bytes % 16 == 0);
-  if (!bulk) {
-    const uint32_t bytes = (uint32_t)n * (uint32_t)a.row_bytes;
-    for (uint32_t i = threadIdx.x; i < bytes; i += blockDim.x) stage[i] = src[i];
-    __syncthreads();
-    return 0;
-  }
-  const int nsub = min(kMaxSub, n);
-  if (threadIdx.x == 0) {
-    // earlier generic-proxy accesses of the stage precede the async-proxy writes
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    // every mbarrier completes exactly one phase per round (unused ones with
-    // zero bytes), so the parity of round r is r & 1 for all of them
-    for (int s = 0; s < kMaxSub; ++s) {
-      if (s < nsub) {
-        const int tb = s * n / nsub, te = (s + 1) * n / nsub;
-        const uint32_t bytes = (uint32_t)(te - tb) * (uint32_t)a.row_bytes;
-        mbar_arrive_expect_tx(&bar[s], bytes);
-        bulk_g2s(stage + (size_t)tb * a.row_bytes, src + (size_t)tb * a.row_bytes, bytes, &bar[s]);
-      } else {
-        mbar_arrive_expect_tx(&bar[s], 0u);
-      }
-    }
-  }
-  return nsub;
-}
-
-// sub-copy holding local token lt when n tokens are split into nsub parts
-__device__ __forceinline__ int sub_of(int lt, int n, int nsub) { return ((lt + 1) * nsub - 1) / n; }
-
-__device__ __forceinline__ bool stage_wait(const RouteArgs& a, uint64_t* bar, int s, uint32_t parity) {
-  if (mbar_wait_bounded(&bar[s], parity, a.timeout_ns)) return true;
-  record_timeout(a.hdr);
-  return false;
 }
 
 __device__ __forceinline__ float stage_val(const RouteArgs& a, const uint8_t* row, int e) {
@@ -193,51 +144,24 @@ __device__ __forceinline__ float stage_val(const RouteArgs& a, const uint8_t* ro
 
 __device__ __forceinline__ float sigmoid_f32(float x) { return 1.0f / (1.0f + expf(-x)); }
 
-// Exact sigmoid of a bf16 input by table: the kernel fills the table with the
-// very expression above for every bf16 value with biased exponent in
-// [kLutExpLo, kLutExpHi], both signs (8448 entries, 33 KB), so a lookup returns
-// exactly what sigmoid_f32 returns.  Inputs outside the range (|x| < 2^-25 or
-// |x| >= 2^8, and non-finite) are evaluated directly.
-constexpr int kLutExpLo = 102, kLutExpHi = 134;
-constexpr int kLutPerSign = (kLutExpHi - kLutExpLo + 1) * 128;
-constexpr int kLutEntries = 2 * kLutPerSign;
-
-__device__ __forceinline__ int lut_index(uint32_t b16) {
-  const int ex = (int)((b16 >> 7) & 0xffu);
-  if (ex < kLutExpLo || ex > kLutExpHi) return -1;
-  return (int)(b16 >> 15) * kLutPerSign + (ex - kLutExpLo) * 128 + (int)(b16 & 0x7fu);
+// expert e belongs to this shard: it gets rows, slots and tiles
+__device__ __forceinline__ bool is_local(const RouteArgs& a, int e) {
+  return (unsigned)(e - a.loc_off) < (unsigned)a.loc_n;
 }
 
-__device__ __forceinline__ uint32_t lut_bits(int idx) {
-  const int sgn = idx / kLutPerSign, r = idx % kLutPerSign;
-  return ((uint32_t)sgn << 15) | ((uint32_t)(r / 128 + kLutExpLo) << 7) | (uint32_t)(r % 128);
-}
-
-// exact score of expert e of a staged bf16 row: table when available
-__device__ __forceinline__ float sigmoid_bf16_row(const float* lut, const uint8_t* row, int e) {
-  const uint32_t b16 = reinterpret_cast<const uint16_t*>(row)[e];
-  const int idx = lut ? lut_index(b16) : -1;
-  return idx >= 0 ? lut[idx] : sigmoid_f32(bf16_bits_to_f32((uint16_t)b16));
+// One selection of expert e by the segment's token lt at slot j: the id in the
+// segment's list, the token's bit in e's mask.
+__device__ __forceinline__ void mark(const RouteArgs& a, uint32_t* masks, uint16_t* ids_s, int lt, int j, int e) {
+  ids_s[lt * a.k + j] = (uint16_t)e;
+  atomicOr(&masks[e * a.MW + (lt >> 5)], 1u << (lt & 31));
 }
 
 // -------------------------------------------------------------------------
 // warp per token (E > 32): lane l owns experts [l*VPL, l*VPL + VPL)
 // -------------------------------------------------------------------------
-// keep a copy of a selection in the block's shared-memory id list (phase 2
-// reads it instead of global memory)
-// expert e belongs to this shard: it gets rows, slots and tiles (phase 1
-// counts every expert; phase 2 gives the others zero width)
-__device__ __forceinline__ bool is_local(const RouteArgs& a, int e) {
-  return (unsigned)(e - a.loc_off) < (unsigned)a.loc_n;
-}
-
-__device__ __forceinline__ void keep_id(uint16_t* ids_s, int local_item, int e) {
-  if (ids_s) ids_s[local_item] = (uint16_t)e;
-}
-
 template <int VPL>
-__device__ void select_token_warp(const RouteArgs& a, const uint8_t* row, int t, const float* bias_s,
-                                  int* hist_cta, int lane, uint16_t* ids_s, int t_base) {
+__device__ void select_token_warp(const RouteArgs& a, const uint8_t* row, long long t, int lt, const float* bias_s,
+                                  uint32_t* masks, uint16_t* ids_s, int lane) {
   const int E = a.E;
   const unsigned FULL = 0xffffffffu;
   float lg[VPL], s[VPL], key[VPL];
@@ -416,9 +340,8 @@ __device__ void select_token_warp(const RouteArgs& a, const uint8_t* row, int t,
   if (has_slot) {
     const size_t o = (size_t)t * a.k + lane;
     a.ids[o] = my_id;
-    keep_id(ids_s, (t - t_base) * a.k + lane, my_id);
     store_from_f32(a.weights, a.weights_dtype, o, v);
-    if ((unsigned)my_id < (unsigned)E) atomicAdd(&hist_cta[my_id], 1); else record_bounds(a.hdr);
+    if ((unsigned)my_id < (unsigned)E) mark(a, masks, ids_s, lt, lane, my_id); else record_bounds(a.hdr);
   }
 }
 
@@ -426,8 +349,8 @@ __device__ void select_token_warp(const RouteArgs& a, const uint8_t* row, int t,
 // thread per token (E <= EMAX <= 32)
 // -------------------------------------------------------------------------
 template <int EMAX>
-__device__ void select_token_thread(const RouteArgs& a, const uint8_t* row, int t, const float* bias_s,
-                                    int* hist_cta, uint16_t* ids_s, int t_base) {
+__device__ void select_token_thread(const RouteArgs& a, const uint8_t* row, long long t, int lt, const float* bias_s,
+                                    uint32_t* masks, uint16_t* ids_s) {
   const int E = a.E;
   float lg[EMAX], s[EMAX], key[EMAX];
 #pragma unroll
@@ -544,9 +467,8 @@ __device__ void select_token_thread(const RouteArgs& a, const uint8_t* row, int 
       const float w = a.renorm ? (val[j] / norm) * a.scale : val[j] * a.scale;
       const size_t o = (size_t)t * a.k + j;
       a.ids[o] = sel[j];
-      keep_id(ids_s, (t - t_base) * a.k + j, sel[j]);
       store_from_f32(a.weights, a.weights_dtype, o, w);
-      if ((unsigned)sel[j] < (unsigned)E) atomicAdd(&hist_cta[sel[j]], 1); else record_bounds(a.hdr);
+      if ((unsigned)sel[j] < (unsigned)E) mark(a, masks, ids_s, lt, j, sel[j]); else record_bounds(a.hdr);
     }
   }
 }
@@ -554,10 +476,41 @@ __device__ void select_token_thread(const RouteArgs& a, const uint8_t* row, int 
 // -------------------------------------------------------------------------
 // sigmoid fast path: 8 lanes per token, lane g owns experts [g*V, (g+1)*V)
 // -------------------------------------------------------------------------
-__device__ __forceinline__ float tanh_approx(float x) {
-  float y;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
+// The proxy key of the fast path, two experts at a time in half precision:
+//   p = 0.5 * tanh.approx(x / 2) + (0.5 + b)   (sigmoid(x) = 0.5 + 0.5 tanh(x/2))
+// with x rounded to f16 (exact for bf16 logits in the f16 range), the tanh and
+// the fused multiply-add in packed f16.  cb2 holds 0.5 + b of both experts in
+// f16.  |p - (sigmoid(x) + b)| <= proxy_delta(...) (see below).
+__device__ __forceinline__ __half2 proxy_pair(float xlo, float xhi, __half2 cb2) {
+  const __half2 half = __float2half2_rn(0.5f);
+  const __half2 h = __hmul2(__floats2half2_rn(xlo, xhi), half);
+  return __hfma2(h2tanh_approx(h), half, cb2);
+}
+
+// Absolute error bound of proxy_pair over a block whose experts have
+// |0.5 + b| <= cbmax: half the assumed tanh.approx.f16 error (|t| <= 1), the
+// f16 rounding of 0.5 + b and of the fused multiply-add's result (|p| <= 0.5 +
+// cbmax), the f16 rounding of fp32 logits (|sigmoid'(x) x| <= 0.224, i.e.
+// <= 2^-13 at 11 bits), and slack for the fp32 sigmoid's own rounding.
+// kTanh16Err is checked against every f16 input by the test suite, and the
+// whole bound against every bf16 logit under a sweep of biases.
+constexpr float kTanh16Err = 1.0f / 1024.0f;
+__host__ __device__ inline float half_ulp16(float v) {
+  // half an f16 ulp at magnitude v (v >= 2^-14): 2^(floor(log2 v) - 11)
+  int e = 0;
+  float m = v;
+  while (m >= 2.0f) { m *= 0.5f; ++e; }
+  while (m < 1.0f && e > -14) { m *= 2.0f; --e; }
+  float r = 1.0f;
+  for (int i = 0; i < 11 - e; ++i) r *= 0.5f;
+  for (int i = 0; i < e - 11; ++i) r *= 2.0f;
+  return r;
+}
+__host__ __device__ inline float proxy_delta(float cbmax, int f32_logits) {
+  if (!(cbmax <= 1024.0f)) return INFINITY;  // f16 too coarse: every expert becomes a candidate
+  const float d = 0.5f * kTanh16Err + half_ulp16(cbmax) + half_ulp16(0.5f + cbmax) +
+                  (f32_logits ? 1.0f / 8192.0f : 0.0f) + 1.0f / (1 << 20);
+  return d;
 }
 
 // A lane reads its NC 16-byte chunks starting at chunk `rot` = g*NC/8, so the 8
@@ -575,205 +528,164 @@ __device__ __forceinline__ int expert_slot(int g, int rot, int e) {
   return (((r / EPC) - rot + NC) & (NC - 1)) * EPC + (r % EPC);
 }
 
-// Per-lane constants 0.5 + bias of the lane's experts, in register-slot order,
-// one padded row of V + 4 floats per lane position g: the 16-byte loads of the
-// 8 lanes of a token fall in distinct bank groups.
+// Per-lane constants 0.5 + bias of the lane's experts in f16, in register-slot
+// order: one row of V halves + 16 bytes of padding per lane position g (the
+// 16-byte loads of the 8 lanes of a token fall in distinct bank groups).
 template <int V>
-__host__ __device__ constexpr int cb_stride() { return V + 4; }
+__host__ __device__ constexpr int cb_stride_bytes() { return V * 2 + 16; }
 
-// Out-of-line exact selection of one token (rare): exact keys for all experts
-// of the lane, exact group scores, k rounds of segment argmax.
-template <int V, int ESZ>
-__device__ __noinline__ void select_token_exact8(const RouteArgs& a, const uint8_t* row, long long t, int g, int rot,
-                                                 int seg, unsigned smask, const float* bias_s, int* hist_cta,
-                                                 uint16_t* ids_s, int t_base) {
-  constexpr uint32_t VMASK = (V >= 32) ? 0xffffffffu : ((1u << V) - 1u);
-  float p[V];
+// Bits of a packed mask: pair i's low half (slot 2i) is bit i, its high half
+// (slot 2i+1) bit 16 + i.
+__device__ __forceinline__ int mask_bit_slot(int b) { return b < 16 ? 2 * b : 2 * (b - 16) + 1; }
+
+// Mask of the lane's slots whose proxy is >= thr (thr rounded down to f16).
+template <int NW>
+__device__ __forceinline__ uint32_t proxy_mask(const __half2 (&p2)[NW], float thr) {
+  const __half t = __float2half_rd(thr);
+  const __half2 t2 = __halves2half2(t, t);
+  uint32_t m = 0;
 #pragma unroll
-  for (int j = 0; j < V; ++j) {
-    const int e = slot_expert<V, ESZ>(g, rot, j);
-    p[j] = sigmoid_f32(stage_val(a, row, e)) + bias_s[e];
-  }
-  uint32_t allowed = VMASK;
-  if (a.grouped) {
-    float e1 = -INFINITY, e2 = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < V; ++j) {
-      const float hi = fmaxf(e1, p[j]);
-      e2 = fmaxf(e2, fminf(e1, p[j]));
-      e1 = hi;
-    }
-    const float gsc = (a.topn == 1) ? e1 : (e1 + e2);
-    int rank = 0;
-    for (int h = 0; h < 8; ++h) {
-      const float o = __shfl_sync(smask, gsc, seg | h);
-      rank += (o > gsc || (o == gsc && h < g)) ? 1 : 0;
-    }
-    if (rank >= a.topk_group) allowed = 0;
-  }
-  float ssum = 0.0f;
-  for (int jr = 0; jr < a.k; ++jr) {
-    unsigned long long best = 0ull;
-#pragma unroll
-    for (int j = 0; j < V; ++j)
-      if ((allowed >> j) & 1u) {
-        const unsigned long long pk = pack_key(p[j], slot_expert<V, ESZ>(g, rot, j));
-        best = pk > best ? pk : best;
-      }
-#pragma unroll
-    for (int off = 1; off < 8; off <<= 1) {
-      const unsigned long long o = shfl_xor_u64(smask, best, off);
-      best = o > best ? o : best;
-    }
-    const int win = packed_expert(best);
-    if (win / V == g) allowed &= ~(1u << expert_slot<V, ESZ>(g, rot, win));
-    if (g == 0) {
-      const float sg = sigmoid_f32(stage_val(a, row, win));
-      a.ids[(size_t)t * a.k + jr] = win;
-      keep_id(ids_s, (int)(t - t_base) * a.k + jr, win);
-      ssum = ssum + sg;
-      if ((unsigned)win < (unsigned)a.E) atomicAdd(&hist_cta[win], 1); else record_bounds(a.hdr);
-    }
-  }
-  if (g == 0) {
-    for (int jr = 0; jr < a.k; ++jr) {
-      const size_t o = (size_t)t * a.k + jr;
-      const float sg = sigmoid_f32(stage_val(a, row, a.ids[o]));
-      store_from_f32(a.weights, a.weights_dtype, o, a.renorm ? (sg / ssum) * a.scale : sg * a.scale);
-    }
-  }
+  for (int i = 0; i < NW; ++i) m |= (__hge2_mask(p2[i], t2) >> (15 - i)) & (0x00010001u << i);
+  return m;
 }
 
+constexpr int kCandSlots = kCandSlotsPerToken;  // more candidates send the token to the exact path
+
+// One quad of tokens (lane = 8*q + g: token q, experts of lane position g),
+// their rows staged in shared memory at `rows`.  cand: per token kCandSlots
+// packed (ordered key, ~expert) words, then kCandSlots fp32 scores.  Returns
+// the mask of the quad's tokens left to the exact path (bit q).
+//
+// 1. Proxy keys p (|p - key| <= delta) of the lane's V experts and the lane's
+//    top-2 proxies m1 >= m2 (the two largest keys lie within delta of them).
+// 2. Groups (lane g = group g): the approximate group scores s = m1 + m2 (or
+//    m1) are within e = 2 delta (delta) of the exact ones.  A group is surely
+//    kept when fewer than topk_group others may reach its score (s_h + e >=
+//    s_g - e), surely dropped when topk_group others surely beat it (s_h - e >
+//    s_g + e); the others are undecided and stay candidates' sources until
+//    their exact scores are known.
+// 3. Threshold: each group that can be kept holds two experts with keys >=
+//    its m2 - delta, and the kept groups hold 2 * topk_group >= k such
+//    experts, so the k-th largest key is >= min m2 - delta over the groups
+//    that can be kept (for ungrouped routing: the k-th largest of the lanes'
+//    m1, m2, minus delta); an expert that can be in the top-k has a proxy >=
+//    that minus delta.
+// 4. Candidates (experts of the groups that can be kept, over the threshold;
+//    at most kCandSlots per token): listed per token, their exact keys (the
+//    stated formula) computed by the token's 8 lanes.  The threshold is below every such group's m2 - 2 delta,
+//    so each undecided group's exact top-2 keys are candidates: its exact
+//    score comes from its candidates, the undecided groups are ranked
+//    exactly (ties -> lower group) and the dropped ones' candidates are
+//    zeroed.  The candidates are ranked by counting on packed (ordered key,
+//    ~expert) words: larger key first, then lower expert.
 template <int V, int ESZ>
-__device__ void select_quad_fast(const RouteArgs& a, const uint8_t* stage, int lt_base, int n, int t_round0,
-                                 const float* cb_s, const float* bias_s, float* cand, int* hist_cta,
-                                 int lane, uint16_t* ids_s, int t_base, const float* lut) {
-  constexpr int EPC = 16 / ESZ, NC = V / EPC;
-  constexpr uint32_t VMASK = (V >= 32) ? 0xffffffffu : ((1u << V) - 1u);
+__device__ unsigned select_quad_fast(const RouteArgs& a, const uint8_t* rows, int lt0, int nq, long long t_seg,
+                                     const uint8_t* cb_s, const float* bias_s, float delta, uint8_t* cand,
+                                     uint32_t* masks, uint16_t* ids_s, int lane) {
+  constexpr int EPC = 16 / ESZ, NC = V / EPC, NW = V / 2, PPC = EPC / 2;  // pairs per chunk
   const unsigned FULL = 0xffffffffu;
   const int q = lane >> 3, g = lane & 7, seg = lane & 24;
   const int rot = (g * NC) >> 3;
-  const int lt = lt_base + q;
-  const bool tv = lt < n;
-  const uint8_t* row = stage + (size_t)(tv ? lt : 0) * a.row_bytes;
-  const long long t = (long long)t_round0 + lt;
+  const bool tv = q < nq;
+  const uint8_t* row = rows + (size_t)(tv ? q : 0) * a.row_bytes;
+  const int lt = lt0 + q;
+  const long long t = t_seg + lt;
+  unsigned long long* ck = reinterpret_cast<unsigned long long*>(cand) + q * kCandSlots;
+  float* cs = reinterpret_cast<float*>(cand + 4 * kCandSlots * 8) + q * kCandSlots;
 
-  // ---- proxy keys (|p - key| <= kProxyDelta) and their top-2 ----
-  float p[V];
-  float m1 = -INFINITY, m2 = -INFINITY, n1 = -INFINITY, n2 = -INFINITY;
-  const float* cbl = cb_s + g * cb_stride<V>();
+  // ---- 1. proxies, packed two per register, and their top-2 (two streams:
+  //         even and odd slots) ----
+  __half2 p2[NW];
+  __half2 m1 = __float2half2_rn(-INFINITY), m2 = m1;
+  const uint8_t* cbl = cb_s + g * cb_stride_bytes<V>();
 #pragma unroll
   for (int c = 0; c < NC; ++c) {
     const int cc = (c + rot) & (NC - 1);
     const uint4 v = *reinterpret_cast<const uint4*>(row + (size_t)g * V * ESZ + cc * 16);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    float cbv[EPC];
-#pragma unroll
-    for (int i = 0; i < EPC; i += 4) {
-      const float4 b4 = *reinterpret_cast<const float4*>(cbl + c * EPC + i);
-      cbv[i] = b4.x; cbv[i + 1] = b4.y; cbv[i + 2] = b4.z; cbv[i + 3] = b4.w;
+    uint32_t cbw[4];
+    if constexpr (PPC == 4) {
+      const uint4 c4 = *reinterpret_cast<const uint4*>(cbl + c * 16);
+      cbw[0] = c4.x; cbw[1] = c4.y; cbw[2] = c4.z; cbw[3] = c4.w;
+    } else {
+      const uint2 c2 = *reinterpret_cast<const uint2*>(cbl + c * 8);
+      cbw[0] = c2.x; cbw[1] = c2.y;
     }
 #pragma unroll
-    for (int i = 0; i < EPC; ++i) {
-      float x;
-      if constexpr (ESZ == 2)
-        x = __uint_as_float((i & 1) ? (w[i >> 1] & 0xffff0000u) : (w[i >> 1] << 16));
-      else
-        x = __uint_as_float(w[i]);
-      const int j = c * EPC + i;
-      const float pj = fmaf(0.5f, tanh_approx(0.5f * x), cbv[i]);
-      p[j] = pj;
-      // two independent top-2 trackers (even / odd slots) shorten the dependency chain
-      if ((i & 1) == 0) {
-        const float hi = fmaxf(m1, pj);
-        m2 = fmaxf(m2, fminf(m1, pj));
-        m1 = hi;
+    for (int i = 0; i < PPC; ++i) {
+      float xlo, xhi;
+      if constexpr (ESZ == 2) {
+        xlo = __uint_as_float(w[i] << 16);
+        xhi = __uint_as_float(w[i] & 0xffff0000u);
       } else {
-        const float hi = fmaxf(n1, pj);
-        n2 = fmaxf(n2, fminf(n1, pj));
-        n1 = hi;
+        xlo = __uint_as_float(w[2 * i]);
+        xhi = __uint_as_float(w[2 * i + 1]);
       }
+      const __half2 p = proxy_pair(xlo, xhi, *reinterpret_cast<const __half2*>(&cbw[i]));
+      p2[c * PPC + i] = p;
+      const __half2 hi = __hmax2(m1, p);
+      m2 = __hmax2(m2, __hmin2(m1, p));
+      m1 = hi;
     }
   }
+  float M1, M2;
   {
-    const float hi = fmaxf(m1, n1);
-    m2 = fmaxf(fminf(m1, n1), fmaxf(m2, n2));
-    m1 = hi;
+    const float a1 = __low2float(m1), b1 = __high2float(m1), a2 = __low2float(m2), b2 = __high2float(m2);
+    M1 = fmaxf(a1, b1);
+    M2 = fmaxf(fminf(a1, b1), fmaxf(a2, b2));
   }
 
-  // ---- exact top-2 keys of the lane: evaluated where the proxy is within
-  //      2*delta of the lane's 2nd-best proxy (the exact top-2 lie there) ----
-  float K1 = -INFINITY, K2 = -INFINITY, S1 = 0.0f, S2 = 0.0f;
-  int j1 = -1, j2 = -1;
-  if (tv) {
-    const float th = m2 - 2.0f * kProxyDelta;
-    uint32_t mq[4] = {0u, 0u, 0u, 0u};  // independent partial masks
-#pragma unroll
-    for (int j = 0; j < V; ++j) mq[j & 3] |= (p[j] >= th ? 1u : 0u) << j;
-    uint32_t m = (mq[0] | mq[1]) | (mq[2] | mq[3]);
-    while (m) {
-      // up to 4 members per pass, their exact keys evaluated side by side
-      int jb[4];
-      float kb4[4], sb4[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        jb[u] = m ? __ffs(m) - 1 : -1;
-        m &= m - 1;
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int e = slot_expert<V, ESZ>(g, rot, max(jb[u], 0));
-        sb4[u] = (ESZ == 2) ? sigmoid_bf16_row(lut, row, e) : sigmoid_f32(stage_val(a, row, e));
-        kb4[u] = sb4[u] + bias_s[e];
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (jb[u] < 0) continue;
-        const float K = kb4[u];
-        if (K > K1) {
-          K2 = K1; S2 = S1; j2 = j1;
-          K1 = K; S1 = sb4[u]; j1 = jb[u];
-        } else if (K > K2) {
-          K2 = K; S2 = sb4[u]; j2 = jb[u];
-        }
-      }
-    }
-  }
-
-  // ---- kept groups from exact group scores (lane g = group g) ----
-  bool kept = true;
-  unsigned kb = 0xffu;
+  // ---- 2. groups: surely kept, surely dropped, undecided ----
+  bool maybe = true;   // this group can be kept
+  bool undec = false;  // undecided: kept or not is settled by exact scores
+  int K = 8;           // groups kept
   if (a.grouped) {
-    const float gsc = (a.topn == 1) ? K1 : (K1 + K2);
-    int rank = 0;
+    K = a.topk_group;
+    const float gsc = (a.topn == 1) ? M1 : (M1 + M2);
+    const float e2 = (a.topn == 1 ? 2.0f : 4.0f) * delta;  // twice the score error
+    int may_beat = 0, beats = 0;
 #pragma unroll
     for (int h = 0; h < 8; ++h) {
       const float o = __shfl_sync(FULL, gsc, seg | h);
-      rank += (o > gsc || (o == gsc && h < g)) ? 1 : 0;
+      may_beat += (h != g && o + e2 >= gsc) ? 1 : 0;
+      beats += (o - e2 > gsc) ? 1 : 0;
     }
-    kept = rank < a.topk_group;
-    kb = (__ballot_sync(FULL, kept) >> seg) & 0xffu;
+    const bool sure = may_beat < K;
+    maybe = beats < K;
+    undec = maybe && !sure;
   }
 
-  // ---- candidates: every kept lane holds two exact keys >= K2min, so the
-  //      k-th largest key is >= K2min when 2 * nkept >= k; any expert that can
-  //      reach the top-k has key >= K2min, hence proxy >= K2min - delta ----
-  float k2min = kept ? K2 : INFINITY;
-  k2min = fminf(k2min, __shfl_xor_sync(FULL, k2min, 1));
-  k2min = fminf(k2min, __shfl_xor_sync(FULL, k2min, 2));
-  k2min = fminf(k2min, __shfl_xor_sync(FULL, k2min, 4));
-  const int nkept = __popc(kb);
-  const float tau = (2 * nkept >= a.k) ? (k2min - kProxyDelta) : -INFINITY;
-  uint32_t mask = 0;
-  if (kept && tv) {
-    uint32_t mq[4] = {0u, 0u, 0u, 0u};
+  // ---- 3. candidate threshold ----
+  float kth;
+  if (a.grouped) {
+    // min m2 over the groups that can be kept (2 * topk_group >= k on this path)
+    float mn = maybe ? M2 : INFINITY;
+    mn = fminf(mn, __shfl_xor_sync(FULL, mn, 1));
+    mn = fminf(mn, __shfl_xor_sync(FULL, mn, 2));
+    kth = fminf(mn, __shfl_xor_sync(FULL, mn, 4));
+  } else {
+    // the k-th largest of the 16 proxies m1, m2 of the token's lanes
+    int gt1 = 0, ge1 = 0, gt2 = 0, ge2 = 0;
 #pragma unroll
-    for (int j = 0; j < V; ++j) mq[j & 3] |= (p[j] >= tau ? 1u : 0u) << j;
-    mask = (mq[0] | mq[1]) | (mq[2] | mq[3]);
-    if (j1 >= 0) mask |= 1u << j1;
-    if (j2 >= 0) mask |= 1u << j2;
+    for (int h = 0; h < 8; ++h) {
+      const float o1 = __shfl_sync(FULL, M1, seg | h), o2 = __shfl_sync(FULL, M2, seg | h);
+      gt1 += (o1 > M1) + (o2 > M1);
+      ge1 += (o1 >= M1) + (o2 >= M1);
+      gt2 += (o1 > M2) + (o2 > M2);
+      ge2 += (o1 >= M2) + (o2 >= M2);
+    }
+    float mine = -INFINITY;
+    if (gt1 < a.k && ge1 >= a.k) mine = M1;
+    if (gt2 < a.k && ge2 >= a.k) mine = fmaxf(mine, M2);
+    mine = fmaxf(mine, __shfl_xor_sync(FULL, mine, 1));
+    mine = fmaxf(mine, __shfl_xor_sync(FULL, mine, 2));
+    kth = fmaxf(mine, __shfl_xor_sync(FULL, mine, 4));
   }
-  const int cnt = __popc(mask);
+
+  // ---- 4. candidates: listed per token (expert ids), then their exact keys
+  //         computed by the token's 8 lanes, entries g, g + 8, ... ----
+  const uint32_t cmask = (maybe && tv) ? proxy_mask<NW>(p2, kth - 2.0f * delta) : 0u;
+  const int cnt = __popc(cmask);
   int incl = cnt;
 #pragma unroll
   for (int off = 1; off < 8; off <<= 1) {
@@ -781,93 +693,132 @@ __device__ void select_quad_fast(const RouteArgs& a, const uint8_t* stage, int l
     if (g >= off) incl += o;
   }
   const int total = __shfl_sync(FULL, incl, seg | 7);
-  const bool slow = tv && (total > kCandMax);
-
-  // ---- fast: exact keys of the candidates, ranked by counting on packed
-  //      (ordered key, ~expert) words: larger key first, then lower expert ----
-  unsigned long long* ck = reinterpret_cast<unsigned long long*>(cand) + q * kCandStride;
-  float* cs = cand + 8 * kCandStride + q * kCandStride;
-  if (tv && !slow) {
-    int pos = incl - cnt;
-    uint32_t m = mask;
-    if (j1 >= 0) m &= ~(1u << j1);
-    if (j2 >= 0) m &= ~(1u << j2);
-    // the lane's top-2 (exact already), then the other candidates 4 per pass
-    if (j1 >= 0 && ((mask >> j1) & 1u)) {
-      ck[pos] = pack_key(K1, slot_expert<V, ESZ>(g, rot, j1));
-      cs[pos++] = S1;
-    }
-    if (j2 >= 0 && ((mask >> j2) & 1u)) {
-      ck[pos] = pack_key(K2, slot_expert<V, ESZ>(g, rot, j2));
-      cs[pos++] = S2;
-    }
-    while (m) {
-      int jb[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        jb[u] = m ? __ffs(m) - 1 : -1;
-        m &= m - 1;
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int e = slot_expert<V, ESZ>(g, rot, max(jb[u], 0));
-        const float sg = (ESZ == 2) ? sigmoid_bf16_row(lut, row, e) : sigmoid_f32(stage_val(a, row, e));
-        if (jb[u] >= 0) {
-          ck[pos] = pack_key(sg + bias_s[e], e);
-          cs[pos++] = sg;
-        }
-      }
-    }
+  const bool slow = tv && (total > kCandSlots || total < a.k);
+  const bool fast = tv && !slow;
+  const int pos0 = incl - cnt;
+  uint16_t* ce = reinterpret_cast<uint16_t*>(cand + 4 * kCandSlots * 12) + q * kCandSlots;
+  if (fast) {
+    uint32_t m = cmask;
+    for (int pos = pos0; m; ++pos, m &= m - 1) ce[pos] = (uint16_t)slot_expert<V, ESZ>(g, rot, mask_bit_slot(__ffs(m) - 1));
   }
   __syncwarp();
-  constexpr int RPL = kCandMax / 8;  // candidates ranked per lane
-  int my_rank[RPL], my_e[RPL];
-  float my_s[RPL];
-  float sel_sum = 0.0f;
+  const int npass = fast ? ((total > 16) ? 2 : 1) : 0;
+  for (int ps = 0; ps < npass; ++ps) {
+    float kx[2], sx[2];
+    int ex[2];
+    bool ok[2];
 #pragma unroll
-  for (int r = 0; r < RPL; ++r) {
-    my_rank[r] = kCandMax;
-    my_e[r] = 0;
-    my_s[r] = 0.0f;
-    const int i = g + 8 * r;
-    if (tv && !slow && i < total) {
-      const unsigned long long ki = ck[i];
-      int rank = 0;
-      for (int jj = 0; jj < total; ++jj) rank += (ck[jj] > ki) ? 1 : 0;
-      my_rank[r] = rank;
-      my_e[r] = packed_expert(ki);
-      my_s[r] = cs[i];
-      if (rank < a.k) sel_sum += my_s[r];
+    for (int u = 0; u < 2; ++u) {
+      const int i = g + 8 * (2 * ps + u);
+      ok[u] = i < total;
+      ex[u] = ok[u] ? ce[i] : 0;
+      sx[u] = sigmoid_f32(stage_val(a, row, ex[u]));
+      kx[u] = sx[u] + bias_s[ex[u]];
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (!ok[u]) continue;
+      const int i = g + 8 * (2 * ps + u);
+      ck[i] = pack_key(kx[u], ex[u]);
+      cs[i] = sx[u];
     }
   }
+  if (fast && g == 0 && (total & 1)) ck[total] = 0ull;  // pads the last pair: ranks below every candidate
+  __syncwarp();
+  // undecided groups: exact scores from their candidates (the lane's own list
+  // entries), ranked among themselves for the slots the surely kept groups
+  // leave; the dropped ones' candidates rank below every other
+  if (__any_sync(FULL, fast && undec)) {
+    float X1 = -INFINITY, X2 = -INFINITY;
+    if (fast && undec)
+      for (int i = pos0; i < pos0 + cnt; ++i) {
+        const uint32_t ok32 = (uint32_t)(ck[i] >> 32);  // ordered key -> fp32 key
+        const float kx = __uint_as_float((ok32 & 0x80000000u) ? (ok32 & 0x7fffffffu) : ~ok32);
+        const float hi = fmaxf(X1, kx);
+        X2 = fmaxf(X2, fminf(X1, kx));
+        X1 = hi;
+      }
+    const unsigned sure_b = (__ballot_sync(FULL, maybe && !undec) >> seg) & 0xffu;
+    const int free_slots = K - __popc(sure_b);
+    const float gx = (a.topn == 1) ? X1 : (X1 + X2);
+    int rx = 0;
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      const float o = __shfl_sync(FULL, gx, seg | h);
+      const bool ou = (__shfl_sync(FULL, undec ? 1 : 0, seg | h) != 0);
+      rx += (ou && (o > gx || (o == gx && h < g))) ? 1 : 0;
+    }
+    __syncwarp();
+    if (fast && undec && rx >= free_slots)
+      for (int i = pos0; i < pos0 + cnt; ++i) ck[i] = 0ull;
+    __syncwarp();
+  }
+
+  // ranks: lane g ranks slots g, g + 8, ... against the token's candidates
+  const int tot2 = (total + 1) & ~1;
+  int rk[4];
+  unsigned long long kk[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int i = g + 8 * r;
+    rk[r] = kCandSlots;
+    kk[r] = 0ull;
+    if (fast && i < total) {
+      kk[r] = ck[i];
+      rk[r] = kk[r] ? 0 : kCandSlots;
+    }
+  }
+  if (fast) {
+    const int nr = (total + 7) >> 3;
+    for (int jj = 0; jj < tot2; jj += 2) {
+      const ulonglong2 o = *reinterpret_cast<const ulonglong2*>(ck + jj);
+      rk[0] += (o.x > kk[0]) + (o.y > kk[0]);
+      rk[1] += (o.x > kk[1]) + (o.y > kk[1]);
+      if (nr > 2) {
+        rk[2] += (o.x > kk[2]) + (o.y > kk[2]);
+        rk[3] += (o.x > kk[3]) + (o.y > kk[3]);
+      }
+    }
+  }
+  float sel_sum = 0.0f;
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+    if (rk[r] < a.k) sel_sum += cs[g + 8 * r];
   sel_sum += __shfl_xor_sync(FULL, sel_sum, 1);
   sel_sum += __shfl_xor_sync(FULL, sel_sum, 2);
   sel_sum += __shfl_xor_sync(FULL, sel_sum, 4);
-  if (tv && !slow) {
 #pragma unroll
-    for (int r = 0; r < RPL; ++r) {
-      if (my_rank[r] < a.k) {
-        const size_t o = (size_t)t * a.k + my_rank[r];
-        const float wv = a.renorm ? (my_s[r] / sel_sum) * a.scale : my_s[r] * a.scale;
-        a.ids[o] = my_e[r];
-        keep_id(ids_s, (int)(t - t_base) * a.k + my_rank[r], my_e[r]);
-        store_from_f32(a.weights, a.weights_dtype, o, wv);
-        atomicAdd(&hist_cta[my_e[r]], 1);
-      }
+  for (int r = 0; r < 4; ++r) {
+    if (rk[r] < a.k) {
+      const size_t o = (size_t)t * a.k + rk[r];
+      const int e = packed_expert(kk[r]);
+      const float sv = cs[g + 8 * r];
+      a.ids[o] = e;
+      store_from_f32(a.weights, a.weights_dtype, o, a.renorm ? (sv / sel_sum) * a.scale : sv * a.scale);
+      mark(a, masks, ids_s, lt, rk[r], e);
     }
   }
-  __syncwarp();
 
-  // ---- slow: exact keys for every expert of the token (rare) ----
-  const unsigned smask = __ballot_sync(FULL, slow);
-  if (slow) select_token_exact8<V, ESZ>(a, row, t, g, rot, seg, smask, bias_s, hist_cta, ids_s, t_base);
-  __syncwarp();
+  // ---- tokens left to the exact path ----
+  const unsigned sb = __ballot_sync(FULL, slow && g == 0);
+  return (sb & 1u) | ((sb >> 7) & 2u) | ((sb >> 14) & 4u) | ((sb >> 21) & 8u);
+}
+
+// The exact path for one token (warp per token, E / 32 experts per lane), its
+// row read from global memory; kept out of line so that its code and registers
+// stay away from the fast path.
+template <int VPL>
+__device__ __noinline__ void select_token_warp_exact(const RouteArgs& a, const uint8_t* lg_bytes, int t_begin,
+                                                     int lt, const float* bias_s, uint32_t* masks, uint16_t* ids_s,
+                                                     int lane) {
+  select_token_warp<VPL>(a, lg_bytes + ((size_t)t_begin + lt) * a.row_bytes, t_begin + lt, lt, bias_s, masks, ids_s,
+                         lane);
 }
 
 // Exclusive scan of padded counts into offs[0..E] (E <= 1024) by warp 0: lane
 // l takes a run of consecutive experts, then one shuffle scan over the lanes.
 // Ends with a block barrier.
-__device__ void scan_padded_offsets(const int* cnt, int* offs, int E, int tile, int* /*scratch*/) {
+__device__ void scan_padded_offsets(const int* cnt, int* offs, int E, int tile) {
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
     const int per = (E + 31) >> 5;
@@ -897,353 +848,273 @@ __device__ void scan_padded_offsets(const int* cnt, int* offs, int E, int tile, 
   __syncthreads();
 }
 
+// After a block's selections: park (expert, rank in the segment) of every
+// selection in expanded_to_permuted, and write the segment's counts row.
+__device__ void finish_segment(const RouteArgs& a, const uint32_t* masks, const uint16_t* ids_s, int n, int t_begin) {
+  const int n_items = n * a.k;
+  const long long i_begin = (long long)t_begin * a.k;
+  for (int i = threadIdx.x; i < n_items; i += blockDim.x) {
+    const int e = ids_s[i];
+    // token of item i: i / k (i < 2^13, so the multiply-high is exact)
+    const int lt = a.k == 1 ? i : (int)__umulhi((uint32_t)i, a.kinv);
+    const uint32_t* m = masks + min(e, a.E - 1) * a.MW;  // ids were range-checked when selected
+    int r = __popc(m[lt >> 5] & ((1u << (lt & 31)) - 1u));
+    for (int w = 0; w < (lt >> 5); ++w) r += __popc(m[w]);
+    a.e2p[i_begin + i] = e < a.E ? (e | (r << 16)) : -1;
+  }
+  uint8_t* trow = a.table + (size_t)blockIdx.x * a.row_stride;
+  uint32_t* grow = a.gtot + (size_t)(blockIdx.x / a.GS) * a.E;
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+    int c = 0;
+    for (int w = 0; w < a.MW; ++w) c += __popc(masks[e * a.MW + w]);
+    if (a.cnt_bytes == 1) trow[e] = (uint8_t)c;
+    else reinterpret_cast<uint16_t*>(trow)[e] = (uint16_t)c;
+    if (c) atomicAdd(&grow[e], (uint32_t)c);  // integer adds: order-free, deterministic
+  }
+}
+
+// bounded wait on a staging barrier; false (recorded) if it gave up
+__device__ __forceinline__ bool stage_wait(const RouteArgs& a, uint64_t* bar, uint32_t parity) {
+  if (mbar_wait_bounded(bar, parity, a.timeout_ns)) return true;
+  record_timeout(a.hdr);
+  return false;
+}
+
 // VPL: experts per lane (0 = a thread per token).  FAST_ESZ: 0 = generic exact
 // path; 2 or 4 = sigmoid fast path with V = VPL and that logits element size.
 template <int VPL, int FAST_ESZ>
-__global__ void __launch_bounds__((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneric, 1) route_kernel(RouteArgs a) {
-  constexpr int kWarps = ((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneric) / 32;
+__global__ void __launch_bounds__((FAST_ESZ > 0) ? kFastWarpsMax * 32 : kGenericThreads, 1)
+    route_select_kernel(RouteArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
+  constexpr bool kFast = FAST_ESZ > 0;
+  constexpr int FV = kFast ? VPL : 1;
   const int E = a.E;
   const int c = blockIdx.x;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  // contiguous token range of this block
-  const int base_n = a.T / a.G, rem = a.T % a.G;
-  const int t_begin = c * base_n + min(c, rem);
-  const int t_end = t_begin + base_n + (c < rem ? 1 : 0);
-  const int n_items = (t_end - t_begin) * a.k;
-  const RouteSmem L = route_smem_layout(E, a.stage_bytes, a.ids_in_smem ? n_items * 2 : 0, kWarps,
-                                       FAST_ESZ == 2 ? kLutEntries * 4 : 0);
-  uint8_t* stage = smem + L.stage;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int t_begin = c * a.B;
+  const int n = max(0, min(a.T, t_begin + a.B) - t_begin);
+  const SelSmem L = sel_smem_layout(E, a.MW, a.B, a.k, kFast ? 1 : 0, FV, a.row_bytes, nwarps);
+  uint32_t* masks = reinterpret_cast<uint32_t*>(smem + L.masks);
+  uint16_t* ids_s = reinterpret_cast<uint16_t*>(smem + L.ids);
   float* bias_s = reinterpret_cast<float*>(smem + L.bias);
-  int* hist_cta = reinterpret_cast<int*>(smem + L.hist_cta);
-  int* hist_w = reinterpret_cast<int*>(smem + L.hist_w);
-  int* offs = reinterpret_cast<int*>(smem + L.offs);
-  int* cnt = reinterpret_cast<int*>(smem + L.cnt);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L.bar);
-  int* flag = reinterpret_cast<int*>(smem + L.flag);
-  int* scan_scratch = reinterpret_cast<int*>(smem + L.scan);
-  uint16_t* ids_s = a.ids_in_smem ? reinterpret_cast<uint16_t*>(smem + L.ids) : nullptr;
-  uint16_t* lrank_s = a.ids_in_smem ? reinterpret_cast<uint16_t*>(smem + L.lrank) : nullptr;
+  uint8_t* cb_s = smem + L.cb;
+  float* delta_s = reinterpret_cast<float*>(smem + L.delta);
+  uint8_t* wbase = smem + L.warp0 + (size_t)warp * L.warp_bytes;
+  uint8_t* cand = wbase + 2 * L.stage_bytes;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(wbase + 2 * L.stage_bytes + kCandBytes);
 
-  // Programmatic dependent launch: the next grid in the stream may be scheduled
-  // at once (its blocks start as this grid's blocks retire), and this grid
-  // touches no global memory before the previous one has completed and its
-  // writes are visible.  Without the launch attribute both are no-ops.
+  // Programmatic dependent launch: the bookkeeping kernel may be scheduled at
+  // once.  Before waiting on the previous grid, only the bias is read (a
+  // preceding kernel that lets its dependents start early must not write it);
+  // the logits are read after the wait.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  // bf16 fast path: the exact-sigmoid table needs no global memory, so all
-  // threads but thread 0 (which waits first and starts the logits copies)
-  // fill it before waiting
-  float* lut = nullptr;
-  if constexpr (FAST_ESZ == 2) {
-    lut = reinterpret_cast<float*>(smem + L.lut);
-    if (threadIdx.x > 0)
-      for (int i = threadIdx.x - 1; i < kLutEntries; i += blockDim.x - 1)
-        lut[i] = sigmoid_f32(bf16_bits_to_f32((uint16_t)lut_bits(i)));
+  for (int i = threadIdx.x; i < E * a.MW; i += blockDim.x) masks[i] = 0u;
+  const int nq = (n + 3) >> 2;
+  if constexpr (kFast) {
+    if (lane == 0) {
+      mbar_init(&bar[0], 1);
+      mbar_init(&bar[1], 1);
+    }
+    __syncwarp();
   }
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-
-  const uint32_t gen = barrier_generation(a.hdr);
-
-  // the first round's logits start streaming before anything else: thread 0
-  // initialises the mbarriers and issues the bulk copies itself
-  const int n0 = min(a.chunk_tokens, t_end - t_begin);
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kMaxSub; ++s) mbar_init(&bar[s], 1);
-    flag[1] = 0;  // set when a staging wait gave up
-  }
-  int nsub = (n0 > 0) ? stage_issue(a, stage, bar, t_begin, n0) : 0;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
     bias_s[e] = a.has_bias ? load_as_f32(a.bias, a.bias_dtype, e) : 0.0f;
-    hist_cta[e] = 0;
-  }
   __syncthreads();
-
-  // fast path: per-lane constants 0.5 + bias, in register-slot order
-  constexpr int FV = (FAST_ESZ > 0) ? VPL : 1;
-  float* cb_s = reinterpret_cast<float*>(smem + L.cand + kWarps * cand_bytes_per_warp());
-  if constexpr (FAST_ESZ > 0) {
+  float delta = 0.0f;
+  if constexpr (kFast) {
+    // per-lane constants 0.5 + bias in f16, in register-slot order; warp 0
+    // also derives the block's proxy error bound from their largest magnitude
     for (int idx = threadIdx.x; idx < 8 * FV; idx += blockDim.x) {
       const int g = idx / FV, j = idx % FV;
       const int rot = (g * (FV / (16 / FAST_ESZ))) >> 3;
-      cb_s[g * cb_stride<FV>() + j] = 0.5f + bias_s[slot_expert<FV, FAST_ESZ>(g, rot, j)];
+      reinterpret_cast<__half*>(cb_s + g * cb_stride_bytes<FV>())[j] =
+          __float2half_rn(0.5f + bias_s[slot_expert<FV, FAST_ESZ>(g, rot, j)]);
+    }
+    if (warp == 0) {
+      float cbmax = 0.0f;
+      for (int e = lane; e < E; e += 32) cbmax = fmaxf(cbmax, fabsf(0.5f + bias_s[e]));
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) cbmax = fmaxf(cbmax, __shfl_xor_sync(0xffffffffu, cbmax, off));
+      if (lane == 0) *delta_s = proxy_delta(cbmax, FAST_ESZ == 4);
     }
     __syncthreads();
+    delta = *delta_s;
   }
-  float* cand = reinterpret_cast<float*>(smem + L.cand + warp * cand_bytes_per_warp());
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  // ---------------- phase 1: select ----------------
-  uint32_t round = 0;
-  for (int t0 = t_begin; t0 < t_end; t0 += a.chunk_tokens, ++round) {
-    const int n = min(a.chunk_tokens, t_end - t0);
-    if (round > 0) nsub = stage_issue(a, stage, bar, t0, n);
-    const uint32_t parity = round & 1u;
-    if constexpr (FAST_ESZ > 0) {
-      const int nquads = (n + 3) >> 2;
-      for (int qd = warp; qd < nquads; qd += kWarps) {
-        if (nsub > 0) {
-          const int s0 = sub_of(qd * 4, n, nsub), s1 = sub_of(min(qd * 4 + 3, n - 1), n, nsub);
-          for (int sb = s0; sb <= s1; ++sb)
-            if (!stage_wait(a, bar, sb, parity)) flag[1] = 1;
+  // fast path: this warp's first two quads start streaming into its slots
+  const uint8_t* lg_bytes = reinterpret_cast<const uint8_t*>(a.logits);
+  if constexpr (kFast) {
+    if (lane == 0) {
+      for (int s = 0; s < 2; ++s) {
+        const int qd = warp + s * nwarps;
+        if (qd < nq) {
+          const uint32_t bytes = (uint32_t)min(4, n - qd * 4) * (uint32_t)a.row_bytes;
+          mbar_arrive_expect_tx(&bar[s], bytes);
+          bulk_g2s(wbase + s * L.stage_bytes, lg_bytes + ((size_t)t_begin + qd * 4) * a.row_bytes, bytes, &bar[s]);
         }
-        select_quad_fast<FV, FAST_ESZ>(a, stage, qd * 4, n, t0, cb_s, bias_s, cand, hist_cta, lane, ids_s, t_begin,
-                                       lut);
-      }
-    } else {
-      for (int sb = 0; sb < nsub; ++sb)
-        if (!stage_wait(a, bar, sb, parity)) flag[1] = 1;
-      if constexpr (VPL == 0) {
-        for (int lt = threadIdx.x; lt < n; lt += blockDim.x) {
-          const uint8_t* row = stage + (size_t)lt * a.row_bytes;
-          if (E <= 8)
-            select_token_thread<8>(a, row, t0 + lt, bias_s, hist_cta, ids_s, t_begin);
-          else if (E <= 16)
-            select_token_thread<16>(a, row, t0 + lt, bias_s, hist_cta, ids_s, t_begin);
-          else
-            select_token_thread<32>(a, row, t0 + lt, bias_s, hist_cta, ids_s, t_begin);
-        }
-      } else {
-        for (int lt = warp; lt < n; lt += kWarps)
-          select_token_warp<VPL>(a, stage + (size_t)lt * a.row_bytes, t0 + lt, bias_s, hist_cta, lane, ids_s,
-                                 t_begin);
       }
     }
-    __syncthreads();
   }
-  const bool staged_ok = flag[1] == 0;
 
-  // ---------------- publish + barrier ----------------
-  uint8_t* trow = reinterpret_cast<uint8_t*>(a.table) + (size_t)c * a.row_stride;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    const int h = hist_cta[e];
-    if (a.cnt_bytes == 1) trow[e] = (uint8_t)h;
-    else if (a.cnt_bytes == 2) reinterpret_cast<uint16_t*>(trow)[e] = (uint16_t)h;
-    else reinterpret_cast<uint32_t*>(trow)[e] = (uint32_t)h;
+  if constexpr (kFast) {
+    uint16_t* pend = reinterpret_cast<uint16_t*>(cand + kCandBytes - 2 * kPendMax - 8);
+    int npend = 0;
+    bool ok = true;
+    int r = 0;
+    for (int qd = warp; qd < nq; qd += nwarps, ++r) {
+      const int s = r & 1;
+      if (!stage_wait(a, &bar[s], (uint32_t)(r >> 1) & 1u)) {
+        ok = false;
+        break;
+      }
+      const uint8_t* slot = wbase + s * L.stage_bytes;
+      const unsigned sq = select_quad_fast<FV, FAST_ESZ>(a, slot, qd * 4, min(4, n - qd * 4), t_begin, cb_s, bias_s,
+                                                         delta, cand, masks, ids_s, lane);
+      // the quad's tokens left to the exact path (rare) wait for the end of the loop
+      for (unsigned m = sq; m; m &= m - 1) {
+        if (lane == 0 && npend < kPendMax) pend[npend] = (uint16_t)(qd * 4 + __ffs(m) - 1);
+        ++npend;
+      }
+      __syncwarp();
+      const int nx = qd + 2 * nwarps;
+      if (lane == 0 && nx < nq) {
+        // this slot's rows were read through the generic proxy: order those
+        // reads before the bulk copy's writes
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        const uint32_t bytes = (uint32_t)min(4, n - nx * 4) * (uint32_t)a.row_bytes;
+        mbar_arrive_expect_tx(&bar[s], bytes);
+        bulk_g2s(wbase + s * L.stage_bytes, lg_bytes + ((size_t)t_begin + nx * 4) * a.row_bytes, bytes, &bar[s]);
+      }
+    }
+    if (!ok) {
+      // a staging wait gave up (recorded; outputs undefined): let the copies
+      // still in flight (rounds r and r + 1) land before the block exits
+      for (int rr = r; rr < r + 2 && warp + rr * nwarps < nq; ++rr)
+        mbar_wait_bounded(&bar[rr & 1], (uint32_t)(rr >> 1) & 1u, a.timeout_ns);
+    }
+    // this warp's tokens left to the exact path
+    __syncwarp();
+    if (npend > kPendMax && lane == 0) record_bounds(a.hdr);  // cannot happen: see kPendMax
+    for (int i = 0; i < min(npend, kPendMax); ++i)
+      select_token_warp_exact<FV / 4>(a, lg_bytes, t_begin, pend[i], bias_s, masks, ids_s, lane);
+    } else if constexpr (VPL == 0) {
+    for (int lt = threadIdx.x; lt < n; lt += blockDim.x) {
+      const uint8_t* row = lg_bytes + ((size_t)t_begin + lt) * a.row_bytes;
+      if (E <= 8)
+        select_token_thread<8>(a, row, t_begin + lt, lt, bias_s, masks, ids_s);
+      else if (E <= 16)
+        select_token_thread<16>(a, row, t_begin + lt, lt, bias_s, masks, ids_s);
+      else
+        select_token_thread<32>(a, row, t_begin + lt, lt, bias_s, masks, ids_s);
+    }
+  } else {
+    for (int lt = warp; lt < n; lt += nwarps)
+      select_token_warp<VPL>(a, lg_bytes + ((size_t)t_begin + lt) * a.row_bytes, t_begin + lt, lt, bias_s, masks,
+                             ids_s, lane);
   }
   __syncthreads();
-  if (threadIdx.x == 0) grid_arrive(a.hdr, (uint32_t)a.G);
+  finish_segment(a, masks, ids_s, n, t_begin);
+}
 
-  // ---- while the other blocks finish: each selection's rank among this
-  //      block's selections of the same expert, in item order (per-warp counts
-  //      over a contiguous split of the items, their exclusive prefix over
-  //      warps, then a walk that ranks equal experts inside each 32-item chunk)
+// ---------------------------------------------------------------------------
+// bookkeeping kernel
+// ---------------------------------------------------------------------------
+__host__ __device__ inline int perm_smem_bytes(int E) { return (3 * E + 1) * 4 + 16; }
+
+__global__ void __launch_bounds__(kPermThreads, 1) route_permute_kernel(RouteArgs a) {
+  extern __shared__ __align__(128) uint8_t psmem[];
+  const int E = a.E;
+  int* cnt = reinterpret_cast<int*>(psmem);
+  int* base = cnt + E;
+  int* offs = base + E;  // [E + 1], then one flag word
+  const int c = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t_begin = c * a.B;
+  const int n = max(0, min(a.T, t_begin + a.B) - t_begin);
+  const int n_items = n * a.k;
   const long long i_begin = (long long)t_begin * a.k;
-  const int w_begin = (int)((long long)n_items * warp / kWarps);
-  const int w_end = (int)((long long)n_items * (warp + 1) / kWarps);
-  if (lrank_s) {
-    for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) hist_w[i] = 0;
-    __syncthreads();
-    for (int i = w_begin + lane; i < w_end; i += 32) {
-      const int e = ids_s[i];
-      if (e < E) atomicAdd(&hist_w[warp * E + e], 1);
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-      int h[kWarps];
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) h[w] = hist_w[w * E + e];
-      int run = 0;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        hist_w[w * E + e] = run;
-        run += h[w];
-      }
-    }
-    __syncthreads();
-    for (int i0 = w_begin; i0 < w_end; i0 += 32) {
-      // rank inside the 32-item chunk = earlier lanes holding the same expert
-      // (inactive lanes hold distinct negative values); the chunk's last item of
-      // each expert then raises the running count
-      const int i = i0 + lane;
-      const bool act = i < w_end;
-      const int e = act ? min((int)ids_s[i], E - 1) : -1 - lane;  // ids were range-checked when selected
-      int rank = 0;
-#pragma unroll
-      for (int d = 1; d < 32; ++d) {
-        const int o = __shfl_up_sync(0xffffffffu, e, d);
-        rank += (lane >= d && o == e) ? 1 : 0;
-      }
-      int slot = 0;
-      if (act) {
-        slot = hist_w[warp * E + e] + rank;
-        lrank_s[i] = (uint16_t)slot;
-      }
-      __syncwarp();
-      if (act) atomicMax(&hist_w[warp * E + e], slot + 1);
-      __syncwarp();
-    }
-  }
-  if (threadIdx.x == 0) flag[0] = grid_wait(a.hdr, (uint32_t)a.G, gen, a.timeout_ns) ? 1 : 0;
-  __syncthreads();
-  if (!flag[0]) return;
-  if (!staged_ok) return;  // a staging wait gave up (recorded); outputs undefined
 
-  // ---------------- phase 2: totals and block base from the table ----------------
-  // Every block reads every row of the table: the sum of all rows gives the
-  // expert counts, the sum of the rows of earlier blocks this block's base.
-  // Thread (row group rg, word w) reads 32-bit word w of rows rg, rg + R, ...
-  // (a warp reads consecutive words: coalesced), all loads in flight, and
-  // keeps per-entry sums; the partial sums go to shared memory word-major so
-  // the stores and the reduction reads hit distinct banks.  Integer sums in a
-  // fixed order: deterministic, no atomics.
-  int P = 0;
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the table and the parked ranks are the selection's output
+
+  // this block's first parked selections, loaded while the table is summed
+  constexpr int kPre = 2;
+  int pre[kPre];
+#pragma unroll
+  for (int u = 0; u < kPre; ++u) {
+    const int i = threadIdx.x + u * kPermThreads;
+    pre[u] = i < n_items ? __ldcg(a.e2p + i_begin + i) : 0;
+  }
+
+  // ---- per expert e (a thread each): cnt[e] = all selections of e (local
+  //      experts; others zero width) = the sum of the group totals; base[e] =
+  //      the selections of e by earlier segments = the groups before this
+  //      segment's group plus this group's segments before this one.  Integer
+  //      sums in a fixed order, 8 loads in flight. ----
   {
-    const int WPR = a.row_stride >> 2;                     // 32-bit words per row
-    const int EPW = 4 / a.cnt_bytes;                       // entries per word
-    const int R = max(1, min((int)blockDim.x / WPR, a.G));  // row groups
-    const int rg = threadIdx.x / WPR, w = threadIdx.x % WPR;
-    int tot[4] = {0, 0, 0, 0}, pre[4] = {0, 0, 0, 0};
-    const bool wide = a.cnt_bytes == 1 && (a.row_stride >> 4) * 16 <= (int)blockDim.x;
-    if (wide) {
-      // byte entries, 16-byte loads: thread (row group rg4 < 16, 16-byte column w4)
-      // reads rows rg4, rg4 + 16, ... (all loads in flight) and keeps two 16-bit
-      // lanes per 32-bit accumulator (a row group's sums stay below 65536)
-      const int W4 = a.row_stride >> 4;
-      const int R4 = min(16, a.G);
-      const int rg4 = threadIdx.x / W4, w4 = threadIdx.x % W4;
-      uint32_t* part_w = reinterpret_cast<uint32_t*>(stage);  // [2][R4][8][W4 + 1] packed pairs
-      const int pstride = W4 + 1;
-      if (rg4 < R4) {
-        uint32_t acc_t[8] = {0, 0, 0, 0, 0, 0, 0, 0}, acc_p[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        constexpr int kB4 = 10;
-        for (int cp0 = rg4; cp0 < a.G; cp0 += R4 * kB4) {
-          uint4 v[kB4];
+    const int grp = c / a.GS, r0 = grp * a.GS;
+    for (int e = threadIdx.x; e < E; e += kPermThreads) {
+      uint32_t tot = 0, pre_e = 0;
+      for (int g0 = 0; g0 < a.NG; g0 += 8) {
+        uint32_t v[8];
 #pragma unroll
-          for (int b = 0; b < kB4; ++b) {
-            const int cp = cp0 + b * R4;
-            v[b] = cp < a.G ? __ldcg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(a.table) +
-                                                                     (size_t)cp * a.row_stride) + w4)
-                            : make_uint4(0, 0, 0, 0);
-          }
-#pragma unroll
-          for (int b = 0; b < kB4; ++b) {
-            const bool before = cp0 + b * R4 < c;
-            const uint32_t vw[4] = {v[b].x, v[b].y, v[b].z, v[b].w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint32_t e02 = vw[j] & 0x00ff00ffu, e13 = (vw[j] >> 8) & 0x00ff00ffu;
-              acc_t[2 * j] += e02;
-              acc_t[2 * j + 1] += e13;
-              if (before) {
-                acc_p[2 * j] += e02;
-                acc_p[2 * j + 1] += e13;
-              }
-            }
-          }
-        }
+        for (int j = 0; j < 8; ++j) v[j] = g0 + j < a.NG ? __ldcg(a.gtot + (size_t)(g0 + j) * E + e) : 0u;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          part_w[(rg4 * 8 + j) * pstride + w4] = acc_t[j];
-          part_w[((R4 + rg4) * 8 + j) * pstride + w4] = acc_p[j];
+          tot += v[j];
+          pre_e += g0 + j < grp ? v[j] : 0u;
         }
       }
-      __syncthreads();
-      // entry e = 16*w4 + 4*j + lo/hi*2 + odd: accumulator 2*j + odd, 16-bit lane lo/hi
-      for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        const int ww = e >> 4, within = e & 15;
-        const int acc = (within >> 2) * 2 + (within & 1), sh = (within & 2) ? 16 : 0;
-        int st = 0, sp = 0;
-        for (int r = 0; r < R4; ++r) {
-          st += (int)((part_w[(r * 8 + acc) * pstride + ww] >> sh) & 0xffffu);
-          sp += (int)((part_w[((R4 + r) * 8 + acc) * pstride + ww] >> sh) & 0xffffu);
+      for (int rb = r0; rb < c; rb += 8) {
+        uint32_t v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int r = rb + j;
+          const uint8_t* trow = a.table + (size_t)r * a.row_stride;
+          v[j] = r < c ? (a.cnt_bytes == 1 ? (uint32_t)__ldcg(trow + e)
+                                           : (uint32_t)__ldcg(reinterpret_cast<const uint16_t*>(trow) + e))
+                       : 0u;
         }
-        cnt[e] = is_local(a, e) ? st : 0;  // another shard's expert: zero width
-        hist_cta[e] = sp;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) pre_e += v[j];
       }
-    } else if (rg < R) {
-      constexpr int kBatch = 20;
-      for (int cp0 = rg; cp0 < a.G; cp0 += R * kBatch) {
-        uint32_t v[kBatch];
-#pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-          const int cp = cp0 + b * R;
-          v[b] = cp < a.G ? __ldcg(reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint8_t*>(a.table) +
-                                                                     (size_t)cp * a.row_stride) + w)
-                          : 0u;
-        }
-        if (a.cnt_bytes == 1) {
-          // byte entries: two 16-bit lanes per 32-bit add (entries 0,2 and
-          // 1,3); totals stay below 65536 because a block holds <= 255 tokens
-          uint32_t t02 = 0, t13 = 0, p02 = 0, p13 = 0;
-#pragma unroll
-          for (int b = 0; b < kBatch; ++b) {
-            const uint32_t e02 = v[b] & 0x00ff00ffu, e13 = (v[b] >> 8) & 0x00ff00ffu;
-            t02 += e02;
-            t13 += e13;
-            if (cp0 + b * R < c) {
-              p02 += e02;
-              p13 += e13;
-            }
-          }
-          tot[0] += (int)(t02 & 0xffffu); tot[2] += (int)(t02 >> 16);
-          tot[1] += (int)(t13 & 0xffffu); tot[3] += (int)(t13 >> 16);
-          pre[0] += (int)(p02 & 0xffffu); pre[2] += (int)(p02 >> 16);
-          pre[1] += (int)(p13 & 0xffffu); pre[3] += (int)(p13 >> 16);
-        } else {
-#pragma unroll
-          for (int b = 0; b < kBatch; ++b) {
-            const bool before = cp0 + b * R < c;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              if (i < EPW) {
-                const int x = a.cnt_bytes == 2 ? (int)((v[b] >> (16 * i)) & 0xffffu) : (int)v[b];
-                tot[i] += x;
-                pre[i] += before ? x : 0;
-              }
-            }
-          }
-        }
-      }
-    }
-    int* part_t = reinterpret_cast<int*>(stage);   // [R][EPW][WPR]
-    int* part_p = part_t + R * EPW * WPR;          // [R][EPW][WPR]
-    if (!wide && rg < R) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (i < EPW) {
-          part_t[(rg * EPW + i) * WPR + w] = tot[i];
-          part_p[(rg * EPW + i) * WPR + w] = pre[i];
-        }
+      cnt[e] = is_local(a, e) ? (int)tot : 0;  // another shard's expert: zero width
+      base[e] = (int)pre_e;
     }
     __syncthreads();
-    for (int x = threadIdx.x; !wide && x < EPW * WPR; x += blockDim.x) {
-      const int i = x / WPR, ww = x % WPR;
-      const int e = ww * EPW + i;
-      if (e < E) {
-        int st = 0, sp = 0;
-        for (int r = 0; r < R; ++r) {
-          st += part_t[(r * EPW + i) * WPR + ww];
-          sp += part_p[(r * EPW + i) * WPR + ww];
-        }
-        cnt[e] = is_local(a, e) ? st : 0;  // another shard's expert: zero width
-        hist_cta[e] = sp;
-      }
-    }
-    if (!lrank_s)
-      for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) hist_w[i] = 0;
+    // the last block to have read the group totals clears them for the next call
+    if (threadIdx.x == 0) base[E + E + 1] = (atomicAdd(&a.hdr->ticket, 1u) == (unsigned)a.G - 1) ? 1 : 0;
     __syncthreads();
-    scan_padded_offsets(cnt, offs, E, a.tile, scan_scratch);
-    P = offs[E];
-    if (c == 0) {
-      // the shard's experts (those before it have no rows: offs[loc_off] == 0)
-      for (int le = threadIdx.x; le < a.loc_n; le += blockDim.x) {
-        a.counts[le] = cnt[a.loc_off + le];
-        a.offsets[le] = offs[a.loc_off + le];
-      }
-      if (threadIdx.x == 0) {
-        a.offsets[a.loc_n] = P;
-        a.totals[0] = P;
-        a.totals[1] = P / a.tile;
-      }
+    if (base[E + E + 1]) {
+      for (int i = threadIdx.x; i < a.NG * E; i += kPermThreads) a.gtot[i] = 0u;
+      if (threadIdx.x == 0) a.hdr->ticket = 0u;
     }
   }
-  const int ntiles = P / a.tile;
+  scan_padded_offsets(cnt, offs, E, a.tile);
+  const int P = offs[E];
+  if (c == 0) {
+    // the shard's experts (those before it have no rows: offs[loc_off] == 0)
+    for (int le = threadIdx.x; le < a.loc_n; le += blockDim.x) {
+      a.counts[le] = cnt[a.loc_off + le];
+      a.offsets[le] = offs[a.loc_off + le];
+    }
+    if (threadIdx.x == 0) {
+      a.offsets[a.loc_n] = P;
+      a.totals[0] = P;
+      a.totals[1] = P / a.tile;
+    }
+  }
 
-  // ---------------- phase 2: slots in token order ----------------
-  if (lrank_s) {
-    // slot = expert offset + earlier blocks' selections of the expert + local rank
-    for (int i = threadIdx.x; i < n_items; i += blockDim.x) {
-      const int e = ids_s[i];
-      if (e >= E) {
+  // ---- slots in token order: offset + earlier segments' rows + rank ----
+  for (int i0 = 0; i0 < n_items; i0 += kPre * kPermThreads) {
+#pragma unroll
+    for (int u = 0; u < kPre; ++u) {
+      const int i = i0 + threadIdx.x + u * kPermThreads;
+      if (i >= n_items) continue;
+      const int v = (i0 == 0) ? pre[u] : __ldcg(a.e2p + i_begin + i);
+      const int e = v & 0xffff, rk = v >> 16;
+      if (v < 0 || e >= E) {
         record_bounds(a.hdr);
         continue;
       }
@@ -1251,79 +1122,31 @@ __global__ void __launch_bounds__((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneri
         a.e2p[i_begin + i] = -1;
         continue;
       }
-      const int slot = offs[e] + hist_cta[e] + lrank_s[i];
+      const int slot = offs[e] + base[e] + rk;
       a.e2p[i_begin + i] = slot;
-      // token of item i: t_begin + i / k (i < 2^16, so the multiply-high is exact)
+      // token of item i: t_begin + i / k
       const int lt = a.k == 1 ? i : (int)__umulhi((uint32_t)i, a.kinv);
       if ((unsigned)slot < (unsigned)a.max_padded) a.p2t[slot] = t_begin + lt;
       else record_bounds(a.hdr);
     }
-  } else {
-    // per-warp counts over a contiguous split of the block's selections, their
-    // exclusive prefix over warps, then a walk that ranks equal experts inside
-    // each 32-item chunk (match + popcount)
-    for (int i = w_begin + lane; i < w_end; i += 32) {
-      const int e = ids_s ? (int)ids_s[i] : a.ids[i_begin + i];
-      if ((unsigned)e < (unsigned)E) atomicAdd(&hist_w[warp * E + e], 1); else record_bounds(a.hdr);
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-      int run = offs[e] + hist_cta[e];
-      for (int w = 0; w < kWarps; ++w) {
-        const int h = hist_w[w * E + e];
-        hist_w[w * E + e] = run;
-        run += h;
-      }
-    }
-    __syncthreads();
-    for (int i0 = w_begin; i0 < w_end; i0 += 32) {
-      const int i = i0 + lane;
-      const bool act = i < w_end;
-      const unsigned amask = __ballot_sync(0xffffffffu, act);
-      if (act) {
-        int e = ids_s ? (int)ids_s[i] : a.ids[i_begin + i];
-        if ((unsigned)e >= (unsigned)E) {
-          record_bounds(a.hdr);
-          e = 0;
-        }
-        const unsigned m = __match_any_sync(amask, e);
-        const int rank = __popc(m & ((1u << lane) - 1u));
-        const int leader = __ffs(m) - 1;
-        const int slot = hist_w[warp * E + e] + rank;
-        __syncwarp(amask);
-        if (lane == leader) hist_w[warp * E + e] += __popc(m);
-        if (is_local(a, e)) {
-          a.e2p[i_begin + i] = slot;
-          if ((unsigned)slot < (unsigned)a.max_padded) a.p2t[slot] = (int)((i_begin + i) / a.k); else record_bounds(a.hdr);
-        } else {
-          a.e2p[i_begin + i] = -1;  // another shard's expert: no slot
-        }
-      }
-      __syncwarp();
-    }
   }
 
-  // ---------------- tile tables and padding rows (a warp per tile) ----------------
-  if (ntiles > a.max_tiles || P > a.max_padded) {
+  // ---- tile tables and padding rows: a warp per expert (experts spread over
+  //      all warps of the grid); the expert's tiles are [offs[e], offs[e+1]) / tile
+  //      and its padding rows follow its count ----
+  if (P / a.tile > a.max_tiles || P > a.max_padded) {
     if (threadIdx.x == 0) record_bounds(a.hdr);
     return;
   }
-  const int tc0 = (int)((long long)ntiles * c / a.G), tc1 = (int)((long long)ntiles * (c + 1) / a.G);
-  for (int tc = tc0 + warp; tc < tc1; tc += kWarps) {
-    const int row = tc * a.tile;
-    int lo = 0, hi = E - 1;  // largest e with offs[e] <= row
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (offs[mid] <= row) lo = mid; else hi = mid - 1;
+  const int nwarps = blockDim.x >> 5;
+  for (int e = c * nwarps + warp; e < E; e += a.G * nwarps) {
+    const int row0 = offs[e], row1 = offs[e + 1], lim = row0 + cnt[e];
+    for (int tc = row0 / a.tile + lane; tc < row1 / a.tile; tc += 32) {
+      a.tile_expert[tc] = e - a.loc_off;  // the local expert (batch index)
+      a.tile_mn[tc] = min((tc + 1) * a.tile, lim);
     }
-    const int lim = min(row + a.tile, offs[lo] + cnt[lo]);
-    if (lane == 0) {
-      a.tile_expert[tc] = lo - a.loc_off;  // the local expert (batch index)
-      a.tile_mn[tc] = lim;
-    }
-    for (int r = lim + lane; r < row + a.tile; r += 32) a.p2t[r] = -1;
+    for (int r = lim + lane; r < row1; r += 32) a.p2t[r] = -1;
   }
-
 }
 
 // ---------------------------------------------------------------------------
@@ -1402,65 +1225,64 @@ int pick_mode(const moe_route_params* p) {
   return -1;
 }
 
-int grid_for(const moe_route_params* p, const DevInfo& d) {
-  const int T = p->num_tokens;
-  int g = (T + 63) / 64;
-  g = std::max(1, std::min(g, d.sms));
-  return g;
+// Segments: about one per SM (at least 32 tokens each, at most kMaxSegment).
+void plan_segments(int T, int sms, int* G, int* B) {
+  if (T <= 0) {
+    *G = 1;
+    *B = 1;
+    return;
+  }
+  const int g = std::max(1, std::min(sms, (T + 31) / 32));
+  const int b = std::min(kMaxSegment, (T + g - 1) / g);
+  *G = (T + b - 1) / b;
+  *B = b;
 }
 
-// workspace: header | table [G][row] (256-byte aligned, rows sized for the
-// widest 4-byte entries; read as 32-bit words)
-size_t table_offset(int) { return 256; }
+// workspace: header | group totals [16][MOE_MAX_EXPERTS] u32 (at a fixed place
+// and size: every call leaves the part it used zero, whatever its shape) |
+// table [G][row] (rows of 1- or 2-byte entries, 16-byte multiples)
+constexpr size_t kHeaderBytes = 256;
+constexpr int kMaxGroups = 16;
+constexpr size_t kTableOffset = kHeaderBytes + (size_t)kMaxGroups * MOE_MAX_EXPERTS * 4;
 
-size_t ws_bytes_for(int E, int G) {
-  const size_t row = ((size_t)E * 4 + 15) & ~(size_t)15;
-  return table_offset(E) + (size_t)G * row;
+size_t table_row_stride(int E, int cnt_bytes) { return ((size_t)E * cnt_bytes + 15) & ~(size_t)15; }
+
+size_t ws_bytes_for(int T, int E, int sms) {
+  int G = 1, B = 1;
+  plan_segments(T, sms, &G, &B);
+  return kTableOffset + (size_t)G * table_row_stride(E, B <= 255 ? 1 : 2);
 }
 
 // sigmoid fast path: 8 lanes per token, one lane per E/8 experts
-bool fast_path_ok(const moe_route_params* p) {
+bool fast_path_ok(const moe_route_params* p, const void* logits) {
   if (p->score_fn != MOE_SIGMOID || !p->softmax_before_topk) return false;
-  if (p->num_experts % 8 != 0) return false;
+  if (p->num_experts % 8 != 0 || p->top_k > 8) return false;
+  if ((reinterpret_cast<uintptr_t>(logits) & 15) != 0) return false;  // rows staged by bulk copies
   const int V = p->num_experts / 8;
   const bool v_ok = p->logits_dtype == MOE_BF16 ? (V == 8 || V == 16 || V == 32) : (V == 8 || V == 16);
   if (!v_ok) return false;
   const bool grouped = p->n_group > 1 && p->topk_group > 0;
-  if (grouped && (p->n_group != 8 || p->group_score_topn > 2)) return false;
-  return p->top_k <= 32;
+  // the candidate bound needs two experts per kept group to cover k
+  if (grouped && (p->n_group != 8 || p->group_score_topn > 2 || 2 * std::min(p->topk_group, 8) < p->top_k))
+    return false;
+  return true;
+}
+
+// Both route kernels ask for the largest shared-memory carveout, so that an
+// SM switching from one to the other need not reconfigure its L1 / shared split.
+template <typename K>
+cudaError_t set_smem_attr(K kernel, int smem) {
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                       (int)cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess || smem <= 48 * 1024) return e;
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
 }
 
 template <int VPL, int FAST_ESZ>
-cudaError_t launch_route(const RouteArgs& a, int smem, cudaStream_t st) {
-  static bool configured[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(route_kernel<VPL, FAST_ESZ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kStageBytesMax + 128 * 1024);
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.G);
-  cfg.blockDim = dim3((FAST_ESZ > 0) ? kThreadsFast : kThreadsGeneric);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, route_kernel<VPL, FAST_ESZ>, a);
-  if (e != cudaSuccess) {
-    // the pair of attributes was refused: a plain cooperative launch
-    cudaGetLastError();
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, route_kernel<VPL, FAST_ESZ>, a);
-  }
-  return e;
+cudaError_t launch_select(const RouteArgs& a, int threads, int smem, cudaStream_t st) {
+  cudaError_t e = set_smem_attr(route_select_kernel<VPL, FAST_ESZ>, smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(route_select_kernel<VPL, FAST_ESZ>, dim3(a.G), dim3(threads), (size_t)smem, st, a);
 }
 
 }  // namespace
@@ -1486,7 +1308,7 @@ extern "C" int moe_route_workspace_bytes(const moe_route_params* p, size_t* byte
   if (!bytes) return MOE_ERR_INVALID_ARG;
   const DevInfo d = device_info();
   if (d.sms <= 0) return MOE_ERR_CUDA;
-  *bytes = ws_bytes_for(p->num_experts, d.sms);
+  *bytes = ws_bytes_for(p->num_tokens, p->num_experts, d.sms);
   return MOE_OK;
 }
 
@@ -1505,7 +1327,8 @@ extern "C" int moe_route(const moe_route_params* p, const void* logits, const vo
   if (mode < 0) return MOE_ERR_UNSUPPORTED;
   const DevInfo d = device_info();
   if (d.sms <= 0) return MOE_ERR_CUDA;
-  if (!ws || ws_bytes < ws_bytes_for(p->num_experts, d.sms)) return MOE_ERR_WORKSPACE;
+  if (!ws || ws_bytes < ws_bytes_for(T, p->num_experts, d.sms)) return MOE_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(ws) & 15) != 0) return MOE_ERR_WORKSPACE;
 
   RouteArgs a = {};
   a.logits = logits;
@@ -1520,8 +1343,7 @@ extern "C" int moe_route(const moe_route_params* p, const void* logits, const vo
   a.tile_mn = tile_mn_limit;
   a.totals = totals;
   a.hdr = reinterpret_cast<WsHeader*>(ws);
-  a.table = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(ws) + table_offset(p->num_experts));
-  if ((reinterpret_cast<uintptr_t>(ws) & 15) != 0) return MOE_ERR_WORKSPACE;
+  a.table = reinterpret_cast<uint8_t*>(ws) + kTableOffset;
   a.T = T;
   a.E = p->num_experts;
   a.k = p->top_k;
@@ -1539,7 +1361,11 @@ extern "C" int moe_route(const moe_route_params* p, const void* logits, const vo
   a.bias_dtype = p->bias_dtype;
   a.weights_dtype = p->weights_dtype;
   a.has_bias = bias != nullptr;
-  a.G = grid_for(p, d);
+  plan_segments(T, d.sms, &a.G, &a.B);
+  a.MW = (a.B + 31) / 32;
+  a.GS = (a.G + kMaxGroups - 1) / kMaxGroups;
+  a.NG = (a.G + a.GS - 1) / a.GS;
+  a.gtot = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(ws) + kHeaderBytes);
   {
     int64_t mp = 0, mt = 0;
     moe_route_capacity(p, &mp, &mt);
@@ -1549,86 +1375,82 @@ extern "C" int moe_route(const moe_route_params* p, const void* logits, const vo
   a.loc_off = p->local_expert_offset;
   a.loc_n = p->local_num_experts > 0 ? p->local_num_experts : p->num_experts;
   a.row_bytes = p->num_experts * esize(p->logits_dtype);
-  const int per_block = (T + a.G - 1) / a.G;
-  a.chunk_tokens = std::max(1, std::min(per_block, kStageBytesMax / a.row_bytes));
-  a.cnt_bytes = per_block <= 255 ? 1 : (per_block <= 65535 ? 2 : 4);
-  a.row_stride = (p->num_experts * a.cnt_bytes + 15) & ~15;
-  a.fast = fast_path_ok(p) ? 1 : 0;
+  a.cnt_bytes = a.B <= 255 ? 1 : 2;
+  a.row_stride = (int)table_row_stride(a.E, a.cnt_bytes);
   a.timeout_ns = kDefaultTimeoutNs;
-  const int nthreads = a.fast ? kThreadsFast : kThreadsGeneric;
-  // the stage region also holds phase 2's per-row-group partial sums (two sets)
-  const int wpr = a.row_stride / 4;
-  const int part_bytes = 2 * std::max(1, std::min(nthreads / wpr, a.G)) * (4 / a.cnt_bytes) * wpr * 4;
-  a.stage_bytes = (std::max(a.chunk_tokens * a.row_bytes, part_bytes) + 15) & ~15;
-  a.ids_in_smem = ((long long)per_block * a.k * 2 <= 32 * 1024) ? 1 : 0;
-  const bool lut = a.fast && p->logits_dtype == MOE_BF16;
-  const RouteSmem L = route_smem_layout(a.E, a.stage_bytes, a.ids_in_smem ? per_block * a.k * 2 : 0, nthreads / 32,
-                                        lut ? kLutEntries * 4 : 0);
-  const int smem = L.total;
-  if (smem > d.smem_optin || smem > kStageBytesMax + 128 * 1024) return MOE_ERR_UNSUPPORTED;
+
+  const bool fast = fast_path_ok(p, logits);
+  int threads;
+  if (fast) {
+    threads = 32 * std::max(1, std::min(kFastWarpsMax, (a.B + 3) / 4));
+  } else if (mode == 0) {
+    threads = std::min(kGenericThreads, std::max(32, (a.B + 31) / 32 * 32));
+  } else {
+    threads = 32 * std::max(1, std::min(kGenericThreads / 32, a.B));
+  }
+  const int V = a.E / 8;
+  const SelSmem L = sel_smem_layout(a.E, a.MW, a.B, a.k, fast ? 1 : 0, fast ? V : 1, a.row_bytes, threads / 32);
+  if (L.total > d.smem_optin) return MOE_ERR_UNSUPPORTED;
+  const int psmem = perm_smem_bytes(a.E);
+  if (psmem > d.smem_optin) return MOE_ERR_UNSUPPORTED;
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t err;
-  if (a.fast) {
-    const int V = a.E / 8;
+  if (fast) {
     if (p->logits_dtype == MOE_BF16)
-      err = V == 8 ? launch_route<8, 2>(a, smem, st) : V == 16 ? launch_route<16, 2>(a, smem, st)
-                                                              : launch_route<32, 2>(a, smem, st);
+      err = V == 8 ? launch_select<8, 2>(a, threads, L.total, st)
+          : V == 16 ? launch_select<16, 2>(a, threads, L.total, st)
+                    : launch_select<32, 2>(a, threads, L.total, st);
     else
-      err = V == 8 ? launch_route<8, 4>(a, smem, st) : launch_route<16, 4>(a, smem, st);
+      err = V == 8 ? launch_select<8, 4>(a, threads, L.total, st) : launch_select<16, 4>(a, threads, L.total, st);
   } else {
     switch (mode) {
-      case 0: err = launch_route<0, 0>(a, smem, st); break;
-      case 2: err = launch_route<2, 0>(a, smem, st); break;
-      case 3: err = launch_route<3, 0>(a, smem, st); break;
-      case 4: err = launch_route<4, 0>(a, smem, st); break;
-      case 5: err = launch_route<5, 0>(a, smem, st); break;  // e.g. 160 experts in groups of 20
-      case 6: err = launch_route<6, 0>(a, smem, st); break;
-      case 8: err = launch_route<8, 0>(a, smem, st); break;
-      case 12: err = launch_route<12, 0>(a, smem, st); break;
-      case 16: err = launch_route<16, 0>(a, smem, st); break;
-      case 24: err = launch_route<24, 0>(a, smem, st); break;
-      case 32: err = launch_route<32, 0>(a, smem, st); break;
+      case 0: err = launch_select<0, 0>(a, threads, L.total, st); break;
+      case 2: err = launch_select<2, 0>(a, threads, L.total, st); break;
+      case 3: err = launch_select<3, 0>(a, threads, L.total, st); break;
+      case 4: err = launch_select<4, 0>(a, threads, L.total, st); break;
+      case 5: err = launch_select<5, 0>(a, threads, L.total, st); break;  // e.g. 160 experts in groups of 20
+      case 6: err = launch_select<6, 0>(a, threads, L.total, st); break;
+      case 8: err = launch_select<8, 0>(a, threads, L.total, st); break;
+      case 12: err = launch_select<12, 0>(a, threads, L.total, st); break;
+      case 16: err = launch_select<16, 0>(a, threads, L.total, st); break;
+      case 24: err = launch_select<24, 0>(a, threads, L.total, st); break;
+      case 32: err = launch_select<32, 0>(a, threads, L.total, st); break;
       default: return MOE_ERR_UNSUPPORTED;
     }
   }
   if (err != cudaSuccess) return MOE_ERR_CUDA;
-  return MOE_OK;
+  err = set_smem_attr(route_permute_kernel, psmem);
+  if (err == cudaSuccess)
+    err = launch_pdl(route_permute_kernel, dim3(a.G), dim3(kPermThreads), (size_t)psmem, st, a);
+  return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------------------
-// barrier test hook: a grid that waits for more arrivals than it has blocks
+// wait test hook: a bounded wait on a barrier that nothing completes
 // ---------------------------------------------------------------------------
 namespace moe {
 namespace {
-__global__ void barrier_probe_kernel(WsHeader* hdr, uint32_t expected, long long timeout_ns) {
-  __shared__ int flag;
-  const uint32_t gen = barrier_generation(hdr);
-  grid_barrier(hdr, expected, gen, timeout_ns, &flag);
+// One block: thread 0 arms a shared-memory mbarrier for one arrival plus
+// `pending` bytes, adds the arrival only when pending == 0, then waits on it
+// the way the kernels wait on their bulk copies (bounded).
+__global__ void wait_probe_kernel(WsHeader* hdr, uint32_t pending, long long timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  mbar_arrive_expect_tx(&bar, pending);  // the arrival; `pending` transaction bytes never come
+  if (!mbar_wait_bounded(&bar, 0, timeout_ns)) record_timeout(hdr);
 }
 }  // namespace
 }  // namespace moe
 
-extern "C" int moe_debug_barrier_wait(int32_t blocks, int32_t extra_arrivals, int64_t timeout_ns, void* ws,
-                                      size_t ws_bytes, void* stream) {
-  if (blocks <= 0 || extra_arrivals < 0 || timeout_ns <= 0 || timeout_ns > 5LL * 1000 * 1000 * 1000)
-    return MOE_ERR_INVALID_ARG;
+extern "C" int moe_debug_wait_timeout(int32_t never_complete, int64_t timeout_ns, void* ws, size_t ws_bytes,
+                                      void* stream) {
+  if (timeout_ns <= 0 || timeout_ns > 5LL * 1000 * 1000 * 1000) return MOE_ERR_INVALID_ARG;
   if (!ws || ws_bytes < sizeof(WsHeader)) return MOE_ERR_WORKSPACE;
-  const DevInfo d = device_info();
-  if (blocks > d.sms) return MOE_ERR_INVALID_ARG;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(blocks);
-  cfg.blockDim = dim3(32);
-  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, barrier_probe_kernel, hdr,
-                                           (uint32_t)(blocks + extra_arrivals), (long long)timeout_ns);
-  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  wait_probe_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<WsHeader*>(ws), never_complete ? 16u : 0u, (long long)timeout_ns);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------------------
@@ -1636,20 +1458,25 @@ extern "C" int moe_debug_barrier_wait(int32_t blocks, int32_t extra_arrivals, in
 // ---------------------------------------------------------------------------
 namespace moe {
 namespace {
-__global__ void proxy_error_kernel(const float* x, long long n, float* out) {
+__global__ void proxy_error_kernel(const float* x, const float* b, long long n, int f32_logits, float* err,
+                                   float* delta) {
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
-    const float v = x[i];
-    out[i] = fmaf(0.5f, tanh_approx(0.5f * v), 0.5f) - sigmoid_f32(v);
+    const float v = x[i], cb = 0.5f + b[i];
+    const __half2 p = proxy_pair(v, v, __float2half2_rn(cb));
+    err[i] = __low2float(p) - (sigmoid_f32(v) + b[i]);
+    delta[i] = proxy_delta(fabsf(cb), f32_logits);
   }
 }
 }  // namespace
 }  // namespace moe
 
-extern "C" int moe_debug_sigmoid_proxy_error(const float* x, int64_t n, float* out, void* stream) {
-  if (n < 0 || (n > 0 && (!x || !out))) return MOE_ERR_INVALID_ARG;
+extern "C" int moe_debug_sigmoid_proxy_error(const float* x, const float* b, int64_t n, int32_t f32_logits, float* err,
+                                             float* delta, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !b || !err || !delta))) return MOE_ERR_INVALID_ARG;
   if (n == 0) return MOE_OK;
   const int grid = (int)std::min<int64_t>((n + 255) / 256, 4096);
-  proxy_error_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, (long long)n, out);
+  proxy_error_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, b, (long long)n, f32_logits, err,
+                                                                               delta);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -1674,9 +1501,10 @@ __device__ __align__(256) uint8_t g_route_scratch[kStaticScratchBytes];
 
 // The array's device address, looked up once per device with that device
 // current.  A failed lookup is not cached: the next call tries again.  The
-// first successful set-up also zero-fills the array's 64-byte header on the
-// caller's stream; after that the status word is sticky across calls (a
-// recorded error stays until moe_route_no_alloc_status clears it).
+// first successful set-up also zero-fills the array's header and group
+// totals on the caller's stream (every call leaves the totals zero again);
+// after that the status word is sticky across calls (a recorded error stays
+// until moe_route_no_alloc_status clears it).
 struct ScratchSlot {
   std::mutex m;
   std::atomic<void*> ptr{nullptr};
@@ -1694,7 +1522,7 @@ void* scratch_address(int dev, cudaStream_t st) {
     cudaGetLastError();
     return nullptr;
   }
-  if (cudaMemsetAsync(p, 0, sizeof(WsHeader), st) != cudaSuccess) return nullptr;
+  if (cudaMemsetAsync(p, 0, kTableOffset, st) != cudaSuccess) return nullptr;  // header and group totals
   slot.ptr.store(p, std::memory_order_release);
   return p;
 }
@@ -1719,7 +1547,7 @@ extern "C" int moe_route_no_alloc(const moe_route_params* p, const void* logits,
   if (v != MOE_OK) return v;
   const DevInfo d = device_info();
   if (d.sms <= 0) return MOE_ERR_CUDA;
-  if (ws_bytes_for(p->num_experts, d.sms) > kStaticScratchBytes) return MOE_ERR_WORKSPACE;
+  if (ws_bytes_for(p->num_tokens, p->num_experts, d.sms) > kStaticScratchBytes) return MOE_ERR_WORKSPACE;
   int dev = 0;
   if (current_device(&dev) != MOE_OK) return MOE_ERR_CUDA;
   void* ws = scratch_address(dev, reinterpret_cast<cudaStream_t>(stream));
