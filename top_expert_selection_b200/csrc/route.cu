@@ -60,6 +60,7 @@ constexpr int kFastWarpsMax = 28;        // fast path: up to 28 warps of 4 token
 constexpr int kGenericThreads = 512;     // generic paths
 constexpr int kPermThreads = 1024;       // bookkeeping kernel
 constexpr int kMaxSegment = 256;         // tokens per segment (8 mask words)
+constexpr int kMaxGroups = 16;           // segment groups whose count totals the selection accumulates
 
 struct RouteArgs {
   const void* logits;
@@ -87,6 +88,7 @@ struct RouteArgs {
   int G, B;          // segments, tokens per segment (segment c: [c*B, min(T, (c+1)*B)))
   int MW;            // 32-bit mask words per expert: ceil(B / 32)
   int GS, NG;        // segments per group, groups
+  int slots;         // fast path: staging slots per warp (1 when every warp has one quad, else 2)
   int max_padded;
   int max_tiles;
   int loc_off, loc_n;  // the local experts [loc_off, loc_off + loc_n): only they get slots and tiles
@@ -115,7 +117,7 @@ constexpr int kCandBytes = 4 * kCandSlotsPerToken * 14 + 2 * kPendMax + 8;
 // candidate keys, 4 x 32 fp32 scores and 4 x 32 u16 expert ids; the warp's
 // pending exact-path tokens; 2 mbarriers
 __host__ __device__ inline SelSmem sel_smem_layout(int E, int MW, int B, int k, int fast, int V, int row_bytes,
-                                                   int nwarps) {
+                                                   int nwarps, int slots) {
   SelSmem L;
   int o = 0;
   L.masks = o;
@@ -131,7 +133,7 @@ __host__ __device__ inline SelSmem sel_smem_layout(int E, int MW, int B, int k, 
   o = (o + 127) & ~127;
   L.warp0 = o;
   L.stage_bytes = fast ? ((4 * row_bytes + 127) & ~127) : 0;
-  L.warp_bytes = fast ? ((2 * L.stage_bytes + kCandBytes + 16 + 127) & ~127) : 0;
+  L.warp_bytes = fast ? ((slots * L.stage_bytes + kCandBytes + 16 + 127) & ~127) : 0;
   o += L.warp_bytes * nwarps;
   L.total = o;
   return L;
@@ -893,15 +895,15 @@ __global__ void __launch_bounds__((FAST_ESZ > 0) ? kFastWarpsMax * 32 : kGeneric
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const int t_begin = c * a.B;
   const int n = max(0, min(a.T, t_begin + a.B) - t_begin);
-  const SelSmem L = sel_smem_layout(E, a.MW, a.B, a.k, kFast ? 1 : 0, FV, a.row_bytes, nwarps);
+  const SelSmem L = sel_smem_layout(E, a.MW, a.B, a.k, kFast ? 1 : 0, FV, a.row_bytes, nwarps, a.slots);
   uint32_t* masks = reinterpret_cast<uint32_t*>(smem + L.masks);
   uint16_t* ids_s = reinterpret_cast<uint16_t*>(smem + L.ids);
   float* bias_s = reinterpret_cast<float*>(smem + L.bias);
   uint8_t* cb_s = smem + L.cb;
   float* delta_s = reinterpret_cast<float*>(smem + L.delta);
   uint8_t* wbase = smem + L.warp0 + (size_t)warp * L.warp_bytes;
-  uint8_t* cand = wbase + 2 * L.stage_bytes;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(wbase + 2 * L.stage_bytes + kCandBytes);
+  uint8_t* cand = wbase + a.slots * L.stage_bytes;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(wbase + a.slots * L.stage_bytes + kCandBytes);
 
   // Programmatic dependent launch: the bookkeeping kernel may be scheduled at
   // once.  Before waiting on the previous grid, only the bias is read (a
@@ -946,7 +948,7 @@ __global__ void __launch_bounds__((FAST_ESZ > 0) ? kFastWarpsMax * 32 : kGeneric
   const uint8_t* lg_bytes = reinterpret_cast<const uint8_t*>(a.logits);
   if constexpr (kFast) {
     if (lane == 0) {
-      for (int s = 0; s < 2; ++s) {
+      for (int s = 0; s < a.slots; ++s) {
         const int qd = warp + s * nwarps;
         if (qd < nq) {
           const uint32_t bytes = (uint32_t)min(4, n - qd * 4) * (uint32_t)a.row_bytes;
@@ -1056,17 +1058,27 @@ __global__ void __launch_bounds__(kPermThreads, 1) route_permute_kernel(RouteArg
     const int grp = c / a.GS, r0 = grp * a.GS;
     for (int e = threadIdx.x; e < E; e += kPermThreads) {
       uint32_t tot = 0, pre_e = 0;
-      for (int g0 = 0; g0 < a.NG; g0 += 8) {
-        uint32_t v[8];
+      // the group totals (at most kMaxGroups) and this group's earlier rows
+      // (fewer than GS): the first 16 of each in flight together
+      uint32_t vg[kMaxGroups], vr[16];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = g0 + j < a.NG ? __ldcg(a.gtot + (size_t)(g0 + j) * E + e) : 0u;
+      for (int j = 0; j < kMaxGroups; ++j) vg[j] = j < a.NG ? __ldcg(a.gtot + (size_t)j * E + e) : 0u;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          tot += v[j];
-          pre_e += g0 + j < grp ? v[j] : 0u;
-        }
+      for (int j = 0; j < 16; ++j) {
+        const int r = r0 + j;
+        const uint8_t* trow = a.table + (size_t)r * a.row_stride;
+        vr[j] = r < c ? (a.cnt_bytes == 1 ? (uint32_t)__ldcg(trow + e)
+                                          : (uint32_t)__ldcg(reinterpret_cast<const uint16_t*>(trow) + e))
+                      : 0u;
       }
-      for (int rb = r0; rb < c; rb += 8) {
+#pragma unroll
+      for (int j = 0; j < kMaxGroups; ++j) {
+        tot += vg[j];
+        pre_e += j < grp ? vg[j] : 0u;
+      }
+#pragma unroll
+      for (int j = 0; j < 16; ++j) pre_e += vr[j];
+      for (int rb = r0 + 16; rb < c; rb += 8) {  // groups of more than 16 segments (very large T)
         uint32_t v[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -1242,7 +1254,6 @@ void plan_segments(int T, int sms, int* G, int* B) {
 // and size: every call leaves the part it used zero, whatever its shape) |
 // table [G][row] (rows of 1- or 2-byte entries, 16-byte multiples)
 constexpr size_t kHeaderBytes = 256;
-constexpr int kMaxGroups = 16;
 constexpr size_t kTableOffset = kHeaderBytes + (size_t)kMaxGroups * MOE_MAX_EXPERTS * 4;
 
 size_t table_row_stride(int E, int cnt_bytes) { return ((size_t)E * cnt_bytes + 15) & ~(size_t)15; }
@@ -1389,7 +1400,9 @@ extern "C" int moe_route(const moe_route_params* p, const void* logits, const vo
     threads = 32 * std::max(1, std::min(kGenericThreads / 32, a.B));
   }
   const int V = a.E / 8;
-  const SelSmem L = sel_smem_layout(a.E, a.MW, a.B, a.k, fast ? 1 : 0, fast ? V : 1, a.row_bytes, threads / 32);
+  a.slots = (fast && (a.B + 3) / 4 > threads / 32) ? 2 : 1;
+  const SelSmem L = sel_smem_layout(a.E, a.MW, a.B, a.k, fast ? 1 : 0, fast ? V : 1, a.row_bytes, threads / 32,
+                                    a.slots);
   if (L.total > d.smem_optin) return MOE_ERR_UNSUPPORTED;
   const int psmem = perm_smem_bytes(a.E);
   if (psmem > d.smem_optin) return MOE_ERR_UNSUPPORTED;
