@@ -51,6 +51,8 @@ def _lib():
                                           P, i32, P, i32, P, P, P, P, P]
         L.oracle_route_capacity.argtypes = [i32, i32, i32, i32, P, P]
         L.oracle_route_bookkeeping.argtypes = [i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P]
+        L.oracle_route_bookkeeping_shared.argtypes = [i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P]
+        L.oracle_append_shared.argtypes = [i32, i32, i32, i32, P, P, P, P]
         L.oracle_aux_scores.argtypes = [i32, i32, i32, i32, P, P, P, P]
         L.oracle_aux_loss_fwd.argtypes = [i32, i32, i32, i32, f32, P, P, P]
         L.oracle_aux_loss_bwd.argtypes = [i32, i32, i32, i32, f32, f32, P, P, P, P]
@@ -59,6 +61,7 @@ def _lib():
         L.oracle_dispatch.argtypes = [i32, i32, i32, P, P, P, i32, P]
         L.oracle_combine.argtypes = [i32, i32, i32, P, P, P, i32, P]
         L.oracle_combine_f32.argtypes = [i32, i32, i32, P, P, P, i32, P]
+        L.oracle_ep_regroup.argtypes = [i32, i32, i32, P, P, ctypes.c_longlong, ctypes.c_longlong, P, P, P, P]
         L.oracle_rmsnorm_router_topk.argtypes = [i32, i32, i32, i32, f32, i32, P, P, P, P, P, P, P, P]
         L.oracle_router_logits.argtypes = [i32, i32, i32, P, P, P, P]
         L.oracle_router_logits.restype = i32
@@ -69,8 +72,9 @@ def _lib():
         L.oracle_f64_to_bf16.argtypes = [ctypes.c_double]
         L.oracle_f64_to_bf16.restype = ctypes.c_uint16
         for name in ("oracle_route_select", "oracle_route_capacity", "oracle_route_bookkeeping",
+                     "oracle_route_bookkeeping_shared", "oracle_append_shared",
                      "oracle_aux_scores", "oracle_aux_loss_fwd", "oracle_aux_loss_bwd", "oracle_aux_scores_bwd", "oracle_route_weights_bwd",
-                     "oracle_dispatch", "oracle_combine", "oracle_combine_f32", "oracle_rmsnorm_router_topk"):
+                     "oracle_dispatch", "oracle_combine", "oracle_combine_f32", "oracle_ep_regroup", "oracle_rmsnorm_router_topk"):
             getattr(L, name).restype = i32
         _lib_handle = L
     return _lib_handle
@@ -159,28 +163,42 @@ def route_capacity(T: int, E: int, k: int, tile: int):
 
 
 def route_bookkeeping(ids, E: int, tile: int, local_expert_offset: int = 0,
-                      local_num_experts: Optional[int] = None) -> dict:
+                      local_num_experts: Optional[int] = None, num_shared: int = 0) -> dict:
     """Bookkeeping of the experts [local_expert_offset, local_expert_offset + local_num_experts)
-    (all E by default); counts/offsets/tile_expert are indexed by the local expert."""
+    (all E by default) and of the num_shared fused shared experts E .. E + num_shared - 1 (local
+    index local_num_experts + s); counts/offsets/tile_expert are indexed by the local expert."""
     ids = as_numpy(ids).astype(np.int32, copy=False)
     T, k = ids.shape
     nl = E if local_num_experts is None else int(local_num_experts)
-    max_padded, max_tiles = route_capacity(T, E, k, tile)
-    counts = np.zeros(nl, np.int32)
-    offsets = np.zeros(nl + 1, np.int32)
+    NL = nl + num_shared
+    rows = T * k
+    max_padded = rows + min(rows, E + num_shared) * (tile - 1)
+    max_tiles = max_padded // tile
+    counts = np.zeros(NL, np.int32)
+    offsets = np.zeros(NL + 1, np.int32)
     e2p = np.zeros(T * k, np.int32)
     p2t = np.full(max(max_padded, 1), -7, np.int32)
     te = np.full(max(max_tiles, 1), -7, np.int32)
     tl = np.full(max(max_tiles, 1), -7, np.int32)
     totals = np.zeros(2, np.int32)
-    rc = _lib().oracle_route_bookkeeping(T, E, k, tile, int(local_expert_offset), nl,
-                                         _ptr(np.ascontiguousarray(ids)), _ptr(counts),
-                                         _ptr(offsets), _ptr(e2p), _ptr(p2t), _ptr(te), _ptr(tl),
-                                         _ptr(totals))
+    rc = _lib().oracle_route_bookkeeping_shared(T, E, num_shared, k, tile, int(local_expert_offset), nl,
+                                                _ptr(np.ascontiguousarray(ids)), _ptr(counts), _ptr(offsets),
+                                                _ptr(e2p), _ptr(p2t), _ptr(te), _ptr(tl), _ptr(totals))
     _check(rc, "route_bookkeeping")
     P, nt = int(totals[0]), int(totals[1])
     return {"counts": counts, "offsets": offsets, "e2p": e2p, "p2t": p2t[:P], "tile_expert": te[:nt],
             "tile_mn_limit": tl[:nt], "totals": totals, "max_padded": max_padded, "max_tiles": max_tiles}
+
+
+def append_shared(ids, weights, E: int, S: int):
+    """The S fused shared-expert slots appended to each token: ids E + s, weights 1.0."""
+    ids = np.ascontiguousarray(as_numpy(ids), dtype=np.int32)
+    w = np.ascontiguousarray(as_numpy(weights), dtype=np.float32)
+    T, k = ids.shape
+    io = np.zeros((T, k + S), np.int32)
+    wo = np.zeros((T, k + S), np.float32)
+    _check(_lib().oracle_append_shared(T, k, S, E, _ptr(ids), _ptr(w), _ptr(io), _ptr(wo)), "append_shared")
+    return io, wo
 
 
 def aux_scores(logits, k: int, score_fn: int = SOFTMAX) -> dict:
@@ -298,3 +316,22 @@ def router_logits(xn, W, bias=None) -> np.ndarray:
     rc = _lib().oracle_router_logits(T, H, E, _ptr(x), _ptr(w), _ptr(b), _ptr(out))
     _check(rc, "router_logits")
     return out
+
+
+def ep_regroup(counts, recv, tile: int) -> dict:
+    """Receive-order rows -> the receiving rank's tile-padded expert layout (expert, source, token)."""
+    c = np.ascontiguousarray(as_numpy(counts), dtype=np.int32)
+    W, L = c.shape
+    r = np.ascontiguousarray(as_numpy(recv))
+    n = r.shape[0]
+    row_bytes = r.dtype.itemsize * int(np.prod(r.shape[1:]))
+    tot = c.sum(0)
+    P = int(sum((int(t) + tile - 1) // tile * tile for t in tot))
+    padded = np.zeros((max(P, 1),) + r.shape[1:], r.dtype)
+    offsets = np.zeros(L + 1, np.int32)
+    totals = np.zeros(2, np.int32)
+    p2r = np.zeros(max(P, 1), np.int32)
+    rc = _lib().oracle_ep_regroup(W, L, tile, _ptr(c), _ptr(r), n, row_bytes, _ptr(padded), _ptr(offsets),
+                                  _ptr(totals), _ptr(p2r))
+    _check(rc, "ep_regroup")
+    return {"padded": padded[:P], "offsets": offsets, "totals": totals, "padded_to_recv": p2r[:P]}

@@ -284,33 +284,46 @@ int oracle_route_capacity(int T, int E, int k, int tile, int64_t* max_padded, in
  * Entries of p2t at or past P and of the tile tables at or past P/tile are
  * left as the caller filled them.
  */
-int oracle_route_bookkeeping(int T, int E, int k, int tile, int off, int nl, const int32_t* ids,
-                             int32_t* counts, int32_t* offsets, int32_t* e2p, int32_t* p2t,
-                             int32_t* tile_expert, int32_t* tile_mn_limit, int32_t* totals) {
-  if (T < 0 || E <= 0 || k <= 0 || !is_pow2(tile)) return -1;
+/*
+ * With S fused shared experts [TRT: Parameters num_fused_shared_experts --
+ * extra shared-expert slots appended per token, DeepSeekV3 path].  READING:
+ * shared expert s has id E + s; it is local on every expert-parallel shard and
+ * is indexed after the shard's routed experts (local index nl + s), so the
+ * bookkeeping runs over nl + S local experts.  ids [T, k] may hold E .. E+S-1.
+ */
+int oracle_route_bookkeeping_shared(int T, int E, int S, int k, int tile, int off, int nl, const int32_t* ids,
+                                    int32_t* counts, int32_t* offsets, int32_t* e2p, int32_t* p2t,
+                                    int32_t* tile_expert, int32_t* tile_mn_limit, int32_t* totals) {
+  if (T < 0 || E <= 0 || S < 0 || k <= 0 || !is_pow2(tile)) return -1;
   if (off < 0 || nl <= 0 || off + nl > E) return -1;
-  for (int le = 0; le < nl; ++le) counts[le] = 0;
+  const int NL = nl + S;  /* local experts: the shard's routed ones, then the shared ones */
+  for (int le = 0; le < NL; ++le) counts[le] = 0;
   for (int64_t i = 0; i < (int64_t)T * k; ++i) {
     int e = ids[i];
-    if (e < 0 || e >= E) return -1;
-    if (e >= off && e < off + nl) counts[e - off] += 1;
+    if (e < 0 || e >= E + S) return -1;
+    if (e >= E) counts[nl + (e - E)] += 1;
+    else if (e >= off && e < off + nl) counts[e - off] += 1;
   }
   offsets[0] = 0;
-  for (int le = 0; le < nl; ++le) {
+  for (int le = 0; le < NL; ++le) {
     int32_t padded = ((counts[le] + tile - 1) / tile) * tile;
     offsets[le + 1] = offsets[le] + padded;
   }
-  int32_t P = offsets[nl];
+  int32_t P = offsets[NL];
   for (int32_t p = 0; p < P; ++p) p2t[p] = -1;
-  int32_t* running = (int32_t*)calloc((size_t)nl, sizeof(int32_t));
+  int32_t* running = (int32_t*)calloc((size_t)NL, sizeof(int32_t));
   for (int t = 0; t < T; ++t) {
     for (int j = 0; j < k; ++j) {
       int e = ids[(size_t)t * k + j];
-      if (e < off || e >= off + nl) {
+      int le;
+      if (e >= E) {
+        le = nl + (e - E);
+      } else if (e >= off && e < off + nl) {
+        le = e - off;
+      } else {
         e2p[(size_t)t * k + j] = -1;
         continue;
       }
-      int le = e - off;
       int32_t slot = offsets[le] + running[le];
       running[le] += 1;
       e2p[(size_t)t * k + j] = slot;
@@ -322,7 +335,7 @@ int oracle_route_bookkeeping(int T, int E, int k, int tile, int off, int nl, con
   for (int32_t c = 0; c < ntiles; ++c) {
     int32_t row = c * tile;
     int le = 0;
-    while (!(offsets[le] <= row && row < offsets[le + 1])) ++le;
+    while (!(offsets[le] <= row && row < offsets[le + 1])) ++le;  /* le < NL */
     int32_t lim = (c + 1) * tile;
     int32_t valid_end = offsets[le] + counts[le];
     tile_expert[c] = le;
@@ -330,6 +343,35 @@ int oracle_route_bookkeeping(int T, int E, int k, int tile, int off, int nl, con
   }
   totals[0] = P;
   totals[1] = ntiles;
+  return 0;
+}
+
+int oracle_route_bookkeeping(int T, int E, int k, int tile, int off, int nl, const int32_t* ids,
+                             int32_t* counts, int32_t* offsets, int32_t* e2p, int32_t* p2t,
+                             int32_t* tile_expert, int32_t* tile_mn_limit, int32_t* totals) {
+  return oracle_route_bookkeeping_shared(T, E, 0, k, tile, off, nl, ids, counts, offsets, e2p, p2t, tile_expert,
+                                         tile_mn_limit, totals);
+}
+
+/*
+ * The fused shared-expert slots [TRT: Parameters num_fused_shared_experts].
+ * READING: each token's S extra slots follow its k routed slots in order;
+ * slot k + s holds expert E + s with weight 1.0 (the shared experts take no
+ * part in selection, renormalisation or the routed scaling factor).
+ */
+int oracle_append_shared(int T, int k, int S, int E, const int32_t* ids, const float* weights, int32_t* ids_out,
+                         float* weights_out) {
+  if (T < 0 || k <= 0 || S < 0 || E <= 0) return -1;
+  for (int t = 0; t < T; ++t) {
+    for (int j = 0; j < k; ++j) {
+      ids_out[(size_t)t * (k + S) + j] = ids[(size_t)t * k + j];
+      weights_out[(size_t)t * (k + S) + j] = weights[(size_t)t * k + j];
+    }
+    for (int s = 0; s < S; ++s) {
+      ids_out[(size_t)t * (k + S) + k + s] = E + s;
+      weights_out[(size_t)t * (k + S) + k + s] = 1.0f;
+    }
+  }
   return 0;
 }
 
@@ -591,6 +633,55 @@ int oracle_combine_f32(int T, int H, int k, const float* expert_out, const int32
       }
     }
   }
+  return 0;
+}
+
+/*
+ * Expert-parallel regroup [NKI: Background, the all-to-all-v MoE dispatch
+ * path; TRT: Parameters local_expert_offset / local_num_experts, Returns].
+ * counts[s*L + e]: rows rank s sends for this rank's local expert e; recv
+ * holds them ordered by source, then expert, then the source's token order.
+ * READING: the receiving rank lays its rows out by local expert, then source
+ * rank, then token (the order a single route of all ranks' tokens,
+ * concatenated in rank order, gives), each expert padded to `tile` rows
+ * (padding rows zero), padded_to_recv = the receive row of each padded row
+ * (-1 on padding).  Rows are `row_bytes` bytes, copied as they are.
+ */
+int oracle_ep_regroup(int W, int L, int tile, const int32_t* counts, const uint8_t* recv, long long n_recv,
+                      long long row_bytes, uint8_t* padded, int32_t* offsets, int32_t* totals,
+                      int32_t* padded_to_recv) {
+  if (W <= 0 || L <= 0 || tile <= 0 || row_bytes <= 0) return -1;
+  long long n = 0;
+  for (int i = 0; i < W * L; ++i) {
+    if (counts[i] < 0) return -1;
+    n += counts[i];
+  }
+  if (n != n_recv) return -1;
+  offsets[0] = 0;
+  for (int e = 0; e < L; ++e) {
+    int tot = 0;
+    for (int s = 0; s < W; ++s) tot += counts[s * L + e];
+    offsets[e + 1] = offsets[e] + (tot + tile - 1) / tile * tile;
+  }
+  int P = offsets[L];
+  for (int p = 0; p < P; ++p) {
+    padded_to_recv[p] = -1;
+    memset(padded + (size_t)p * row_bytes, 0, (size_t)row_bytes);
+  }
+  long long r = 0;
+  for (int s = 0; s < W; ++s) {
+    for (int e = 0; e < L; ++e) {
+      int before = 0;  /* rows of expert e from earlier sources */
+      for (int s2 = 0; s2 < s; ++s2) before += counts[s2 * L + e];
+      for (int i = 0; i < counts[s * L + e]; ++i, ++r) {
+        int p = offsets[e] + before + i;
+        memcpy(padded + (size_t)p * row_bytes, recv + (size_t)r * row_bytes, (size_t)row_bytes);
+        padded_to_recv[p] = (int32_t)r;
+      }
+    }
+  }
+  totals[0] = P;
+  totals[1] = P / tile;
   return 0;
 }
 

@@ -728,3 +728,82 @@ def test_decode_rejects_page_constraints():
     x = np.zeros((4, 100), np.uint16)
     with pytest.raises(ValueError):
         oracle.rmsnorm_router_topk(x, np.zeros(100, np.uint16), np.zeros((100, 8), np.uint16), None, k=2)
+
+
+# --------------------------------------------------------------------------- expert-parallel regroup
+
+
+def test_ep_regroup_handworked():
+    # two ranks send to a rank owning two experts, tile 2: rank 0 sends one row for expert 0 and two for
+    # expert 1, rank 1 one row for expert 1.  Receive order r0 (s0,e0), r1 r2 (s0,e1), r3 (s1,e1).
+    # Expert 0: 1 row -> 2 padded rows; expert 1: 3 rows -> 4, ordered by source then token.
+    counts = np.array([[1, 2], [0, 1]], np.int32)
+    recv = np.array([[10, 11], [20, 21], [30, 31], [40, 41]], np.uint16)
+    out = oracle.ep_regroup(counts, recv, 2)
+    assert out["offsets"].tolist() == [0, 2, 6] and out["totals"].tolist() == [6, 3]
+    assert out["padded_to_recv"].tolist() == [0, -1, 1, 2, 3, -1]
+    assert out["padded"].tolist() == [[10, 11], [0, 0], [20, 21], [30, 31], [40, 41], [0, 0]]
+    # no rows at all, and a rank that sends nothing
+    e = oracle.ep_regroup(np.zeros((3, 2), np.int32), np.zeros((0, 8), np.float32), 4)
+    assert e["offsets"].tolist() == [0, 0, 0] and e["totals"].tolist() == [0, 0]
+
+
+def test_ep_regroup_equals_single_route_of_the_concatenation():
+    """Rows sent by W ranks (each routed over all experts with tile 1 and dispatched) and regrouped by the
+    receiving rank equal the shard bookkeeping + dispatch of all ranks' tokens concatenated in rank order:
+    two definitions written separately (the shard route of the pages' local_expert_offset /
+    local_num_experts, and the exchange) must agree."""
+    rng = np.random.default_rng(7)
+    W, E, k, H, tile = 3, 12, 3, 4, 4
+    L = E // W
+    Ts = [9, 0, 14]
+    ids_r = [np.array([rng.choice(E, k, replace=False) for _ in range(T)], np.int32).reshape(T, k) for T in Ts]
+    hid_r = [rng.integers(0, 60000, (T, H)).astype(np.uint16) for T in Ts]
+    ids_all = np.concatenate(ids_r)
+    hid_all = np.concatenate(hid_r)
+    for d in range(W):
+        # the sender side: tile-1 bookkeeping over all experts, dispatch, this destination's expert range
+        counts = np.zeros((W, L), np.int32)
+        parts = []
+        for s in range(W):
+            bk = oracle.route_bookkeeping(ids_r[s], E, 1)
+            send = oracle.dispatch(hid_r[s], bk["e2p"], bk["p2t"], int(bk["totals"][0]), max(int(bk["totals"][0]), 1))
+            lo, hi = int(bk["offsets"][d * L]), int(bk["offsets"][(d + 1) * L])
+            parts.append(send[lo:hi])
+            counts[s] = bk["counts"][d * L:(d + 1) * L]
+        recv = np.concatenate(parts) if sum(p.shape[0] for p in parts) else np.zeros((0, H), np.uint16)
+        got = oracle.ep_regroup(counts, recv, tile)
+        ref_bk = oracle.route_bookkeeping(ids_all, E, tile, d * L, L)
+        P = int(ref_bk["totals"][0])
+        ref = oracle.dispatch(hid_all, ref_bk["e2p"], ref_bk["p2t"], P, P)
+        assert got["offsets"].tolist() == ref_bk["offsets"].tolist()
+        assert got["totals"].tolist() == ref_bk["totals"].tolist()
+        assert np.array_equal(got["padded"], ref[:P])
+        assert np.array_equal(got["padded_to_recv"] >= 0, ref_bk["p2t"] >= 0)
+
+
+# --------------------------------------------------------------------------- fused shared experts
+
+
+def test_fused_shared_experts_handworked():
+    """Reading of num_fused_shared_experts (trtllm_gen_routing, Parameters): one shared expert (id E = 4)
+    appended to every token after its k routed slots, weight 1.0, local on every shard after the shard's
+    routed experts.  Hand-worked from T=3, k=2, E=4, tile 4, ids [[1,0],[1,2],[3,1]]."""
+    ids, w = oracle.append_shared(np.array([[1, 0], [1, 2], [3, 1]], np.int32),
+                                  np.array([[0.5, 0.25], [0.6, 0.4], [0.7, 0.3]], np.float32), 4, 1)
+    assert ids.tolist() == [[1, 0, 4], [1, 2, 4], [3, 1, 4]]
+    assert w[:, 2].tolist() == [1.0, 1.0, 1.0] and w[0, :2].tolist() == [0.5, 0.25]
+    bk = oracle.route_bookkeeping(ids, 4, 4, num_shared=1)
+    assert bk["counts"].tolist() == [1, 3, 1, 1, 3]
+    assert bk["offsets"].tolist() == [0, 4, 8, 12, 16, 20]
+    assert bk["e2p"].tolist() == [4, 0, 16, 5, 8, 17, 12, 6, 18]
+    assert bk["p2t"].tolist() == [0, -1, -1, -1, 0, 1, 2, -1, 1, -1, -1, -1, 2, -1, -1, -1, 0, 1, 2, -1]
+    assert bk["tile_expert"].tolist() == [0, 1, 2, 3, 4] and bk["tile_mn_limit"].tolist() == [1, 7, 9, 13, 19]
+    assert bk["totals"].tolist() == [20, 5]
+    # a shard owning experts 1 and 2: the shared expert is local there too, after them
+    sh = oracle.route_bookkeeping(ids, 4, 4, 1, 2, num_shared=1)
+    assert sh["counts"].tolist() == [3, 1, 3] and sh["offsets"].tolist() == [0, 4, 8, 12]
+    assert sh["e2p"].tolist() == [0, -1, 8, 1, 4, 9, -1, 2, 10]
+    assert sh["p2t"].tolist() == [0, 1, 2, -1, 1, -1, -1, -1, 0, 1, 2, -1]
+    assert sh["tile_expert"].tolist() == [0, 1, 2] and sh["tile_mn_limit"].tolist() == [3, 5, 11]
+    assert sh["totals"].tolist() == [12, 3]
