@@ -331,6 +331,39 @@ int moe_combine(int32_t T, int32_t H, int32_t k, int32_t dtype, const void* expe
                 void* out, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * moe_ep_regroup -- the receiving side of an expert-parallel all-to-all-v
+ * dispatch (direction 0) and the sending side of its return (direction 1)
+ * [NKI: Background -- the router top-k feeds the all-to-all-v MoE dispatch
+ * path; TRT: Parameters local_expert_offset / local_num_experts, Returns --
+ * the tile-padded expert-contiguous layout; LMD: invokeMoeDispatch /
+ * invokeMoeCombine].
+ * A world of `world` ranks; this rank owns `local_experts` experts.
+ * counts [world][local_experts] int32 (device): rows rank s sends for local
+ * expert e.  recv [n_recv, H] holds them ordered by source rank, then expert,
+ * then the source's token order, n_recv = sum of counts (what every rank's
+ * route over all experts with tile 1, followed by moe_dispatch, sends to this
+ * rank).  Direction 0 writes padded [max_padded, H]: the rows ordered by local
+ * expert, then source rank, then token, each expert padded to `tile` rows
+ * (padding rows zero) -- exactly the layout moe_route gives this rank's
+ * experts for all ranks' tokens concatenated in rank order -- and
+ * padded_offsets [local_experts + 1], totals [2] (P, P / tile) and
+ * padded_to_recv [max_padded] (receive row of each padded row, -1 on padding;
+ * rows >= P untouched).  Direction 1 reads padded (the expert outputs in that
+ * layout) and writes recv (receive order), for the return all-to-all-v; the
+ * offsets, totals and padded_to_recv arguments are ignored.
+ * dtype MOE_BF16 | MOE_F32; H * element size a multiple of 16 bytes; recv and
+ * padded 16-byte aligned; tile a power of two <= 4096; world * local_experts
+ * <= 8192.  If the counts disagree with n_recv, or the padded rows exceed
+ * max_padded, nothing is moved and ws (optional, >= 64 bytes) records
+ * MOE_ERR_DEVICE_BOUNDS.  Reads the counts after waiting on the preceding
+ * kernel (programmatic dependent launch).
+ */
+int moe_ep_regroup(int32_t world, int32_t local_experts, int32_t H, int32_t dtype, int32_t tile, const int32_t* counts,
+                   int32_t direction, void* recv, int64_t n_recv, void* padded, int64_t max_padded,
+                   int32_t* padded_offsets, int32_t* totals, int32_t* padded_to_recv, void* ws, size_t ws_bytes,
+                   void* stream);
+
+/*
  * Workspace bytes of moe_rmsnorm_router_topk (header and the fp32 partial
  * logits of the K-split projection; depends on T, H and E).  The workspace
  * must be zero before its first use (moe_workspace_init).

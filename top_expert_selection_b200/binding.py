@@ -39,7 +39,7 @@ EXPORTED = (
     "moe_aux_loss_fwd", "moe_aux_loss_bwd", "moe_dispatch", "moe_combine",
     "moe_rmsnorm_router_topk_workspace_bytes", "moe_rmsnorm_router_topk", "moe_debug_wait_timeout",
     "moe_debug_sigmoid_proxy_error", "moe_route_no_alloc", "moe_route_no_alloc_status",
-    "moe_debug_no_alloc_record",
+    "moe_debug_no_alloc_record", "moe_ep_regroup",
 )
 
 
@@ -87,6 +87,7 @@ def lib() -> ctypes.CDLL:
             "moe_route_no_alloc": ([RP, P, P, P, P, P, P, P, P, P, P, P, P], ctypes.c_int),
             "moe_route_no_alloc_status": ([P, ctypes.POINTER(i32), ctypes.c_int], ctypes.c_int),
             "moe_debug_no_alloc_record": ([i32, P], ctypes.c_int),
+            "moe_ep_regroup": ([i32, i32, i32, i32, i32, P, i32, P, i64, P, i64, P, P, P, P, sz, P], ctypes.c_int),
             "moe_aux_workspace_bytes": ([i32, i32, ctypes.POINTER(sz)], ctypes.c_int),
             "moe_aux_scores": ([i32, i32, i32, i32, P, P, P, P, P, sz, P], ctypes.c_int),
             "moe_aux_loss_fwd": ([i32, i32, i32, i32, f32, P, P, P, P, sz, P], ctypes.c_int),
@@ -402,3 +403,26 @@ def route_no_alloc_status(clear: bool = True, stream=None) -> int:
     st = ctypes.c_int32(0)
     _check(lib().moe_route_no_alloc_status(_stream(stream), ctypes.byref(st), int(clear)), "moe_route_no_alloc_status")
     return int(st.value)
+
+
+# ---------------------------------------------------------------------------- expert-parallel exchange
+
+def ep_regroup_into(counts: torch.Tensor, recv: torch.Tensor, padded: torch.Tensor, tile: int, offsets: torch.Tensor,
+                    totals: torch.Tensor, padded_to_recv: torch.Tensor, ws: Optional[torch.Tensor] = None,
+                    stream=None) -> None:
+    """Receive order -> tile-padded expert layout (moe_ep_regroup, direction 0)."""
+    W, L = counts.shape
+    H = recv.shape[1]
+    _check(lib().moe_ep_regroup(W, L, H, _DT[recv.dtype], tile, _p(counts), 0, _p(recv), recv.shape[0], _p(padded),
+                                padded.shape[0], _p(offsets), _p(totals), _p(padded_to_recv), _p(ws),
+                                ctypes.c_size_t(0 if ws is None else ws.numel()), _stream(stream)), "moe_ep_regroup")
+
+
+def ep_ungroup_into(counts: torch.Tensor, padded: torch.Tensor, recv: torch.Tensor, tile: int,
+                    ws: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Tile-padded expert layout -> receive order (moe_ep_regroup, direction 1)."""
+    W, L = counts.shape
+    H = recv.shape[1]
+    _check(lib().moe_ep_regroup(W, L, H, _DT[recv.dtype], tile, _p(counts), 1, _p(recv), recv.shape[0], _p(padded),
+                                padded.shape[0], None, None, None, _p(ws),
+                                ctypes.c_size_t(0 if ws is None else ws.numel()), _stream(stream)), "moe_ep_regroup")
