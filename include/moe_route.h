@@ -92,6 +92,14 @@ typedef struct moe_route_params {
                                   global expert = it + local_expert_offset [TRT: Notes]); a
                                   selection of another shard's expert gets
                                   expanded_to_permuted = -1 */
+  int32_t num_fused_shared_experts; /* S >= 0 [TRT: num_fused_shared_experts -- extra fused
+                                  shared-expert slots appended per token].  Each token's S slots
+                                  follow its k routed ones: expert E + s, weight 1.0 (outside
+                                  selection, renormalisation and scaling); every token selects
+                                  every shared expert; the shared experts are local on every
+                                  shard, after its routed experts (local index L + s).  The
+                                  outputs then hold k + S slots per token and L + S local
+                                  experts; E + S <= MOE_MAX_EXPERTS, k + S <= MOE_MAX_TOPK */
 } moe_route_params;
 
 /* Human-readable name of a status code (static string). */
@@ -108,7 +116,8 @@ int moe_status(void* ws, void* stream, int32_t* status, int clear);
 
 /*
  * Upper bounds for the permutation outputs of moe_route:
- *   max_padded = T*k + min(E, T*k) * (tile - 1)   (rows of permuted_to_token)
+ *   max_padded = T*k' + min(E + S, T*k') * (tile - 1)   (rows of permuted_to_token;
+ *                k' = k + S slots per token, S fused shared experts)
  *   max_tiles  = max_padded / tile                (entries of the tile tables)
  * [TRT: tile_tokens_dim -- each expert's rows are padded to the tile].
  */
@@ -178,8 +187,12 @@ int moe_route_workspace_bytes(const moe_route_params* p, size_t* bytes);
  * MOE_ERR_UNSUPPORTED (E or k past the build limits, a group layout the
  * kernels do not map: with groups, a lane holds v in {2,3,4,5,6,8,12,16,24,32}
  * experts (the least with 32v >= E) and a group must span a power of two of
- * whole lanes or a lane whole groups), MOE_ERR_WORKSPACE, MOE_ERR_CUDA;
- * device timeout via moe_status.
+ * whole lanes or a lane whole groups; k + S past the slot limit or E + S past
+ * the expert limit), MOE_ERR_WORKSPACE (ws smaller than
+ * moe_route_workspace_bytes), MOE_ERR_CUDA (a launch failed).  Device-side
+ * errors (MOE_ERR_DEVICE_TIMEOUT from a bounded wait on a bulk copy) are not
+ * returned here: they are recorded in the status word at the start of ws and
+ * read with moe_status.
  */
 int moe_route(const moe_route_params* p, const void* logits, const void* bias, int32_t* topk_ids,
               void* topk_weights, int32_t* expert_counts, int32_t* padded_offsets,

@@ -113,6 +113,31 @@ def test_other_entry_points_validate():
     assert L.moe_debug_wait_timeout(1, 1000, d, ctypes.c_size_t(8), None) == B.MOE_ERR_WORKSPACE
 
 
+def test_fused_shared_experts_validation():
+    L = B.lib()
+    mp, mt = ctypes.c_int64(), ctypes.c_int64()
+    p = B.route_params(16, 8, 2, tile_tokens_dim=4, num_fused_shared_experts=2)
+    assert L.moe_route_capacity(ctypes.byref(p), ctypes.byref(mp), ctypes.byref(mt)) == 0
+    assert mp.value == 16 * 4 + min(64, 10) * 3 and mt.value == mp.value // 4
+    assert L.moe_route_capacity(ctypes.byref(B.route_params(16, 8, 2, num_fused_shared_experts=-1)),
+                                ctypes.byref(mp), ctypes.byref(mt)) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_route_capacity(ctypes.byref(B.route_params(16, 1020, 2, num_fused_shared_experts=5)),
+                                ctypes.byref(mp), ctypes.byref(mt)) == B.MOE_ERR_UNSUPPORTED
+    assert L.moe_route_capacity(ctypes.byref(B.route_params(16, 64, 30, num_fused_shared_experts=3)),
+                                ctypes.byref(mp), ctypes.byref(mt)) == B.MOE_ERR_UNSUPPORTED
+
+
+def test_ep_regroup_validates():
+    L = B.lib()
+    d = ctypes.c_void_p(16)
+    args = lambda W, Lx, H, dt, tile, direction: (W, Lx, H, dt, tile, d, direction, d, 4, d, 16, d, d, d, None, 0, None)
+    assert L.moe_ep_regroup(*args(0, 4, 8, 1, 4, 0)) == -1
+    assert L.moe_ep_regroup(*args(2, 4, 8, 1, 3, 0)) == -1      # tile not a power of two
+    assert L.moe_ep_regroup(*args(2, 4, 4, 1, 4, 0)) == -1      # 8-byte rows
+    assert L.moe_ep_regroup(*args(2, 4, 8, 1, 4, 2)) == -1      # no such direction
+    assert L.moe_ep_regroup(*args(64, 1024, 8, 1, 4, 0)) == B.MOE_ERR_UNSUPPORTED
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises((ValueError, RuntimeError)):

@@ -377,3 +377,45 @@ def test_route_expert_parallel_shard_bad_range():
         p = B.route_params(16, 8, 2, local_expert_offset=off, local_num_experts=nl)
         with pytest.raises(B.MoeError):
             B.Router(p)(torch.randn(16, 8, device="cuda"))
+
+
+@pytest.mark.parametrize("name,S,off,nl", [("dsv3", 1, 0, 0), ("dsv3", 2, 64, 64), ("mixtral", 2, 0, 0),
+                                           ("e64", 1, 16, 16), ("e64", 3, 0, 0)])
+def test_route_fused_shared_experts(name, S, off, nl):
+    """num_fused_shared_experts (trtllm_gen_routing, Parameters): the routed slots equal the plain route's,
+    each token's S appended slots hold experts E .. E+S-1 with weight 1.0, and the whole bookkeeping
+    (routed local experts, then the shared ones) equals the oracle's on the GPU's ids, bit-exactly."""
+    if name == "dsv3":
+        spec = W.DSV3_GROUPED_SIGMOID.with_(T=3000, seed=77)
+    elif name == "mixtral":
+        spec = W.MIXTRAL_ROUTE.with_(T=999, seed=78)
+    else:
+        spec = W.RouteSpec(T=777, E=64, k=6, score_fn=W.SOFTMAX, softmax_before_topk=1, n_group=0, topk_group=0,
+                           group_score_topn=2, renormalize=1, scaling_factor=1.0, tile_tokens_dim=16,
+                           logits_dtype=W.F32, bias_dtype=W.F32, weights_dtype=W.F32, seed=79)
+    inp = W.route_inputs(spec)
+    kw = dict(score_fn=spec.score_fn, softmax_before_topk=spec.softmax_before_topk, n_group=spec.n_group,
+              topk_group=spec.topk_group, group_score_topn=spec.group_score_topn, renormalize=spec.renormalize,
+              scaling_factor=spec.scaling_factor, tile_tokens_dim=spec.tile_tokens_dim,
+              logits_dtype=spec.logits_dtype, bias_dtype=spec.bias_dtype, weights_dtype=spec.weights_dtype,
+              local_expert_offset=off, local_num_experts=nl)
+    lg = inp["logits"].cuda()
+    b = inp["bias"].cuda() if inp["bias"] is not None else None
+    plain = B.Router(B.route_params(spec.T, spec.E, spec.k, **kw))(lg, b)
+    plain = {n: v.clone() for n, v in plain.items()}
+    r = B.Router(B.route_params(spec.T, spec.E, spec.k, num_fused_shared_experts=S, **kw))
+    got = r(lg, b)
+    torch.cuda.synchronize()
+    assert B.status(r.ws) == B.MOE_OK
+    k, E, T = spec.k, spec.E, spec.T
+    ids = to_np(got["ids"]).reshape(T, k + S)
+    w = got["weights"].float().cpu().numpy().reshape(T, k + S)
+    assert np.array_equal(ids[:, :k], to_np(plain["ids"]).reshape(T, k))
+    assert np.array_equal(w[:, :k], plain["weights"].float().cpu().numpy().reshape(T, k))
+    assert np.all(ids[:, k:] == np.arange(E, E + S)) and np.all(w[:, k:] == 1.0)
+    bk = oracle.route_bookkeeping(ids, E, spec.tile_tokens_dim, off, nl or E, num_shared=S)
+    P, nt = int(bk["totals"][0]), int(bk["totals"][1])
+    assert to_np(got["totals"]).tolist() == [P, nt]
+    for name_, n in (("counts", (nl or E) + S), ("offsets", (nl or E) + S + 1), ("e2p", T * (k + S)),
+                     ("p2t", P), ("tile_expert", nt), ("tile_mn_limit", nt)):
+        assert np.array_equal(to_np(got[name_])[:n], bk[name_][:n]), f"{name_} differs from the oracle"

@@ -58,6 +58,7 @@ class RouteParams(ctypes.Structure):
         ("tile_tokens_dim", ctypes.c_int32), ("logits_dtype", ctypes.c_int32), ("bias_dtype", ctypes.c_int32),
         ("weights_dtype", ctypes.c_int32),
         ("local_expert_offset", ctypes.c_int32), ("local_num_experts", ctypes.c_int32),
+        ("num_fused_shared_experts", ctypes.c_int32),
     ]
 
 
@@ -154,11 +155,11 @@ def route_params(T: int, E: int, k: int, *, score_fn: int = SOFTMAX, softmax_bef
                  n_group: int = 0, topk_group: int = 0, group_score_topn: int = 2, renormalize: int = 1,
                  scaling_factor: float = 1.0, tile_tokens_dim: int = 8, logits_dtype: int = F32,
                  bias_dtype: int = F32, weights_dtype: int = F32, local_expert_offset: int = 0,
-                 local_num_experts: int = 0) -> RouteParams:
+                 local_num_experts: int = 0, num_fused_shared_experts: int = 0) -> RouteParams:
     """local_num_experts == 0: every expert is local (single GPU)."""
     return RouteParams(T, E, k, score_fn, softmax_before_topk, n_group, topk_group, group_score_topn,
                        renormalize, scaling_factor, tile_tokens_dim, logits_dtype, bias_dtype, weights_dtype,
-                       local_expert_offset, local_num_experts)
+                       local_expert_offset, local_num_experts, num_fused_shared_experts)
 
 
 def route_capacity(p: RouteParams):
@@ -179,8 +180,9 @@ class Router:
         with torch.cuda.device(self.device):
             _check(L.moe_route_workspace_bytes(ctypes.byref(p), ctypes.byref(nb)), "moe_route_workspace_bytes")
         dev = self.device
-        T, E, k = p.num_tokens, p.num_experts, p.top_k
-        L_e = p.local_num_experts if p.local_num_experts > 0 else E  # the local experts' bookkeeping
+        T, E, S = p.num_tokens, p.num_experts, p.num_fused_shared_experts
+        k = p.top_k + S  # slots per token: the routed ones, then the fused shared ones
+        L_e = (p.local_num_experts if p.local_num_experts > 0 else E) + S  # the local experts' bookkeeping
         self.ws = make_workspace(nb.value, dev)
         self.out = {
             "ids": torch.empty((T, k), dtype=torch.int32, device=dev),

@@ -78,11 +78,12 @@ struct RouteArgs {
   uint8_t* table;    // [G][row_stride]: per-segment expert counts (cnt_bytes wide)
   uint32_t* gtot;    // [NG][E]: per-group expert counts (groups of GS segments), zero between calls
   int T, E, k;
+  int S, kt, E2;     // fused shared experts (ids E .. E+S-1), slots per token k + S, experts counted E + S
   int score_fn, pre, grouped, n_group, topk_group, topn;
   int renorm;
   float scale;
   int tile;          // power of two
-  uint32_t kinv;     // ceil(2^32 / k): item -> token by a multiply-high
+  uint32_t kinv;     // ceil(2^32 / kt): item -> token by a multiply-high
   int logits_dtype, bias_dtype, weights_dtype;
   int has_bias;
   int G, B;          // segments, tokens per segment (segment c: [c*B, min(T, (c+1)*B)))
@@ -121,7 +122,7 @@ __host__ __device__ inline SelSmem sel_smem_layout(int E, int MW, int B, int k, 
   SelSmem L;
   int o = 0;
   L.masks = o;
-  o += E * MW * 4;
+  o += ((E * MW * 4) + 15) & ~15;  // every region starts on 16 bytes (the constants are read as 16-byte vectors)
   L.ids = o;
   o += ((B * k * 2) + 15) & ~15;
   L.bias = o;
@@ -146,15 +147,20 @@ __device__ __forceinline__ float stage_val(const RouteArgs& a, const uint8_t* ro
 
 __device__ __forceinline__ float sigmoid_f32(float x) { return 1.0f / (1.0f + expf(-x)); }
 
-// expert e belongs to this shard: it gets rows, slots and tiles
+// expert e belongs to this shard: it gets rows, slots and tiles (a fused
+// shared expert, e >= E, is local on every shard)
 __device__ __forceinline__ bool is_local(const RouteArgs& a, int e) {
-  return (unsigned)(e - a.loc_off) < (unsigned)a.loc_n;
+  return (unsigned)(e - a.loc_off) < (unsigned)a.loc_n || e >= a.E;
+}
+// the local index of a local expert: the shard's routed experts, then the shared ones
+__device__ __forceinline__ int local_index(const RouteArgs& a, int e) {
+  return e >= a.E ? a.loc_n + (e - a.E) : e - a.loc_off;
 }
 
 // One selection of expert e by the segment's token lt at slot j: the id in the
 // segment's list, the token's bit in e's mask.
 __device__ __forceinline__ void mark(const RouteArgs& a, uint32_t* masks, uint16_t* ids_s, int lt, int j, int e) {
-  ids_s[lt * a.k + j] = (uint16_t)e;
+  ids_s[lt * a.kt + j] = (uint16_t)e;
   atomicOr(&masks[e * a.MW + (lt >> 5)], 1u << (lt & 31));
 }
 
@@ -340,7 +346,7 @@ __device__ void select_token_warp(const RouteArgs& a, const uint8_t* row, long l
     v = v * a.scale;
   }
   if (has_slot) {
-    const size_t o = (size_t)t * a.k + lane;
+    const size_t o = (size_t)t * a.kt + lane;
     a.ids[o] = my_id;
     store_from_f32(a.weights, a.weights_dtype, o, v);
     if ((unsigned)my_id < (unsigned)E) mark(a, masks, ids_s, lt, lane, my_id); else record_bounds(a.hdr);
@@ -467,7 +473,7 @@ __device__ void select_token_thread(const RouteArgs& a, const uint8_t* row, long
   for (int j = 0; j < EMAX; ++j) {
     if (j < a.k) {
       const float w = a.renorm ? (val[j] / norm) * a.scale : val[j] * a.scale;
-      const size_t o = (size_t)t * a.k + j;
+      const size_t o = (size_t)t * a.kt + j;
       a.ids[o] = sel[j];
       store_from_f32(a.weights, a.weights_dtype, o, w);
       if ((unsigned)sel[j] < (unsigned)E) mark(a, masks, ids_s, lt, j, sel[j]); else record_bounds(a.hdr);
@@ -792,7 +798,7 @@ __device__ unsigned select_quad_fast(const RouteArgs& a, const uint8_t* rows, in
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
     if (rk[r] < a.k) {
-      const size_t o = (size_t)t * a.k + rk[r];
+      const size_t o = (size_t)t * a.kt + rk[r];
       const int e = packed_expert(kk[r]);
       const float sv = cs[g + 8 * r];
       a.ids[o] = e;
@@ -853,20 +859,20 @@ __device__ void scan_padded_offsets(const int* cnt, int* offs, int E, int tile) 
 // After a block's selections: park (expert, rank in the segment) of every
 // selection in expanded_to_permuted, and write the segment's counts row.
 __device__ void finish_segment(const RouteArgs& a, const uint32_t* masks, const uint16_t* ids_s, int n, int t_begin) {
-  const int n_items = n * a.k;
-  const long long i_begin = (long long)t_begin * a.k;
+  const int n_items = n * a.kt;
+  const long long i_begin = (long long)t_begin * a.kt;
   for (int i = threadIdx.x; i < n_items; i += blockDim.x) {
     const int e = ids_s[i];
     // token of item i: i / k (i < 2^13, so the multiply-high is exact)
-    const int lt = a.k == 1 ? i : (int)__umulhi((uint32_t)i, a.kinv);
-    const uint32_t* m = masks + min(e, a.E - 1) * a.MW;  // ids were range-checked when selected
+    const int lt = a.kt == 1 ? i : (int)__umulhi((uint32_t)i, a.kinv);
+    const uint32_t* m = masks + min(e, a.E2 - 1) * a.MW;  // ids were range-checked when selected
     int r = __popc(m[lt >> 5] & ((1u << (lt & 31)) - 1u));
     for (int w = 0; w < (lt >> 5); ++w) r += __popc(m[w]);
-    a.e2p[i_begin + i] = e < a.E ? (e | (r << 16)) : -1;
+    a.e2p[i_begin + i] = e < a.E2 ? (e | (r << 16)) : -1;
   }
   uint8_t* trow = a.table + (size_t)blockIdx.x * a.row_stride;
-  uint32_t* grow = a.gtot + (size_t)(blockIdx.x / a.GS) * a.E;
-  for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+  uint32_t* grow = a.gtot + (size_t)(blockIdx.x / a.GS) * a.E2;
+  for (int e = threadIdx.x; e < a.E2; e += blockDim.x) {
     int c = 0;
     for (int w = 0; w < a.MW; ++w) c += __popc(masks[e * a.MW + w]);
     if (a.cnt_bytes == 1) trow[e] = (uint8_t)c;
@@ -895,7 +901,7 @@ __global__ void __launch_bounds__((FAST_ESZ > 0) ? kFastWarpsMax * 32 : kGeneric
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const int t_begin = c * a.B;
   const int n = max(0, min(a.T, t_begin + a.B) - t_begin);
-  const SelSmem L = sel_smem_layout(E, a.MW, a.B, a.k, kFast ? 1 : 0, FV, a.row_bytes, nwarps, a.slots);
+  const SelSmem L = sel_smem_layout(a.E2, a.MW, a.B, a.kt, kFast ? 1 : 0, FV, a.row_bytes, nwarps, a.slots);
   uint32_t* masks = reinterpret_cast<uint32_t*>(smem + L.masks);
   uint16_t* ids_s = reinterpret_cast<uint16_t*>(smem + L.ids);
   float* bias_s = reinterpret_cast<float*>(smem + L.bias);
@@ -910,7 +916,7 @@ __global__ void __launch_bounds__((FAST_ESZ > 0) ? kFastWarpsMax * 32 : kGeneric
   // preceding kernel that lets its dependents start early must not write it);
   // the logits are read after the wait.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  for (int i = threadIdx.x; i < E * a.MW; i += blockDim.x) masks[i] = 0u;
+  for (int i = threadIdx.x; i < a.E2 * a.MW; i += blockDim.x) masks[i] = 0u;
   const int nq = (n + 3) >> 2;
   if constexpr (kFast) {
     if (lane == 0) {
@@ -1015,6 +1021,22 @@ __global__ void __launch_bounds__((FAST_ESZ > 0) ? kFastWarpsMax * 32 : kGeneric
       select_token_warp<VPL>(a, lg_bytes + ((size_t)t_begin + lt) * a.row_bytes, t_begin + lt, lt, bias_s, masks,
                              ids_s, lane);
   }
+  // the fused shared experts' slots: every token of the segment, after its k
+  // routed slots, expert E + s with weight 1.0 (their masks hold every token)
+  if (a.S > 0) {
+    for (int i = threadIdx.x; i < n * a.S; i += blockDim.x) {
+      const int lt = i / a.S, s = i % a.S;
+      const size_t o = ((size_t)t_begin + lt) * a.kt + a.k + s;
+      a.ids[o] = E + s;
+      store_from_f32(a.weights, a.weights_dtype, o, 1.0f);
+      ids_s[lt * a.kt + a.k + s] = (uint16_t)(E + s);
+    }
+    for (int i = threadIdx.x; i < a.S * a.MW; i += blockDim.x) {
+      const int s = i / a.MW, w = i % a.MW;
+      const int lo = w * 32, cntw = max(0, min(32, n - lo));
+      masks[(E + s) * a.MW + w] = cntw >= 32 ? 0xffffffffu : ((1u << cntw) - 1u);
+    }
+  }
   __syncthreads();
   finish_segment(a, masks, ids_s, n, t_begin);
 }
@@ -1026,7 +1048,7 @@ __host__ __device__ inline int perm_smem_bytes(int E) { return (3 * E + 1) * 4 +
 
 __global__ void __launch_bounds__(kPermThreads, 1) route_permute_kernel(RouteArgs a) {
   extern __shared__ __align__(128) uint8_t psmem[];
-  const int E = a.E;
+  const int E = a.E2;  // experts counted: the routed ones, then the fused shared ones
   int* cnt = reinterpret_cast<int*>(psmem);
   int* base = cnt + E;
   int* offs = base + E;  // [E + 1], then one flag word
@@ -1034,8 +1056,8 @@ __global__ void __launch_bounds__(kPermThreads, 1) route_permute_kernel(RouteArg
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int t_begin = c * a.B;
   const int n = max(0, min(a.T, t_begin + a.B) - t_begin);
-  const int n_items = n * a.k;
-  const long long i_begin = (long long)t_begin * a.k;
+  const int n_items = n * a.kt;
+  const long long i_begin = (long long)t_begin * a.kt;
 
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");  // the table and the parked ranks are the selection's output
@@ -1106,13 +1128,15 @@ __global__ void __launch_bounds__(kPermThreads, 1) route_permute_kernel(RouteArg
   scan_padded_offsets(cnt, offs, E, a.tile);
   const int P = offs[E];
   if (c == 0) {
-    // the shard's experts (those before it have no rows: offs[loc_off] == 0)
-    for (int le = threadIdx.x; le < a.loc_n; le += blockDim.x) {
-      a.counts[le] = cnt[a.loc_off + le];
-      a.offsets[le] = offs[a.loc_off + le];
+    // the shard's experts, then the shared ones (the others have no rows:
+    // offs[loc_off] == 0, and the shared experts follow the shard's)
+    for (int le = threadIdx.x; le < a.loc_n + a.S; le += blockDim.x) {
+      const int e = le < a.loc_n ? a.loc_off + le : a.E + (le - a.loc_n);
+      a.counts[le] = cnt[e];
+      a.offsets[le] = offs[e];
     }
     if (threadIdx.x == 0) {
-      a.offsets[a.loc_n] = P;
+      a.offsets[a.loc_n + a.S] = P;
       a.totals[0] = P;
       a.totals[1] = P / a.tile;
     }
@@ -1137,7 +1161,7 @@ __global__ void __launch_bounds__(kPermThreads, 1) route_permute_kernel(RouteArg
       const int slot = offs[e] + base[e] + rk;
       a.e2p[i_begin + i] = slot;
       // token of item i: t_begin + i / k
-      const int lt = a.k == 1 ? i : (int)__umulhi((uint32_t)i, a.kinv);
+      const int lt = a.kt == 1 ? i : (int)__umulhi((uint32_t)i, a.kinv);
       if ((unsigned)slot < (unsigned)a.max_padded) a.p2t[slot] = t_begin + lt;
       else record_bounds(a.hdr);
     }
@@ -1154,7 +1178,7 @@ __global__ void __launch_bounds__(kPermThreads, 1) route_permute_kernel(RouteArg
   for (int e = c * nwarps + warp; e < E; e += a.G * nwarps) {
     const int row0 = offs[e], row1 = offs[e + 1], lim = row0 + cnt[e];
     for (int tc = row0 / a.tile + lane; tc < row1 / a.tile; tc += 32) {
-      a.tile_expert[tc] = e - a.loc_off;  // the local expert (batch index)
+      a.tile_expert[tc] = local_index(a, e);  // the local expert (batch index)
       a.tile_mn[tc] = min((tc + 1) * a.tile, lim);
     }
     for (int r = lim + lane; r < row1; r += 32) a.p2t[r] = -1;
@@ -1209,9 +1233,11 @@ int validate(const moe_route_params* p) {
     if ((long long)p->top_k > (long long)kept * gs) return MOE_ERR_INVALID_ARG;
     if (p->group_score_topn > 2) return MOE_ERR_UNSUPPORTED;
   }
-  if (p->num_experts > MOE_MAX_EXPERTS || p->top_k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
-  const long long items = (long long)p->num_tokens * p->top_k;
-  if (items + std::min<long long>(p->num_experts, items) * (p->tile_tokens_dim - 1) > 0x7fffffffLL)
+  if (p->num_fused_shared_experts < 0) return MOE_ERR_INVALID_ARG;
+  const int S = p->num_fused_shared_experts;
+  if (p->num_experts + S > MOE_MAX_EXPERTS || p->top_k + S > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+  const long long items = (long long)p->num_tokens * (p->top_k + S);
+  if (items + std::min<long long>(p->num_experts + S, items) * (p->tile_tokens_dim - 1) > 0x7fffffffLL)
     return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
@@ -1306,8 +1332,8 @@ extern "C" int moe_route_capacity(const moe_route_params* p, int64_t* max_padded
   const int v = validate(p);
   if (v != MOE_OK) return v;
   if (!max_padded || !max_tiles) return MOE_ERR_INVALID_ARG;
-  const int64_t rows = (int64_t)p->num_tokens * p->top_k;
-  const int64_t nz = std::min<int64_t>(rows, p->num_experts);
+  const int64_t rows = (int64_t)p->num_tokens * (p->top_k + p->num_fused_shared_experts);
+  const int64_t nz = std::min<int64_t>(rows, p->num_experts + p->num_fused_shared_experts);
   *max_padded = rows + nz * (p->tile_tokens_dim - 1);
   *max_tiles = *max_padded / p->tile_tokens_dim;
   return MOE_OK;
@@ -1319,7 +1345,7 @@ extern "C" int moe_route_workspace_bytes(const moe_route_params* p, size_t* byte
   if (!bytes) return MOE_ERR_INVALID_ARG;
   const DevInfo d = device_info();
   if (d.sms <= 0) return MOE_ERR_CUDA;
-  *bytes = ws_bytes_for(p->num_tokens, p->num_experts, d.sms);
+  *bytes = ws_bytes_for(p->num_tokens, p->num_experts + p->num_fused_shared_experts, d.sms);
   return MOE_OK;
 }
 
@@ -1338,7 +1364,7 @@ extern "C" int moe_route(const moe_route_params* p, const void* logits, const vo
   if (mode < 0) return MOE_ERR_UNSUPPORTED;
   const DevInfo d = device_info();
   if (d.sms <= 0) return MOE_ERR_CUDA;
-  if (!ws || ws_bytes < ws_bytes_for(T, p->num_experts, d.sms)) return MOE_ERR_WORKSPACE;
+  if (!ws || ws_bytes < ws_bytes_for(T, p->num_experts + p->num_fused_shared_experts, d.sms)) return MOE_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(ws) & 15) != 0) return MOE_ERR_WORKSPACE;
 
   RouteArgs a = {};
@@ -1358,6 +1384,9 @@ extern "C" int moe_route(const moe_route_params* p, const void* logits, const vo
   a.T = T;
   a.E = p->num_experts;
   a.k = p->top_k;
+  a.S = p->num_fused_shared_experts;
+  a.kt = a.k + a.S;
+  a.E2 = a.E + a.S;
   a.score_fn = p->score_fn;
   a.pre = p->softmax_before_topk ? 1 : 0;
   a.grouped = (p->n_group > 1 && p->topk_group > 0) ? 1 : 0;
@@ -1367,7 +1396,7 @@ extern "C" int moe_route(const moe_route_params* p, const void* logits, const vo
   a.renorm = p->renormalize ? 1 : 0;
   a.scale = p->scaling_factor;
   a.tile = p->tile_tokens_dim;
-  a.kinv = p->top_k > 1 ? (uint32_t)((0x100000000ull + (uint64_t)p->top_k - 1) / (uint64_t)p->top_k) : 0u;
+  a.kinv = a.kt > 1 ? (uint32_t)((0x100000000ull + (uint64_t)a.kt - 1) / (uint64_t)a.kt) : 0u;
   a.logits_dtype = p->logits_dtype;
   a.bias_dtype = p->bias_dtype;
   a.weights_dtype = p->weights_dtype;
@@ -1387,7 +1416,7 @@ extern "C" int moe_route(const moe_route_params* p, const void* logits, const vo
   a.loc_n = p->local_num_experts > 0 ? p->local_num_experts : p->num_experts;
   a.row_bytes = p->num_experts * esize(p->logits_dtype);
   a.cnt_bytes = a.B <= 255 ? 1 : 2;
-  a.row_stride = (int)table_row_stride(a.E, a.cnt_bytes);
+  a.row_stride = (int)table_row_stride(a.E2, a.cnt_bytes);
   a.timeout_ns = kDefaultTimeoutNs;
 
   const bool fast = fast_path_ok(p, logits);
@@ -1401,10 +1430,11 @@ extern "C" int moe_route(const moe_route_params* p, const void* logits, const vo
   }
   const int V = a.E / 8;
   a.slots = (fast && (a.B + 3) / 4 > threads / 32) ? 2 : 1;
-  const SelSmem L = sel_smem_layout(a.E, a.MW, a.B, a.k, fast ? 1 : 0, fast ? V : 1, a.row_bytes, threads / 32,
+  const SelSmem L = sel_smem_layout(a.E2, a.MW, a.B, a.kt, fast ? 1 : 0, fast ? V : 1, a.row_bytes, threads / 32,
                                     a.slots);
   if (L.total > d.smem_optin) return MOE_ERR_UNSUPPORTED;
-  const int psmem = perm_smem_bytes(a.E);
+  if ((L.ids | L.bias | L.cb | L.delta | L.warp0) & 15) return MOE_ERR_UNSUPPORTED;  // layout invariant
+  const int psmem = perm_smem_bytes(a.E2);
   if (psmem > d.smem_optin) return MOE_ERR_UNSUPPORTED;
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -1560,7 +1590,8 @@ extern "C" int moe_route_no_alloc(const moe_route_params* p, const void* logits,
   if (v != MOE_OK) return v;
   const DevInfo d = device_info();
   if (d.sms <= 0) return MOE_ERR_CUDA;
-  if (ws_bytes_for(p->num_tokens, p->num_experts, d.sms) > kStaticScratchBytes) return MOE_ERR_WORKSPACE;
+  if (ws_bytes_for(p->num_tokens, p->num_experts + p->num_fused_shared_experts, d.sms) > kStaticScratchBytes)
+    return MOE_ERR_WORKSPACE;
   int dev = 0;
   if (current_device(&dev) != MOE_OK) return MOE_ERR_CUDA;
   void* ws = scratch_address(dev, reinterpret_cast<cudaStream_t>(stream));
