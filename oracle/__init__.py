@@ -57,6 +57,7 @@ def _lib():
         L.oracle_aux_loss_fwd.argtypes = [i32, i32, i32, i32, f32, P, P, P]
         L.oracle_aux_loss_bwd.argtypes = [i32, i32, i32, i32, f32, f32, P, P, P, P]
         L.oracle_aux_scores_bwd.argtypes = [i32, i32, i32, P, P, P]
+        L.oracle_aux_scores_bwd_logits.argtypes = [i32, i32, i32, P, P, P]
         L.oracle_route_weights_bwd.argtypes = [i32, i32, i32, i32, i32, i32, f32, P, P, P, P]
         L.oracle_dispatch.argtypes = [i32, i32, i32, P, P, P, i32, P]
         L.oracle_combine.argtypes = [i32, i32, i32, P, P, P, i32, P]
@@ -73,7 +74,8 @@ def _lib():
         L.oracle_f64_to_bf16.restype = ctypes.c_uint16
         for name in ("oracle_route_select", "oracle_route_capacity", "oracle_route_bookkeeping",
                      "oracle_route_bookkeeping_shared", "oracle_append_shared",
-                     "oracle_aux_scores", "oracle_aux_loss_fwd", "oracle_aux_loss_bwd", "oracle_aux_scores_bwd", "oracle_route_weights_bwd",
+                     "oracle_aux_scores", "oracle_aux_loss_fwd", "oracle_aux_loss_bwd", "oracle_aux_scores_bwd", "oracle_aux_scores_bwd_logits",
+                     "oracle_route_weights_bwd",
                      "oracle_dispatch", "oracle_combine", "oracle_combine_f32", "oracle_ep_regroup", "oracle_rmsnorm_router_topk"):
             getattr(L, name).restype = i32
         _lib_handle = L
@@ -247,6 +249,18 @@ def route_weights_bwd(logits, ids, grad_weights, *, score_fn: int, softmax_befor
     _check(_lib().oracle_route_weights_bwd(T, E, k, int(score_fn), int(softmax_before_topk), int(renormalize),
                                            float(scaling_factor), _ptr(lg), _ptr(idv), _ptr(gw), _ptr(gl)),
            "route_weights_bwd")
+    return gl
+
+
+def aux_scores_bwd_logits(logits, grad_probs, score_fn: int = 0) -> np.ndarray:
+    """dL/dlogits of the aux scores (softmax, or sigmoid over the row sum) given dL/dprobs, the scores
+    recomputed from the logits."""
+    x = np.ascontiguousarray(as_numpy(logits), dtype=np.float32)
+    g = np.ascontiguousarray(as_numpy(grad_probs), dtype=np.float32)
+    T, E = x.shape
+    gl = np.zeros((T, E), np.float32)
+    _check(_lib().oracle_aux_scores_bwd_logits(T, E, int(score_fn), _ptr(x), _ptr(g), _ptr(gl)),
+           "aux_scores_bwd_logits")
     return gl
 
 

@@ -561,6 +561,60 @@ int oracle_aux_scores_bwd(int T, int E, int score_fn, const float* probs, const 
 }
 
 /*
+ * Backward of the aux scores from the logits [TE: Description,
+ * fused_compute_score_for_moe_aux_loss, "both forward and backward"; I/O
+ * Contract, score_function "softmax" or "sigmoid"]: the vector-Jacobian
+ * product of the forward's scores p(x) with the upstream gradient g, the
+ * scores recomputed from the logits (READING: for sigmoid the scores are the
+ * sigmoids divided by their row sum, as the forward states, so the row sum --
+ * which the probs do not carry -- comes from the logits).
+ *   softmax: p = softmax(x);          grad_i = p_i * (g_i - sum_e g_e p_e)
+ *   sigmoid: s = sigmoid(x), S = sum s, p = s / S;
+ *            dp_e/dx_i = s_i (1 - s_i) (delta_ei - p_e) / S
+ *            grad_i = s_i (1 - s_i) / S * (g_i - sum_e g_e p_e)
+ * All in double from the fp32 inputs, rounded once.
+ */
+int oracle_aux_scores_bwd_logits(int T, int E, int score_fn, const float* logits, const float* grad_probs,
+                                 float* grad_logits) {
+  if (T < 0 || E <= 0) return -1;
+  if (score_fn != ORC_SOFTMAX && score_fn != ORC_SIGMOID) return -1;
+  double* p = (double*)malloc(sizeof(double) * (size_t)E);
+  double* d = (double*)malloc(sizeof(double) * (size_t)E);  /* dp_i/dx_i without the -p_i part */
+  for (int t = 0; t < T; ++t) {
+    const float* x = logits + (size_t)t * E;
+    const float* g = grad_probs + (size_t)t * E;
+    double sum = 0.0;
+    if (score_fn == ORC_SOFTMAX) {
+      double m = x[0];
+      for (int e = 1; e < E; ++e) m = x[e] > m ? x[e] : m;
+      for (int e = 0; e < E; ++e) {
+        p[e] = exp((double)x[e] - m);
+        sum += p[e];
+      }
+      for (int e = 0; e < E; ++e) {
+        p[e] /= sum;
+        d[e] = p[e];
+      }
+    } else {
+      for (int e = 0; e < E; ++e) {
+        p[e] = 1.0 / (1.0 + exp(-(double)x[e]));
+        sum += p[e];
+      }
+      for (int e = 0; e < E; ++e) {
+        d[e] = p[e] * (1.0 - p[e]) / sum;
+        p[e] /= sum;
+      }
+    }
+    double dot = 0.0;
+    for (int e = 0; e < E; ++e) dot += (double)g[e] * p[e];
+    for (int e = 0; e < E; ++e) grad_logits[(size_t)t * E + e] = (float)(d[e] * ((double)g[e] - dot));
+  }
+  free(p);
+  free(d);
+  return 0;
+}
+
+/*
  * Dispatch [LMD: invokeMoeDispatch]: copy each token's hidden row to each of
  * its k permuted rows; padding rows below P (p2t == -1) are zero (READING);
  * rows at or past P are left untouched.  Rows are raw 16-bit elements.

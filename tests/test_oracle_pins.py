@@ -475,6 +475,55 @@ def test_aux_scores_backward_special_cases():
         oracle.aux_scores_bwd(probs, onehot, score_fn=W.SIGMOID)
 
 
+@pytest.mark.parametrize("score_fn", [W.SOFTMAX, W.SIGMOID])
+def test_aux_scores_backward_from_logits_finite_differences(score_fn):
+    """aux_scores_bwd_logits is d/dlogits of sum_t sum_e p(l_t)_e * G[t,e], with p the softmax or the
+    sigmoids over their row sum (central differences of a float64 forward written here from that
+    definition)."""
+    T, E = 4, 11
+    rng = np.random.default_rng(21 + score_fn)
+    lg = (rng.standard_normal((T, E)) * 2).astype(np.float32)
+    G = rng.standard_normal((T, E)).astype(np.float32)
+    gl = oracle.aux_scores_bwd_logits(lg, G, score_fn=score_fn)
+
+    def f64(x):
+        if score_fn == W.SOFTMAX:
+            z = np.exp(x - x.max(1, keepdims=True))
+        else:
+            z = 1.0 / (1.0 + np.exp(-x))
+        return float(((z / z.sum(1, keepdims=True)) * G.astype(np.float64)).sum())
+
+    x0 = lg.astype(np.float64)
+    h = 1e-6
+    fd = np.zeros_like(x0)
+    for t in range(T):
+        for e in range(E):
+            xp = x0.copy(); xp[t, e] += h
+            xm = x0.copy(); xm[t, e] -= h
+            fd[t, e] = (f64(xp) - f64(xm)) / (2 * h)
+    np.testing.assert_allclose(gl, fd, rtol=2e-5, atol=2e-7)
+
+
+def test_aux_scores_backward_from_logits_special_cases():
+    """Normalised scores sum to 1 for any logits, so a constant upstream gradient moves no logit and a
+    single expert (E = 1) has no gradient; for softmax, the entry that recomputes the scores agrees with
+    the one given the probs; saturated sigmoids (|x| = 30) leave finite gradients."""
+    rng = np.random.default_rng(6)
+    lg = rng.standard_normal((5, 10)).astype(np.float32)
+    for sf in (W.SOFTMAX, W.SIGMOID):
+        z = oracle.aux_scores_bwd_logits(lg, np.full_like(lg, -1.75), score_fn=sf)
+        assert np.all(np.abs(z) <= 1e-7)
+        one = oracle.aux_scores_bwd_logits(lg[:, :1].copy(), rng.standard_normal((5, 1)).astype(np.float32), sf)
+        assert np.all(one == 0)
+    G = rng.standard_normal(lg.shape).astype(np.float32)
+    a = oracle.aux_scores_bwd_logits(lg, G, score_fn=W.SOFTMAX)
+    b = oracle.aux_scores_bwd(oracle.aux_scores(lg, 2)["probs"], G)
+    np.testing.assert_allclose(a, b, rtol=1e-5, atol=1e-7)
+    sat = np.array([[30.0, -30.0, 0.0, 30.0]], np.float32)
+    g = oracle.aux_scores_bwd_logits(sat, np.array([[1.0, 2.0, 3.0, 4.0]], np.float32), score_fn=W.SIGMOID)
+    assert np.all(np.isfinite(g)) and abs(g[0, 1]) < 1e-12 and g[0, 2] != 0
+
+
 def test_aux_sigmoid_scores_closed_forms():
     E = 8
     sc = oracle.aux_scores(np.zeros((2, E), np.float32), 2, score_fn=W.SIGMOID)
