@@ -610,6 +610,8 @@ def secondary_rows(dev, hbm):
                                           z[4])) for z in sets], 20, stream)
     rows["aux_scores_bwd_us"] = _time_calls(
         [(lambda z=z: B.aux_scores_bwd_into(z[2]["probs"], z[4], z[5])) for z in sets], 20, stream)
+    rows["aux_scores_bwd_sigmoid_from_logits_us"] = _time_calls(
+        [(lambda z=z: B.aux_scores_bwd_logits_into(z[0], z[4], z[5], score_fn=W.SIGMOID)) for z in sets], 20, stream)
     del sets
     # the headline workload routed for one expert-parallel shard of four (experts 64..127): selection of
     # all 256 experts, bookkeeping of the shard's 64 (24 rotated logit sets, as the headline)
@@ -655,6 +657,18 @@ def secondary_rows(dev, hbm):
         [(lambda z=z: B.rmsnorm_router_topk_into(z[0], z[1], z[2], z[3], d.k, d.eps, d.act, z[4]["out_norm"],
                                                  z[4]["ids"], z[4]["affinities"], None, z[4]["ws"]))
          for z in dsets], 20, stream)
+    # decode with 384 experts (T=128, H=7168, k=8; two rounds of 256 in the top-k stage)
+    d384 = W.DECODE_FUSED.with_(E=384, seed=91)
+    di = W.decode_inputs(d384)
+    dsets = []
+    for _ in range(16):
+        x, gam, Wm, bb = (di[n].to(dev) for n in ("hidden", "gamma", "W", "bias"))
+        dsets.append((x, gam, Wm, bb, B.rmsnorm_router_topk(x, gam, Wm, bb, k=d384.k)))
+    rows["decode_e384_us"] = _time_calls(
+        [(lambda z=z: B.rmsnorm_router_topk_into(z[0], z[1], z[2], z[3], d384.k, d384.eps, d384.act,
+                                                 z[4]["out_norm"], z[4]["ids"], z[4]["affinities"], None,
+                                                 z[4]["ws"])) for z in dsets], 20, stream)
+    del dsets
     rows["note"] = ("us per call, device time of CUDA-graph replays over input/output sets rotated past the "
                     "126 MB L2 (dispatch/combine inputs exceed it alone)")
     return rows

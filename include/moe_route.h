@@ -290,11 +290,28 @@ int moe_route_weights_bwd(const moe_route_params* p, const void* logits, const i
  *   grad_logits[t,e] = p[t,e] * (grad_probs[t,e] - sum_j p[t,j] grad_probs[t,j])
  * probs, grad_probs, grad_logits [T,E] fp32 (probs as moe_aux_scores wrote
  * them).  score_fn MOE_SIGMOID returns MOE_ERR_UNSUPPORTED: the sigmoid scores
- * normalised by their row sum need that sum, which the probs do not carry.
+ * normalised by their row sum need that sum, which the probs do not carry
+ * (moe_aux_scores_bwd_logits computes it from the logits).
  * No workspace; returns MOE_ERR_INVALID_ARG for bad sizes or null pointers.
  */
 int moe_aux_scores_bwd(int32_t T, int32_t E, int32_t score_fn, const float* probs, const float* grad_probs,
                        float* grad_logits, void* stream);
+
+/*
+ * moe_aux_scores_bwd_logits -- backward of the aux scores from the logits
+ * [TE: Description, fused_compute_score_for_moe_aux_loss, forward and
+ * backward; I/O Contract, score_function "softmax" or "sigmoid"]: the scores
+ * are recomputed from the logits as moe_aux_scores computes them, so the
+ * sigmoid scores (divided by their row sum) have a backward too:
+ *   softmax: p = softmax(x);             grad = p * (g - sum_e p_e g_e)
+ *   sigmoid: s = sigmoid(x), S = sum s;  grad = s (1 - s) / S * (g - sum_e p_e g_e)
+ * logits, grad_probs (dL/dprobs), grad_logits [T,E] fp32, device,
+ * caller-owned; rows may start anywhere (16-byte vectors when aligned).
+ * No workspace.  Returns MOE_ERR_INVALID_ARG for bad sizes, an unknown
+ * score_fn or null pointers; MOE_ERR_UNSUPPORTED for E > MOE_MAX_EXPERTS.
+ */
+int moe_aux_scores_bwd_logits(int32_t T, int32_t E, int32_t score_fn, const float* logits,
+                              const float* grad_probs, float* grad_logits, void* stream);
 
 /*
  * moe_aux_loss_bwd -- gradient of the loss [TE: Description, forward and
@@ -396,7 +413,7 @@ int moe_rmsnorm_router_topk_workspace_bytes(int32_t T, int32_t H, int32_t E, siz
  * hidden [T,H], gamma [H], W [H,E], bias [E] or NULL, out_norm [T,H],
  * affinities [T,E] -- bf16; ids [T,k] int32; debug_logits [T,E] fp32 or NULL
  * (receives the logits when given).  T <= 128 and H % 128 == 0 [NKI: Notes];
- * this build also needs E % 16 == 0, E <= 256 and H <= 32768, and every
+ * this build also needs E % 16 == 0, E <= 1024 and H <= 32768, and every
  * pointer 16-byte aligned.  Three launches chained by programmatic dependent
  * launch: a row-parallel RMSNorm writing out_norm; the projection split over
  * K-slices (one CTA per token group x 64 experts x slice, all resident at

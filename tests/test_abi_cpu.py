@@ -94,6 +94,10 @@ def test_other_entry_points_validate():
     assert L.moe_rmsnorm_router_topk(4, 100, 16, 2, 1e-6, 1, d, d, d, None, d, d, d, None, d, sz, None) == -1
     assert L.moe_rmsnorm_router_topk(4, 128, 24, 2, 1e-6, 1, d, d, d, None, d, d, d, None, d, sz, None) == -2
     assert L.moe_rmsnorm_router_topk(4, 128, 16, 17, 1e-6, 1, d, d, d, None, d, d, d, None, d, sz, None) == -1
+    assert L.moe_rmsnorm_router_topk(4, 128, 1040, 8, 1e-6, 1, d, d, d, None, d, d, d, None, d, sz, None) == -2
+    nb = ctypes.c_size_t()
+    assert L.moe_rmsnorm_router_topk_workspace_bytes(128, 7168, 1024, ctypes.byref(nb)) == 0 and nb.value > 0
+    assert L.moe_rmsnorm_router_topk_workspace_bytes(128, 7168, 1040, ctypes.byref(nb)) == -2
     # dispatch / combine: rows must be 16-byte multiples
     assert L.moe_dispatch(4, 3, 2, 1, d, d, d, d, 16, d, None) == -1
     assert L.moe_combine(4, 12, 2, 1, d, 16, d, d, 0, d, None, 0, None) == -1
@@ -125,6 +129,16 @@ def test_fused_shared_experts_validation():
                                 ctypes.byref(mp), ctypes.byref(mt)) == B.MOE_ERR_UNSUPPORTED
     assert L.moe_route_capacity(ctypes.byref(B.route_params(16, 64, 30, num_fused_shared_experts=3)),
                                 ctypes.byref(mp), ctypes.byref(mt)) == B.MOE_ERR_UNSUPPORTED
+
+
+def test_aux_scores_bwd_logits_validates():
+    L = B.lib()
+    d = ctypes.c_void_p(16)
+    assert L.moe_aux_scores_bwd_logits(-1, 8, 0, d, d, d, None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_aux_scores_bwd_logits(4, 8, 7, d, d, d, None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_aux_scores_bwd_logits(4, 8, 1, None, d, d, None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_aux_scores_bwd_logits(4, 4096, 1, d, d, d, None) == B.MOE_ERR_UNSUPPORTED
+    assert L.moe_aux_scores_bwd_logits(0, 8, 1, None, None, None, None) == B.MOE_OK
 
 
 def test_ep_regroup_validates():

@@ -141,6 +141,47 @@ def test_aux_scores_backward(T, E):
     assert np.all(err <= RTOL * scale + 1e-30), f"err/scale max {np.max(err / (scale + 1e-30))}"
 
 
+@pytest.mark.parametrize("score_fn", [W.SIGMOID, W.SOFTMAX])
+@pytest.mark.parametrize("T,E", [(1, 8), (77, 33), (1000, 128), (32768, 128), (129, 1024), (300, 5)])
+def test_aux_scores_backward_from_logits(score_fn, T, E):
+    """moe_aux_scores_bwd_logits against the oracle's vector-Jacobian product of the scores recomputed from
+    the logits, relative to the terms before cancellation: d_e * (|g_e| + sum_j p_j |g_j|), with
+    d = p (softmax) or s (1 - s) / S (sigmoid over the row sum)."""
+    g = torch.Generator().manual_seed(T * 11 + E + 3 * score_fn)
+    lg = torch.randn(T, E, generator=g) * 2.0
+    G = torch.randn(T, E, generator=g)
+    got = to_np(B.aux_scores_bwd_logits(lg.cuda(), G.cuda(), score_fn=score_fn))
+    torch.cuda.synchronize()
+    ref = oracle.aux_scores_bwd_logits(lg, G, score_fn=score_fn)
+    x = lg.double().numpy()
+    if score_fn == W.SOFTMAX:
+        z = np.exp(x - x.max(1, keepdims=True))
+        p = z / z.sum(1, keepdims=True)
+        d = p
+    else:
+        s = 1.0 / (1.0 + np.exp(-x))
+        p = s / s.sum(1, keepdims=True)
+        d = s * (1 - s) / s.sum(1, keepdims=True)
+    ag = np.abs(G.double().numpy())
+    scale = d * (ag + (p * ag).sum(1, keepdims=True))
+    err = np.abs(got.astype(np.float64) - ref.astype(np.float64))
+    assert np.all(err <= RTOL * scale + 1e-30), f"err/scale max {np.max(err / (scale + 1e-30))}"
+
+
+def test_aux_scores_backward_from_logits_unaligned_rows():
+    # rows that start off 16 bytes (a view one element in) take the scalar loads, same values
+    T, E = 64, 128
+    g = torch.Generator().manual_seed(5)
+    big = torch.randn(T * E + 1, generator=g).cuda()
+    Gbig = torch.randn(T * E + 1, generator=g).cuda()
+    lg, G = big[1:].view(T, E), Gbig[1:].view(T, E)
+    out = torch.empty(T * E + 1, device="cuda")[1:].view(T, E)
+    B.aux_scores_bwd_logits_into(lg, G, out, score_fn=W.SIGMOID)
+    ref = B.aux_scores_bwd_logits(lg.contiguous().clone(), G.clone(), score_fn=W.SIGMOID)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+
+
 def test_aux_scores_backward_sigmoid_unsupported():
     p = torch.full((4, 8), 0.125, device="cuda")
     with pytest.raises(Exception):

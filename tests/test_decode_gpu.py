@@ -67,10 +67,13 @@ def test_decode_workload_full_size():
 @pytest.mark.parametrize("T,H,E,k,act,bias", [
     (1, 128, 16, 1, W.SIGMOID, False), (7, 256, 64, 4, W.SIGMOID, True), (128, 7168, 256, 8, W.SOFTMAX, True),
     (33, 1024, 96, 6, W.SIGMOID, False), (128, 19200, 128, 8, W.SIGMOID, True), (64, 640, 48, 3, W.SOFTMAX, False),
-    (100, 2048, 160, 6, W.SIGMOID, True), (65, 512, 256, 8, W.SIGMOID, True), (128, 32768, 64, 4, W.SIGMOID, True)])
+    (100, 2048, 160, 6, W.SIGMOID, True), (65, 512, 256, 8, W.SIGMOID, True), (128, 32768, 64, 4, W.SIGMOID, True),
+    (128, 7168, 384, 8, W.SIGMOID, True), (40, 2048, 272, 8, W.SOFTMAX, True), (128, 4096, 512, 8, W.SIGMOID, True),
+    (17, 1024, 784, 6, W.SOFTMAX, False), (128, 2048, 1024, 8, W.SIGMOID, True)])
 def test_decode_shapes(T, H, E, k, act, bias):
-    # cluster sizes 2..16 (H/64 chunks), one or two 64-token groups, partial expert groups, and slices
-    # longer than the staging ring (H=19200, 32768)
+    # cluster sizes 2..16 (H/64 chunks), one or two 64-token groups, partial expert groups, slices
+    # longer than the staging ring (H=19200, 32768), and 272 .. 1024 experts (two to four rounds of 256
+    # in the top-k stage, the last one partial for 272 and 784)
     run_decode(W.DecodeSpec(T=T, H=H, E=E, k=k, act=act, has_bias=bias, seed=T + H + E))
 
 

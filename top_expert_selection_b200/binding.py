@@ -35,7 +35,8 @@ _TORCH = {F32: torch.float32, BF16: torch.bfloat16}
 # every symbol the C header declares (checked by the CPU test suite)
 EXPORTED = (
     "moe_error_string", "moe_workspace_init", "moe_status", "moe_route_capacity",
-    "moe_route_workspace_bytes", "moe_route", "moe_aux_workspace_bytes", "moe_aux_scores", "moe_aux_scores_bwd", "moe_route_weights_bwd",
+    "moe_route_workspace_bytes", "moe_route", "moe_aux_workspace_bytes", "moe_aux_scores", "moe_aux_scores_bwd", "moe_aux_scores_bwd_logits",
+    "moe_route_weights_bwd",
     "moe_aux_loss_fwd", "moe_aux_loss_bwd", "moe_dispatch", "moe_combine",
     "moe_rmsnorm_router_topk_workspace_bytes", "moe_rmsnorm_router_topk", "moe_debug_wait_timeout",
     "moe_debug_sigmoid_proxy_error", "moe_route_no_alloc", "moe_route_no_alloc_status",
@@ -94,6 +95,7 @@ def lib() -> ctypes.CDLL:
             "moe_aux_loss_fwd": ([i32, i32, i32, i32, f32, P, P, P, P, sz, P], ctypes.c_int),
             "moe_aux_loss_bwd": ([i32, i32, i32, i32, f32, P, P, P, P, P, P], ctypes.c_int),
             "moe_aux_scores_bwd": ([i32, i32, i32, P, P, P, P], ctypes.c_int),
+            "moe_aux_scores_bwd_logits": ([i32, i32, i32, P, P, P, P], ctypes.c_int),
             "moe_route_weights_bwd": ([RP, P, P, P, P, P, sz, P], ctypes.c_int),
             "moe_dispatch": ([i32, i32, i32, i32, P, P, P, P, i64, P, P], ctypes.c_int),
             "moe_combine": ([i32, i32, i32, i32, P, i64, P, P, i32, P, P, sz, P], ctypes.c_int),
@@ -333,6 +335,19 @@ def aux_scores_bwd_into(probs: torch.Tensor, grad_probs: torch.Tensor, grad_logi
     T, E = probs.shape
     _check(lib().moe_aux_scores_bwd(T, E, score_fn, _p(probs), _p(grad_probs), _p(grad_logits), _stream(stream)),
            "moe_aux_scores_bwd")
+
+
+def aux_scores_bwd_logits_into(logits: torch.Tensor, grad_probs: torch.Tensor, grad_logits: torch.Tensor,
+                               score_fn: int = SOFTMAX, stream=None) -> None:
+    T, E = logits.shape
+    _check(lib().moe_aux_scores_bwd_logits(T, E, score_fn, _p(logits), _p(grad_probs), _p(grad_logits),
+                                           _stream(stream)), "moe_aux_scores_bwd_logits")
+
+
+def aux_scores_bwd_logits(logits: torch.Tensor, grad_probs: torch.Tensor, score_fn: int = SOFTMAX) -> torch.Tensor:
+    gl = torch.empty_like(logits)
+    aux_scores_bwd_logits_into(logits, grad_probs, gl, score_fn)
+    return gl
 
 
 def aux_scores_bwd(probs: torch.Tensor, grad_probs: torch.Tensor, score_fn: int = SOFTMAX) -> torch.Tensor:

@@ -400,10 +400,10 @@ __global__ void __launch_bounds__(kAuxThreads) aux_loss_bwd_kernel(int T, int E,
 template <int VPL>
 __global__ void __launch_bounds__(kAuxThreads) aux_scores_bwd_kernel(int T, int E, const float* __restrict__ probs,
                                                                      const float* __restrict__ grad_probs,
-                                                                     float* __restrict__ grad_logits) {
+                                                                     float* __restrict__ grad_logits, bool aligned) {
   pdl_entry();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const bool vec = (VPL % 4 == 0) && ((E & 3) == 0) && (lane * VPL + VPL <= E);
+  const bool vec = aligned && (VPL % 4 == 0) && ((E & 3) == 0) && (lane * VPL + VPL <= E);
   for (long long t = (long long)blockIdx.x * kAuxWarps + warp; t < T; t += (long long)gridDim.x * kAuxWarps) {
     const float* prow = probs + t * E;
     const float* grow = grad_probs + t * E;
@@ -440,6 +440,100 @@ __global__ void __launch_bounds__(kAuxThreads) aux_scores_bwd_kernel(int T, int 
                              p[i + 3] * (g[i + 3] - dot)));
       } else if (e < E) {
         __stcs(grad_logits + t * E + e, p[i] * (g[i] - dot));
+      }
+    }
+  }
+}
+
+// --------------------------------------------------------------------------
+// backward of the scores from the logits (softmax, or sigmoid over the row
+// sum): warp per row, the scores recomputed as the forward computes them,
+// dot = sum_e p_e g_e (lane partials, then a shuffle tree),
+// grad = d * (g - dot) with d = p (softmax) or p * (1 - s) = s (1 - s) / S
+// (sigmoid; 1 - s formed as exp(-x) * s, without cancellation)
+// --------------------------------------------------------------------------
+template <int VPL>
+__device__ __forceinline__ void load_row_f32(const float* __restrict__ row, int E, int lane, bool vec, float* v) {
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int e = lane * VPL + i;
+    if (vec) {
+      if ((i & 3) == 0) {
+        const float4 q = __ldcs(reinterpret_cast<const float4*>(row + e));
+        v[i] = q.x;
+        if (i + 1 < VPL) v[i + 1] = q.y;
+        if (i + 2 < VPL) v[i + 2] = q.z;
+        if (i + 3 < VPL) v[i + 3] = q.w;
+      }
+    } else {
+      v[i] = e < E ? __ldcs(row + e) : 0.0f;
+    }
+  }
+}
+
+template <int VPL>
+__global__ void __launch_bounds__(kAuxThreads) aux_scores_bwd_logits_kernel(int T, int E, int score_fn,
+                                                                            const float* __restrict__ logits,
+                                                                            const float* __restrict__ grad_probs,
+                                                                            float* __restrict__ grad_logits,
+                                                                            bool aligned) {
+  const unsigned FULL = 0xffffffffu;
+  pdl_entry();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const bool vec = aligned && (VPL % 4 == 0) && ((E & 3) == 0) && (lane * VPL + VPL <= E);
+  uint32_t valid = 0;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) valid |= ((lane * VPL + i < E) ? 1u : 0u) << i;
+  for (long long t = (long long)blockIdx.x * kAuxWarps + warp; t < T; t += (long long)gridDim.x * kAuxWarps) {
+    float x[VPL], g[VPL], p[VPL], d[VPL];
+    load_row_f32<VPL>(logits + t * E, E, lane, vec, x);
+    load_row_f32<VPL>(grad_probs + t * E, E, lane, vec, g);
+    float sum = 0.0f;
+    if (score_fn == MOE_SOFTMAX) {
+      float m = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i)
+        if (valid & (1u << i)) m = fmaxf(m, x[i]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, off));
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        p[i] = (valid & (1u << i)) ? expf(x[i] - m) : 0.0f;
+        sum += p[i];
+      }
+    } else {
+      // s = 1 / (1 + u) with u = exp(-x) (the forward's sigmoid); 1 - s = u * s
+      // keeps its relative precision where s rounds close to 1 (d[] holds it)
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const float u = expf(-x[i]);
+        p[i] = (valid & (1u << i)) ? 1.0f / (1.0f + u) : 0.0f;
+        d[i] = p[i] > 0.0f ? u * p[i] : 1.0f;
+        sum += p[i];
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(FULL, sum, off);
+    float dot = 0.0f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      p[i] = p[i] / sum;
+      d[i] = score_fn == MOE_SOFTMAX ? p[i] : p[i] * d[i];
+      dot = fmaf(p[i], g[i], dot);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(FULL, dot, off);
+    float* out = grad_logits + t * E;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int e = lane * VPL + i;
+      if (vec) {
+        if ((i & 3) == 0 && i + 3 < VPL)
+          __stcs(reinterpret_cast<float4*>(out + e),
+                 make_float4(d[i] * (g[i] - dot), d[i + 1] * (g[i + 1] - dot), d[i + 2] * (g[i + 2] - dot),
+                             d[i + 3] * (g[i + 3] - dot)));
+      } else if (e < E) {
+        __stcs(out + e, d[i] * (g[i] - dot));
       }
     }
   }
@@ -681,8 +775,28 @@ extern "C" int moe_aux_scores_bwd(int32_t T, int32_t E, int32_t score_fn, const 
   const int grid = std::max(1, std::min((T + kAuxWarps - 1) / kAuxWarps, sm_count() * 8));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t err = cudaSuccess;
+  const bool aligned = ((reinterpret_cast<uintptr_t>(probs) | reinterpret_cast<uintptr_t>(grad_probs) |
+                         reinterpret_cast<uintptr_t>(grad_logits)) & 15) == 0;
   MOE_VPL_SWITCH(vpl, (err = launch_pdl(aux_scores_bwd_kernel<V>, dim3(grid), dim3(kAuxThreads), 0, st, T, E, probs,
-                                        grad_probs, grad_logits)));
+                                        grad_probs, grad_logits, aligned)));
+  return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+extern "C" int moe_aux_scores_bwd_logits(int32_t T, int32_t E, int32_t score_fn, const float* logits,
+                                         const float* grad_probs, float* grad_logits, void* stream) {
+  if (T < 0 || E <= 0) return MOE_ERR_INVALID_ARG;
+  if (score_fn != MOE_SOFTMAX && score_fn != MOE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (!logits || !grad_probs || !grad_logits) return MOE_ERR_INVALID_ARG;
+  const int vpl = pick_vpl(E);
+  const int grid = std::max(1, std::min((T + kAuxWarps - 1) / kAuxWarps, sm_count() * 8));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool aligned = ((reinterpret_cast<uintptr_t>(logits) | reinterpret_cast<uintptr_t>(grad_probs) |
+                         reinterpret_cast<uintptr_t>(grad_logits)) & 15) == 0;
+  cudaError_t err = cudaSuccess;
+  MOE_VPL_SWITCH(vpl, (err = launch_pdl(aux_scores_bwd_logits_kernel<V>, dim3(grid), dim3(kAuxThreads), 0, st, T,
+                                        E, score_fn, logits, grad_probs, grad_logits, aligned)));
   return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

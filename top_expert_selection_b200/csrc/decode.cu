@@ -54,13 +54,13 @@ constexpr int kProjThreads = 256;  // 8 warps: 4 TMEM lane quarters x 2 column h
 constexpr int kChunk = 64;         // hidden columns per staged chunk (one 128-byte swizzle atom)
 constexpr int kExpGroup = 64;      // experts per CTA (MMA N <= 64)
 constexpr int kM = 128;            // MMA M: token rows (a 64-token group pads with zero rows)
-constexpr int kMaxE = 256;         // top-k stage: 8 experts per lane
+constexpr int kMaxE = 1024;        // top-k stage: 8 experts per lane per round of 256
 constexpr int kMaxStages = 8;      // staged chunks in flight
 constexpr int kMaxKS = 48;         // K-slices (bounds the partial-logit workspace)
 constexpr int kATile = kM * 128;      // 16 KB
 constexpr int kBTile = kChunk * 128;  // 8 KB (64 K rows x 64 experts)
 constexpr int kSmemLimit = 227 * 1024;  // opt-in shared memory per CTA
-constexpr int kSelThreads = 256;        // K3: one thread per expert
+constexpr int kSelThreads = 256;        // K3: threads summing the partial logits
 constexpr int kMaxH = 32768;            // hidden size limit
 
 struct DecodeArgs {
@@ -240,53 +240,62 @@ __device__ __forceinline__ double sumsq8(uint4 v) {
 
 // K3: ids, affinities (and debug logits) of one token from its logits row in
 // shared memory; outputs are written only while the workspace status is
-// MOE_OK.
-__device__ void select_row(const DecodeArgs& a, int t, int lane, const float* row, int status, uint4 bv) {
-  float lg[8];
+// MOE_OK.  R rounds of 256 experts: lane l holds experts r*256 + 8l .. +7 of
+// round r in slots 8r .. 8r+7 (E is a multiple of 16, so a lane's 8 experts
+// of a round are all present or all absent).
+template <int R>
+__device__ void select_row(const DecodeArgs& a, int t, int lane, const float* row, int status, const uint4* bv) {
+  constexpr int NS = 8 * R;
+  float lg[NS];
   uint32_t valid = 0;
-  if (lane * 8 < a.E) {
-    const float4 u = reinterpret_cast<const float4*>(row + lane * 8)[0];
-    const float4 w = reinterpret_cast<const float4*>(row + lane * 8)[1];
-    lg[0] = u.x; lg[1] = u.y; lg[2] = u.z; lg[3] = u.w;
-    lg[4] = w.x; lg[5] = w.y; lg[6] = w.z; lg[7] = w.w;
-    valid = 0xffu;
-    if (a.bias) {
-      const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        lg[2 * i] += __uint_as_float(bw[i] << 16);
-        lg[2 * i + 1] += __uint_as_float(bw[i] & 0xffff0000u);
+  for (int r = 0; r < R; ++r) {
+    const int e0 = r * 256 + lane * 8;
+    if (e0 < a.E) {
+      const float4 u = reinterpret_cast<const float4*>(row + e0)[0];
+      const float4 w = reinterpret_cast<const float4*>(row + e0)[1];
+      lg[8 * r + 0] = u.x; lg[8 * r + 1] = u.y; lg[8 * r + 2] = u.z; lg[8 * r + 3] = u.w;
+      lg[8 * r + 4] = w.x; lg[8 * r + 5] = w.y; lg[8 * r + 6] = w.z; lg[8 * r + 7] = w.w;
+      valid |= 0xffu << (8 * r);
+      if (a.bias) {
+        const uint32_t bw[4] = {bv[r].x, bv[r].y, bv[r].z, bv[r].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          lg[8 * r + 2 * i] += __uint_as_float(bw[i] << 16);
+          lg[8 * r + 2 * i + 1] += __uint_as_float(bw[i] & 0xffff0000u);
+        }
       }
-    }
-  } else {
+    } else {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) lg[i] = 0.0f;
+      for (int i = 0; i < 8; ++i) lg[8 * r + i] = 0.0f;
+    }
   }
   // top-k on the raw logits: k rounds of (warp max of the order-preserving
   // key, then the lowest expert holding it), ties -> lower expert
-  uint32_t key[8];
+  uint32_t key[NS];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) key[i] = ordered_key(lg[i]);
+  for (int i = 0; i < NS; ++i) key[i] = ordered_key(lg[i]);
   uint32_t chosen = 0, avail = valid;
   int my_id = 0;
   uint32_t bk = 0u;
-  int bi = 8;  // this lane's best remaining (key, slot); slot 8 = none
+  int bi = NS;  // this lane's best remaining (key, slot); slot NS = none
   auto lane_best = [&]() {
     bk = 0u;
-    bi = 8;
+    bi = NS;
 #pragma unroll
-    for (int i = 7; i >= 0; --i)
-      if (((avail >> i) & 1u) && key[i] >= bk) {
+    for (int i = NS - 1; i >= 0; --i)
+      if (((avail >> i) & 1u) && key[i] >= bk) {  // from the top down: ties -> the lower slot (lower expert)
         bk = key[i];
         bi = i;
       }
   };
+  auto slot_expert = [&](int i) { return (i >> 3) * 256 + lane * 8 + (i & 7); };
   lane_best();
   for (int j = 0; j < a.k; ++j) {
     const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
     const uint32_t win =
-        __reduce_min_sync(0xffffffffu, (bi < 8 && bk == m) ? (uint32_t)(lane * 8 + bi) : 0xffffffffu);
-    if (bi < 8 && (uint32_t)(lane * 8 + bi) == win) {
+        __reduce_min_sync(0xffffffffu, (bi < NS && bk == m) ? (uint32_t)slot_expert(bi) : 0xffffffffu);
+    if (bi < NS && (uint32_t)slot_expert(bi) == win) {
       avail &= ~(1u << bi);
       chosen |= 1u << bi;
       lane_best();
@@ -294,39 +303,49 @@ __device__ void select_row(const DecodeArgs& a, int t, int lane, const float* ro
     if (lane == j) my_id = (int)win;
   }
   if (status != MOE_OK) return;
-  if (a.dbg_logits && lane * 8 < a.E) {
-    float* d = a.dbg_logits + (size_t)t * a.E + lane * 8;
-    *reinterpret_cast<float4*>(d) = make_float4(lg[0], lg[1], lg[2], lg[3]);
-    *reinterpret_cast<float4*>(d + 4) = make_float4(lg[4], lg[5], lg[6], lg[7]);
+  if (a.dbg_logits) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int e0 = r * 256 + lane * 8;
+      if (e0 < a.E) {
+        float* d = a.dbg_logits + (size_t)t * a.E + e0;
+        *reinterpret_cast<float4*>(d) = make_float4(lg[8 * r], lg[8 * r + 1], lg[8 * r + 2], lg[8 * r + 3]);
+        *reinterpret_cast<float4*>(d + 4) = make_float4(lg[8 * r + 4], lg[8 * r + 5], lg[8 * r + 6], lg[8 * r + 7]);
+      }
+    }
   }
   // activation over the selected only (ACT2): sigmoid each, or softmax over the k
   float m = -INFINITY, ssum = 0.0f;
   if (a.act == MOE_SOFTMAX) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < NS; ++i)
       if ((chosen >> i) & 1u) m = fmaxf(m, lg[i]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < NS; ++i)
       if ((chosen >> i) & 1u) ssum += expf(lg[i] - m);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, off);
   }
   if (lane < a.k) a.ids[(size_t)t * a.k + lane] = my_id;
-  if (lane * 8 < a.E) {
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int e0 = r * 256 + lane * 8;
+    if (e0 >= a.E) continue;
     uint32_t ow[4];
 #pragma unroll
     for (int i = 0; i < 8; i += 2) {
+      const int s0 = 8 * r + i;
       float v0 = 0.0f, v1 = 0.0f;
-      if ((chosen >> i) & 1u) v0 = (a.act == MOE_SOFTMAX) ? expf(lg[i] - m) / ssum : sigmoid_f32(lg[i]);
-      if ((chosen >> (i + 1)) & 1u)
-        v1 = (a.act == MOE_SOFTMAX) ? expf(lg[i + 1] - m) / ssum : sigmoid_f32(lg[i + 1]);
+      if ((chosen >> s0) & 1u) v0 = (a.act == MOE_SOFTMAX) ? expf(lg[s0] - m) / ssum : sigmoid_f32(lg[s0]);
+      if ((chosen >> (s0 + 1)) & 1u)
+        v1 = (a.act == MOE_SOFTMAX) ? expf(lg[s0 + 1] - m) / ssum : sigmoid_f32(lg[s0 + 1]);
       const __nv_bfloat16 h0 = __float2bfloat16_rn(v0), h1 = __float2bfloat16_rn(v1);
       ow[i / 2] = (uint32_t)(*reinterpret_cast<const uint16_t*>(&h0)) |
                   ((uint32_t)(*reinterpret_cast<const uint16_t*>(&h1)) << 16);
     }
-    *reinterpret_cast<uint4*>(a.aff + (size_t)t * a.E + lane * 8) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+    *reinterpret_cast<uint4*>(a.aff + (size_t)t * a.E + e0) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
   }
 }
 
@@ -538,17 +557,23 @@ __global__ void __launch_bounds__(kProjThreads, 1)
 }
 
 // K3: the logits of one token (its partials summed in slice order) and its top-k.
+template <int R>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const DecodeArgs a) {
   __shared__ __align__(16) float row[kMaxE];
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int t = blockIdx.x, e = threadIdx.x;
-  uint4 bv = make_uint4(0, 0, 0, 0);  // the bias of lane l's experts 8l..8l+7 (warp 0), a weight
-  if (e < 32 && a.bias && e * 8 < a.E) bv = __ldg(reinterpret_cast<const uint4*>(a.bias + e * 8));
+  const int t = blockIdx.x;
+  uint4 bv[R];  // the bias of lane l's experts r*256 + 8l .. +7 (warp 0), a weight
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    bv[r] = make_uint4(0, 0, 0, 0);
+    const int e0 = r * 256 + threadIdx.x * 8;
+    if (threadIdx.x < 32 && a.bias && e0 < a.E) bv[r] = __ldg(reinterpret_cast<const uint4*>(a.bias + e0));
+  }
   asm volatile("griddepcontrol.wait;" ::: "memory");  // the partial logits are K2's output
   int status = MOE_OK;
-  if (e < 32) status = *reinterpret_cast<const volatile int32_t*>(&a.hdr->status);
+  if (threadIdx.x < 32) status = *reinterpret_cast<const volatile int32_t*>(&a.hdr->status);
   const int tp = a.TG * a.TGS, ep = a.NG * kExpGroup;
-  if (e < a.E) {
+  for (int e = threadIdx.x; e < a.E; e += kSelThreads) {
     const float* p = a.part + (size_t)t * ep + e;
     float sum = 0.0f;  // slice order (a deeper unroll measured slower)
 #pragma unroll 4
@@ -556,7 +581,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const DecodeArgs a)
     row[e] = sum;
   }
   __syncthreads();
-  if (e < 32) select_row(a, t, e, row, status, bv);
+  if (threadIdx.x < 32) select_row<R>(a, t, threadIdx.x, row, status, bv);
 }
 
 // ---- host ----
@@ -729,6 +754,11 @@ extern "C" int moe_rmsnorm_router_topk(int32_t T, int32_t H, int32_t E, int32_t 
   if (launch_pdl(project_kernel, dim3(plan.KS * plan.NG * plan.TG), dim3(kProjThreads), (size_t)plan.smem, st, a,
                  xmap, wmap) != cudaSuccess)
     return MOE_ERR_CUDA;
-  if (launch_pdl(select_kernel, dim3(T), dim3(kSelThreads), 0, st, a) != cudaSuccess) return MOE_ERR_CUDA;
+  const int R = (E + 255) / 256;
+  const cudaError_t e3 = R == 1   ? launch_pdl(select_kernel<1>, dim3(T), dim3(kSelThreads), 0, st, a)
+                         : R == 2 ? launch_pdl(select_kernel<2>, dim3(T), dim3(kSelThreads), 0, st, a)
+                         : R == 3 ? launch_pdl(select_kernel<3>, dim3(T), dim3(kSelThreads), 0, st, a)
+                                  : launch_pdl(select_kernel<4>, dim3(T), dim3(kSelThreads), 0, st, a);
+  if (e3 != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }

@@ -125,6 +125,9 @@ class DecodeSpec:
     has_bias: bool = True
     seed: int = 4
 
+    def with_(self, **kw) -> "DecodeSpec":
+        return replace(self, **kw)
+
 
 DECODE_FUSED = DecodeSpec()
 
