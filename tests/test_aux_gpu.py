@@ -76,7 +76,8 @@ def check_backward(p, tpe, T_total, k, coeff, grad, got_gp, got_gl):
 
 
 @pytest.mark.parametrize("T,E,k", [(1, 8, 2), (33, 64, 6), (1000, 128, 8), (257, 96, 4), (300, 256, 8),
-                                   (129, 1024, 16), (77, 33, 3)])
+                                   (129, 1024, 16), (77, 33, 3), (1, 64, 1), (5, 128, 8), (4097, 256, 7),
+                                   (999, 64, 8), (2, 128, 3), (6, 256, 1)])
 def test_aux_shapes(T, E, k):
     g = torch.Generator().manual_seed(T + E)
     lg = torch.randn(T, E, generator=g) * 1.5
@@ -90,6 +91,68 @@ def test_aux_shapes(T, E, k):
         gr = B.aux_loss_bwd(gl, probs, tpe, T_total, k, 0.37)
         check_backward(to_np(probs), to_np(tpe), T_total, k, 0.37, 0.75, to_np(gr["grad_probs"]),
                        to_np(gr["grad_logits"]))
+
+
+@pytest.mark.parametrize("score_fn", [W.SOFTMAX, W.SIGMOID])
+@pytest.mark.parametrize("E", [64, 128, 256])
+def test_aux_scores_masked_and_tied_rows(E, score_fn):
+    """Rows the per-lane top-3 threshold cannot settle alone: exact ties (all equal; a block of equal
+    maxima wider than k; ties at zero probability after -inf logits), one dominant expert, and the top k
+    held by one lane's experts.  The routing map equals the oracle's exactly (ties -> lower expert)."""
+    k = 8
+    rng = np.random.default_rng(E + score_fn)
+    lg = rng.standard_normal((13, E)).astype(np.float32)
+    lg[0] = 0.5                                    # all equal
+    lg[1] = -np.inf
+    lg[1, [5, 77 % E, 40]] = [1.0, 2.0, 0.5]       # three finite: then ties at 0 -> lowest experts
+    lg[2] = 0.0
+    lg[2, rng.permutation(E)[:20]] = 1.0           # 20 equal maxima
+    lg[3] = 0.0
+    lg[3, 9] = 100.0                               # one dominant expert, the rest equal
+    lane_experts = [c * 32 + 4 * 2 + r for c in range(E // 32) for r in range(4)]
+    lg[4, lane_experts] += 6.0                     # the top k all in one lane's experts
+    if score_fn == W.SIGMOID:
+        lg[1] = np.where(np.isinf(lg[1]), -30.0, lg[1])  # sigmoid(-inf) = 0 is a tie as well; keep finite
+    g = B.aux_scores(torch.from_numpy(lg).cuda(), k, score_fn)
+    torch.cuda.synchronize()
+    o = oracle.aux_scores(lg, k, score_fn)
+    assert np.array_equal(to_np(g["routing_map"]), o["routing_map"])
+    assert np.array_equal(to_np(g["tokens_per_expert"]), o["tokens_per_expert"])
+    ref = o["probs"]
+    assert np.all(np.abs(to_np(g["probs"]) - ref) <= RTOL * np.abs(ref) + 1e-30)
+
+
+def test_aux_scores_rows_with_non_finite_logits():
+    """A NaN or +inf logit makes the row's score sum non-finite: that row is redone by the whole warp and
+    still marks exactly k experts; the other rows of the same four-token group match the oracle."""
+    T, E, k = 9, 128, 8
+    rng = np.random.default_rng(3)
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    lg[2, 17] = np.nan
+    lg[5, 100] = np.inf
+    g = B.aux_scores(torch.from_numpy(lg).cuda(), k)
+    torch.cuda.synchronize()
+    o = oracle.aux_scores(lg, k)
+    gm = to_np(g["routing_map"])
+    assert np.all(gm.sum(1) == k)
+    assert np.array_equal(to_np(g["tokens_per_expert"]), gm.sum(0).astype(np.int32))
+    ok = [t for t in range(T) if t not in (2, 5)]
+    assert np.array_equal(gm[ok], o["routing_map"][ok])
+    assert np.all(np.abs(to_np(g["probs"])[ok] - o["probs"][ok]) <= RTOL * np.abs(o["probs"][ok]) + 1e-30)
+
+
+def test_aux_loss_fwd_unaligned_counts_and_ragged_rows():
+    # counts that start off 16 bytes take the shared-memory column path; both paths agree with the oracle
+    T, E, k = 1001, 128, 8
+    g = torch.Generator().manual_seed(9)
+    lg = torch.randn(T, E, generator=g)
+    sc = B.aux_scores(lg.cuda(), k)
+    big = torch.zeros(E + 1, dtype=torch.int32, device="cuda")
+    big[1:] = sc["tokens_per_expert"]
+    for tpe in (sc["tokens_per_expert"], big[1:]):
+        loss = B.aux_loss_fwd(sc["probs"], tpe, 3 * T, k, 0.01)
+        ref = oracle.aux_loss_fwd(to_np(sc["probs"]), to_np(sc["tokens_per_expert"]), 3 * T, k, 0.01)
+        assert abs(float(loss.item()) - ref) <= RTOL * abs(ref)
 
 
 def test_aux_uniform_closed_form_on_gpu():

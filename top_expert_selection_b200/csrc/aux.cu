@@ -114,28 +114,20 @@ __device__ __forceinline__ bool topk_mask_by_threshold(const float* p, uint32_t 
   return true;
 }
 
+// One row by a whole warp (lane l: entries [l*VPL, l*VPL+VPL)): scores, the
+// top-k mask, probs and routing-map stores, the mask counted into hist.
 template <int VPL>
-__global__ void __launch_bounds__(kScoreThreads, 3) aux_scores_kernel(int T, int E, int k, int score_fn,
-                                                                 const float* __restrict__ logits,
-                                                                 float* __restrict__ probs,
-                                                                 uint8_t* __restrict__ rmap,
-                                                                 int32_t* __restrict__ tpe, void* ws) {
-  extern __shared__ int hist[];  // [E], then per warp 32 packed candidate keys
+__device__ __forceinline__ void score_row_warp(long long t, int E, int k, int score_fn, const float* __restrict__ logits,
+                                               float* __restrict__ probs, uint8_t* __restrict__ rmap, int* hist,
+                                               unsigned long long* list, int lane) {
   const unsigned FULL = 0xffffffffu;
-  pdl_entry();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
-  AuxWs w = aux_ws(ws, E);
-  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
-  __syncthreads();
-
-  const int nw = blockDim.x >> 5;
   uint32_t valid = 0;
 #pragma unroll
   for (int i = 0; i < VPL; ++i) valid |= ((lane * VPL + i < E) ? 1u : 0u) << i;
   // a lane's VPL experts are contiguous: 16-byte loads when the row allows it
   const bool vec = (VPL % 4 == 0) && ((E & 3) == 0) && (lane * VPL + VPL <= E);
-  auto load_row = [&](long long t, float* x) {
+  float x[VPL], p[VPL];
+  {
     const float* row = logits + t * E;
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
@@ -152,97 +144,97 @@ __global__ void __launch_bounds__(kScoreThreads, 3) aux_scores_kernel(int T, int
         x[i] = e < E ? __ldcs(row + e) : 0.0f;
       }
     }
-  };
-  for (long long t = (long long)blockIdx.x * nw + warp; t < T; t += (long long)gridDim.x * nw) {
-    float x[VPL], p[VPL];
-    load_row(t, x);
-    float sum = 0.0f;
-    if (score_fn == MOE_SOFTMAX) {
-      float m = -INFINITY;
+  }
+  float sum = 0.0f;
+  if (score_fn == MOE_SOFTMAX) {
+    float m = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < VPL; ++i)
-        if (valid & (1u << i)) m = fmaxf(m, x[i]);
+    for (int i = 0; i < VPL; ++i)
+      if (valid & (1u << i)) m = fmaxf(m, x[i]);
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, off));
-#pragma unroll
-      for (int i = 0; i < VPL; ++i) {
-        p[i] = (valid & (1u << i)) ? expf(x[i] - m) : 0.0f;
-        sum += p[i];
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < VPL; ++i) {
-        p[i] = (valid & (1u << i)) ? sigmoid_f32(x[i]) : 0.0f;
-        sum += p[i];
-      }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(FULL, sum, off);
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) p[i] = p[i] / sum;
-
-    // top-k mask over probs, ties -> lower expert: threshold + counting, else
-    // k rounds of warp argmax
-    uint32_t avail = valid, chosen = 0;
-    bool done = false;
-    if constexpr (VPL <= 8) {
-      unsigned long long* list = reinterpret_cast<unsigned long long*>(hist + ((E + 1) & ~1)) + warp * 32;
-      if (k <= 8) done = topk_mask_by_threshold<VPL>(p, valid, lane, k, list, &chosen);
-    }
-    for (int j = 0; j < k && !done; ++j) {
-      unsigned long long best = 0ull;
-#pragma unroll
-      for (int i = 0; i < VPL; ++i)
-        if (avail & (1u << i)) {
-          const unsigned long long pk = pack_key(p[i], lane * VPL + i);
-          best = pk > best ? pk : best;
-        }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const unsigned long long o = shfl_xor_u64(FULL, best, off);
-        best = o > best ? o : best;
-      }
-      const int win = packed_expert(best);
-      if (win / VPL == lane) {
-        const uint32_t bit = 1u << (win - lane * VPL);
-        avail &= ~bit;
-        chosen |= bit;
-      }
-    }
-    float* prow = probs + t * E;
-    uint8_t* mrow = rmap + t * E;
-    if constexpr (VPL % 4 == 0) {
-      const bool vec = ((E & 3) == 0) && (lane * VPL + VPL <= E);
-      if (vec) {
-#pragma unroll
-        for (int i = 0; i < VPL; i += 4) {
-          const int e = lane * VPL + i;
-          __stcs(reinterpret_cast<float4*>(prow + e), make_float4(p[i], p[i + 1], p[i + 2], p[i + 3]));
-          const uint32_t m4 = ((chosen >> i) & 1u) | (((chosen >> (i + 1)) & 1u) << 8) |
-                              (((chosen >> (i + 2)) & 1u) << 16) | (((chosen >> (i + 3)) & 1u) << 24);
-          *reinterpret_cast<uint32_t*>(mrow + e) = m4;
-        }
-#pragma unroll
-        for (int i = 0; i < VPL; ++i)
-          if ((chosen >> i) & 1u) atomicAdd(&hist[lane * VPL + i], 1);
-        continue;
-      }
-    }
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, off));
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
-      const int e = lane * VPL + i;
-      if (valid & (1u << i)) {
-        __stcs(prow + e, p[i]);
-        const bool c = (chosen >> i) & 1u;
-        mrow[e] = c ? 1 : 0;
-        if (c) atomicAdd(&hist[e], 1);
-      }
+      p[i] = (valid & (1u << i)) ? expf(x[i] - m) : 0.0f;
+      sum += p[i];
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      p[i] = (valid & (1u << i)) ? sigmoid_f32(x[i]) : 0.0f;
+      sum += p[i];
     }
   }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(FULL, sum, off);
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) p[i] = p[i] / sum;
+
+  // top-k mask over probs, ties -> lower expert: threshold + counting, else
+  // k rounds of warp argmax
+  uint32_t avail = valid, chosen = 0;
+  bool done = false;
+  if constexpr (VPL <= 8) {
+    if (k <= 8) done = topk_mask_by_threshold<VPL>(p, valid, lane, k, list, &chosen);
+  }
+  for (int j = 0; j < k && !done; ++j) {
+    unsigned long long best = 0ull;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i)
+      if (avail & (1u << i)) {
+        const unsigned long long pk = pack_key(p[i], lane * VPL + i);
+        best = pk > best ? pk : best;
+      }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const unsigned long long o = shfl_xor_u64(FULL, best, off);
+      best = o > best ? o : best;
+    }
+    const int win = packed_expert(best);
+    if (win / VPL == lane) {
+      const uint32_t bit = 1u << (win - lane * VPL);
+      avail &= ~bit;
+      chosen |= bit;
+    }
+  }
+  float* prow = probs + t * E;
+  uint8_t* mrow = rmap + t * E;
+  if constexpr (VPL % 4 == 0) {
+    if (vec) {
+#pragma unroll
+      for (int i = 0; i < VPL; i += 4) {
+        const int e = lane * VPL + i;
+        __stcs(reinterpret_cast<float4*>(prow + e), make_float4(p[i], p[i + 1], p[i + 2], p[i + 3]));
+        const uint32_t m4 = ((chosen >> i) & 1u) | (((chosen >> (i + 1)) & 1u) << 8) |
+                            (((chosen >> (i + 2)) & 1u) << 16) | (((chosen >> (i + 3)) & 1u) << 24);
+        *reinterpret_cast<uint32_t*>(mrow + e) = m4;
+      }
+#pragma unroll
+      for (int i = 0; i < VPL; ++i)
+        if ((chosen >> i) & 1u) atomicAdd(&hist[lane * VPL + i], 1);
+      return;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int e = lane * VPL + i;
+    if (valid & (1u << i)) {
+      __stcs(prow + e, p[i]);
+      const bool c = (chosen >> i) & 1u;
+      mrow[e] = c ? 1 : 0;
+      if (c) atomicAdd(&hist[e], 1);
+    }
+  }
+}
+
+// The block's counts into the accumulator; the last block to finish publishes
+// them to tokens_per_expert and clears the accumulator.
+__device__ __forceinline__ void publish_counts(int E, const int* hist, int32_t* __restrict__ tpe, void* ws) {
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
+  AuxWs w = aux_ws(ws, E);
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x)
     if (hist[e]) atomicAdd(&w.tpe_acc[e], hist[e]);
-  // the last block to finish publishes the counts and clears the accumulator
   __shared__ int last;
   __threadfence();
   __syncthreads();
@@ -258,6 +250,219 @@ __global__ void __launch_bounds__(kScoreThreads, 3) aux_scores_kernel(int T, int
   }
 }
 
+template <int VPL>
+__global__ void __launch_bounds__(kScoreThreads, 3) aux_scores_kernel(int T, int E, int k, int score_fn,
+                                                                 const float* __restrict__ logits,
+                                                                 float* __restrict__ probs,
+                                                                 uint8_t* __restrict__ rmap,
+                                                                 int32_t* __restrict__ tpe, void* ws) {
+  extern __shared__ int hist[];  // [E], then per warp 32 packed candidate keys
+  pdl_entry();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int nw = blockDim.x >> 5;
+  unsigned long long* list = reinterpret_cast<unsigned long long*>(hist + ((E + 1) & ~1)) + warp * 32;
+  for (long long t = (long long)blockIdx.x * nw + warp; t < T; t += (long long)gridDim.x * nw)
+    score_row_warp<VPL>(t, E, k, score_fn, logits, probs, rmap, hist, list, lane);
+  publish_counts(E, hist, tpe, ws);
+}
+
+// --------------------------------------------------------------------------
+// scores, four tokens per warp (E = 8V, k <= 8): the 8 lanes of group g take
+// token 4q + g; lane j holds experts c*32 + 4j + r (c < V/4, r < 4), so each
+// 16-byte load or store of a chunk c covers 128 contiguous bytes of the row.
+//
+// Top-k mask without k argmax rounds: every lane keeps the three largest of
+// its V probs; k extraction rounds over those lists (each round the group's
+// largest head is popped) give a value tau with at least k entries >= tau
+// (the k popped ones), so the entries >= tau include the top k.  The head
+// keys carry the lane in their 3 low bits so that one head is popped per
+// round; tau is the k-th popped key with those bits cleared, which is at most
+// the popped entries' values.  When exactly k entries are >= tau, they are
+// the mask; otherwise (a lane held more than three of the top k, or ties)
+// the least candidate -- smallest prob, then highest expert -- is dropped
+// until k remain.  A row whose score sum is not finite is redone by the whole
+// warp with the per-row path above.
+// --------------------------------------------------------------------------
+constexpr int kQuadThreads = 256;
+
+template <int V>
+__device__ __noinline__ void score_row_warp_out_of_line(long long t, int k, int score_fn, const float* logits,
+                                                        float* probs, uint8_t* rmap, int* hist,
+                                                        unsigned long long* list, int lane) {
+  score_row_warp<V / 4>(t, 8 * V, k, score_fn, logits, probs, rmap, hist, list, lane);
+}
+
+template <int V>
+__global__ void __launch_bounds__(kQuadThreads, V >= 32 ? 2 : 3) aux_scores_quad_kernel(int T, int k, int score_fn,
+                                                                      const float* __restrict__ logits,
+                                                                      float* __restrict__ probs,
+                                                                      uint8_t* __restrict__ rmap,
+                                                                      int32_t* __restrict__ tpe, void* ws) {
+  constexpr int E = 8 * V, NC = V / 4;
+  extern __shared__ int hist[];  // [E], then per warp 32 keys for the per-row path
+  const unsigned FULL = 0xffffffffu;
+  pdl_entry();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 3, j = lane & 7;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int nw = blockDim.x >> 5;
+  unsigned long long* list = reinterpret_cast<unsigned long long*>(hist + E) + warp * 32;
+
+  // routing-map bytes of this lane's experts summed over its tokens, 4 per word
+  uint32_t cnt4[NC];
+#pragma unroll
+  for (int c = 0; c < NC; ++c) cnt4[c] = 0u;
+  auto flush = [&]() {  // 4 groups x at most 63 tokens per byte: no carry
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+      uint32_t v = cnt4[c];
+      v += __shfl_xor_sync(FULL, v, 8);
+      v += __shfl_xor_sync(FULL, v, 16);
+      if (g == 0 && v) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int n = (v >> (8 * r)) & 255;
+          if (n) atomicAdd(&hist[c * 32 + 4 * j + r], n);
+        }
+      }
+      cnt4[c] = 0u;
+    }
+  };
+
+  const long long nq = ((long long)T + 3) >> 2;
+  const long long qstride = (long long)gridDim.x * nw;
+  int since_flush = 0;
+  // the next group's rows are loaded while this one is scored
+  float4 nx[NC];
+  auto load_quad = [&](long long qq) {
+    const long long tt = 4 * qq + g;
+    const float* row = logits + tt * E + 4 * j;
+#pragma unroll
+    for (int c = 0; c < NC; ++c)
+      nx[c] = (qq < nq && tt < T) ? __ldcs(reinterpret_cast<const float4*>(row + c * 32))
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+  load_quad((long long)blockIdx.x * nw + warp);
+  for (long long q = (long long)blockIdx.x * nw + warp; q < nq; q += qstride) {
+    const long long t = 4 * q + g;
+    const bool tv = t < T;
+    float p[V];
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+      p[4 * c] = nx[c].x;
+      p[4 * c + 1] = nx[c].y;
+      p[4 * c + 2] = nx[c].z;
+      p[4 * c + 3] = nx[c].w;
+    }
+    load_quad(q + qstride);
+    float sum = 0.0f;
+    if (score_fn == MOE_SOFTMAX) {
+      float m = p[0];
+#pragma unroll
+      for (int i = 1; i < V; ++i) m = fmaxf(m, p[i]);
+      m = fmaxf(m, __shfl_xor_sync(FULL, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(FULL, m, 2));
+      m = fmaxf(m, __shfl_xor_sync(FULL, m, 4));
+#pragma unroll
+      for (int i = 0; i < V; ++i) {
+        p[i] = expf(p[i] - m);
+        sum += p[i];
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < V; ++i) {
+        p[i] = sigmoid_f32(p[i]);
+        sum += p[i];
+      }
+    }
+    sum += __shfl_xor_sync(FULL, sum, 1);
+    sum += __shfl_xor_sync(FULL, sum, 2);
+    sum += __shfl_xor_sync(FULL, sum, 4);
+#pragma unroll
+    for (int i = 0; i < V; ++i) p[i] = p[i] / sum;
+    const bool hard = tv && !isfinite(sum);  // group-uniform
+    const bool fast = tv && !hard;
+
+    // the three largest probs of this lane (fast rows: every prob >= 0)
+    float a1 = -1.0f, a2 = -1.0f, a3 = -1.0f;
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+      a3 = fmaxf(a3, fminf(a2, p[i]));
+      a2 = fmaxf(a2, fminf(a1, p[i]));
+      a1 = fmaxf(a1, p[i]);
+    }
+    const uint32_t tag = 7u - (uint32_t)j;  // distinct per lane of a group
+    uint32_t h1 = (__float_as_uint(a1) & ~7u) | tag, h2 = (__float_as_uint(a2) & ~7u) | tag,
+             h3 = (__float_as_uint(a3) & ~7u) | tag, mx = 0u;
+    for (int r = 0; r < k; ++r) {
+      mx = h1;
+      mx = max(mx, __shfl_xor_sync(FULL, mx, 1));
+      mx = max(mx, __shfl_xor_sync(FULL, mx, 2));
+      mx = max(mx, __shfl_xor_sync(FULL, mx, 4));
+      const bool win = h1 == mx;
+      h1 = win ? h2 : h1;
+      h2 = win ? h3 : h2;
+      h3 = win ? 0u : h3;
+    }
+    const float tau = __uint_as_float(mx & ~7u);
+    uint32_t cm = 0u;
+#pragma unroll
+    for (int i = 0; i < V; ++i) cm |= (p[i] >= tau ? 1u : 0u) << i;
+    int cnt = __popc(cm);
+    cnt += __shfl_xor_sync(FULL, cnt, 1);
+    cnt += __shfl_xor_sync(FULL, cnt, 2);
+    cnt += __shfl_xor_sync(FULL, cnt, 4);
+    int excess = fast ? cnt - k : 0;  // >= 0; group-uniform
+    while (__any_sync(FULL, excess > 0)) {
+      // drop the group's least candidate: smallest prob, then highest expert
+      unsigned long long lk = ~0ull;
+      int li = 0;
+#pragma unroll
+      for (int i = 0; i < V; ++i) {
+        const unsigned long long key =
+            ((unsigned long long)__float_as_uint(p[i]) << 32) | (uint32_t)(0xffff - ((i >> 2) * 32 + 4 * j + (i & 3)));
+        if (((cm >> i) & 1u) && key < lk) {
+          lk = key;
+          li = i;
+        }
+      }
+      unsigned long long gk = lk;
+#pragma unroll
+      for (int off = 1; off < 8; off <<= 1) {
+        const unsigned long long o = shfl_xor_u64(FULL, gk, off);
+        gk = o < gk ? o : gk;
+      }
+      if (excess > 0 && lk == gk) cm &= ~(1u << li);
+      excess -= excess > 0 ? 1 : 0;
+    }
+    if (fast) {
+      float* prow = probs + t * E + 4 * j;
+      uint8_t* mrow = rmap + t * E + 4 * j;
+#pragma unroll
+      for (int c = 0; c < NC; ++c) {
+        __stcs(reinterpret_cast<float4*>(prow + c * 32), make_float4(p[4 * c], p[4 * c + 1], p[4 * c + 2], p[4 * c + 3]));
+        const uint32_t b = (((cm >> (4 * c)) & 15u) * 0x00204081u) & 0x01010101u;  // bit r -> byte r
+        __stcs(reinterpret_cast<unsigned int*>(mrow + c * 32), b);
+        cnt4[c] += b;
+      }
+    }
+    // rows with a non-finite sum: the whole warp, one row at a time
+    for (uint32_t hb = __ballot_sync(FULL, hard && j == 0); hb; hb &= hb - 1) {
+      const int gg = (__ffs(hb) - 1) >> 3;
+      score_row_warp_out_of_line<V>(4 * q + gg, k, score_fn, logits, probs, rmap, hist, list, lane);
+    }
+    if (++since_flush == 63) {
+      flush();
+      since_flush = 0;
+    }
+  }
+  flush();
+  publish_counts(E, hist, tpe, ws);
+}
+
 // --------------------------------------------------------------------------
 // loss forward: one pass over probs; fixed grid; deterministic reduction
 // --------------------------------------------------------------------------
@@ -271,12 +476,47 @@ __global__ void __launch_bounds__(kAuxThreads, 2) aux_loss_fwd_kernel(long long 
   __shared__ int last;
   WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
   AuxWs w = aux_ws(ws, E);
-  for (int e = threadIdx.x; e < E; e += blockDim.x) tpe_s[e] = (float)tpe[e];
-  __syncthreads();
-  // each block owns a contiguous range of elements; threads stride through it
-  const long long per = (((n + gridDim.x - 1) / gridDim.x) + 3) & ~3LL;  // multiple of 4: float4 ranges
+  // each block owns a contiguous range of elements (whole rows when E is a
+  // multiple of 4); threads stride through it
+  const long long rows = n / E;
+  const long long per = (E & 3) == 0 ? ((rows + gridDim.x - 1) / gridDim.x) * E
+                                     : (((n + gridDim.x - 1) / gridDim.x) + 3) & ~3LL;  // float4 ranges
   const long long b0 = (long long)blockIdx.x * per, b1 = min(n, b0 + per);
   float acc = 0.0f;
+  if ((E & 3) == 0 && ((blockDim.x * 4) % (unsigned)E) == 0 && (reinterpret_cast<uintptr_t>(tpe) & 15) == 0) {
+    // every float4 a thread loads covers the same four columns: sum the
+    // float4s, then one dot product with those columns' counts
+    const long long q1 = b1 >> 2;
+    const float4* base = reinterpret_cast<const float4*>(probs) + (b0 >> 2);
+    const int nq = (int)(q1 - (b0 >> 2));
+    constexpr int kB = 16;
+    float4 v[kB];
+#pragma unroll
+    for (int b = 0; b < kB; ++b) {
+      const int l = threadIdx.x + b * (int)blockDim.x;
+      v[b] = l < nq ? __ldcs(base + l) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const int e = (int)((threadIdx.x * 4) % (unsigned)E);
+    const int4 c4 = __ldg(reinterpret_cast<const int4*>(tpe + e));
+    float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int b = 0; b < kB; ++b) {
+      s4.x += v[b].x;
+      s4.y += v[b].y;
+      s4.z += v[b].z;
+      s4.w += v[b].w;
+    }
+    for (int l = threadIdx.x + kB * (int)blockDim.x; l < nq; l += (int)blockDim.x) {
+      const float4 u = __ldcs(base + l);
+      s4.x += u.x;
+      s4.y += u.y;
+      s4.z += u.z;
+      s4.w += u.w;
+    }
+    acc = fmaf(s4.x, (float)c4.x, fmaf(s4.y, (float)c4.y, fmaf(s4.z, (float)c4.z, s4.w * (float)c4.w)));
+  } else {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) tpe_s[e] = (float)tpe[e];
+  __syncthreads();
   if ((E & 3) == 0 && (b0 & 3) == 0) {
     const long long q1 = b1 >> 2;
     const float4* base = reinterpret_cast<const float4*>(probs) + (b0 >> 2);
@@ -307,6 +547,7 @@ __global__ void __launch_bounds__(kAuxThreads, 2) aux_loss_fwd_kernel(long long 
     for (long long i = (q1 << 2) + threadIdx.x; i < b1; i += blockDim.x) acc = fmaf(probs[i], tpe_s[i % E], acc);
   } else {
     for (long long i = b0 + threadIdx.x; i < b1; i += blockDim.x) acc = fmaf(probs[i], tpe_s[i % E], acc);
+  }
   }
   double d = (double)acc;
 #pragma unroll
@@ -737,9 +978,29 @@ extern "C" int moe_aux_scores(int32_t T, int32_t E, int32_t k, int32_t score_fn,
   if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
   if (!tokens_per_expert || (T > 0 && (!logits || !probs || !routing_map))) return MOE_ERR_INVALID_ARG;
   if (!ws || ws_bytes < aux_ws_bytes(E)) return MOE_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool aligned = ((reinterpret_cast<uintptr_t>(logits) | reinterpret_cast<uintptr_t>(probs) |
+                         reinterpret_cast<uintptr_t>(routing_map)) & 15) == 0;
+  if (aligned && k <= 8 && (E == 64 || E == 128 || E == 256)) {
+    // four tokens per warp; enough warps for every SM, each taking a few quads
+    const long long nq = ((long long)T + 3) / 4;
+    const int grid = (int)std::max(1LL, std::min<long long>((nq + kQuadThreads / 32 - 1) / (kQuadThreads / 32),
+                                                            (long long)sm_count() * 3));
+    const size_t smem = (size_t)E * sizeof(int) + (size_t)(kQuadThreads / 32) * 32 * 8;
+    cudaError_t err = cudaSuccess;
+    if (E == 64)
+      err = launch_pdl(aux_scores_quad_kernel<8>, dim3(grid), dim3(kQuadThreads), smem, st, T, k, score_fn, logits,
+                       probs, routing_map, tokens_per_expert, ws);
+    else if (E == 128)
+      err = launch_pdl(aux_scores_quad_kernel<16>, dim3(grid), dim3(kQuadThreads), smem, st, T, k, score_fn, logits,
+                       probs, routing_map, tokens_per_expert, ws);
+    else
+      err = launch_pdl(aux_scores_quad_kernel<32>, dim3(grid), dim3(kQuadThreads), smem, st, T, k, score_fn, logits,
+                       probs, routing_map, tokens_per_expert, ws);
+    return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  }
   const int vpl = pick_vpl(E);
   const int grid = std::max(1, std::min((T + 15) / 16, sm_count() * 3));  // 3 blocks per SM (40 registers)
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   // histogram, then 32 packed candidate keys per warp
   const size_t smem = (size_t)((E + 1) & ~1) * sizeof(int) + (size_t)(kScoreThreads / 32) * 32 * 8;
   cudaError_t err = cudaSuccess;
