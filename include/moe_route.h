@@ -459,6 +459,18 @@ int moe_debug_sigmoid_proxy_error(const float* x, const float* b, int64_t n, int
                                   float* delta, void* stream);
 
 /*
+ * Test hook for the division the aux-scores kernel uses in place of one IEEE
+ * division per entry: a / b from the reciprocal 1/b (one IEEE division per
+ * row) and two fused-multiply-add corrections (Markstein's method), within
+ * its range (a >= 2^-60, 2^-20 <= b <= 2^20).  Counts, into *mismatches
+ * (device uint32, zeroed by the caller), the pairs in range whose result
+ * differs in any bit from the IEEE quotient a[i] / b[i]; pairs out of range
+ * are skipped.  a, b: n device floats.  MOE_ERR_INVALID_ARG for null
+ * pointers with n > 0.
+ */
+int moe_debug_div_check(const float* a, const float* b, int64_t n, uint32_t* mismatches, void* stream);
+
+/*
  * Test hook for moe_route_no_alloc_status: records `code` (negative) in the
  * status word of the no-alloc workspace on the current device, as a kernel's
  * bounds check would (first error wins), without running a route.

@@ -155,6 +155,39 @@ def test_aux_loss_fwd_unaligned_counts_and_ragged_rows():
         assert abs(float(loss.item()) - ref) <= RTOL * abs(ref)
 
 
+def test_division_by_reciprocal_matches_ieee_quotient():
+    """The aux-scores kernel divides a row's entries by their sum through one reciprocal and two fused
+    multiply-add corrections (Markstein's method); that must give the IEEE quotient bit for bit.  Random
+    pairs over the method's whole range, pairs whose first product is least accurate (numerator mantissa
+    near 2, denominator mantissa near 1 and near 2), exact and near-exact multiples, and the softmax
+    rows of the aux workload."""
+    g = torch.Generator().manual_seed(17)
+    n = 1 << 24
+
+    def rand_float(lo_exp, hi_exp, mant=None):
+        e = torch.randint(lo_exp, hi_exp + 1, (n,), generator=g).to(torch.float64)
+        m = torch.rand(n, generator=g, dtype=torch.float64) + 1.0 if mant is None else mant
+        return (m * torch.pow(2.0, e)).to(torch.float32)
+
+    cases = []
+    b = rand_float(-20, 19)
+    cases.append((rand_float(-60, 19), b))                                   # anything in range
+    cases.append((b * rand_float(-40, 0), b))                                # quotients <= 2
+    near2 = 2.0 - torch.rand(n, generator=g, dtype=torch.float64) * 2.0 ** -10
+    near1 = 1.0 + torch.rand(n, generator=g, dtype=torch.float64) * 2.0 ** -10
+    cases.append((rand_float(-30, 0, near2), rand_float(-10, 10, near1)))
+    cases.append((rand_float(-30, 0, near2), rand_float(-10, 10, near2)))
+    cases.append((rand_float(-30, 0, near1), rand_float(-10, 10, near2)))
+    k = torch.randint(1, 1 << 20, (n,), generator=g).to(torch.float32)
+    cases.append((b * k, b))                                                 # exact multiples
+    cases.append((torch.nextafter(b * k, torch.full_like(b, float("inf"))), b))
+    lg = W.aux_inputs(W.QWEN3_AUX)["logits"]
+    z = torch.exp(lg.double() - lg.double().max(1, keepdim=True).values).float()
+    cases.append((z.reshape(-1), z.sum(1, keepdim=True).expand_as(z).reshape(-1).contiguous()))
+    for a_, b_ in cases:
+        assert B.debug_div_check(a_.contiguous().cuda(), b_.contiguous().cuda()) == 0
+
+
 def test_aux_uniform_closed_form_on_gpu():
     T, E, k, coeff = 4096, 128, 8, 1e-2
     g = B.aux_scores(torch.zeros(T, E, device="cuda"), k)

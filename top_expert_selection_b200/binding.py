@@ -35,7 +35,7 @@ _TORCH = {F32: torch.float32, BF16: torch.bfloat16}
 # every symbol the C header declares (checked by the CPU test suite)
 EXPORTED = (
     "moe_error_string", "moe_workspace_init", "moe_status", "moe_route_capacity",
-    "moe_route_workspace_bytes", "moe_route", "moe_aux_workspace_bytes", "moe_aux_scores", "moe_aux_scores_bwd", "moe_aux_scores_bwd_logits",
+    "moe_route_workspace_bytes", "moe_route", "moe_aux_workspace_bytes", "moe_aux_scores", "moe_aux_scores_bwd", "moe_aux_scores_bwd_logits", "moe_debug_div_check",
     "moe_route_weights_bwd",
     "moe_aux_loss_fwd", "moe_aux_loss_bwd", "moe_dispatch", "moe_combine",
     "moe_rmsnorm_router_topk_workspace_bytes", "moe_rmsnorm_router_topk", "moe_debug_wait_timeout",
@@ -96,6 +96,7 @@ def lib() -> ctypes.CDLL:
             "moe_aux_loss_bwd": ([i32, i32, i32, i32, f32, P, P, P, P, P, P], ctypes.c_int),
             "moe_aux_scores_bwd": ([i32, i32, i32, P, P, P, P], ctypes.c_int),
             "moe_aux_scores_bwd_logits": ([i32, i32, i32, P, P, P, P], ctypes.c_int),
+            "moe_debug_div_check": ([P, P, ctypes.c_int64, P, P], ctypes.c_int),
             "moe_route_weights_bwd": ([RP, P, P, P, P, P, sz, P], ctypes.c_int),
             "moe_dispatch": ([i32, i32, i32, i32, P, P, P, P, i64, P, P], ctypes.c_int),
             "moe_combine": ([i32, i32, i32, i32, P, i64, P, P, i32, P, P, sz, P], ctypes.c_int),
@@ -348,6 +349,13 @@ def aux_scores_bwd_logits(logits: torch.Tensor, grad_probs: torch.Tensor, score_
     gl = torch.empty_like(logits)
     aux_scores_bwd_logits_into(logits, grad_probs, gl, score_fn)
     return gl
+
+
+def debug_div_check(a: torch.Tensor, b: torch.Tensor) -> int:
+    """Pairs (in the method's range) where the reciprocal-and-corrections quotient differs from a / b."""
+    bad = torch.zeros(1, dtype=torch.int32, device=a.device)
+    _check(lib().moe_debug_div_check(_p(a), _p(b), a.numel(), _p(bad), _stream(None)), "moe_debug_div_check")
+    return int(bad.item())
 
 
 def aux_scores_bwd(probs: torch.Tensor, grad_probs: torch.Tensor, score_fn: int = SOFTMAX) -> torch.Tensor:

@@ -229,6 +229,10 @@ __device__ __forceinline__ void score_row_warp(long long t, int E, int k, int sc
 
 // The block's counts into the accumulator; the last block to finish publishes
 // them to tokens_per_expert and clears the accumulator.
+// The block's atomics are ordered before its ticket by the barrier and thread
+// 0's fence (a fence orders what its thread has observed, which the barrier
+// makes the other threads' atomics); the other threads do not fence, so they
+// do not wait for their own probs and routing-map stores to drain.
 __device__ __forceinline__ void publish_counts(int E, const int* hist, int32_t* __restrict__ tpe, void* ws) {
   WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
   AuxWs w = aux_ws(ws, E);
@@ -236,9 +240,11 @@ __device__ __forceinline__ void publish_counts(int E, const int* hist, int32_t* 
   for (int e = threadIdx.x; e < E; e += blockDim.x)
     if (hist[e]) atomicAdd(&w.tpe_acc[e], hist[e]);
   __shared__ int last;
-  __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) last = (atomicAdd(&hdr->ticket, 1u) == gridDim.x - 1);
+  if (threadIdx.x == 0) {
+    __threadfence();
+    last = (atomicAdd(&hdr->ticket, 1u) == gridDim.x - 1);
+  }
   __syncthreads();
   if (last) {
     __threadfence();
@@ -295,7 +301,7 @@ __device__ __noinline__ void score_row_warp_out_of_line(long long t, int k, int 
 }
 
 template <int V>
-__global__ void __launch_bounds__(kQuadThreads, V >= 32 ? 2 : 3) aux_scores_quad_kernel(int T, int k, int score_fn,
+__global__ void __launch_bounds__(kQuadThreads, V >= 32 ? 2 : 4) aux_scores_quad_kernel(int T, int k, int score_fn,
                                                                       const float* __restrict__ logits,
                                                                       float* __restrict__ probs,
                                                                       uint8_t* __restrict__ rmap,
@@ -381,8 +387,22 @@ __global__ void __launch_bounds__(kQuadThreads, V >= 32 ? 2 : 3) aux_scores_quad
     sum += __shfl_xor_sync(FULL, sum, 1);
     sum += __shfl_xor_sync(FULL, sum, 2);
     sum += __shfl_xor_sync(FULL, sum, 4);
+    // p / sum: one reciprocal per row and two corrections per entry give the
+    // IEEE quotient; rows with an entry or sum outside that method's range
+    // divide directly
+    {
+      bool direct = !(sum >= kDivMinDen && sum <= kDivMaxDen);
 #pragma unroll
-    for (int i = 0; i < V; ++i) p[i] = p[i] / sum;
+      for (int i = 0; i < V; ++i) direct |= p[i] < kDivMinNum;
+      if (__any_sync(FULL, direct)) {
+#pragma unroll
+        for (int i = 0; i < V; ++i) p[i] = p[i] / sum;
+      } else {
+        const float y = 1.0f / sum;
+#pragma unroll
+        for (int i = 0; i < V; ++i) p[i] = div_rn_by_recip(p[i], sum, y);
+      }
+    }
     const bool hard = tv && !isfinite(sum);  // group-uniform
     const bool fast = tv && !hard;
 
@@ -970,6 +990,30 @@ extern "C" int moe_aux_workspace_bytes(int32_t num_tokens, int32_t num_experts, 
   return MOE_OK;
 }
 
+// Test hook: div_rn_by_recip(a[i], b[i], 1/b[i]) against the IEEE quotient
+// a[i] / b[i], bit for bit, for pairs inside the method's range; counts the
+// mismatches into *mismatches (device, zeroed by the caller).
+static __global__ void div_check_kernel(const float* __restrict__ a, const float* __restrict__ b, long long n,
+                                 unsigned int* mismatches) {
+  unsigned int bad = 0;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const float x = a[i], d = b[i];
+    if (!(x >= kDivMinNum && d >= kDivMinDen && d <= kDivMaxDen)) continue;
+    const float y = 1.0f / d;
+    bad += __float_as_uint(div_rn_by_recip(x, d, y)) != __float_as_uint(x / d);
+  }
+  if (bad) atomicAdd(mismatches, bad);
+}
+
+extern "C" int moe_debug_div_check(const float* a, const float* b, int64_t n, uint32_t* mismatches, void* stream) {
+  if (n < 0 || (n > 0 && (!a || !b || !mismatches))) return MOE_ERR_INVALID_ARG;
+  if (n == 0) return MOE_OK;
+  const int grid = (int)std::min<int64_t>((n + 255) / 256, 4096);
+  div_check_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a, b, (long long)n,
+                                                                            reinterpret_cast<unsigned int*>(mismatches));
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 extern "C" int moe_aux_scores(int32_t T, int32_t E, int32_t k, int32_t score_fn, const float* logits, float* probs,
                               uint8_t* routing_map, int32_t* tokens_per_expert, void* ws, size_t ws_bytes,
                               void* stream) {
@@ -984,8 +1028,9 @@ extern "C" int moe_aux_scores(int32_t T, int32_t E, int32_t k, int32_t score_fn,
   if (aligned && k <= 8 && (E == 64 || E == 128 || E == 256)) {
     // four tokens per warp; enough warps for every SM, each taking a few quads
     const long long nq = ((long long)T + 3) / 4;
+    const int per_sm = E == 256 ? 2 : 4;  // resident blocks (the kernel's launch bounds)
     const int grid = (int)std::max(1LL, std::min<long long>((nq + kQuadThreads / 32 - 1) / (kQuadThreads / 32),
-                                                            (long long)sm_count() * 3));
+                                                            (long long)sm_count() * per_sm));
     const size_t smem = (size_t)E * sizeof(int) + (size_t)(kQuadThreads / 32) * 32 * 8;
     cudaError_t err = cudaSuccess;
     if (E == 64)

@@ -73,6 +73,24 @@ __device__ __forceinline__ unsigned long long shfl_xor_u64(unsigned mask, unsign
   return ((unsigned long long)hi << 32) | lo;
 }
 
+// a / b rounded to nearest even, given y = 1/b rounded to nearest (one IEEE
+// division shared by every a over the same b).  q0 = a*y is within 1.5 ulp of
+// a/b; the correction q1 = q0 + (a - b*q0)*y (two fused multiply-adds) is
+// within half an ulp plus a tiny fraction of one, so q1 is a faithful
+// quotient, the remainder a - b*q1 is exact, and q1 + (a - b*q1)*y rounded to
+// nearest is the correctly rounded quotient (Markstein, "Computation of
+// elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
+// Dev. 34(1), 1990).  Away from underflow only: callers keep a >= 2^-60 and
+// 2^-20 <= b <= 2^20 (positive), and take the IEEE division otherwise.
+__device__ __forceinline__ float div_rn_by_recip(float a, float b, float y) {
+  const float q0 = a * y;
+  const float q1 = fmaf(fmaf(-q0, b, a), y, q0);
+  return fmaf(fmaf(-q1, b, a), y, q1);
+}
+constexpr float kDivMinNum = 0x1p-60f;  // div_rn_by_recip's range: a >= kDivMinNum,
+constexpr float kDivMinDen = 0x1p-20f;  // kDivMinDen <= b <= kDivMaxDen
+constexpr float kDivMaxDen = 0x1p20f;
+
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
   return __uint_as_float(((uint32_t)b) << 16);
 }
