@@ -78,7 +78,7 @@ def route_source_hash() -> str:
 
 def ncu_traffic_per_launch():
     """DRAM bytes per launch from the committed ncu summary, if it was taken on this exact source."""
-    path = os.path.join(ROOT, "profiles", "route_kernel_dsv3_grouped_sigmoid.txt")
+    path = os.path.join(ROOT, "profiles", "route_select_permute_dsv3_grouped_sigmoid.txt")
     try:
         kv = {}
         with open(path) as f:
