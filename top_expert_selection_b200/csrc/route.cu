@@ -1062,6 +1062,17 @@ __global__ void __launch_bounds__(kPermThreads, 1) route_permute_kernel(RouteArg
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");  // the table and the parked ranks are the selection's output
 
+  unsigned int ticket = 0u;  // thread 0: this block's place among those that have read the group totals
+  auto release_totals = [&]() {
+    __syncthreads();
+    if (threadIdx.x == 0) base[E + E + 1] = ticket == (unsigned)a.G - 1 ? 1 : 0;
+    __syncthreads();
+    if (base[E + E + 1]) {
+      for (int i = threadIdx.x; i < a.NG * E; i += kPermThreads) a.gtot[i] = 0u;
+      if (threadIdx.x == 0) a.hdr->ticket = 0u;
+    }
+  };
+
   // this block's first parked selections, loaded while the table is summed
   constexpr int kPre = 2;
   int pre[kPre];
@@ -1117,13 +1128,9 @@ __global__ void __launch_bounds__(kPermThreads, 1) route_permute_kernel(RouteArg
       base[e] = (int)pre_e;
     }
     __syncthreads();
-    // the last block to have read the group totals clears them for the next call
-    if (threadIdx.x == 0) base[E + E + 1] = (atomicAdd(&a.hdr->ticket, 1u) == (unsigned)a.G - 1) ? 1 : 0;
-    __syncthreads();
-    if (base[E + E + 1]) {
-      for (int i = threadIdx.x; i < a.NG * E; i += kPermThreads) a.gtot[i] = 0u;
-      if (threadIdx.x == 0) a.hdr->ticket = 0u;
-    }
+    // this block has read the group totals: take a ticket now, look at it at
+    // the end (the last block to have read them clears them for the next call)
+    if (threadIdx.x == 0) ticket = atomicAdd(&a.hdr->ticket, 1u);
   }
   scan_padded_offsets(cnt, offs, E, a.tile);
   const int P = offs[E];
@@ -1172,6 +1179,7 @@ __global__ void __launch_bounds__(kPermThreads, 1) route_permute_kernel(RouteArg
   //      and its padding rows follow its count ----
   if (P / a.tile > a.max_tiles || P > a.max_padded) {
     if (threadIdx.x == 0) record_bounds(a.hdr);
+    release_totals();
     return;
   }
   const int nwarps = blockDim.x >> 5;
@@ -1183,6 +1191,7 @@ __global__ void __launch_bounds__(kPermThreads, 1) route_permute_kernel(RouteArg
     }
     for (int r = lim + lane; r < row1; r += 32) a.p2t[r] = -1;
   }
+  release_totals();
 }
 
 // ---------------------------------------------------------------------------
