@@ -354,8 +354,8 @@ __device__ void select_row(const DecodeArgs& a, int t, int lane, const float* ro
 // eps) in double kept as r_hi + r_lo, then x*gamma*r rounded once to bf16
 // (normalize8 / normalize8_exact) into out_norm.  gamma is read before the
 // dependency wait (a weight, not written by the preceding kernel).
-constexpr int kNormThreads = 256;
-constexpr int kNormKeep = 4;  // 16-byte groups a thread keeps in registers (H <= 8192)
+constexpr int kNormThreads = 512;
+constexpr int kNormKeep = 2;  // 16-byte groups a thread keeps in registers (H <= 8192)
 
 __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const DecodeArgs a) {
   __shared__ double red[kNormThreads / 32];
@@ -575,9 +575,22 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const DecodeArgs a)
   const int tp = a.TG * a.TGS, ep = a.NG * kExpGroup;
   for (int e = threadIdx.x; e < a.E; e += kSelThreads) {
     const float* p = a.part + (size_t)t * ep + e;
-    float sum = 0.0f;  // slice order (a deeper unroll measured slower)
+    float sum = 0.0f;  // slice order
+    if constexpr (R == 1) {
+      // up to 256 experts: 4 loads in flight per thread (measured faster here than 16)
 #pragma unroll 4
-    for (int s = 0; s < a.KS; ++s) sum += __ldcg(p + (size_t)s * tp * ep);
+      for (int s = 0; s < a.KS; ++s) sum += __ldcg(p + (size_t)s * tp * ep);
+    } else {
+      // more experts: 16 slices' loads in flight at a time (one L2 round trip for KS <= 16)
+      for (int s0 = 0; s0 < a.KS; s0 += 16) {
+        float v[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = s0 + j < a.KS ? __ldcg(p + (size_t)(s0 + j) * tp * ep) : 0.0f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (s0 + j < a.KS) sum += v[j];
+      }
+    }
     row[e] = sum;
   }
   __syncthreads();
