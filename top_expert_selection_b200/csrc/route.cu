@@ -35,12 +35,17 @@
 //       for all its experts;
 //     - generic: a warp per token (E > 32) or a thread per token (E <= 32)
 //       with exact keys and k rounds of argmax, logits read from global memory.
+//   The segments form groups of GS consecutive segments; each selection block
+//   also adds its counts into its group's row of per-group totals (integer
+//   atomics: order-free, so the totals are deterministic).
 // route_permute_kernel (one block per segment, launched as the dependent)
-//   Every block sums all rows of the table (the expert counts) and the rows of
-//   the segments before its own (its base per expert), scans the tile-padded
-//   offsets, and turns each parked (expert, rank) into the slot offset + base +
-//   rank (deterministic, token order, no atomics); it also writes its share of
-//   the tile tables and of the padding rows of permuted_to_token.
+//   Every block adds the group totals (the expert counts; those of the groups
+//   before its own plus the table rows of its group's earlier segments give its
+//   base per expert), scans the tile-padded offsets, and turns each parked
+//   (expert, rank) into the slot offset + base + rank (deterministic, token
+//   order); it also writes its share of the tile tables and of the padding
+//   rows of permuted_to_token.  The last block to have read the group totals
+//   (a ticket) clears them for the next call.
 // Neither kernel waits on another block, so no device-side wait can time out
 // (the only bounded waits are on the block's own bulk copies).
 #include <cuda_fp16.h>
