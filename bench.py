@@ -669,6 +669,28 @@ def secondary_rows(dev, hbm):
                                                  z[4]["out_norm"], z[4]["ids"], z[4]["affinities"], None,
                                                  z[4]["ws"])) for z in dsets], 20, stream)
     del dsets
+    # expert-parallel regroup (one rank of eight, 32 local experts, H=4096 bf16, tile 128): the received
+    # rows (seeded per-(source, expert) counts summing to 65 536) into the tile-padded expert layout and
+    # back; 2 rotated sets of 537 MB in + out
+    g = torch.Generator().manual_seed(7)
+    Wr, Lr, Hr, tile = 8, 32, 4096, 128
+    cnt = torch.multinomial(torch.ones(Wr * Lr), 65536, replacement=True, generator=g).bincount(minlength=Wr * Lr)
+    counts = cnt.view(Wr, Lr).to(torch.int32).to(dev)
+    n_recv = int(cnt.sum())
+    max_pad = n_recv + Lr * (tile - 1)
+    esets = []
+    for _ in range(2):
+        recv = torch.empty((n_recv, Hr), dtype=torch.bfloat16, device=dev).normal_()
+        padded = torch.empty((max_pad, Hr), dtype=torch.bfloat16, device=dev)
+        esets.append((recv, padded, torch.empty(Lr + 1, dtype=torch.int32, device=dev),
+                      torch.empty(2, dtype=torch.int32, device=dev), torch.empty(max_pad, dtype=torch.int32, device=dev)))
+    ep_bytes = 2 * n_recv * Hr * 2 + max_pad * 4
+    us_ep = _time_calls([(lambda z=z: B.ep_regroup_into(counts, z[0], z[1], tile, z[2], z[3], z[4])) for z in esets],
+                        10, stream)
+    us_back = _time_calls([(lambda z=z: B.ep_ungroup_into(counts, z[1], z[0], tile)) for z in esets], 10, stream)
+    rows["ep_regroup"] = {"us": us_ep, "GBps": ep_bytes / us_ep / 1e3, "frac": ep_bytes / us_ep / 1e3 / hbm,
+                          "return_us": us_back, "rows": n_recv, "H": Hr, "world": Wr, "local_experts": Lr}
+    del esets
     rows["note"] = ("us per call, device time of CUDA-graph replays over input/output sets rotated past the "
                     "126 MB L2 (dispatch/combine inputs exceed it alone)")
     return rows

@@ -23,7 +23,8 @@
 //
 // Every block derives the plan (per-expert totals, padded offsets, and each
 // (source, expert) run's receive and padded starts) from the counts in shared
-// memory, then moves rows a warp each in 16-byte vectors.
+// memory, then moves rows a warp each in 16-byte vectors (four loads in flight
+// per lane before their stores).
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -35,6 +36,7 @@ namespace {
 
 constexpr int kEpThreads = 256;
 constexpr int kEpMaxRuns = 8192;  // world * local experts
+constexpr int kVec = 4;           // row copy: 16-byte vectors in flight per lane
 
 struct EpArgs {
   const int32_t* counts;  // [W][L]
@@ -159,20 +161,34 @@ __global__ void __launch_bounds__(kEpThreads) ep_regroup_kernel(EpArgs a) {
     // (a run with no rows shares its start with the next run, so the largest
     // run with start <= r < n_recv always has rows)
     const long long pr = (long long)p.pad_start[lo] + (r - p.recv_start[lo]);
-    const uint4* s = a.direction == 0 ? a.src + r * V : a.src + pr * V;
-    uint4* d = a.direction == 0 ? a.dst + pr * V : a.dst + r * V;
-    for (int v = lane; v < V; v += 32) d[v] = __ldcs(s + v);
+    const uint4* __restrict__ s = a.direction == 0 ? a.src + r * V : a.src + pr * V;
+    uint4* __restrict__ d = a.direction == 0 ? a.dst + pr * V : a.dst + r * V;
+    // kVec 16-byte loads in flight per lane before their stores
+    for (int v0 = lane; v0 < V; v0 += 32 * kVec) {
+      uint4 t[kVec];
+#pragma unroll
+      for (int u = 0; u < kVec; ++u)
+        if (v0 + 32 * u < V) t[u] = __ldcs(s + v0 + 32 * u);
+#pragma unroll
+      for (int u = 0; u < kVec; ++u)
+        if (v0 + 32 * u < V) __stcs(d + v0 + 32 * u, t[u]);
+    }
     if (a.direction == 0 && lane == 0) a.p2r[pr] = (int32_t)r;
   }
-  // padding rows of each expert (direction 0): zero, receive row -1
+  // padding rows (direction 0): zero, receive row -1; a warp per padded row,
+  // spread over the whole grid (the padded row's expert is the largest with
+  // off[e] <= row, so experts without rows are passed over)
   if (a.direction == 0) {
     const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-    for (long long e = warp_g; e < a.L; e += nwarps) {
-      const int b = p.off[e] + p.tot[e], en = p.off[e + 1];
-      for (int row = b; row < en; ++row) {
-        for (int v = lane; v < V; v += 32) a.dst[(long long)row * V + v] = z;
-        if (lane == 0) a.p2r[row] = -1;
+    for (long long row = warp_g; row < P; row += nwarps) {
+      int lo = 0, hi = a.L - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.off[mid] <= row) lo = mid; else hi = mid - 1;
       }
+      if (row < (long long)p.off[lo] + p.tot[lo]) continue;  // a received row, moved above
+      for (int v = lane; v < V; v += 32) __stcs(a.dst + row * V + v, z);
+      if (lane == 0) a.p2r[row] = -1;
     }
   }
 }
@@ -218,7 +234,7 @@ extern "C" int moe_ep_regroup(int32_t world, int32_t local_experts, int32_t H, i
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const long long warps = std::max<long long>(n_recv, local_experts);
+  const long long warps = std::max<long long>(n_recv, max_padded);
   const int grid = (int)std::max(1LL, std::min<long long>((warps * 32 + kEpThreads - 1) / kEpThreads, 4LL * sms));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (smem > 48 * 1024 &&
