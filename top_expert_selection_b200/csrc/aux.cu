@@ -26,7 +26,8 @@ namespace {
 
 constexpr int kAuxThreads = 256;
 constexpr int kAuxWarps = kAuxThreads / 32;
-constexpr int kLossBlocks = 296;  // fixed: 2 per SM on a 148-SM part; the reduction order depends on it
+constexpr int kLossBlocks = 148;  // fixed: one per SM on a 148-SM part; the reduction order depends on it
+constexpr int kLossThreads = 512;  // loss forward block (measured faster than 2 x 256 per SM)
 
 // workspace layout after the 64-byte header
 struct AuxWs {
@@ -486,12 +487,12 @@ __global__ void __launch_bounds__(kQuadThreads, V >= 32 ? 2 : 3) aux_scores_quad
 // --------------------------------------------------------------------------
 // loss forward: one pass over probs; fixed grid; deterministic reduction
 // --------------------------------------------------------------------------
-__global__ void __launch_bounds__(kAuxThreads, 2) aux_loss_fwd_kernel(long long n, int E, double C,
+__global__ void __launch_bounds__(kLossThreads, 1) aux_loss_fwd_kernel(long long n, int E, double C,
                                                                    const float* __restrict__ probs,
                                                                    const int32_t* __restrict__ tpe, float* loss,
                                                                    void* ws) {
   extern __shared__ float tpe_s[];  // [E]
-  __shared__ double red[kAuxWarps];
+  __shared__ double red[kLossThreads / 32];
   pdl_entry();
   __shared__ int last;
   WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
@@ -576,7 +577,7 @@ __global__ void __launch_bounds__(kAuxThreads, 2) aux_loss_fwd_kernel(long long 
   __syncthreads();
   if (threadIdx.x == 0) {
     double s = 0.0;
-    for (int i = 0; i < kAuxWarps; ++i) s += red[i];
+    for (int i = 0; i < kLossThreads / 32; ++i) s += red[i];
     w.partials[blockIdx.x] = s;
     __threadfence();
     last = (atomicAdd(&hdr->ticket, 1u) == gridDim.x - 1);
@@ -1064,7 +1065,7 @@ extern "C" int moe_aux_loss_fwd(int32_t T_rows, int32_t T_total, int32_t E, int3
   if (reinterpret_cast<uintptr_t>(probs) & 15) return MOE_ERR_INVALID_ARG;
   const double C = (double)coeff * (double)E / ((double)T_total * (double)k);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const cudaError_t err = launch_pdl(aux_loss_fwd_kernel, dim3(kLossBlocks), dim3(kAuxThreads),
+  const cudaError_t err = launch_pdl(aux_loss_fwd_kernel, dim3(kLossBlocks), dim3(kLossThreads),
                                      (size_t)E * sizeof(float), st, (long long)T_rows * E, E, C, probs,
                                      tokens_per_expert, loss, ws);
   return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
