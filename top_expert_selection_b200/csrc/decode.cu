@@ -275,32 +275,77 @@ __device__ void select_row(const DecodeArgs& a, int t, int lane, const float* ro
   uint32_t key[NS];
 #pragma unroll
   for (int i = 0; i < NS; ++i) key[i] = ordered_key(lg[i]);
-  uint32_t chosen = 0, avail = valid;
+  uint32_t chosen = 0;
   int my_id = 0;
-  uint32_t bk = 0u;
-  int bi = NS;  // this lane's best remaining (key, slot); slot NS = none
-  auto lane_best = [&]() {
-    bk = 0u;
-    bi = NS;
+  if constexpr (R == 1) {
+    // up to 256 experts: the lane's 8 keys sorted once, descending, by an
+    // odd-even transposition network that swaps only on a strictly larger key
+    // (stable: equal keys keep the lower slot, the lower expert, first;
+    // absent slots carry key 0 and sink), so that each round pops the head in
+    // one step instead of rescanning the lane
+    uint32_t sk[8];
+    int ss[8];
 #pragma unroll
-    for (int i = NS - 1; i >= 0; --i)
-      if (((avail >> i) & 1u) && key[i] >= bk) {  // from the top down: ties -> the lower slot (lower expert)
-        bk = key[i];
-        bi = i;
-      }
-  };
-  auto slot_expert = [&](int i) { return (i >> 3) * 256 + lane * 8 + (i & 7); };
-  lane_best();
-  for (int j = 0; j < a.k; ++j) {
-    const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
-    const uint32_t win =
-        __reduce_min_sync(0xffffffffu, (bi < NS && bk == m) ? (uint32_t)slot_expert(bi) : 0xffffffffu);
-    if (bi < NS && (uint32_t)slot_expert(bi) == win) {
-      avail &= ~(1u << bi);
-      chosen |= 1u << bi;
-      lane_best();
+    for (int i = 0; i < 8; ++i) {
+      const bool v = (valid >> i) & 1u;
+      sk[i] = v ? key[i] : 0u;
+      ss[i] = v ? i : NS;
     }
-    if (lane == j) my_id = (int)win;
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+      for (int i = r & 1; i + 1 < 8; i += 2)
+        if (sk[i + 1] > sk[i]) {
+          const uint32_t tk = sk[i];
+          sk[i] = sk[i + 1];
+          sk[i + 1] = tk;
+          const int ts = ss[i];
+          ss[i] = ss[i + 1];
+          ss[i + 1] = ts;
+        }
+    for (int j = 0; j < a.k; ++j) {
+      const uint32_t m = __reduce_max_sync(0xffffffffu, sk[0]);
+      const uint32_t win =
+          __reduce_min_sync(0xffffffffu, (ss[0] < NS && sk[0] == m) ? (uint32_t)(lane * 8 + ss[0]) : 0xffffffffu);
+      if (ss[0] < NS && (uint32_t)(lane * 8 + ss[0]) == win) {
+        chosen |= 1u << ss[0];
+#pragma unroll
+        for (int i = 0; i < 7; ++i) {
+          sk[i] = sk[i + 1];
+          ss[i] = ss[i + 1];
+        }
+        sk[7] = 0u;
+        ss[7] = NS;
+      }
+      if (lane == j) my_id = (int)win;
+    }
+  } else {
+    uint32_t avail = valid;
+    uint32_t bk = 0u;
+    int bi = NS;  // this lane's best remaining (key, slot); slot NS = none
+    auto lane_best = [&]() {
+      bk = 0u;
+      bi = NS;
+#pragma unroll
+      for (int i = NS - 1; i >= 0; --i)
+        if (((avail >> i) & 1u) && key[i] >= bk) {  // from the top down: ties -> the lower slot (lower expert)
+          bk = key[i];
+          bi = i;
+        }
+    };
+    auto slot_expert = [&](int i) { return (i >> 3) * 256 + lane * 8 + (i & 7); };
+    lane_best();
+    for (int j = 0; j < a.k; ++j) {
+      const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+      const uint32_t win =
+          __reduce_min_sync(0xffffffffu, (bi < NS && bk == m) ? (uint32_t)slot_expert(bi) : 0xffffffffu);
+      if (bi < NS && (uint32_t)slot_expert(bi) == win) {
+        avail &= ~(1u << bi);
+        chosen |= 1u << bi;
+        lane_best();
+      }
+      if (lane == j) my_id = (int)win;
+    }
   }
   if (status != MOE_OK) return;
   if (a.dbg_logits) {
