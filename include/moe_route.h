@@ -28,7 +28,8 @@
  *     (moe_workspace_init or any memset); the library leaves it consistent
  *     for the next call.  One workspace serves one stream at a time: calls
  *     that may overlap on the GPU need separate workspaces.
- *   - Inputs must be finite (no NaN or Inf logits or hidden states).
+ *   - Inputs must be finite (no NaN or Inf logits or hidden states) unless an
+ *     entry point states otherwise (moe_aux_scores).
  */
 #ifndef MOE_ROUTE_H
 #define MOE_ROUTE_H
@@ -245,6 +246,9 @@ int moe_aux_workspace_bytes(int32_t num_tokens, int32_t num_experts, size_t* byt
  *   routing_map [T,E] u8  = 1 at the token's k largest probs (ties -> lower e)
  *   tokens_per_expert [E] = column sums of routing_map (int32)
  * logits [T,E] fp32.  All pointers device, caller-owned; ws as above.
+ * A logit of -inf (a masked expert) gives a zero prob; a row whose score sum
+ * is not finite (a NaN or +inf logit) still marks exactly k experts (probs
+ * undefined).
  */
 int moe_aux_scores(int32_t T, int32_t E, int32_t k, int32_t score_fn, const float* logits,
                    float* probs, uint8_t* routing_map, int32_t* tokens_per_expert, void* ws,
